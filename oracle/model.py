@@ -1,0 +1,72 @@
+"""Oracle decode step of a whole synthetic model (TEST INFRASTRUCTURE ONLY).
+
+Drives the C oracle layer by layer; each layer's packed weights, norm weights
+and prefilled fp16 KV cache are regenerated on the host from the seed (synth/),
+so host memory holds one layer at a time even for the 70B shapes.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+import synth
+from synth import GLOBAL_LAYER, ModelSpec, tensor_id
+
+from . import decode_layer, dims_of, embed, lm_head
+
+
+def layer_tensors(spec: ModelSpec, layer: int) -> dict:
+    """Host copies of one layer's tensors, generated from the seed."""
+    q, s, hd = spec.qtype, spec.seed, spec.head_dim
+    t = {}
+    for kind in ("w_qkv", "w_o", "w_gate", "w_up", "w_down"):
+        rows, cols, qp = spec.packed(kind)
+        t[kind] = synth.blocks_host(q, s, tensor_id(layer, kind), rows, cols, qp)
+    for kind in ("attn_norm", "ffn_norm"):
+        t[kind] = synth.uniform_f32_host(s, tensor_id(layer, kind), spec.hidden, *synth.NORM_W)
+    n = spec.n_kv_heads * spec.max_ctx * hd
+    for kind in ("k_cache", "v_cache"):
+        t[kind] = synth.normal_f16_host(s, tensor_id(layer, kind), n).reshape(spec.n_kv_heads, spec.max_ctx, hd)
+    return t
+
+
+def embedding_row(spec: ModelSpec, token: int) -> np.ndarray:
+    rows, cols, qp = spec.packed("tok_embd")
+    row = synth.blocks_host(spec.qtype, spec.seed, tensor_id(GLOBAL_LAYER, "tok_embd"), 1, cols, qp, row0=token)
+    return embed(spec.qtype, row, spec.hidden, 0)
+
+
+def head_tensors(spec: ModelSpec, rows=None):
+    """(out_norm, packed LM-head rows); rows = (row0, n) for a slice of the vocabulary."""
+    vocab, cols, qp = spec.packed("output")
+    row0, n = (0, vocab) if rows is None else rows
+    W = synth.blocks_host(spec.qtype, spec.seed, tensor_id(GLOBAL_LAYER, "output"), n, cols, qp, row0=row0)
+    norm = synth.uniform_f32_host(spec.seed, tensor_id(GLOBAL_LAYER, "out_norm"), spec.hidden, *synth.NORM_W)
+    return norm, W
+
+
+def decode(spec: ModelSpec, pos: int | None = None, token: int | None = None, n_layers: int | None = None,
+           head_rows=None, keep_hidden: bool = False, layer_hook=None):
+    """Logits of one decode step (token at position pos, default n_prefill).
+
+    Returns (logits, hidden_states) where hidden_states[l] is h after layer l
+    when keep_hidden is set.  layer_hook(l, tensors) may inspect the layer's
+    tensors after the step (e.g. the KV rows written at pos).
+    """
+    pos = spec.n_prefill if pos is None else pos
+    token = spec.token() if token is None else token
+    n_layers = spec.n_layers if n_layers is None else n_layers
+    dims = dims_of(spec)
+    h = embedding_row(spec, token).copy()
+    hidden = []
+    for layer in range(n_layers):
+        t = layer_tensors(spec, layer)
+        decode_layer(dims, spec.qtype, h, pos, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"], t["w_gate"],
+                     t["w_up"], t["w_down"], t["k_cache"], t["v_cache"])
+        if keep_hidden:
+            hidden.append(h.copy())
+        if layer_hook is not None:
+            layer_hook(layer, t)
+    norm, W = head_tensors(spec, head_rows)
+    n_rows = W.shape[0]
+    logits = lm_head(spec.qtype, norm, W, n_rows, spec.hidden, spec.rms_eps, h)
+    return logits, hidden
