@@ -1,0 +1,423 @@
+#!/usr/bin/env python
+"""Benchmark of the batch-1 quantized decode path on B200.
+
+Workloads (synthetic, seeded; shapes of the ntransformer news summary's
+workloads, random weights of the Llama architecture):
+  llama70b_q6k_decode (default)  80 layers, hidden 8192, 64 q / 8 kv heads, FFN 28672,
+                                 Q6_K weights, fp16 KV cache prefilled to 8192 positions
+  llama8b_q8_0_decode            32 layers, hidden 4096, 32 q / 8 kv heads, FFN 14336,
+                                 Q8_0 weights, KV cache prefilled to 4096 positions
+  llama70b_q4k_stream            70B shape in Q4_K, layers 0-35 resident, 36-79 streamed
+                                 from pinned host memory through the two-slot HBM ring
+  gemv_q8_0_4096                 Q8_0 GEMV 4096 x 4096 (rotating over weight copies)
+
+One step = one decode step (one token); the metric is tokens per second.
+`--impl reference` times the CPU oracle (as it stands) on a bounded sample of
+the same workload instead.  Multi-GPU runs are independent replicas (the path
+does not shard): each rank decodes its own sequence; value = tokens of all ranks
+/ the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+METRIC = "batch-1 decode tok/s"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return PEAKS_FALLBACK["hbm_gbs"], "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=clocks.sm,clocks.max.sm,clocks_event_reasons.active",
+                 "--format=csv,noheader,nounits", "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        for l in self.lines:
+            parts = [p.strip() for p in l.split(",")]
+            if len(parts) < 3:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+                bits = int(parts[2], 16)
+            except ValueError:
+                continue
+            for b, name in REASON_BITS.items():
+                if bits & b and name != "gpu_idle":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- distributed
+
+def dist_setup(n_gpus):
+    rank, world = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v, world):
+    if world == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------- workloads
+
+def spec_for(name):
+    import synth
+    if name == "llama70b_q6k_decode":
+        return synth.ModelSpec(**synth.LLAMA_70B_Q6_K)
+    if name == "llama8b_q8_0_decode":
+        return synth.ModelSpec(**synth.LLAMA_8B_Q8_0)
+    if name == "llama70b_q4k_stream":
+        return synth.ModelSpec(**synth.LLAMA_70B_Q4_K)
+    raise ValueError(name)
+
+
+def kv_read_bytes(spec):
+    return spec.n_layers * 2 * spec.n_kv_heads * (spec.n_prefill + 1) * spec.head_dim * 2
+
+
+def step_bytes(spec):
+    """Algorithmic bytes of one decode step: packed weights read + KV cache read
+    (positions 0..pos) + the embedding row (vectors are negligible)."""
+    import synth
+    w = spec.n_layers * spec.layer_weight_bytes() + spec.vocab * synth.row_bytes(spec.qtype, spec.hidden)
+    return w + kv_read_bytes(spec) + synth.row_bytes(spec.qtype, spec.hidden)
+
+
+def gemv_shapes(spec):
+    """(rows, cols, launches per step) of the decode GEMVs."""
+    return [(spec.qkv_rows, spec.hidden, spec.n_layers), (spec.hidden, spec.q_dim, spec.n_layers),
+            (spec.ffn, spec.hidden, 2 * spec.n_layers), (spec.hidden, spec.ffn, spec.n_layers),
+            (spec.vocab, spec.hidden, 1)]
+
+
+def measure_gemv_roofline(ntx, model, spec, stream, iters=3):
+    """Time every decode GEMV of one step on its own (same weights, same shapes, same
+    stream) with CUDA events: the dominant kernel's achieved HBM bandwidth."""
+    import torch
+    import synth
+    x = torch.randn(max(spec.hidden, spec.ffn, spec.q_dim), device="cuda")
+    y = torch.empty(max(spec.vocab, spec.ffn, spec.qkv_rows), device="cuda")
+    launches = []
+    for t in model.layers:
+        launches.append((t["w_qkv"], spec.qkv_rows, spec.hidden))
+        launches.append((t["w_o"], spec.hidden, spec.q_dim))
+        launches.append((t["w_gate"], spec.ffn, spec.hidden))
+        launches.append((t["w_up"], spec.ffn, spec.hidden))
+        launches.append((t["w_down"], spec.hidden, spec.ffn))
+    launches.append((model.output, spec.vocab, spec.hidden))
+    nbytes = sum(r * synth.row_bytes(spec.qtype, c) + 4 * (c + r) for _, r, c in launches)
+    with torch.cuda.stream(stream):
+        for W, r, c in launches[:20]:
+            ntx.ntx_gemv_q(spec.qtype, W, r, c, x, y, stream.cuda_stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(iters):
+            for W, r, c in launches:
+                ntx.ntx_gemv_q(spec.qtype, W, r, c, x, y, stream.cuda_stream)
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / (iters * len(launches))
+    per_launch = nbytes / len(launches)
+    return per_launch / (ms * 1e-3) / 1e9, per_launch, ms
+
+
+def run_decode_bench(args, rank, world, local):
+    import torch
+    import quantized_weight_gemv_block_b200 as ntx
+    from synth.device_model import DeviceModel
+
+    name = args.workload
+    spec = spec_for(name)
+    streamed = name == "llama70b_q4k_stream"
+    n_res = 36 if streamed else None
+    t0 = time.time()
+    model = DeviceModel(spec, n_resident=n_res)
+    setup_s = time.time() - t0
+    token, pos = spec.token(), spec.n_prefill
+    stream = torch.cuda.Stream()
+    copy_stream = torch.cuda.Stream() if streamed else None
+    logits = torch.empty(spec.vocab, dtype=torch.float32, device="cuda")
+    launches_per_step = 2 + 5 * spec.n_layers + 1
+
+    def step():
+        if streamed:
+            ntx.ntx_stream_layers(model.handle, token, pos, logits, stream.cuda_stream, copy_stream.cuda_stream, 0)
+        else:
+            ntx.ntx_decode_step(model.handle, token, pos, logits, stream.cuda_stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    ms = e0.elapsed_time(e1) / args.steps
+    ms = max_over_ranks(ms, world)
+    dev_err = ntx.ntx_device_error()
+
+    # end to end through the public API: token in from the host, logits back to pinned host memory
+    host_logits = torch.empty(spec.vocab, dtype=torch.float32, pin_memory=True)
+    e2e_steps = max(3, min(args.steps, 10))
+    torch.cuda.synchronize()
+    t_e2e = time.perf_counter()
+    for _ in range(e2e_steps):
+        step()
+        with torch.cuda.stream(stream):
+            host_logits.copy_(logits, non_blocking=True)
+        stream.synchronize()
+    e2e_ms = (time.perf_counter() - t_e2e) * 1e3 / e2e_steps
+    e2e_ms = max_over_ranks(e2e_ms, world)
+
+    out = {"ms_per_step": ms, "tok_s": world * 1e3 / ms, "e2e_tok_s": world * 1e3 / e2e_ms, "setup_s": setup_s,
+           "clocks": clk.summary(), "launches": launches_per_step * args.steps, "device_error": dev_err,
+           "bytes": step_bytes(spec), "spec": spec, "model": model, "stream": stream}
+    if streamed:
+        h2d, step_ms = ntx.ntx_stream_stats(model.handle)
+        out["h2d_bytes"] = h2d
+        out["h2d_gbs"] = h2d / (ms * 1e-3) / 1e9
+        out["h2d_peak_gbs"] = measure_h2d()
+    return out
+
+
+def measure_h2d():
+    """Pinned host -> device copy bandwidth of this machine (1 GiB, best of 3)."""
+    import torch
+    n = 1 << 30
+    h = torch.empty(n, dtype=torch.uint8, pin_memory=True)
+    d = torch.empty(n, dtype=torch.uint8, device="cuda")
+    best = 0.0
+    for _ in range(3):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        d.copy_(h, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        best = max(best, n / (e0.elapsed_time(e1) * 1e-3) / 1e9)
+    del h, d
+    return best
+
+
+def cpu_baseline(spec, budget_s=20.0):
+    """The CPU oracle, as it stands, on a bounded sample of the decode step: whole
+    layers at the workload's shape (weights generated before timing) and a slice of
+    the LM head; extrapolated to one token."""
+    import numpy as np
+    import oracle
+    from oracle import model as om
+    import synth
+    oracle.build()
+    dims = oracle.dims_of(spec)
+    t = om.layer_tensors(spec, 0)
+    h = om.embedding_row(spec, spec.token()).copy()
+    n_layers_timed, t_layers = 0, 0.0
+    while t_layers < budget_s * 0.7 and n_layers_timed < spec.n_layers:
+        t0 = time.perf_counter()
+        oracle.decode_layer(dims, spec.qtype, h, spec.n_prefill, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"],
+                            t["w_gate"], t["w_up"], t["w_down"], t["k_cache"], t["v_cache"])
+        t_layers += time.perf_counter() - t0
+        n_layers_timed += 1
+    head_rows = max(256, spec.vocab // 32)
+    norm, W = om.head_tensors(spec, (0, head_rows))
+    t0 = time.perf_counter()
+    oracle.lm_head(spec.qtype, norm, W, head_rows, spec.hidden, spec.rms_eps, h)
+    t_head = (time.perf_counter() - t0) * spec.vocab / head_rows
+    s_per_tok = t_layers / n_layers_timed * spec.n_layers + t_head
+    return {"value": 1.0 / s_per_tok, "unit": "tok/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": f"{n_layers_timed} of {spec.n_layers} layers (full shape, ctx {spec.n_prefill + 1}) "
+                      f"+ {head_rows} of {spec.vocab} LM-head rows, extrapolated to one token"}
+
+
+def gemv_bench(ntx, iters=50):
+    """Q8_0 4096 x 4096 GEMV rotating over 16 weight copies (> 2 x L2)."""
+    import torch
+    import synth
+    rows = cols = 4096
+    qp = synth.sweep_qparams(synth.Q8_0)
+    rb = synth.row_bytes(synth.Q8_0, cols)
+    copies = [torch.empty(rows * rb, dtype=torch.uint8, device="cuda") for _ in range(16)]
+    for i, c in enumerate(copies):
+        synth.blocks_dev(c, synth.Q8_0, 0, 1, rows, cols, qp)
+    x = torch.empty(cols, device="cuda")
+    synth.normal_f32_dev(x, 0, 2)
+    y = torch.empty(rows, device="cuda")
+    s = torch.cuda.current_stream()
+    for c in copies:
+        ntx.ntx_gemv_q(synth.Q8_0, c, rows, cols, x, y)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(s)
+    for i in range(iters):
+        ntx.ntx_gemv_q(synth.Q8_0, copies[i % 16], rows, cols, x, y)
+    e1.record(s)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / iters
+    nbytes = rows * rb + 4 * (rows + cols)
+    return {"us": us, "gbs": nbytes / (us * 1e-6) / 1e9}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ntx", choices=["ntx", "reference"])
+    ap.add_argument("--workload", default="llama70b_q6k_decode",
+                    choices=["llama70b_q6k_decode", "llama8b_q8_0_decode", "llama70b_q4k_stream"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extras", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    rank, world, local = dist_setup(args.gpus)
+    spec = spec_for(args.workload)
+    config = {"workload": args.workload, "layers": spec.n_layers, "hidden": spec.hidden, "ffn": spec.ffn,
+              "q_heads": spec.n_q_heads, "kv_heads": spec.n_kv_heads, "vocab": spec.vocab, "format": ["q8_0", "q4_0",
+              "q4_k", "q6_k"][spec.qtype], "context": spec.n_prefill + 1, "batch": 1,
+              "l2": "inputs larger than L2 (weights %.1f GB per step)" % (step_bytes(spec) / 1e9),
+              "parallelism": "replicas" if world > 1 else "single"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        cb = None
+        vals = []
+        for i in range(args.warmup + args.steps):
+            cb = cpu_baseline(spec, budget_s=6.0)
+            if i >= args.warmup:
+                vals.append(cb["value"])
+        v = statistics.median(vals)
+        cb["value"] = v
+        print(json.dumps({"metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps,
+                          "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+                          "impl": "reference", "config": config, "cpu_baseline": cb,
+                          "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        return
+
+    import torch
+    import quantized_weight_gemv_block_b200 as ntx
+    from quantized_weight_gemv_block_b200 import build
+    import synth
+    build.build()
+    synth.build_dev()
+    torch.cuda.set_device(local)
+    r = run_decode_bench(args, rank, world, local)
+    spec, model, stream = r["spec"], r["model"], r["stream"]
+    peak, peak_kind = load_peaks()
+
+    line = {"metric": METRIC, "value": r["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded random weights and KV cache)",
+            "config": config, "clocks": r["clocks"], "gpu_launches": r["launches"],
+            "e2e": {"value": r["e2e_tok_s"], "unit": "tok/s", "h2d_bytes_per_step": 8,
+                    "d2h_bytes_per_step": 4 * spec.vocab}}
+    step_gbs = r["bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
+    line["step_hbm"] = {"bytes_per_step": r["bytes"], "achieved_gbs": step_gbs, "frac_of_%s" % peak_kind:
+                        step_gbs / peak, "frac_of_8000": step_gbs / 8000.0}
+    if args.workload == "llama70b_q4k_stream":
+        line["host_link"] = {"h2d_bytes_per_step": r["h2d_bytes"], "achieved_gbs": r["h2d_gbs"],
+                             "measured_pinned_h2d_gbs": r["h2d_peak_gbs"], "frac": r["h2d_gbs"] / r["h2d_peak_gbs"]}
+    if rank == 0:
+        gbs, per_launch, ms = measure_gemv_roofline(ntx, model, spec, stream)
+        line["roofline"] = {"bound": "hbm", "kernel": "gemv_kernel<%s>" % config["format"], "achieved": gbs,
+                            "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / peak,
+                            "traffic": None, "bytes_per_launch": per_launch, "avg_launch_us": ms * 1e3}
+        if not args.no_extras:
+            line["gemv_q8_0_4096x4096"] = gemv_bench(ntx)
+        if not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(spec)
+        if r["device_error"]:
+            line["device_error"] = r["device_error"]
+        print(json.dumps(line))
+    model.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

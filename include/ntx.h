@@ -1,0 +1,223 @@
+/*
+ * ntx.h - C ABI of the B200 (sm_100a) batch-1 quantized decode library (libntx.so).
+ *
+ * Source of the operations: the ntransformer news summary (news.hada.io topic
+ * 26894).  "Descripción general de NTransformer" lists the GGUF weight formats
+ * (Q4_0, Q8_0, Q4_K_M, Q6_K, ...); "Arquitectura y estructura del código" lists the
+ * CUDA kernels (GEMV, RMSNorm, RoPE, SwiGLU, softmax) and the model pieces
+ * (attention, FFN, normalization); "Funciones principales" names the Llama
+ * architecture pieces (RoPE, GQA, SwiGLU, RMSNorm, KV cache) and the SLEP
+ * double-buffered streaming; "Hoja de ruta de desarrollo" gives the F16 KV cache
+ * (Fase 3) and the planned public C API (Fase 5).  The pages print no formula,
+ * layout or signature; the readings used are stated per function below.
+ *
+ * Conventions (every function):
+ *  - returns ntx_status; NTX_OK = 0.  A failing call sets a thread-local message
+ *    readable with ntx_last_error().  Nothing aborts or throws across the ABI.
+ *  - arguments are checked on the host before anything is launched; a rejected
+ *    call launches nothing.
+ *  - device pointers are owned by the caller (the library never frees them) and
+ *    must stay valid until the work queued on the stream has finished.
+ *  - work is queued asynchronously on the caller's stream (`stream`, a
+ *    cudaStream_t passed as void*; NULL = legacy default stream).  Launch errors
+ *    are returned as NTX_ECUDA; errors raised while kernels run surface at the
+ *    caller's next synchronisation.  Kernels that wait on a barrier give up
+ *    after a bounded time and record a code readable with ntx_device_error().
+ *  - packed weights are row-major: row r occupies ntx_row_bytes(qtype, cols)
+ *    bytes starting at W + r * ntx_row_bytes(qtype, cols); inside a row, blocks
+ *    follow one another in the GGUF-style layouts below.
+ *
+ * Block layouts (little-endian; one block covers consecutive elements of a row):
+ *   NTX_Q8_0  34 B / 32:  fp16 d | 32 x int8 q                w = d q
+ *   NTX_Q4_0  18 B / 32:  fp16 d | 16 B; byte j: element j in the low nibble,
+ *                         element j+16 in the high nibble     w = d (q - 8)
+ *   NTX_Q4_K 144 B / 256: fp16 d | fp16 dmin | 12 B of 6-bit scales and mins |
+ *                         128 B of 4-bit codes                w = d sc_j q - dmin m_j
+ *                         (j = element / 32; code byte 32c+l holds element 64c+l in
+ *                         its low nibble and 64c+32+l in its high nibble; scales /
+ *                         mins of sub-blocks 0..3 in the low 6 bits of bytes 0..3 /
+ *                         4..7, sub-blocks 4..7 split between bytes 8..11 (low 4
+ *                         bits) and the top 2 bits of bytes 0..7)
+ *   NTX_Q6_K 210 B / 256: 128 B low code bits | 64 B high code bits | 16 x int8
+ *                         scales | fp16 d                     w = d sc_j (q - 32)
+ *                         (j = element / 16; element e, t = e % 128, h = e / 128:
+ *                         low 4 bits from ql[64h + t % 64], low nibble if t < 64
+ *                         else high nibble; high 2 bits = bits 2 (t / 32) of
+ *                         qh[32h + t % 32])
+ */
+#ifndef NTX_H
+#define NTX_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum ntx_status {
+    NTX_OK = 0,
+    NTX_EINVAL = 1,        /* bad argument (null pointer, bad size, misalignment, range) */
+    NTX_EUNSUPPORTED = 2,  /* valid but not supported (format, shape) */
+    NTX_ENOMEM = 3,        /* library-owned allocation failed */
+    NTX_ECUDA = 4,         /* a CUDA runtime call failed; see ntx_last_error() */
+    NTX_ETIMEOUT = 5       /* a bounded wait ran out */
+} ntx_status;
+
+typedef enum ntx_qtype {
+    NTX_Q8_0 = 0,
+    NTX_Q4_0 = 1,
+    NTX_Q4_K = 2,
+    NTX_Q6_K = 3
+} ntx_qtype;
+
+/* Message of the last failing ntx_* call on this thread ("" if none). */
+const char* ntx_last_error(void);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int ntx_version(void);
+
+/* Bytes of one packed row of `cols` elements; 0 if qtype is unknown or cols is
+ * not a positive multiple of the format's block size (32 or 256). */
+size_t ntx_row_bytes(int qtype, int64_t cols);
+
+/* Elements per block of qtype (32 or 256), 0 if unknown. */
+int ntx_block_elems(int qtype);
+
+/* Error code recorded by a kernel on the current device whose bounded wait ran
+ * out (0 = none), and reset it.  Synchronises the current device. */
+ntx_status ntx_device_error(uint32_t* code);
+
+/* ---------------------------------------------------------------- quantized GEMV
+ * y = W x: y[r] = sum_k dequant(W)[r, k] * x[k] for r < rows, k < cols
+ * (the GEMV kernel of "Arquitectura y estructura del código"; batch 1).
+ *   W    device, packed [rows, cols] in `qtype`; 16-byte aligned
+ *   x    device fp32 [cols];  y  device fp32 [rows] (must not overlap x or W)
+ * Accumulation is fp32; results match the exact dot product to a normwise
+ * relative error far below 2e-3.  rows >= 1; cols a multiple of the block size.
+ * Rows whose byte length is a multiple of 16 take the bulk-copy pipeline; other
+ * shapes take a simpler kernel. */
+ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t cols, const float* x, float* y,
+                      void* stream);
+
+/* Dequantize W [rows, cols] to fp32 out [rows, cols] (row-major).  The result
+ * is bit-exact: every weight is one fp32 product of exact factors (Q4_K: one
+ * rounding of d sc q - dmin m). */
+ntx_status ntx_dequant_q(int qtype, const void* W, int64_t rows, int64_t cols, float* out, void* stream);
+
+/* ------------------------------------------------------------------ decode ops */
+
+/* RMSNorm (listed in "Arquitectura y estructura del código"):
+ * y_i = x_i / sqrt(mean(x^2) + eps) * w_i, fp32, n >= 1.  x, w, y device fp32 [n];
+ * y may equal x. */
+ntx_status ntx_rmsnorm(const float* x, const float* w, float* y, int64_t n, float eps, void* stream);
+
+/* RoPE on adjacent pairs (2i, 2i+1) of every head of q [n_q_heads, head_dim] and
+ * k [n_kv_heads, head_dim], in place: rotation by pos * theta^(-2i/head_dim),
+ * the angle and its sine / cosine evaluated in double.  k may be NULL
+ * (n_kv_heads ignored).  head_dim even, pos >= 0. */
+ntx_status ntx_rope(float* q, float* k, int n_q_heads, int n_kv_heads, int head_dim, int32_t pos, float theta,
+                    void* stream);
+
+/* GQA decode attention of one query token (attention with GQA of "Funciones
+ * principales", F16 KV cache of "Hoja de ruta de desarrollo" Fase 3):
+ * q head h reads kv head g = h / (n_q_heads / n_kv_heads);
+ * out_h = sum_t softmax_t(q_h . K[g][t] / sqrt(head_dim)) V[g][t], t < n_ctx.
+ *   q       device fp32 [n_q_heads, head_dim]
+ *   k_cache, v_cache  device fp16 [n_kv_heads, max_ctx, head_dim]
+ *   out     device fp32 [n_q_heads, head_dim]
+ *   workspace / workspace_bytes: device scratch of at least
+ *           ntx_attn_workspace_bytes(...) bytes, 16-byte aligned; zero-initialised
+ *           by the caller once before first use (the kernel leaves it zeroed).
+ * head_dim == 128, n_q_heads a multiple of n_kv_heads with at most 8 q heads per
+ * kv head, 1 <= n_ctx <= max_ctx.  Calls sharing a workspace must not overlap. */
+ntx_status ntx_attn_decode(const float* q, const void* k_cache, const void* v_cache, float* out, int n_q_heads,
+                           int n_kv_heads, int head_dim, int32_t n_ctx, int32_t max_ctx, void* workspace,
+                           size_t workspace_bytes, void* stream);
+size_t ntx_attn_workspace_bytes(int n_q_heads, int n_kv_heads, int head_dim, int32_t max_ctx);
+
+/* SwiGLU (listed in "Arquitectura y estructura del código"):
+ * out_i = gate_i / (1 + e^-gate_i) * up_i, fp32 [n]. */
+ntx_status ntx_swiglu(const float* gate, const float* up, float* out, int64_t n, void* stream);
+
+/* softmax (listed in "Arquitectura y estructura del código") over one row:
+ * y_i = e^(x_i - max x) / sum_j e^(x_j - max x), fp32 [n], 1 <= n <= 2^26. */
+ntx_status ntx_softmax(const float* x, float* y, int64_t n, void* stream);
+
+/* Greedy token pick: *out_index = argmax_i x_i (lowest index among ties), device
+ * int32 output; n <= 2^26. */
+ntx_status ntx_argmax(const float* x, int64_t n, int32_t* out_index, void* stream);
+
+/* Embedding lookup: h = dequant(row `token` of E [vocab, hidden]); token is read
+ * from device memory (`token_dev`, int32) so the call can be replayed. */
+ntx_status ntx_embed(int qtype, const void* E, int64_t vocab, int64_t hidden, const int32_t* token_dev, float* h,
+                     void* stream);
+
+/* ------------------------------------------------------------------ decode step
+ * A Llama-architecture model ("Funciones principales"; model/ of "Arquitectura y
+ * estructura del código") with per-layer packed weights.  One call runs one
+ * batch-1 decode step: embedding, then per layer
+ *   xn = RMSNorm(h); [q|k|v] = W_qkv xn; RoPE(q, k, pos); K[pos] = fp16(k),
+ *   V[pos] = fp16(v); a = attention over positions 0..pos; h += W_o a;
+ *   xn = RMSNorm(h); h += W_down (silu(W_gate xn) * (W_up xn)),
+ * then logits = W_out RMSNorm(h). */
+typedef struct ntx_layer_desc {
+    const float* attn_norm;   /* device fp32 [hidden] */
+    const void* w_qkv;        /* packed [(n_q + 2 n_kv) * head_dim, hidden]: q rows, k rows, v rows */
+    const void* w_o;          /* packed [hidden, n_q * head_dim] */
+    const float* ffn_norm;    /* device fp32 [hidden] */
+    const void* w_gate;       /* packed [ffn, hidden] */
+    const void* w_up;         /* packed [ffn, hidden] */
+    const void* w_down;       /* packed [hidden, ffn] */
+    void* k_cache;            /* device fp16 [n_kv, max_ctx, head_dim] */
+    void* v_cache;            /* device fp16 [n_kv, max_ctx, head_dim] */
+} ntx_layer_desc;
+
+typedef struct ntx_model_desc {
+    int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab, max_ctx;
+    float rms_eps, rope_theta;
+    int32_t qtype;                 /* format of every packed tensor */
+    const void* tok_embd;          /* packed [vocab, hidden], device */
+    const float* out_norm;         /* device fp32 [hidden] */
+    const void* output;            /* packed [vocab, hidden], device */
+    const ntx_layer_desc* layers;  /* host array [n_layers], copied by ntx_model_create */
+    /* Layer streaming ("Streaming SLEP" of "Funciones principales"): layers
+     * [n_resident, n_layers) hold their five packed weight pointers in pinned host
+     * memory and are copied each step through a two-slot HBM ring by
+     * ntx_stream_layers.  Norm weights and KV caches of every layer stay in HBM.
+     * n_resident == n_layers: fully resident model. */
+    int32_t n_resident;
+} ntx_model_desc;
+
+typedef struct ntx_model ntx_model;
+
+/* Validate the descriptor and allocate the model's scratch (activations,
+ * attention partials, and the HBM ring when n_resident < n_layers).  The model
+ * must be used on the device that was current at creation. */
+ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** model);
+ntx_status ntx_model_destroy(ntx_model* model);
+
+/* One decode step of a fully resident model: token at position pos (attends to
+ * 0..pos, writes K/V at pos), logits device fp32 [vocab].  0 <= pos < max_ctx,
+ * 0 <= token < vocab.  Queued on `stream`.  The first call on a stream records a
+ * CUDA graph of the step that later calls replay. */
+ntx_status ntx_decode_step(ntx_model* model, int32_t token, int32_t pos, float* logits, void* stream);
+
+/* One decode step of a partly resident model: resident layers on `compute`,
+ * streamed layers copied host -> HBM ring on `copy` (cudaMemcpyAsync, one slot
+ * ahead) and computed on `compute` once their copy event has fired.  Returns
+ * after queueing if timeout_ms == 0; otherwise waits up to timeout_ms for the
+ * step to finish and returns NTX_ETIMEOUT if it has not (work stays queued). */
+ntx_status ntx_stream_layers(ntx_model* model, int32_t token, int32_t pos, float* logits, void* compute,
+                             void* copy, int64_t timeout_ms);
+
+/* Per-step counters of the last ntx_stream_layers call: bytes copied host ->
+ * device, and device milliseconds of the whole step (between the step's first
+ * and last event; valid once the step finished). */
+ntx_status ntx_stream_stats(ntx_model* model, int64_t* h2d_bytes, float* step_ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NTX_H */

@@ -1,0 +1,432 @@
+// decode.cu - the batch-1 decode step of a Llama-architecture model (model/ and
+// inference/ of the ntransformer news summary, "Arquitectura y estructura del
+// código"), and the layer-streaming ring (SLEP streaming, "Funciones
+// principales": host read, PCIe DMA and GPU compute overlapped with double
+// buffering; here pinned host memory -> a two-slot HBM ring on a copy stream).
+//
+// Per layer, five kernels:
+//   1. fused QKV GEMV: RMSNorm(h) prologue, RoPE + fp16 K/V append epilogue
+//   2. split-KV GQA attention (merge by the last CTA of each kv head)
+//   3. O GEMV, residual add into h
+//   4. fused gate/up GEMV: RMSNorm(h) prologue, SwiGLU epilogue
+//   5. down GEMV, residual add into h
+// plus the embedding before layer 0 and the RMSNorm + LM-head GEMV after the
+// last layer.  Kernels use programmatic dependent launch so each one's weight
+// stream starts while the previous one drains; the resident step is recorded
+// once as a CUDA graph and replayed, with token and position read from device
+// memory.
+#include <chrono>
+#include <cstdlib>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "ops.h"
+
+struct ntx_model {
+    ntx_model_desc d;
+    std::vector<ntx_layer_desc> layers;
+    int device = 0;
+    int64_t rb_h = 0, rb_q = 0, rb_f = 0;
+    float* h = nullptr;
+    float* q = nullptr;
+    float* att = nullptr;
+    float* act = nullptr;
+    int32_t* step = nullptr;
+    void* attn_ws = nullptr;
+    int n_split = 1;
+    bool pdl = true;
+    bool use_graph = true;
+    // CUDA graph of the resident step
+    cudaGraphExec_t graph = nullptr;
+    float* graph_logits = nullptr;
+    // streaming ring
+    uint8_t* ring = nullptr;
+    size_t slot_bytes = 0;
+    size_t off_qkv = 0, off_o = 0, off_gate = 0, off_up = 0, off_down = 0;
+    size_t sz_qkv = 0, sz_o = 0, sz_ffn = 0, sz_down = 0;
+    cudaEvent_t copy_done[2] = {nullptr, nullptr};
+    cudaEvent_t slot_free[2] = {nullptr, nullptr};
+    cudaEvent_t ev_start = nullptr, ev_end = nullptr;
+    int64_t last_h2d = 0;
+};
+
+namespace ntx {
+namespace {
+
+using gemv::Params;
+
+size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
+
+struct LayerW {
+    const void *qkv, *o, *gate, *up, *down;
+};
+
+ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl)
+{
+    const ntx_model_desc& d = m->d;
+    const ntx_layer_desc& L = m->layers[l];
+    const int qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim;
+    ntx_status st;
+    {
+        Params P{};
+        P.W = (const uint8_t*)w.qkv;
+        P.row_bytes = m->rb_h;
+        P.M = qd + 2 * kvd;
+        P.K = d.hidden;
+        P.x = m->h;
+        P.norm_w = L.attn_norm;
+        P.eps = d.rms_eps;
+        P.q_rows = qd;
+        P.kv_rows = kvd;
+        P.head_dim = d.head_dim;
+        P.max_ctx = d.max_ctx;
+        P.pos_dev = m->step + 1;
+        P.theta = d.rope_theta;
+        P.k_cache = (__half*)L.k_cache;
+        P.v_cache = (__half*)L.v_cache;
+        P.q_out = m->q;
+        P.use_pdl = pdl;
+        if ((st = gemv_launch(d.qtype, gemv::EPI_QKV, gemv::PRO_RMSNORM, P, s)) != NTX_OK) return st;
+    }
+    {
+        AttnArgs a{};
+        a.q = m->q;
+        a.k_cache = (const __half*)L.k_cache;
+        a.v_cache = (const __half*)L.v_cache;
+        a.out = m->att;
+        a.n_q_heads = d.n_q_heads;
+        a.n_kv_heads = d.n_kv_heads;
+        a.head_dim = d.head_dim;
+        a.max_ctx = d.max_ctx;
+        a.pos_dev = m->step + 1;
+        a.workspace = m->attn_ws;
+        a.n_split = m->n_split;
+        a.pdl = pdl;
+        if ((st = attn_launch(a, s)) != NTX_OK) return st;
+    }
+    {
+        Params P{};
+        P.W = (const uint8_t*)w.o;
+        P.row_bytes = m->rb_q;
+        P.M = d.hidden;
+        P.K = qd;
+        P.x = m->att;
+        P.y = m->h;
+        P.use_pdl = pdl;
+        if ((st = gemv_launch(d.qtype, gemv::EPI_ADD, gemv::PRO_X, P, s)) != NTX_OK) return st;
+    }
+    {
+        Params P{};
+        P.W = (const uint8_t*)w.gate;
+        P.W2 = (const uint8_t*)w.up;
+        P.row_bytes = m->rb_h;
+        P.M = d.ffn;
+        P.K = d.hidden;
+        P.x = m->h;
+        P.norm_w = L.ffn_norm;
+        P.eps = d.rms_eps;
+        P.y = m->act;
+        P.use_pdl = pdl;
+        if ((st = gemv_launch(d.qtype, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, P, s)) != NTX_OK) return st;
+    }
+    {
+        Params P{};
+        P.W = (const uint8_t*)w.down;
+        P.row_bytes = m->rb_f;
+        P.M = d.hidden;
+        P.K = d.ffn;
+        P.x = m->act;
+        P.y = m->h;
+        P.use_pdl = pdl;
+        if ((st = gemv_launch(d.qtype, gemv::EPI_ADD, gemv::PRO_X, P, s)) != NTX_OK) return st;
+    }
+    return NTX_OK;
+}
+
+ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
+{
+    const ntx_model_desc& d = m->d;
+    Params P{};
+    P.W = (const uint8_t*)d.output;
+    P.row_bytes = m->rb_h;
+    P.M = d.vocab;
+    P.K = d.hidden;
+    P.x = m->h;
+    P.norm_w = d.out_norm;
+    P.eps = d.rms_eps;
+    P.y = logits;
+    P.use_pdl = pdl;
+    return gemv_launch(d.qtype, gemv::EPI_STORE, gemv::PRO_RMSNORM, P, s);
+}
+
+LayerW resident_w(const ntx_layer_desc& L) { return {L.w_qkv, L.w_o, L.w_gate, L.w_up, L.w_down}; }
+
+// Embedding + resident layers [0, n) (+ head if with_head), token/pos from m->step.
+ntx_status enqueue_resident(ntx_model* m, int n, float* logits, cudaStream_t s, bool with_head)
+{
+    ntx_status st = embed_launch(m->d.qtype, m->d.tok_embd, m->d.hidden, m->step, m->h, s, m->pdl);
+    if (st != NTX_OK) return st;
+    for (int l = 0; l < n; ++l)
+        if ((st = enqueue_layer(m, l, resident_w(m->layers[l]), s, m->pdl)) != NTX_OK) return st;
+    if (with_head) return enqueue_head(m, logits, s, m->pdl);
+    return NTX_OK;
+}
+
+bool env_flag(const char* name)
+{
+    const char* v = std::getenv(name);
+    return v && v[0] && v[0] != '0';
+}
+
+ntx_status check_desc(const ntx_model_desc* d)
+{
+    if (!d) return fail(NTX_EINVAL, "model: null descriptor");
+    if (qtraits(d->qtype).block_elems == 0) return fail(NTX_EINVAL, "model: unknown qtype");
+    if (d->n_layers < 1 || d->hidden < 1 || d->n_q_heads < 1 || d->n_kv_heads < 1 || d->ffn < 1 || d->vocab < 1)
+        return fail(NTX_EINVAL, "model: dimensions must be positive");
+    if (d->head_dim != 128) return fail(NTX_EUNSUPPORTED, "model: head_dim must be 128");
+    if (d->n_q_heads % d->n_kv_heads) return fail(NTX_EINVAL, "model: n_q_heads must be a multiple of n_kv_heads");
+    const int G = d->n_q_heads / d->n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8) return fail(NTX_EUNSUPPORTED, "model: q heads per kv head must be 1, 2, 4 or 8");
+    if (d->n_kv_heads > 64) return fail(NTX_EUNSUPPORTED, "model: at most 64 kv heads");
+    if (d->max_ctx < 1) return fail(NTX_EINVAL, "model: max_ctx must be >= 1");
+    if (!(d->rms_eps >= 0.f) || !(d->rope_theta > 0.f)) return fail(NTX_EINVAL, "model: bad eps / theta");
+    if (d->n_resident < 0 || d->n_resident > d->n_layers) return fail(NTX_EINVAL, "model: n_resident out of range");
+    if (!d->tok_embd || !d->out_norm || !d->output || !d->layers) return fail(NTX_EINVAL, "model: null pointer");
+    const int qd = d->n_q_heads * d->head_dim;
+    for (int64_t k : {(int64_t)d->hidden, (int64_t)qd, (int64_t)d->ffn}) {
+        if (row_bytes(d->qtype, k) == 0) return fail(NTX_EINVAL, "model: a row length is not a multiple of the block size");
+        if (row_bytes(d->qtype, k) % 16) return fail(NTX_EUNSUPPORTED, "model: packed rows must be multiples of 16 bytes");
+        if (k > 32768) return fail(NTX_EUNSUPPORTED, "model: row length above 32768");
+    }
+    if (!aligned(d->tok_embd, 16) || !aligned(d->output, 16)) return fail(NTX_EINVAL, "model: tensors must be 16-byte aligned");
+    for (int l = 0; l < d->n_layers; ++l) {
+        const ntx_layer_desc& L = d->layers[l];
+        if (!L.attn_norm || !L.ffn_norm || !L.w_qkv || !L.w_o || !L.w_gate || !L.w_up || !L.w_down || !L.k_cache || !L.v_cache)
+            return fail(NTX_EINVAL, "model: null layer pointer (layer " + std::to_string(l) + ")");
+        if (!aligned(L.w_qkv, 16) || !aligned(L.w_o, 16) || !aligned(L.w_gate, 16) || !aligned(L.w_up, 16) ||
+            !aligned(L.w_down, 16) || !aligned(L.k_cache, 16) || !aligned(L.v_cache, 16))
+            return fail(NTX_EINVAL, "model: tensors must be 16-byte aligned (layer " + std::to_string(l) + ")");
+    }
+    return NTX_OK;
+}
+
+void free_model(ntx_model* m)
+{
+    if (!m) return;
+    if (m->graph) cudaGraphExecDestroy(m->graph);
+    for (int i = 0; i < 2; ++i) {
+        if (m->copy_done[i]) cudaEventDestroy(m->copy_done[i]);
+        if (m->slot_free[i]) cudaEventDestroy(m->slot_free[i]);
+    }
+    if (m->ev_start) cudaEventDestroy(m->ev_start);
+    if (m->ev_end) cudaEventDestroy(m->ev_end);
+    cudaFree(m->h);
+    cudaFree(m->q);
+    cudaFree(m->att);
+    cudaFree(m->act);
+    cudaFree(m->step);
+    cudaFree(m->attn_ws);
+    cudaFree(m->ring);
+    delete m;
+}
+
+}  // namespace
+
+cudaError_t take_device_error_decode(uint32_t* out) { return take_tu_device_error(out); }
+
+}  // namespace ntx
+
+using namespace ntx;
+
+NTX_EXPORT ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** model)
+{
+    if (!model) return fail(NTX_EINVAL, "ntx_model_create: null output pointer");
+    *model = nullptr;
+    ntx_status st = check_desc(desc);
+    if (st != NTX_OK) return st;
+    ntx_model* m = new ntx_model();
+    m->d = *desc;
+    m->layers.assign(desc->layers, desc->layers + desc->n_layers);
+    m->d.layers = nullptr;
+    cudaGetDevice(&m->device);
+    const ntx_model_desc& d = m->d;
+    const int qd = d.n_q_heads * d.head_dim;
+    m->rb_h = row_bytes(d.qtype, d.hidden);
+    m->rb_q = row_bytes(d.qtype, qd);
+    m->rb_f = row_bytes(d.qtype, d.ffn);
+    m->pdl = !env_flag("NTX_NO_PDL");
+    m->use_graph = !env_flag("NTX_NO_GRAPH");
+    m->n_split = attn_split_for(d.n_kv_heads, d.max_ctx);
+    const size_t ws = attn_workspace_bytes_for(d.n_q_heads, d.n_kv_heads, d.head_dim, m->n_split);
+    cudaError_t e = cudaSuccess;
+    auto alloc = [&](void** p, size_t n) {
+        if (e == cudaSuccess) e = cudaMalloc(p, n);
+    };
+    alloc((void**)&m->h, (size_t)d.hidden * 4);
+    alloc((void**)&m->q, (size_t)qd * 4);
+    alloc((void**)&m->att, (size_t)qd * 4);
+    alloc((void**)&m->act, (size_t)d.ffn * 4);
+    alloc((void**)&m->step, 16);
+    alloc(&m->attn_ws, ws);
+    if (e == cudaSuccess) e = cudaMemset(m->attn_ws, 0, ws);
+    if (e == cudaSuccess) e = cudaMemset(m->step, 0, 16);
+    if (e == cudaSuccess && d.n_resident < d.n_layers) {
+        const int kvd = d.n_kv_heads * d.head_dim;
+        m->sz_qkv = (size_t)(qd + 2 * kvd) * m->rb_h;
+        m->sz_o = (size_t)d.hidden * m->rb_q;
+        m->sz_ffn = (size_t)d.ffn * m->rb_h;
+        m->sz_down = (size_t)d.hidden * m->rb_f;
+        m->off_qkv = 0;
+        m->off_o = align256(m->sz_qkv);
+        m->off_gate = m->off_o + align256(m->sz_o);
+        m->off_up = m->off_gate + align256(m->sz_ffn);
+        m->off_down = m->off_up + align256(m->sz_ffn);
+        m->slot_bytes = m->off_down + align256(m->sz_down);
+        alloc((void**)&m->ring, 2 * m->slot_bytes);
+        for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+            e = cudaEventCreateWithFlags(&m->copy_done[i], cudaEventDisableTiming);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&m->slot_free[i], cudaEventDisableTiming);
+        }
+    }
+    if (e == cudaSuccess) e = cudaEventCreate(&m->ev_start);
+    if (e == cudaSuccess) e = cudaEventCreate(&m->ev_end);
+    if (e != cudaSuccess) {
+        const ntx_status code = (e == cudaErrorMemoryAllocation) ? NTX_ENOMEM : NTX_ECUDA;
+        free_model(m);
+        return fail(code, std::string("ntx_model_create: ") + cudaGetErrorString(e));
+    }
+    *model = m;
+    return NTX_OK;
+}
+
+NTX_EXPORT ntx_status ntx_model_destroy(ntx_model* model)
+{
+    if (!model) return fail(NTX_EINVAL, "ntx_model_destroy: null model");
+    cudaDeviceSynchronize();
+    free_model(model);
+    return NTX_OK;
+}
+
+NTX_EXPORT ntx_status ntx_decode_step(ntx_model* m, int32_t token, int32_t pos, float* logits, void* stream)
+{
+    if (!m || !logits) return fail(NTX_EINVAL, "ntx_decode_step: null pointer");
+    if (m->d.n_resident != m->d.n_layers)
+        return fail(NTX_EINVAL, "ntx_decode_step: model has streamed layers; use ntx_stream_layers");
+    if (token < 0 || token >= m->d.vocab) return fail(NTX_EINVAL, "ntx_decode_step: token out of range");
+    if (pos < 0 || pos >= m->d.max_ctx) return fail(NTX_EINVAL, "ntx_decode_step: pos out of range");
+    if (!aligned(logits, 4)) return fail(NTX_EINVAL, "ntx_decode_step: logits must be 4-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    ntx_status st = set_step_launch(m->step, token, pos, s);
+    if (st != NTX_OK) return st;
+    if (!m->use_graph) return enqueue_resident(m, m->d.n_layers, logits, s, true);
+    if (!m->graph || m->graph_logits != logits) {
+        if (m->graph) {
+            cudaGraphExecDestroy(m->graph);
+            m->graph = nullptr;
+        }
+        cudaStream_t cap;
+        NTX_CUDA_TRY(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
+        cudaGraph_t g = nullptr;
+        cudaError_t e = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal);
+        if (e != cudaSuccess) {
+            cudaStreamDestroy(cap);
+            return fail(NTX_ECUDA, std::string("ntx_decode_step: begin capture: ") + cudaGetErrorString(e));
+        }
+        st = enqueue_resident(m, m->d.n_layers, logits, cap, true);
+        e = cudaStreamEndCapture(cap, &g);
+        cudaStreamDestroy(cap);
+        if (st != NTX_OK) {
+            if (g) cudaGraphDestroy(g);
+            return st;
+        }
+        if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("ntx_decode_step: end capture: ") + cudaGetErrorString(e));
+        e = cudaGraphInstantiate(&m->graph, g, 0);
+        cudaGraphDestroy(g);
+        if (e != cudaSuccess) {
+            m->graph = nullptr;
+            return fail(NTX_ECUDA, std::string("ntx_decode_step: instantiate: ") + cudaGetErrorString(e));
+        }
+        m->graph_logits = logits;
+    }
+    NTX_CUDA_TRY(cudaGraphLaunch(m->graph, s));
+    return NTX_OK;
+}
+
+NTX_EXPORT ntx_status ntx_stream_layers(ntx_model* m, int32_t token, int32_t pos, float* logits, void* compute,
+                                        void* copy, int64_t timeout_ms)
+{
+    if (!m || !logits) return fail(NTX_EINVAL, "ntx_stream_layers: null pointer");
+    if (token < 0 || token >= m->d.vocab) return fail(NTX_EINVAL, "ntx_stream_layers: token out of range");
+    if (pos < 0 || pos >= m->d.max_ctx) return fail(NTX_EINVAL, "ntx_stream_layers: pos out of range");
+    if (timeout_ms < 0) return fail(NTX_EINVAL, "ntx_stream_layers: timeout_ms must be >= 0");
+    if (compute == copy && m->d.n_resident < m->d.n_layers)
+        return fail(NTX_EINVAL, "ntx_stream_layers: compute and copy streams must differ");
+    cudaStream_t cs = (cudaStream_t)compute, ks = (cudaStream_t)copy;
+    const ntx_model_desc& d = m->d;
+    const int nres = d.n_resident;
+    NTX_CUDA_TRY(cudaEventRecord(m->ev_start, cs));
+    ntx_status st = set_step_launch(m->step, token, pos, cs);
+    if (st != NTX_OK) return st;
+    int64_t h2d = 0;
+    // copies of streamed layer j into slot (j - nres) % 2; the slot is free once
+    // the compute of the layer that used it before has finished
+    auto enqueue_copy = [&](int j) -> ntx_status {
+        const int slot = (j - nres) & 1;
+        const ntx_layer_desc& L = m->layers[j];
+        uint8_t* base = m->ring + (size_t)slot * m->slot_bytes;
+        NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->slot_free[slot], 0));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_qkv, L.w_qkv, m->sz_qkv, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_o, L.w_o, m->sz_o, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_gate, L.w_gate, m->sz_ffn, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_up, L.w_up, m->sz_ffn, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_down, L.w_down, m->sz_down, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaEventRecord(m->copy_done[slot], ks));
+        h2d += (int64_t)(m->sz_qkv + m->sz_o + 2 * m->sz_ffn + m->sz_down);
+        return NTX_OK;
+    };
+    if (nres < d.n_layers) {
+        NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->ev_start, 0));
+        for (int j = nres; j < std::min(d.n_layers, nres + 2); ++j)
+            if ((st = enqueue_copy(j)) != NTX_OK) return st;
+    }
+    if ((st = enqueue_resident(m, nres, logits, cs, false)) != NTX_OK) return st;
+    for (int j = nres; j < d.n_layers; ++j) {
+        const int slot = (j - nres) & 1;
+        uint8_t* base = m->ring + (size_t)slot * m->slot_bytes;
+        NTX_CUDA_TRY(cudaStreamWaitEvent(cs, m->copy_done[slot], 0));
+        const LayerW w{base + m->off_qkv, base + m->off_o, base + m->off_gate, base + m->off_up, base + m->off_down};
+        if ((st = enqueue_layer(m, j, w, cs, false)) != NTX_OK) return st;
+        NTX_CUDA_TRY(cudaEventRecord(m->slot_free[slot], cs));
+        if (j + 2 < d.n_layers)
+            if ((st = enqueue_copy(j + 2)) != NTX_OK) return st;
+    }
+    if ((st = enqueue_head(m, logits, cs, false)) != NTX_OK) return st;
+    NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
+    m->last_h2d = h2d;
+    if (timeout_ms > 0) {
+        const auto deadline = std::chrono::steady_clock::now() + std::chrono::milliseconds(timeout_ms);
+        for (;;) {
+            cudaError_t q = cudaEventQuery(m->ev_end);
+            if (q == cudaSuccess) break;
+            if (q != cudaErrorNotReady) return fail(NTX_ECUDA, std::string("ntx_stream_layers: ") + cudaGetErrorString(q));
+            if (std::chrono::steady_clock::now() > deadline)
+                return fail(NTX_ETIMEOUT, "ntx_stream_layers: step not finished within timeout_ms (work stays queued)");
+            std::this_thread::sleep_for(std::chrono::microseconds(200));
+        }
+    }
+    return NTX_OK;
+}
+
+NTX_EXPORT ntx_status ntx_stream_stats(ntx_model* m, int64_t* h2d_bytes, float* step_ms)
+{
+    if (!m) return fail(NTX_EINVAL, "ntx_stream_stats: null model");
+    if (h2d_bytes) *h2d_bytes = m->last_h2d;
+    if (step_ms) {
+        float ms = 0.f;
+        NTX_CUDA_TRY(cudaEventElapsedTime(&ms, m->ev_start, m->ev_end));
+        *step_ms = ms;
+    }
+    return NTX_OK;
+}

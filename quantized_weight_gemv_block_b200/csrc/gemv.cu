@@ -1,0 +1,174 @@
+// gemv.cu - host side of the quantized GEMV (launch shaping, C ABI), the simple
+// kernel for rows that are not 16-byte multiples, and the dequantization kernel.
+#include <algorithm>
+#include <mutex>
+
+#include "blocks.cuh"
+#include "gemv_kernel.cuh"
+#include "launch.h"
+
+namespace ntx {
+namespace gemv {
+
+template <int QT>
+__global__ void dequant_kernel(const uint8_t* W, int64_t rows, int64_t cols, int64_t rb, float* out)
+{
+    using F = Fmt<QT>;
+    const int64_t nb_row = cols / F::BE;
+    const int64_t total = rows * nb_row;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total * F::BE;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t blk = i / F::BE;
+        const int e = (int)(i % F::BE);
+        const int64_t r = blk / nb_row, kb = blk % nb_row;
+        out[r * cols + kb * F::BE + e] = weight_at<QT>(W + r * rb + kb * F::BB, e);
+    }
+}
+
+// Simple GEMV: one warp per row, lanes stride over blocks; any row length.
+template <int QT>
+__global__ void gemv_simple_kernel(const uint8_t* W, int rows, int cols, int64_t rb, const float* x, float* y)
+{
+    using F = Fmt<QT>;
+    const int warps = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int nb = cols / F::BE;
+    for (int r = blockIdx.x * warps + (threadIdx.x >> 5); r < rows; r += gridDim.x * warps) {
+        const uint8_t* row = W + (int64_t)r * rb;
+        float acc = 0.f;
+        for (int i = lane; i < nb * F::BE; i += 32) {
+            const int kb = i / F::BE, e = i % F::BE;
+            acc = fmaf(weight_at<QT>(row + (int64_t)kb * F::BB, e), x[i], acc);
+        }
+        acc = warp_sum(acc);
+        if (lane == 0) y[r] = acc;
+    }
+}
+
+// ------------------------------------------------------------------ launch shaping
+
+template <int QT>
+bool shape(Params& P, int n_sm_unused)
+{
+    (void)n_sm_unused;
+    using F = Fmt<QT>;
+    P.chunk_elems = kConsumers * F::E;
+    P.n_chunks = (P.K + P.chunk_elems - 1) / P.chunk_elems;
+    P.chunk_bytes = P.chunk_elems / F::BE * F::BB;
+    P.stage_bytes = kSlots * P.chunk_bytes;
+    P.x_bytes = ((P.K * 4 + 127) / 128) * 128;
+    const int fixed = 1024 + P.x_bytes + 128;   // barriers / reduction, x, tail padding
+    int ns = (kSmemLimit - fixed) / P.stage_bytes;
+    ns = std::min(ns, kMaxStages);
+    if (ns < 2) return false;
+    P.n_stages = ns;
+    return true;
+}
+
+int smem_bytes(const Params& P) { return 1024 + P.x_bytes + P.n_stages * P.stage_bytes + 128; }
+
+template <int QT, int EPI, int PRO>
+ntx_status launch_t(Params P, cudaStream_t s, int grid_cap)
+{
+    if (!shape<QT>(P, 0)) return fail(NTX_EUNSUPPORTED, "gemv: row too long for the shared-memory pipeline");
+    auto kern = gemv_kernel<QT, EPI, PRO>;
+    const int smem = smem_bytes(P);
+    static std::once_flag once[4][4][2];
+    std::call_once(once[QT][EPI][PRO], [&] {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    });
+    const int outs = EPI == EPI_SWIGLU ? kSlots / 2 : kSlots;
+    int grid = std::min(grid_cap, (P.M + outs - 1) / outs);
+    grid = std::max(grid, 1);
+    return launch_kernel(kern, dim3(grid), dim3(kThreads), smem, s, P.use_pdl != 0, P);
+}
+
+template <int EPI, int PRO>
+ntx_status launch_q(int qtype, const Params& P, cudaStream_t s, int grid_cap)
+{
+    switch (qtype) {
+    case NTX_Q8_0: return launch_t<NTX_Q8_0, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q4_0: return launch_t<NTX_Q4_0, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q4_K: return launch_t<NTX_Q4_K, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q6_K: return launch_t<NTX_Q6_K, EPI, PRO>(P, s, grid_cap);
+    default: return fail(NTX_EINVAL, "unknown qtype");
+    }
+}
+
+}  // namespace gemv
+
+ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s)
+{
+    using namespace gemv;
+    const int cap = num_sms();
+    if (epi == EPI_STORE && pro == PRO_X) return launch_q<EPI_STORE, PRO_X>(qtype, P, s, cap);
+    if (epi == EPI_ADD && pro == PRO_X) return launch_q<EPI_ADD, PRO_X>(qtype, P, s, cap);
+    if (epi == EPI_SWIGLU && pro == PRO_RMSNORM) return launch_q<EPI_SWIGLU, PRO_RMSNORM>(qtype, P, s, cap);
+    if (epi == EPI_QKV && pro == PRO_RMSNORM) return launch_q<EPI_QKV, PRO_RMSNORM>(qtype, P, s, cap);
+    if (epi == EPI_STORE && pro == PRO_RMSNORM) return launch_q<EPI_STORE, PRO_RMSNORM>(qtype, P, s, cap);
+    return fail(NTX_EUNSUPPORTED, "gemv: unsupported prologue / epilogue combination");
+}
+
+cudaError_t take_device_error_gemv(uint32_t* out) { return take_tu_device_error(out); }
+
+bool gemv_fast_path_ok(int qtype, const void* W, int64_t cols)
+{
+    return aligned(W, 16) && row_bytes(qtype, cols) % 16 == 0;
+}
+
+}  // namespace ntx
+
+using namespace ntx;
+
+NTX_EXPORT ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t cols, const float* x, float* y,
+                                 void* stream)
+{
+    if (qtraits(qtype).block_elems == 0) return fail(NTX_EINVAL, "ntx_gemv_q: unknown qtype");
+    if (!W || !x || !y) return fail(NTX_EINVAL, "ntx_gemv_q: null pointer");
+    if (rows < 1 || rows > (1 << 30)) return fail(NTX_EINVAL, "ntx_gemv_q: rows out of range");
+    if (row_bytes(qtype, cols) == 0 || cols > (1 << 28))
+        return fail(NTX_EINVAL, "ntx_gemv_q: cols must be a positive multiple of the block size");
+    if (!aligned(x, 4) || !aligned(y, 4)) return fail(NTX_EINVAL, "ntx_gemv_q: x / y must be 4-byte aligned");
+    if (!aligned(W, 2)) return fail(NTX_EINVAL, "ntx_gemv_q: W must be at least 2-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t rb = row_bytes(qtype, cols);
+    if (gemv_fast_path_ok(qtype, W, cols) && cols <= 32768) {
+        gemv::Params P{};
+        P.W = (const uint8_t*)W;
+        P.row_bytes = rb;
+        P.M = (int)rows;
+        P.K = (int)cols;
+        P.x = x;
+        P.y = y;
+        return gemv_launch(qtype, gemv::EPI_STORE, gemv::PRO_X, P, s);
+    }
+    const int threads = 256, warps = threads / 32;
+    int grid = (int)std::min<int64_t>((rows + warps - 1) / warps, (int64_t)num_sms() * 8);
+    switch (qtype) {
+    case NTX_Q8_0: gemv::gemv_simple_kernel<NTX_Q8_0><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y); break;
+    case NTX_Q4_0: gemv::gemv_simple_kernel<NTX_Q4_0><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y); break;
+    case NTX_Q4_K: gemv::gemv_simple_kernel<NTX_Q4_K><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y); break;
+    case NTX_Q6_K: gemv::gemv_simple_kernel<NTX_Q6_K><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y); break;
+    }
+    return check_launch("ntx_gemv_q (simple kernel)");
+}
+
+NTX_EXPORT ntx_status ntx_dequant_q(int qtype, const void* W, int64_t rows, int64_t cols, float* out, void* stream)
+{
+    if (qtraits(qtype).block_elems == 0) return fail(NTX_EINVAL, "ntx_dequant_q: unknown qtype");
+    if (!W || !out) return fail(NTX_EINVAL, "ntx_dequant_q: null pointer");
+    if (rows < 1 || row_bytes(qtype, cols) == 0) return fail(NTX_EINVAL, "ntx_dequant_q: bad shape");
+    if (!aligned(out, 4)) return fail(NTX_EINVAL, "ntx_dequant_q: out must be 4-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    const int64_t rb = row_bytes(qtype, cols);
+    const int64_t n = rows * cols;
+    const int threads = 256;
+    const int grid = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)num_sms() * 32);
+    switch (qtype) {
+    case NTX_Q8_0: gemv::dequant_kernel<NTX_Q8_0><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out); break;
+    case NTX_Q4_0: gemv::dequant_kernel<NTX_Q4_0><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out); break;
+    case NTX_Q4_K: gemv::dequant_kernel<NTX_Q4_K><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out); break;
+    case NTX_Q6_K: gemv::dequant_kernel<NTX_Q6_K><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out); break;
+    }
+    return check_launch("ntx_dequant_q");
+}

@@ -1,0 +1,32 @@
+// ops.h - internal launchers shared by the op, attention and decode-step files.
+#pragma once
+
+#include "common.cuh"
+#include "gemv.cuh"
+
+namespace ntx {
+
+ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t* token_dev, float* h, cudaStream_t s,
+                        bool pdl);
+ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, cudaStream_t s);
+ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
+bool gemv_fast_path_ok(int qtype, const void* W, int64_t cols);
+
+// Split-KV decode attention (attn.cu).
+struct AttnArgs {
+    const float* q;
+    const __half* k_cache;
+    const __half* v_cache;
+    float* out;
+    int n_q_heads, n_kv_heads, head_dim, max_ctx;
+    int32_t n_ctx;              // used when n_ctx_from_pos is null
+    const int32_t* pos_dev;     // if set: n_ctx = *pos_dev + 1 (read on the device)
+    void* workspace;            // counters + partials, zeroed once
+    int n_split;                // CTAs per kv head
+    bool pdl;
+};
+int attn_split_for(int n_kv_heads, int32_t max_ctx);
+size_t attn_workspace_bytes_for(int n_q_heads, int n_kv_heads, int head_dim, int n_split);
+ntx_status attn_launch(const AttnArgs& a, cudaStream_t s);
+
+}  // namespace ntx

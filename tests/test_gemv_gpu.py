@@ -1,0 +1,163 @@
+"""GPU parity of the quantized GEMV and dequantization (through the C ABI) with
+the CPU oracle, on inputs from the seeded generator."""
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import GEMV_TIGHT, TOL, ntx_module, rel_err
+
+pytestmark = pytest.mark.gpu
+
+Q8_0, Q4_0, Q4_K, Q6_K = 0, 1, 2, 3
+NAMES = {Q8_0: "q8_0", Q4_0: "q4_0", Q4_K: "q4_k", Q6_K: "q6_k"}
+
+
+@pytest.fixture(scope="module")
+def ntx():
+    return ntx_module()
+
+
+def make(syn, qtype, rows, cols, seed=1, decode=False):
+    qp = syn.decode_qparams(qtype, cols) if decode else syn.sweep_qparams(qtype)
+    host = syn.blocks_host(qtype, seed, 11, rows, cols, qp)
+    dev = torch.empty(host.size, dtype=torch.uint8, device="cuda")
+    syn.blocks_dev(dev, qtype, seed, 11, rows, cols, qp)
+    torch.cuda.synchronize()
+    assert np.array_equal(dev.cpu().numpy().reshape(host.shape), host), "device generator differs from host"
+    return host, dev
+
+
+def gpu_gemv(ntx, qtype, W, rows, cols, x):
+    xd = torch.from_numpy(x).cuda()
+    y = torch.full((rows,), float("nan"), dtype=torch.float32, device="cuda")
+    ntx.ntx_gemv_q(qtype, W, rows, cols, xd, y)
+    torch.cuda.synchronize()
+    return y.cpu().numpy()
+
+
+# fast path: rows that are 16-byte multiples, several groups + a partial group,
+# several chunks + a partial chunk
+FAST = [(Q8_0, 37, 4096 + 256), (Q4_0, 37, 4096 + 256), (Q4_K, 37, 8192 + 256), (Q6_K, 37, 8192 + 2048),
+        (Q8_0, 1, 32 * 8), (Q4_K, 3, 256), (Q6_K, 2, 2048), (Q8_0, 150, 4096), (Q4_0, 300, 1024)]
+
+
+@pytest.mark.parametrize("qtype,rows,cols", FAST, ids=[f"{NAMES[q]}-{r}x{c}" for q, r, c in FAST])
+def test_gemv_fast_path(ntx, orc, syn, qtype, rows, cols):
+    host, dev = make(syn, qtype, rows, cols)
+    x = syn.normal_f32_host(1, 12, cols)
+    y = gpu_gemv(ntx, qtype, dev, rows, cols, x)
+    o = orc.gemv(qtype, host, rows, cols, x)
+    e = rel_err(y, o)
+    assert e <= TOL and e <= GEMV_TIGHT, e
+    assert ntx.ntx_device_error() == 0
+
+
+# simple kernel: rows that are not 16-byte multiples, or W only 2-byte aligned
+SIMPLE = [(Q8_0, 5, 96), (Q4_0, 9, 160), (Q6_K, 4, 256 * 3), (Q4_K, 5, 256 * 3)]
+
+
+@pytest.mark.parametrize("qtype,rows,cols", SIMPLE, ids=[f"{NAMES[q]}-{r}x{c}" for q, r, c in SIMPLE])
+def test_gemv_simple_path(ntx, orc, syn, qtype, rows, cols):
+    host, dev = make(syn, qtype, rows, cols)
+    if qtype == Q4_K:      # 144-byte rows take the fast path when aligned: offset W by 2 bytes
+        buf = torch.zeros(dev.numel() + 16, dtype=torch.uint8, device="cuda")
+        buf[2:2 + dev.numel()] = dev
+        W = buf.data_ptr() + 2
+    else:
+        W = dev
+    x = syn.normal_f32_host(2, 12, cols)
+    y = gpu_gemv(ntx, qtype, W, rows, cols, x)
+    o = orc.gemv(qtype, host, rows, cols, x)
+    assert rel_err(y, o) <= GEMV_TIGHT
+
+
+@pytest.mark.parametrize("qtype", [Q8_0, Q4_0, Q4_K, Q6_K], ids=list(NAMES.values()))
+def test_one_hot_input_returns_the_dequantized_column(ntx, syn, qtype):
+    """x = e_k: every product and the offset subtraction are exact, so y == W[:, k] bit for bit."""
+    rows, cols = 24, 8192 + (2048 if qtype == Q6_K else 256)
+    host, dev = make(syn, qtype, rows, cols)
+    dq = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    ntx.ntx_dequant_q(qtype, dev, rows, cols, dq)
+    for k in (0, 17, cols // 2 + 3, cols - 1):
+        x = np.zeros(cols, dtype=np.float32)
+        x[k] = 1.0
+        y = gpu_gemv(ntx, qtype, dev, rows, cols, x)
+        assert np.array_equal(y, dq[:, k].cpu().numpy()), k
+
+
+@pytest.mark.parametrize("qtype", [Q8_0, Q4_K])
+def test_gemv_input_edge_cases(ntx, orc, syn, qtype):
+    rows, cols = 40, 8192
+    host, dev = make(syn, qtype, rows, cols)
+    zero = np.zeros(cols, dtype=np.float32)
+    assert np.array_equal(gpu_gemv(ntx, qtype, dev, rows, cols, zero), np.zeros(rows, dtype=np.float32))
+    # wide dynamic range: tiny and huge inputs mixed (exercises the input scaling)
+    x = syn.normal_f32_host(3, 12, cols)
+    x[::7] *= 1e20
+    x[1::7] *= 1e-20
+    assert rel_err(gpu_gemv(ntx, qtype, dev, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)) <= GEMV_TIGHT
+    for scale in (1e-30, 1e25):
+        xs = (syn.normal_f32_host(4, 12, cols) * np.float32(scale)).astype(np.float32)
+        assert rel_err(gpu_gemv(ntx, qtype, dev, rows, cols, xs), orc.gemv(qtype, host, rows, cols, xs)) <= GEMV_TIGHT
+
+
+# ----------------------------------------------------------------- dequantization
+
+DQ = [(Q8_0, 37, 4096 + 256), (Q4_0, 37, 4096 + 256), (Q4_K, 37, 8192 + 256), (Q6_K, 37, 8192 + 2048),
+      (Q8_0, 3, 96), (Q6_K, 3, 768), (Q4_K, 4096, 4096), (Q4_0, 4096, 4096)]
+
+
+@pytest.mark.parametrize("qtype,rows,cols", DQ, ids=[f"{NAMES[q]}-{r}x{c}" for q, r, c in DQ])
+def test_dequant_bit_exact(ntx, orc, syn, qtype, rows, cols):
+    host, dev = make(syn, qtype, rows, cols)
+    out = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    ntx.ntx_dequant_q(qtype, dev, rows, cols, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), orc.dequant(qtype, host, rows, cols).view(np.uint32))
+
+
+def test_dequant_decode_recipe_subnormal_scales(ntx, orc, syn):
+    """Q6_K at K = 28672 under the decode recipe has fp16-subnormal scales."""
+    host, dev = make(syn, Q6_K, 8, 28672, decode=True)
+    d = host.reshape(-1, 210)[:, 208:210].copy().view(np.uint16)
+    assert np.any((d & 0x7C00) == 0)
+    out = torch.empty((8, 28672), dtype=torch.float32, device="cuda")
+    ntx.ntx_dequant_q(Q6_K, dev, 8, 28672, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), orc.dequant(Q6_K, host, 8, 28672).view(np.uint32))
+
+
+# ------------------------------------------------------- full-size workload shapes
+
+# (K -> N): Llama-8B layer shapes of the GEMV sweep, and the Llama-70B shapes of the Q6_K decode
+SWEEP = [(q, n, k) for q in (Q4_0, Q4_K) for (k, n) in ((4096, 6144), (4096, 4096), (4096, 14336), (14336, 4096))]
+SWEEP += [(Q8_0, 4096, 4096), (Q8_0, 6144, 4096), (Q8_0, 4096, 14336), (Q6_K, 10240, 8192), (Q6_K, 8192, 28672),
+          (Q6_K, 28672, 8192)]
+
+
+@pytest.mark.parametrize("qtype,rows,cols", SWEEP, ids=[f"{NAMES[q]}-{r}x{c}" for q, r, c in SWEEP])
+def test_gemv_full_shapes(ntx, orc, syn, qtype, rows, cols):
+    host, dev = make(syn, qtype, rows, cols)
+    x = syn.normal_f32_host(5, 12, cols)
+    y = gpu_gemv(ntx, qtype, dev, rows, cols, x)
+    e = rel_err(y, orc.gemv(qtype, host, rows, cols, x))
+    assert e <= GEMV_TIGHT, e
+
+
+@pytest.mark.parametrize("qtype", [Q4_0, Q4_K, Q8_0, Q6_K], ids=["q4_0", "q4_k", "q8_0", "q6_k"])
+def test_gemv_lm_head_sampled_rows(ntx, orc, syn, qtype):
+    """The 4096 -> 128256 (8192 -> 128256 for Q6_K) LM-head GEMV at full size, checked on
+    sampled rows the oracle computes one by one."""
+    rows, cols = 128256, (8192 if qtype == Q6_K else 4096)
+    qp = syn.sweep_qparams(qtype)
+    dev = torch.empty(rows * syn.row_bytes(qtype, cols), dtype=torch.uint8, device="cuda")
+    syn.blocks_dev(dev, qtype, 9, 21, rows, cols, qp)
+    x = syn.normal_f32_host(9, 22, cols)
+    y = gpu_gemv(ntx, qtype, dev, rows, cols, x)
+    rng = np.random.default_rng(0)
+    sample = np.unique(np.concatenate([[0, 1, rows // 2, rows - 2, rows - 1], rng.integers(0, rows, 300)]))
+    o = np.empty(sample.size, dtype=np.float32)
+    for i, r in enumerate(sample):
+        Wr = syn.blocks_host(qtype, 9, 21, 1, cols, qp, row0=int(r))
+        o[i] = orc.gemv(qtype, Wr, 1, cols, x)[0]
+    assert rel_err(y[sample], o) <= GEMV_TIGHT
