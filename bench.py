@@ -338,6 +338,35 @@ def gemv_bench(ntx, iters=50):
     return {"us": us, "gbs": nbytes / (us * 1e-6) / 1e9}
 
 
+def profile_gemv(what, launches):
+    """A few launches of one GEMV (weights larger than L2), nothing else: the case
+    that profiler captures of the GEMV kernel run."""
+    import torch
+    import synth
+    import quantized_weight_gemv_block_b200 as ntx
+    from quantized_weight_gemv_block_b200 import build
+    build.build()
+    synth.build_dev()
+    fmt, shape = what.split(":")
+    rows, cols = (int(v) for v in shape.split("x"))
+    q = synth.qtype_of(fmt)
+    W = torch.empty(rows * synth.row_bytes(q, cols), dtype=torch.uint8, device="cuda")
+    synth.blocks_dev(W, q, 0, 1, rows, cols, synth.sweep_qparams(q))
+    x = torch.empty(cols, device="cuda")
+    synth.normal_f32_dev(x, 0, 2)
+    y = torch.empty(rows, device="cuda")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ntx.ntx_gemv_q(q, W, rows, cols, x, y)
+    torch.cuda.synchronize()
+    e0.record()
+    for _ in range(launches):
+        ntx.ntx_gemv_q(q, W, rows, cols, x, y)
+    e1.record()
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / launches
+    print(json.dumps({"gemv": what, "bytes": W.numel(), "us": us, "gbs": W.numel() / (us * 1e-6) / 1e9}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -348,7 +377,11 @@ def main():
                     choices=["llama70b_q6k_decode", "llama8b_q8_0_decode", "llama70b_q4k_stream"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--profile-gemv", default=None, metavar="FMT:ROWSxCOLS",
+                    help="only run the GEMV kernel on one matrix (for profilers), e.g. q6_k:28672x8192")
     args = ap.parse_args()
+    if args.profile_gemv:
+        return profile_gemv(args.profile_gemv, args.steps)
     if args.warmup < 3:
         args.warmup = 3
 

@@ -24,7 +24,7 @@ constexpr int HD = 128;
 constexpr int kThreads = 256;
 constexpr int kMaxRows = 256;       // positions per CTA (V rows in shared memory)
 constexpr int kCounterBytes = 256;  // ticket counters at the start of the workspace
-constexpr int kPartFloats = 2 + HD;
+constexpr int kPartFloats = 4 + HD;   // m, l, 2 pad, acc[128]: 528 B, 16-byte aligned records
 
 struct KArgs {
     const float* q;
@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const KArgs a)
                 acc[i] = s;
             }
         }
-        *reinterpret_cast<float4*>(pp + 2 + 4 * lane) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        *reinterpret_cast<float4*>(pp + 4 + 4 * lane) = make_float4(acc[0], acc[1], acc[2], acc[3]);
         if (lane == 0) {
             pp[0] = stat[h];
             pp[1] = stat[G + h];
@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const KArgs a)
                 if (ls > 0.f) {
                     const float w = expf(__ldcg(ps) - M);
                     L = fmaf(ls, w, L);
-                    o = fmaf(__ldcg(ps + 2 + d), w, o);
+                    o = fmaf(__ldcg(ps + 4 + d), w, o);
                 }
             }
             a.out[(int64_t)(g * G + hh) * HD + d] = o / L;
