@@ -135,15 +135,20 @@ def max_over_ranks(v, world):
 
 # --------------------------------------------------------------------------- workloads
 
-def spec_for(name):
+def spec_for(name, layout="tiled"):
     import synth
+    tiled = layout == "tiled"
     if name == "llama70b_q6k_decode":
-        return synth.ModelSpec(**synth.LLAMA_70B_Q6_K)
+        return synth.ModelSpec(**synth.LLAMA_70B_Q6_K, tiled=tiled)
     if name == "llama8b_q8_0_decode":
-        return synth.ModelSpec(**synth.LLAMA_8B_Q8_0)
+        return synth.ModelSpec(**synth.LLAMA_8B_Q8_0, tiled=tiled)
     if name == "llama70b_q4k_stream":
-        return synth.ModelSpec(**synth.LLAMA_70B_Q4_K)
+        return synth.ModelSpec(**synth.LLAMA_70B_Q4_K, tiled=tiled)
     raise ValueError(name)
+
+
+def lib_qtype(spec):
+    return spec.qtype | (16 if spec.tiled else 0)
 
 
 def kv_read_bytes(spec):
@@ -181,15 +186,16 @@ def measure_gemv_roofline(ntx, model, spec, stream, iters=3):
         launches.append((t["w_down"], spec.hidden, spec.ffn))
     launches.append((model.output, spec.vocab, spec.hidden))
     nbytes = sum(r * synth.row_bytes(spec.qtype, c) + 4 * (c + r) for _, r, c in launches)
+    q = lib_qtype(spec)
     with torch.cuda.stream(stream):
         for W, r, c in launches[:20]:
-            ntx.ntx_gemv_q(spec.qtype, W, r, c, x, y, stream.cuda_stream)
+            ntx.ntx_gemv_q(q, W, r, c, x, y, stream.cuda_stream)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         torch.cuda.synchronize()
         e0.record(stream)
         for _ in range(iters):
             for W, r, c in launches:
-                ntx.ntx_gemv_q(spec.qtype, W, r, c, x, y, stream.cuda_stream)
+                ntx.ntx_gemv_q(q, W, r, c, x, y, stream.cuda_stream)
         e1.record(stream)
         torch.cuda.synchronize()
     ms = e0.elapsed_time(e1) / (iters * len(launches))
@@ -203,7 +209,7 @@ def run_decode_bench(args, rank, world, local):
     from synth.device_model import DeviceModel
 
     name = args.workload
-    spec = spec_for(name)
+    spec = spec_for(name, args.layout)
     streamed = name == "llama70b_q4k_stream"
     n_res = 36 if streamed else None
     t0 = time.time()
@@ -310,7 +316,7 @@ def cpu_baseline(spec, budget_s=20.0):
                       f"+ {head_rows} of {spec.vocab} LM-head rows, extrapolated to one token"}
 
 
-def gemv_bench(ntx, iters=50):
+def gemv_bench(ntx, iters=50, tiled=True):
     """Q8_0 4096 x 4096 GEMV rotating over 16 weight copies (> 2 x L2)."""
     import torch
     import synth
@@ -318,19 +324,25 @@ def gemv_bench(ntx, iters=50):
     qp = synth.sweep_qparams(synth.Q8_0)
     rb = synth.row_bytes(synth.Q8_0, cols)
     copies = [torch.empty(rows * rb, dtype=torch.uint8, device="cuda") for _ in range(16)]
+    tmp = torch.empty(rows * rb, dtype=torch.uint8, device="cuda")
     for i, c in enumerate(copies):
-        synth.blocks_dev(c, synth.Q8_0, 0, 1, rows, cols, qp)
+        if tiled:
+            synth.blocks_dev(tmp, synth.Q8_0, 0, 1, rows, cols, qp)
+            ntx.ntx_repack_q(synth.Q8_0, tmp, c, rows, cols)
+        else:
+            synth.blocks_dev(c, synth.Q8_0, 0, 1, rows, cols, qp)
+    q = synth.Q8_0 | (16 if tiled else 0)
     x = torch.empty(cols, device="cuda")
     synth.normal_f32_dev(x, 0, 2)
     y = torch.empty(rows, device="cuda")
     s = torch.cuda.current_stream()
     for c in copies:
-        ntx.ntx_gemv_q(synth.Q8_0, c, rows, cols, x, y)
+        ntx.ntx_gemv_q(q, c, rows, cols, x, y)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
     e0.record(s)
     for i in range(iters):
-        ntx.ntx_gemv_q(synth.Q8_0, copies[i % 16], rows, cols, x, y)
+        ntx.ntx_gemv_q(q, copies[i % 16], rows, cols, x, y)
     e1.record(s)
     torch.cuda.synchronize()
     us = e0.elapsed_time(e1) * 1e3 / iters
@@ -349,9 +361,15 @@ def profile_gemv(what, launches):
     synth.build_dev()
     fmt, shape = what.split(":")
     rows, cols = (int(v) for v in shape.split("x"))
-    q = synth.qtype_of(fmt)
+    tiled = fmt.endswith("_t")
+    q = synth.qtype_of(fmt[:-2] if tiled else fmt)
     W = torch.empty(rows * synth.row_bytes(q, cols), dtype=torch.uint8, device="cuda")
     synth.blocks_dev(W, q, 0, 1, rows, cols, synth.sweep_qparams(q))
+    if tiled:
+        Wt = torch.empty_like(W)
+        ntx.ntx_repack_q(q, W, Wt, rows, cols)
+        W = Wt
+        q |= 16
     x = torch.empty(cols, device="cuda")
     synth.normal_f32_dev(x, 0, 2)
     y = torch.empty(rows, device="cuda")
@@ -375,6 +393,8 @@ def main():
     ap.add_argument("--impl", default="ntx", choices=["ntx", "reference"])
     ap.add_argument("--workload", default="llama70b_q6k_decode",
                     choices=["llama70b_q6k_decode", "llama8b_q8_0_decode", "llama70b_q4k_stream"])
+    ap.add_argument("--layout", default="tiled", choices=["tiled", "gguf"],
+                    help="weights handed to the library as tiled (repacked once at load) or GGUF-style blocks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--profile-gemv", default=None, metavar="FMT:ROWSxCOLS",
@@ -386,10 +406,10 @@ def main():
         args.warmup = 3
 
     rank, world, local = dist_setup(args.gpus)
-    spec = spec_for(args.workload)
+    spec = spec_for(args.workload, args.layout)
     config = {"workload": args.workload, "layers": spec.n_layers, "hidden": spec.hidden, "ffn": spec.ffn,
               "q_heads": spec.n_q_heads, "kv_heads": spec.n_kv_heads, "vocab": spec.vocab, "format": ["q8_0", "q4_0",
-              "q4_k", "q6_k"][spec.qtype], "context": spec.n_prefill + 1, "batch": 1,
+              "q4_k", "q6_k"][spec.qtype], "layout": args.layout, "context": spec.n_prefill + 1, "batch": 1,
               "l2": "inputs larger than L2 (weights %.1f GB per step)" % (step_bytes(spec) / 1e9),
               "parallelism": "replicas" if world > 1 else "single"}
 
@@ -440,7 +460,7 @@ def main():
                             "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / peak,
                             "traffic": None, "bytes_per_launch": per_launch, "avg_launch_us": ms * 1e3}
         if not args.no_extras:
-            line["gemv_q8_0_4096x4096"] = gemv_bench(ntx)
+            line["gemv_q8_0_4096x4096"] = {"tiled": gemv_bench(ntx, tiled=True), "gguf": gemv_bench(ntx, tiled=False)}
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(spec)
         if r["device_error"]:

@@ -68,7 +68,24 @@ typedef enum ntx_qtype {
     NTX_Q8_0 = 0,
     NTX_Q4_0 = 1,
     NTX_Q4_K = 2,
-    NTX_Q6_K = 3
+    NTX_Q6_K = 3,
+    /* Tiled layouts (flag NTX_TILED): the same blocks, the same bytes per row,
+     * regrouped inside fixed tiles so every code run starts on a 16-byte boundary.
+     * Produced from the GGUF-style layout by ntx_repack_q, lossless.
+     *   NTX_Q8_0_T tile = 8 blocks (256 weights, 272 B): 256 int8 codes in element
+     *              order | the 8 fp16 d
+     *   NTX_Q4_0_T tile = 8 blocks (256 weights, 144 B): the 8 blocks' 16 code bytes
+     *              (nibble order unchanged) | the 8 fp16 d
+     *   NTX_Q4_K_T tile = 1 superblock: identical to NTX_Q4_K
+     *   NTX_Q6_K_T tile = 8 superblocks (2048 weights, 1680 B): 8 x 128 B low code
+     *              bits | 8 x 64 B high code bits | 8 x 16 int8 scales | 8 fp16 d
+     * A row of a tiled tensor must hold whole tiles (cols a multiple of 256, 2048
+     * for Q6_K). */
+    NTX_TILED = 16,
+    NTX_Q8_0_T = 16,
+    NTX_Q4_0_T = 17,
+    NTX_Q4_K_T = 18,
+    NTX_Q6_K_T = 19
 } ntx_qtype;
 
 /* Message of the last failing ntx_* call on this thread ("" if none). */
@@ -78,7 +95,8 @@ const char* ntx_last_error(void);
 int ntx_version(void);
 
 /* Bytes of one packed row of `cols` elements; 0 if qtype is unknown or cols is
- * not a positive multiple of the format's block size (32 or 256). */
+ * not a positive multiple of the format's block size (32 or 256; for a tiled
+ * qtype, of the tile size).  Tiled and GGUF-style rows have the same length. */
 size_t ntx_row_bytes(int qtype, int64_t cols);
 
 /* Elements per block of qtype (32 or 256), 0 if unknown. */
@@ -99,6 +117,12 @@ ntx_status ntx_device_error(uint32_t* code);
  * shapes take a simpler kernel. */
 ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t cols, const float* x, float* y,
                       void* stream);
+
+/* Repack W [rows, cols] from the GGUF-style layout of `qtype` (NTX_Q8_0 ..
+ * NTX_Q6_K) into the tiled layout qtype | NTX_TILED, device to device: W_tiled
+ * receives rows * ntx_row_bytes(qtype, cols) bytes and must not overlap W.
+ * cols must be a multiple of the tile size.  A pure byte permutation. */
+ntx_status ntx_repack_q(int qtype, const void* W, void* W_tiled, int64_t rows, int64_t cols, void* stream);
 
 /* Dequantize W [rows, cols] to fp32 out [rows, cols] (row-major).  The result
  * is bit-exact: every weight is one fp32 product of exact factors (Q4_K: one

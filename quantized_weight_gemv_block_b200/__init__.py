@@ -15,12 +15,14 @@ from .build import LIB
 
 NTX_OK, NTX_EINVAL, NTX_EUNSUPPORTED, NTX_ENOMEM, NTX_ECUDA, NTX_ETIMEOUT = range(6)
 NTX_Q8_0, NTX_Q4_0, NTX_Q4_K, NTX_Q6_K = range(4)
+NTX_TILED = 16
+NTX_Q8_0_T, NTX_Q4_0_T, NTX_Q4_K_T, NTX_Q6_K_T = 16, 17, 18, 19
 STATUS_NAMES = {0: "NTX_OK", 1: "NTX_EINVAL", 2: "NTX_EUNSUPPORTED", 3: "NTX_ENOMEM", 4: "NTX_ECUDA",
                 5: "NTX_ETIMEOUT"}
 
 # Every symbol of include/ntx.h.
 EXPORTS = ("ntx_last_error", "ntx_version", "ntx_row_bytes", "ntx_block_elems", "ntx_device_error", "ntx_gemv_q",
-           "ntx_dequant_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_workspace_bytes", "ntx_swiglu",
+           "ntx_dequant_q", "ntx_repack_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_workspace_bytes", "ntx_swiglu",
            "ntx_softmax", "ntx_argmax", "ntx_embed", "ntx_model_create", "ntx_model_destroy", "ntx_decode_step",
            "ntx_stream_layers", "ntx_stream_stats")
 
@@ -66,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "ntx_device_error": ([ctypes.POINTER(ctypes.c_uint32)], ci),
             "ntx_gemv_q": ([ci, vp, i64, i64, vp, vp, vp], ci),
             "ntx_dequant_q": ([ci, vp, i64, i64, vp, vp], ci),
+            "ntx_repack_q": ([ci, vp, vp, i64, i64, vp], ci),
             "ntx_rmsnorm": ([vp, vp, vp, i64, cf, vp], ci),
             "ntx_rope": ([vp, vp, ci, ci, ci, i32, cf, vp], ci),
             "ntx_attn_decode": ([vp, vp, vp, vp, ci, ci, ci, i32, i32, vp, sz, vp], ci),
@@ -138,6 +141,10 @@ def ntx_gemv_q(qtype, W, rows, cols, x, y, stream=None) -> None:
 
 def ntx_dequant_q(qtype, W, rows, cols, out, stream=None) -> None:
     check(lib().ntx_dequant_q(qtype, _p(W), rows, cols, _p(out), _s(stream)))
+
+
+def ntx_repack_q(qtype, W, W_tiled, rows, cols, stream=None) -> None:
+    check(lib().ntx_repack_q(qtype, _p(W), _p(W_tiled), rows, cols, _s(stream)))
 
 
 def ntx_rmsnorm(x, w, y, n, eps, stream=None) -> None:

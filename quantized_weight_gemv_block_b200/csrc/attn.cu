@@ -33,7 +33,7 @@ struct KArgs {
     float* out;
     uint32_t* cnt;
     float* part;
-    int max_ctx, n_split, p_alloc;
+    int max_ctx, n_split, p_alloc, sc_len;   // sc_len = max(p_alloc, n_split)
     int32_t n_ctx;
     const int32_t* pos_dev;
     int use_pdl;
@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const KArgs a)
     int* flag = reinterpret_cast<int*>(sm + 8);
     __half* vbuf = reinterpret_cast<__half*>(sm + 128);
     float* sc = reinterpret_cast<float*>(sm + 128 + (size_t)a.p_alloc * HD * 2);   // [G][p_alloc]
-    float* red = sc + G * a.p_alloc;                                                // [8][HD]
+    float* red = sc + G * a.sc_len;                                                 // [8][HD]
     float* stat = red + 8 * HD;                                                     // m[G], l[G]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -195,33 +195,82 @@ __global__ void __launch_bounds__(kThreads, 2) attn_kernel(const KArgs a)
     __syncthreads();
     if (*flag) {
         __threadfence();
+        // (1) all (m, l) of this kv head's splits in parallel; weights e^(m_s - M_h)
         const float* base = a.part + (size_t)g * a.n_split * G * kPartFloats;
-        for (int idx = tid; idx < G * HD; idx += kThreads) {
-            const int hh = idx / HD, d = idx % HD;
+        float* wsm = sc;                         // [n_split][G] weights (score buffer is free now)
+        for (int r = tid; r < a.n_split * G; r += kThreads) {
+            const float2 ml = __ldcg(reinterpret_cast<const float2*>(base + (size_t)r * kPartFloats));
+            wsm[r] = ml.y > 0.f ? ml.x : -INFINITY;
+            red[r] = ml.y;                       // l (red has 8 * 128 >= 64 * 8 floats)
+        }
+        __syncthreads();
+        for (int hh = warp; hh < G; hh += kThreads / 32) {
             float M = -INFINITY;
-            for (int s = 0; s < a.n_split; ++s) M = fmaxf(M, __ldcg(base + ((size_t)s * G + hh) * kPartFloats));
-            float L = 0.f, o = 0.f;
-            for (int s = 0; s < a.n_split; ++s) {
-                const float* ps = base + ((size_t)s * G + hh) * kPartFloats;
-                const float ls = __ldcg(ps + 1);
-                if (ls > 0.f) {
-                    const float w = expf(__ldcg(ps) - M);
-                    L = fmaf(ls, w, L);
-                    o = fmaf(__ldcg(ps + 4 + d), w, o);
+            for (int s2 = lane; s2 < a.n_split; s2 += 32) M = fmaxf(M, wsm[s2 * G + hh]);
+            M = gemv::warp_max(M);
+            float L = 0.f;
+            for (int s2 = lane; s2 < a.n_split; s2 += 32) {
+                const int r = s2 * G + hh;
+                const float w = wsm[r] == -INFINITY ? 0.f : expf(wsm[r] - M);
+                L = fmaf(red[r], w, L);
+                wsm[r] = w;
+            }
+            L = gemv::warp_sum(L);
+            if (lane == 0) stat[hh] = L;
+        }
+        __syncthreads();
+        // (2) acc: warp -> head h, lane -> 4 dims; splits interleaved over the WPH warps of
+        // the head; independent 16-byte loads, eight in flight
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
+        constexpr int UM = 8;
+        for (int s0 = sub; s0 < a.n_split; s0 += WPH * UM) {
+            float4 v[UM];
+            float w[UM];
+#pragma unroll
+            for (int u = 0; u < UM; ++u) {
+                const int s2 = s0 + u * WPH;
+                const bool ok = s2 < a.n_split;
+                w[u] = ok ? wsm[s2 * G + h] : 0.f;
+                v[u] = ok ? __ldcg(reinterpret_cast<const float4*>(base + ((size_t)s2 * G + h) * kPartFloats + 4) + lane)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < UM; ++u) {
+                o[0] = fmaf(w[u], v[u].x, o[0]);
+                o[1] = fmaf(w[u], v[u].y, o[1]);
+                o[2] = fmaf(w[u], v[u].z, o[2]);
+                o[3] = fmaf(w[u], v[u].w, o[3]);
+            }
+        }
+        __syncthreads();
+        if (WPH > 1) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) red[warp * HD + 4 * lane + i] = o[i];
+        }
+        __syncthreads();
+        if (sub == 0) {
+            if (WPH > 1) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float s3 = 0.f;
+                    for (int w2 = 0; w2 < WPH; ++w2) s3 += red[(warp + w2) * HD + 4 * lane + i];
+                    o[i] = s3;
                 }
             }
-            a.out[(int64_t)(g * G + hh) * HD + d] = o / L;
+            const float invL = 1.0f / stat[h];
+            *reinterpret_cast<float4*>(a.out + (int64_t)(g * G + h) * HD + 4 * lane) =
+                make_float4(o[0] * invL, o[1] * invL, o[2] * invL, o[3] * invL);
         }
         if (tid == 0) a.cnt[g] = 0u;
     }
 }
 
-int smem_for(int G, int p_alloc) { return 128 + p_alloc * HD * 2 + (G * p_alloc + 8 * HD + 2 * G) * 4 + 64; }
+int smem_for(int G, int p_alloc, int sc_len) { return 128 + p_alloc * HD * 2 + (G * sc_len + 8 * HD + 2 * G) * 4 + 64; }
 
 template <int G>
 ntx_status launch_g(const KArgs& k, int grid, int p_alloc, cudaStream_t s, bool pdl)
 {
-    const int smem = smem_for(G, p_alloc);
+    const int smem = smem_for(G, p_alloc, k.sc_len);
     static bool configured = false;
     if (!configured) {
         cudaFuncSetAttribute(attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
@@ -250,7 +299,7 @@ int attn_split_for(int n_kv_heads, int32_t max_ctx)
 {
     const int target = (2 * num_sms() + n_kv_heads - 1) / n_kv_heads;
     const int by_rows = (max_ctx + kMaxRows - 1) / kMaxRows;
-    return std::max(1, std::max(target, by_rows));
+    return std::min(128, std::max(1, std::max(target, by_rows)));
 }
 
 size_t attn_workspace_bytes_for(int n_q_heads, int n_kv_heads, int head_dim, int n_split)
@@ -273,6 +322,9 @@ ntx_status attn_launch(const AttnArgs& a, cudaStream_t s)
     k.max_ctx = a.max_ctx;
     k.n_split = a.n_split;
     k.p_alloc = ((a.max_ctx + a.n_split - 1) / a.n_split + 1) & ~1;
+    k.sc_len = std::max(k.p_alloc, a.n_split);
+    if (a.n_split * G > 8 * HD || smem_for(G, k.p_alloc, k.sc_len) > 200 * 1024)
+        return fail(NTX_EUNSUPPORTED, "attention: context too long for one split pass");
     k.n_ctx = a.n_ctx;
     k.pos_dev = a.pos_dev;
     k.use_pdl = a.pdl ? 1 : 0;

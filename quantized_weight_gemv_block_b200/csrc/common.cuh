@@ -63,8 +63,26 @@ struct QTraits {
     int block_bytes;
 };
 
+inline bool is_tiled(int qtype) { return (qtype & NTX_TILED) != 0; }
+inline int base_qtype(int qtype) { return qtype & ~NTX_TILED; }
+
+// Elements per tile of a tiled layout (8 blocks, one Q4_K superblock, 8 Q6_K superblocks).
+inline int tile_elems(int qtype)
+{
+    switch (base_qtype(qtype)) {
+    case NTX_Q8_0: case NTX_Q4_0: case NTX_Q4_K: return 256;
+    case NTX_Q6_K: return 2048;
+    default: return 0;
+    }
+}
+
 inline QTraits qtraits(int qtype)
 {
+    if (is_tiled(qtype)) {
+        const int b = base_qtype(qtype);
+        if (b < NTX_Q8_0 || b > NTX_Q6_K) return {0, 0};
+        qtype = b;
+    }
     switch (qtype) {
     case NTX_Q8_0: return {32, 34};
     case NTX_Q4_0: return {32, 18};
@@ -78,6 +96,7 @@ inline int64_t row_bytes(int qtype, int64_t cols)
 {
     QTraits t = qtraits(qtype);
     if (t.block_elems == 0 || cols <= 0 || cols % t.block_elems) return 0;
+    if (is_tiled(qtype) && cols % tile_elems(qtype)) return 0;
     return cols / t.block_elems * t.block_bytes;
 }
 
@@ -190,7 +209,21 @@ __device__ __forceinline__ void fma2(uint64_t& acc, uint64_t a, uint64_t b)
     asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
 }
 
-__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi) { return (uint64_t)lo | ((uint64_t)hi << 32); }
+// Two 32-bit values as one register pair (no arithmetic).
+__device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi)
+{
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+    return r;
+}
+
+// a + b, lane-wise.
+__device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
 
 __device__ __forceinline__ float f16_bits_to_f32(uint16_t h) { return __half2float(__ushort_as_half(h)); }
 

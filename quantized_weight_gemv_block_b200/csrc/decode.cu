@@ -200,12 +200,14 @@ ntx_status check_desc(const ntx_model_desc* d)
         if (row_bytes(d->qtype, k) % 16) return fail(NTX_EUNSUPPORTED, "model: packed rows must be multiples of 16 bytes");
         if (k > 32768) return fail(NTX_EUNSUPPORTED, "model: row length above 32768");
     }
-    if (!aligned(d->tok_embd, 16) || !aligned(d->output, 16)) return fail(NTX_EINVAL, "model: tensors must be 16-byte aligned");
+    if (!aligned(d->tok_embd, 16) || !aligned(d->output, 16) || !aligned(d->out_norm, 16))
+        return fail(NTX_EINVAL, "model: tensors must be 16-byte aligned");
     for (int l = 0; l < d->n_layers; ++l) {
         const ntx_layer_desc& L = d->layers[l];
         if (!L.attn_norm || !L.ffn_norm || !L.w_qkv || !L.w_o || !L.w_gate || !L.w_up || !L.w_down || !L.k_cache || !L.v_cache)
             return fail(NTX_EINVAL, "model: null layer pointer (layer " + std::to_string(l) + ")");
         if (!aligned(L.w_qkv, 16) || !aligned(L.w_o, 16) || !aligned(L.w_gate, 16) || !aligned(L.w_up, 16) ||
+            !aligned(L.attn_norm, 16) || !aligned(L.ffn_norm, 16) ||
             !aligned(L.w_down, 16) || !aligned(L.k_cache, 16) || !aligned(L.v_cache, 16))
             return fail(NTX_EINVAL, "model: tensors must be 16-byte aligned (layer " + std::to_string(l) + ")");
     }

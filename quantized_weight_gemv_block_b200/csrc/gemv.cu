@@ -13,35 +13,49 @@ namespace gemv {
 template <int QT>
 __global__ void dequant_kernel(const uint8_t* W, int64_t rows, int64_t cols, int64_t rb, float* out)
 {
-    using F = Fmt<QT>;
-    const int64_t nb_row = cols / F::BE;
-    const int64_t total = rows * nb_row;
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total * F::BE;
-         i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t blk = i / F::BE;
-        const int e = (int)(i % F::BE);
-        const int64_t r = blk / nb_row, kb = blk % nb_row;
-        out[r * cols + kb * F::BE + e] = weight_at<QT>(W + r * rb + kb * F::BB, e);
+    const int64_t total = rows * cols;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / cols, e = i % cols;
+        out[i] = weight_in_row<QT>(W + r * rb, e);
     }
 }
 
-// Simple GEMV: one warp per row, lanes stride over blocks; any row length.
+// Simple GEMV: one warp per row, lanes stride over the elements; any row length.
 template <int QT>
 __global__ void gemv_simple_kernel(const uint8_t* W, int rows, int cols, int64_t rb, const float* x, float* y)
 {
-    using F = Fmt<QT>;
     const int warps = blockDim.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int nb = cols / F::BE;
     for (int r = blockIdx.x * warps + (threadIdx.x >> 5); r < rows; r += gridDim.x * warps) {
         const uint8_t* row = W + (int64_t)r * rb;
         float acc = 0.f;
-        for (int i = lane; i < nb * F::BE; i += 32) {
-            const int kb = i / F::BE, e = i % F::BE;
-            acc = fmaf(weight_at<QT>(row + (int64_t)kb * F::BB, e), x[i], acc);
-        }
+        for (int i = lane; i < cols; i += 32) acc = fmaf(weight_in_row<QT>(row, i), x[i], acc);
         acc = warp_sum(acc);
         if (lane == 0) y[r] = acc;
+    }
+}
+
+// GGUF-style -> tiled: out byte o of a tile comes from byte src(o) of the same
+// tile in the GGUF-style layout.
+template <int B>
+__device__ __forceinline__ int repack_src(int o)
+{
+    if (B == NTX_Q8_0) return o < 256 ? 34 * (o >> 5) + 2 + (o & 31) : 34 * ((o - 256) >> 1) + ((o - 256) & 1);
+    if (B == NTX_Q4_0) return o < 128 ? 18 * (o >> 4) + 2 + (o & 15) : 18 * ((o - 128) >> 1) + ((o - 128) & 1);
+    if (B == NTX_Q4_K) return o;
+    if (o < 1024) return 210 * (o >> 7) + (o & 127);
+    if (o < 1536) return 210 * ((o - 1024) >> 6) + 128 + ((o - 1024) & 63);
+    if (o < 1664) return 210 * ((o - 1536) >> 4) + 192 + ((o - 1536) & 15);
+    return 210 * ((o - 1664) >> 1) + 208 + ((o - 1664) & 1);
+}
+
+template <int B>
+__global__ void repack_kernel(const uint8_t* in, uint8_t* out, int64_t n_bytes, int tile_bytes)
+{
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_bytes; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t tile = i / tile_bytes;
+        const int o = (int)(i - tile * tile_bytes);
+        out[i] = in[tile * tile_bytes + repack_src<B>(o)];
     }
 }
 
@@ -52,12 +66,12 @@ bool shape(Params& P, int n_sm_unused)
 {
     (void)n_sm_unused;
     using F = Fmt<QT>;
-    P.chunk_elems = kConsumers * F::E;
+    P.chunk_elems = kOwners * F::E;
     P.n_chunks = (P.K + P.chunk_elems - 1) / P.chunk_elems;
     P.chunk_bytes = P.chunk_elems / F::BE * F::BB;
-    P.stage_bytes = kSlots * P.chunk_bytes;
+    P.stage_bytes = Slots<QT>::value * P.chunk_bytes;
     P.x_bytes = ((P.K * 4 + 127) / 128) * 128;
-    const int fixed = 1024 + P.x_bytes + 128;   // barriers / reduction, x, tail padding
+    const int fixed = kHeader + P.x_bytes + 128;   // barriers / reduction, x, tail padding
     int ns = (kSmemLimit - fixed) / P.stage_bytes;
     ns = std::min(ns, kMaxStages);
     if (ns < 2) return false;
@@ -65,7 +79,7 @@ bool shape(Params& P, int n_sm_unused)
     return true;
 }
 
-int smem_bytes(const Params& P) { return 1024 + P.x_bytes + P.n_stages * P.stage_bytes + 128; }
+int smem_bytes(const Params& P) { return kHeader + P.x_bytes + P.n_stages * P.stage_bytes + 128; }
 
 template <int QT, int EPI, int PRO>
 ntx_status launch_t(Params P, cudaStream_t s, int grid_cap)
@@ -73,11 +87,20 @@ ntx_status launch_t(Params P, cudaStream_t s, int grid_cap)
     if (!shape<QT>(P, 0)) return fail(NTX_EUNSUPPORTED, "gemv: row too long for the shared-memory pipeline");
     auto kern = gemv_kernel<QT, EPI, PRO>;
     const int smem = smem_bytes(P);
-    static std::once_flag once[4][4][2];
+    static std::once_flag once[20][4][2];
     std::call_once(once[QT][EPI][PRO], [&] {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     });
-    const int outs = EPI == EPI_SWIGLU ? kSlots / 2 : kSlots;
+    P.m24 = 1u << 24;
+    P.m28 = 1u << 28;
+    P.m30 = 1u << 30;
+    P.m16 = 16u;
+    for (int i = 0; i < 3; ++i) {
+        P.kb[i] = 0xFFu << (8 * i);
+        P.ks[i] = 0x80u << (8 * i);
+    }
+    P.k0f = 0x0F0F0F0Fu;
+    const int outs = Outs<QT, EPI>::value;
     int grid = std::min(grid_cap, (P.M + outs - 1) / outs);
     grid = std::max(grid, 1);
     return launch_kernel(kern, dim3(grid), dim3(kThreads), smem, s, P.use_pdl != 0, P);
@@ -91,6 +114,10 @@ ntx_status launch_q(int qtype, const Params& P, cudaStream_t s, int grid_cap)
     case NTX_Q4_0: return launch_t<NTX_Q4_0, EPI, PRO>(P, s, grid_cap);
     case NTX_Q4_K: return launch_t<NTX_Q4_K, EPI, PRO>(P, s, grid_cap);
     case NTX_Q6_K: return launch_t<NTX_Q6_K, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q8_0_T: return launch_t<NTX_Q8_0_T, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q4_0_T: return launch_t<NTX_Q4_0_T, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q4_K_T: return launch_t<NTX_Q4_K, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q6_K_T: return launch_t<NTX_Q6_K_T, EPI, PRO>(P, s, grid_cap);
     default: return fail(NTX_EINVAL, "unknown qtype");
     }
 }
@@ -132,7 +159,7 @@ NTX_EXPORT ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t
     if (!aligned(W, 2)) return fail(NTX_EINVAL, "ntx_gemv_q: W must be at least 2-byte aligned");
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t rb = row_bytes(qtype, cols);
-    if (gemv_fast_path_ok(qtype, W, cols) && cols <= 32768) {
+    if (gemv_fast_path_ok(qtype, W, cols) && cols <= 32768 && aligned(x, 16)) {
         gemv::Params P{};
         P.W = (const uint8_t*)W;
         P.row_bytes = rb;
@@ -144,12 +171,17 @@ NTX_EXPORT ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t
     }
     const int threads = 256, warps = threads / 32;
     int grid = (int)std::min<int64_t>((rows + warps - 1) / warps, (int64_t)num_sms() * 8);
+#define NTX_SIMPLE(Q) gemv::gemv_simple_kernel<Q><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y)
     switch (qtype) {
-    case NTX_Q8_0: gemv::gemv_simple_kernel<NTX_Q8_0><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y); break;
-    case NTX_Q4_0: gemv::gemv_simple_kernel<NTX_Q4_0><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y); break;
-    case NTX_Q4_K: gemv::gemv_simple_kernel<NTX_Q4_K><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y); break;
-    case NTX_Q6_K: gemv::gemv_simple_kernel<NTX_Q6_K><<<grid, threads, 0, s>>>((const uint8_t*)W, (int)rows, (int)cols, rb, x, y); break;
+    case NTX_Q8_0: NTX_SIMPLE(NTX_Q8_0); break;
+    case NTX_Q4_0: NTX_SIMPLE(NTX_Q4_0); break;
+    case NTX_Q4_K: case NTX_Q4_K_T: NTX_SIMPLE(NTX_Q4_K); break;
+    case NTX_Q6_K: NTX_SIMPLE(NTX_Q6_K); break;
+    case NTX_Q8_0_T: NTX_SIMPLE(NTX_Q8_0_T); break;
+    case NTX_Q4_0_T: NTX_SIMPLE(NTX_Q4_0_T); break;
+    case NTX_Q6_K_T: NTX_SIMPLE(NTX_Q6_K_T); break;
     }
+#undef NTX_SIMPLE
     return check_launch("ntx_gemv_q (simple kernel)");
 }
 
@@ -164,11 +196,40 @@ NTX_EXPORT ntx_status ntx_dequant_q(int qtype, const void* W, int64_t rows, int6
     const int64_t n = rows * cols;
     const int threads = 256;
     const int grid = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)num_sms() * 32);
+#define NTX_DQ(Q) gemv::dequant_kernel<Q><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out)
     switch (qtype) {
-    case NTX_Q8_0: gemv::dequant_kernel<NTX_Q8_0><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out); break;
-    case NTX_Q4_0: gemv::dequant_kernel<NTX_Q4_0><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out); break;
-    case NTX_Q4_K: gemv::dequant_kernel<NTX_Q4_K><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out); break;
-    case NTX_Q6_K: gemv::dequant_kernel<NTX_Q6_K><<<grid, threads, 0, s>>>((const uint8_t*)W, rows, cols, rb, out); break;
+    case NTX_Q8_0: NTX_DQ(NTX_Q8_0); break;
+    case NTX_Q4_0: NTX_DQ(NTX_Q4_0); break;
+    case NTX_Q4_K: case NTX_Q4_K_T: NTX_DQ(NTX_Q4_K); break;
+    case NTX_Q6_K: NTX_DQ(NTX_Q6_K); break;
+    case NTX_Q8_0_T: NTX_DQ(NTX_Q8_0_T); break;
+    case NTX_Q4_0_T: NTX_DQ(NTX_Q4_0_T); break;
+    case NTX_Q6_K_T: NTX_DQ(NTX_Q6_K_T); break;
     }
+#undef NTX_DQ
     return check_launch("ntx_dequant_q");
+}
+
+NTX_EXPORT ntx_status ntx_repack_q(int qtype, const void* W, void* W_tiled, int64_t rows, int64_t cols, void* stream)
+{
+    if (qtype < NTX_Q8_0 || qtype > NTX_Q6_K) return fail(NTX_EINVAL, "ntx_repack_q: qtype must be a GGUF-style format");
+    if (!W || !W_tiled) return fail(NTX_EINVAL, "ntx_repack_q: null pointer");
+    if (rows < 1 || row_bytes(qtype | NTX_TILED, cols) == 0)
+        return fail(NTX_EINVAL, "ntx_repack_q: cols must be a positive multiple of the tile size");
+    const int64_t n = rows * row_bytes(qtype, cols);
+    const char* a = (const char*)W;
+    const char* b = (const char*)W_tiled;
+    if (a < b + n && b < a + n) return fail(NTX_EINVAL, "ntx_repack_q: W and W_tiled overlap");
+    cudaStream_t s = (cudaStream_t)stream;
+    const int threads = 256;
+    const int grid = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)num_sms() * 32);
+    const uint8_t* in = (const uint8_t*)W;
+    uint8_t* out = (uint8_t*)W_tiled;
+    switch (qtype) {
+    case NTX_Q8_0: gemv::repack_kernel<NTX_Q8_0><<<grid, threads, 0, s>>>(in, out, n, 272); break;
+    case NTX_Q4_0: gemv::repack_kernel<NTX_Q4_0><<<grid, threads, 0, s>>>(in, out, n, 144); break;
+    case NTX_Q4_K: gemv::repack_kernel<NTX_Q4_K><<<grid, threads, 0, s>>>(in, out, n, 144); break;
+    case NTX_Q6_K: gemv::repack_kernel<NTX_Q6_K><<<grid, threads, 0, s>>>(in, out, n, 1680); break;
+    }
+    return check_launch("ntx_repack_q");
 }

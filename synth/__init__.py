@@ -260,6 +260,7 @@ class ModelSpec:
     rms_eps: float = 1e-5
     rope_theta: float = 500000.0
     seed: int = 0
+    tiled: bool = False       # weights handed to the library in the tiled layout (same bytes, regrouped)
     extra: dict = field(default_factory=dict)
 
     @property

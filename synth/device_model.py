@@ -16,6 +16,11 @@ def _alloc_packed(spec: ModelSpec, kind: str, layer: int, device, host: bool = F
     nbytes = rows * row_bytes(spec.qtype, cols)
     t = torch.empty(nbytes, dtype=torch.uint8, device=device)
     blocks_dev(t, spec.qtype, spec.seed, tensor_id(layer, kind), rows, cols, qp)
+    if spec.tiled:
+        import quantized_weight_gemv_block_b200 as ntx
+        tt = torch.empty_like(t)
+        ntx.ntx_repack_q(spec.qtype, t, tt, rows, cols)
+        t = tt
     if host:
         h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
         h.copy_(t)
@@ -59,7 +64,8 @@ class DeviceModel:
                                                                             "w_gate", "w_up", "w_down", "k_cache",
                                                                             "v_cache")])
         self.desc = ntx.ModelDesc(self.n_layers, s.hidden, s.n_q_heads, s.n_kv_heads, s.head_dim, s.ffn, s.vocab,
-                                  s.max_ctx, s.rms_eps, s.rope_theta, s.qtype, self.tok_embd.data_ptr(),
+                                  s.max_ctx, s.rms_eps, s.rope_theta, s.qtype | (16 if s.tiled else 0),
+                                  self.tok_embd.data_ptr(),
                                   self.out_norm.data_ptr(), self.output.data_ptr(),
                                   ctypes.cast(self._layer_descs, ctypes.POINTER(ntx.LayerDesc)), self.n_resident)
         self.handle = ntx.ntx_model_create(self.desc)

@@ -52,6 +52,20 @@ def test_decode_step_small(ntx, syn, qtype):
     m.close()
 
 
+@pytest.mark.parametrize("qtype", [0, 1, 2, 3], ids=["q8_0_t", "q4_0_t", "q4_k_t", "q6_k_t"])
+def test_decode_step_tiled(ntx, syn, qtype):
+    """Weights repacked to the tiled layout: same logits as the oracle on the GGUF-style bytes."""
+    from oracle import model as om
+    from synth.device_model import DeviceModel
+    kw = dict(hidden=8192, ffn=8192 * 2, n_q_heads=64) if qtype == 3 else {}
+    spec = small_spec(syn, qtype, n_layers=2, tiled=True, **kw)
+    m = DeviceModel(spec)
+    got = run_decode(ntx, m, spec.token(), spec.n_prefill)
+    m.close()
+    want, _ = om.decode(spec)
+    assert rel_err(got, want) <= TOL
+
+
 def test_decode_positions_and_tokens(ntx, syn):
     """pos 0 (one key), a middle position, and a different token."""
     from oracle import model as om
@@ -83,7 +97,7 @@ def test_graph_and_direct_launches_agree(ntx, syn, monkeypatch):
 def test_streamed_equals_resident(ntx, syn):
     """Same kernels, same bytes: streaming layers through the HBM ring is bit-identical."""
     from synth.device_model import DeviceModel
-    spec = small_spec(syn, 2, n_layers=6, hidden=8192, n_q_heads=64, ffn=28672, vocab=2000)
+    spec = small_spec(syn, 2, n_layers=6, hidden=8192, n_q_heads=64, ffn=28672, vocab=2000, tiled=True)
     res = DeviceModel(spec)
     lr = run_decode(ntx, res, 11, spec.n_prefill)
     res.close()

@@ -161,3 +161,78 @@ def test_gemv_lm_head_sampled_rows(ntx, orc, syn, qtype):
         Wr = syn.blocks_host(qtype, 9, 21, 1, cols, qp, row0=int(r))
         o[i] = orc.gemv(qtype, Wr, 1, cols, x)[0]
     assert rel_err(y[sample], o) <= GEMV_TIGHT
+
+
+# ------------------------------------------------------------------ tiled layouts
+
+T = 16      # tiled flag
+
+
+def make_tiled(ntx, syn, qtype, rows, cols, seed=1):
+    host, dev = make(syn, qtype, rows, cols, seed)
+    tiled = torch.empty_like(dev)
+    ntx.ntx_repack_q(qtype, dev, tiled, rows, cols)
+    torch.cuda.synchronize()
+    return host, tiled
+
+
+TILED_FAST = [(Q8_0, 37, 4096 + 256), (Q4_0, 37, 4096 + 256), (Q4_K, 37, 8192 + 256), (Q6_K, 37, 8192 + 2048),
+              (Q8_0, 150, 4096), (Q6_K, 2, 2048), (Q4_0, 300, 1024), (Q8_0, 1, 256)]
+
+
+@pytest.mark.parametrize("qtype,rows,cols", TILED_FAST, ids=[f"{NAMES[q]}_t-{r}x{c}" for q, r, c in TILED_FAST])
+def test_gemv_tiled(ntx, orc, syn, qtype, rows, cols):
+    host, W = make_tiled(ntx, syn, qtype, rows, cols)
+    x = syn.normal_f32_host(1, 13, cols)
+    e = rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x))
+    assert e <= TOL and e <= GEMV_TIGHT, e
+
+
+@pytest.mark.parametrize("qtype", [Q8_0, Q4_0, Q4_K, Q6_K], ids=list(NAMES.values()))
+def test_tiled_dequant_bit_exact_and_simple_path(ntx, orc, syn, qtype):
+    rows, cols = 19, 4096 if qtype != Q6_K else 6144
+    host, W = make_tiled(ntx, syn, qtype, rows, cols)
+    out = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    ntx.ntx_dequant_q(qtype | T, W, rows, cols, out)
+    torch.cuda.synchronize()
+    want = orc.dequant(qtype, host, rows, cols)
+    assert np.array_equal(out.cpu().numpy().view(np.uint32), want.view(np.uint32))
+    # the same tiled bytes at a 2-byte-aligned address take the simple kernel
+    buf = torch.zeros(W.numel() + 16, dtype=torch.uint8, device="cuda")
+    buf[2:2 + W.numel()] = W
+    x = syn.normal_f32_host(2, 13, cols)
+    y = gpu_gemv(ntx, qtype | T, buf.data_ptr() + 2, rows, cols, x)
+    assert rel_err(y, orc.gemv(qtype, host, rows, cols, x)) <= GEMV_TIGHT
+
+
+@pytest.mark.parametrize("qtype", [Q8_0, Q4_0, Q4_K, Q6_K], ids=list(NAMES.values()))
+def test_tiled_one_hot_bit_exact(ntx, syn, qtype):
+    rows, cols = 16, 8192 + (2048 if qtype == Q6_K else 256)
+    host, W = make_tiled(ntx, syn, qtype, rows, cols)
+    dq = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    ntx.ntx_dequant_q(qtype | T, W, rows, cols, dq)
+    for k in (0, 33, cols // 2 + 5, cols - 1):
+        x = np.zeros(cols, dtype=np.float32)
+        x[k] = 1.0
+        assert np.array_equal(gpu_gemv(ntx, qtype | T, W, rows, cols, x), dq[:, k].cpu().numpy()), k
+
+
+TSWEEP = [(q, n, k) for q in (Q4_0, Q4_K, Q8_0) for (k, n) in ((4096, 6144), (4096, 14336), (14336, 4096))]
+TSWEEP += [(Q6_K, 10240, 8192), (Q6_K, 8192, 28672), (Q6_K, 28672, 8192), (Q8_0, 4096, 4096)]
+
+
+@pytest.mark.parametrize("qtype,rows,cols", TSWEEP, ids=[f"{NAMES[q]}_t-{r}x{c}" for q, r, c in TSWEEP])
+def test_gemv_tiled_full_shapes(ntx, orc, syn, qtype, rows, cols):
+    host, W = make_tiled(ntx, syn, qtype, rows, cols)
+    x = syn.normal_f32_host(6, 12, cols)
+    assert rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)) <= GEMV_TIGHT
+
+
+def test_repack_is_a_byte_permutation(ntx, syn):
+    for qtype, cols in ((Q8_0, 512), (Q4_0, 512), (Q4_K, 512), (Q6_K, 4096)):
+        host, W = make_tiled(ntx, syn, qtype, 3, cols)
+        a = np.sort(host.ravel())
+        b = np.sort(W.cpu().numpy())
+        assert np.array_equal(a, b)
+        if qtype == Q4_K:
+            assert np.array_equal(host.ravel(), W.cpu().numpy())
