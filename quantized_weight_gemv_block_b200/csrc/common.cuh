@@ -217,6 +217,14 @@ __device__ __forceinline__ uint64_t pack2(uint32_t lo, uint32_t hi)
     return r;
 }
 
+// a * b, lane-wise.
+__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b)
+{
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
 // a + b, lane-wise.
 __device__ __forceinline__ uint64_t add2(uint64_t a, uint64_t b)
 {

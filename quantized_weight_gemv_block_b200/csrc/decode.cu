@@ -260,7 +260,7 @@ NTX_EXPORT ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** m
     m->rb_f = row_bytes(d.qtype, d.ffn);
     m->pdl = !env_flag("NTX_NO_PDL");
     m->use_graph = !env_flag("NTX_NO_GRAPH");
-    m->n_split = attn_split_for(d.n_kv_heads, d.max_ctx);
+    m->n_split = attn_split_for(d.n_q_heads, d.n_kv_heads, d.max_ctx);
     const size_t ws = attn_workspace_bytes_for(d.n_q_heads, d.n_kv_heads, d.head_dim, m->n_split);
     cudaError_t e = cudaSuccess;
     auto alloc = [&](void** p, size_t n) {

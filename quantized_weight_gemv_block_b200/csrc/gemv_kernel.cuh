@@ -43,7 +43,7 @@ __device__ __forceinline__ bool slot_valid(int slot, int n_out)
 // Epilogue for one finished output (thread i < outs of warp 0 after the reduction).
 template <int QT, int EPI>
 __device__ __forceinline__ void epilogue(const Params& P, const float* tot, int out_row, int i, int n_out,
-                                         int32_t pos)
+                                         int32_t pos, const float* rope_cs)
 {
     if (EPI == EPI_STORE) {
         if (i < n_out) P.y[out_row + i] = tot[i];
@@ -63,10 +63,7 @@ __device__ __forceinline__ void epilogue(const Params& P, const float* tot, int 
             const int hd = P.head_dim;
             if (r < P.q_rows + P.kv_rows) {
                 const int pi = (r % hd) / 2;
-                const double ang = (double)pos * pow((double)P.theta, -(2.0 * pi) / (double)hd);
-                double s, c;
-                sincos(ang, &s, &c);
-                const float cf = (float)c, sf = (float)s;
+                const float cf = rope_cs[2 * pi], sf = rope_cs[2 * pi + 1];
                 const float ra = a * cf - b * sf, rb = a * sf + b * cf;
                 a = ra;
                 b = rb;
@@ -104,6 +101,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params P)
     uint64_t* empty = full + kMaxStages;
     float* red = reinterpret_cast<float*>(empty + kMaxStages);          // [2][16 warps][R]
     float* tot = red + 2 * kConsumerWarps * R;                            // [2][SL]
+    float* rope_cs = reinterpret_cast<float*>(smem + kHeader - 512);       // [head_dim / 2 <= 64][cos, sin]
     float4* xs = reinterpret_cast<float4*>(smem + kHeader);               // x, P.x_bytes
     uint8_t* stages = smem + kHeader + P.x_bytes;                         // n_stages * stage_bytes
 
@@ -246,6 +244,14 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params P)
     }
 
     const int32_t pos = (EPI == EPI_QKV) ? (P.pos_dev ? *P.pos_dev : P.pos) : 0;
+    if (EPI == EPI_QKV && tid < P.head_dim / 2) {
+        // RoPE angles of this position, pos * theta^(-2i/head_dim), in double; read by the epilogue
+        const double ang = (double)pos * pow((double)P.theta, -(2.0 * tid) / (double)P.head_dim);
+        double sn, cs;
+        sincos(ang, &sn, &cs);
+        rope_cs[2 * tid] = (float)cs;
+        rope_cs[2 * tid + 1] = (float)sn;
+    }
     bool dead = false;
     // this thread's x pieces of a chunk, and the offset / min sums of its elements
     uint64_t xr[2 * NP];
@@ -345,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params P)
             if (warp == 0) {
                 __syncwarp();
                 const float* tg = tot + (g & 1) * SL;
-                if (tid < OUTS) epilogue<QT, EPI>(P, tg, out_row, tid, n_out, pos);
+                if (tid < OUTS) epilogue<QT, EPI>(P, tg, out_row, tid, n_out, pos, rope_cs);
             }
         }
     }

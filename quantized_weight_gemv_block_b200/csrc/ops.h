@@ -25,7 +25,7 @@ struct AttnArgs {
     int n_split;                // CTAs per kv head
     bool pdl;
 };
-int attn_split_for(int n_kv_heads, int32_t max_ctx);
+int attn_split_for(int n_q_heads, int n_kv_heads, int32_t max_ctx);
 size_t attn_workspace_bytes_for(int n_q_heads, int n_kv_heads, int head_dim, int n_split);
 ntx_status attn_launch(const AttnArgs& a, cudaStream_t s);
 
