@@ -160,6 +160,24 @@ ntx_status ntx_attn_decode(const float* q, const void* k_cache, const void* v_ca
                            size_t workspace_bytes, void* stream);
 size_t ntx_attn_workspace_bytes(int n_q_heads, int n_kv_heads, int head_dim, int32_t max_ctx);
 
+/* The same attention as ntx_attn_decode, for callers that cannot allocate device
+ * memory: code that runs under a fixed, pre-planned memory budget or inside a
+ * host framework whose allocator hands out no scratch, and so has no workspace
+ * to pass.  (The pages have no counterpart; this is an addition of this library.)
+ * The split partials and counters live in a device array of 512 KiB that the
+ * library holds on every GPU that loads it, until the process exits.  Shapes
+ * whose workspace (ntx_attn_workspace_bytes) exceeds 512 KiB are rejected with
+ * NTX_EUNSUPPORTED (on a 148-SM B200: 8 q heads per kv head with 8 kv heads, as
+ * in Llama-70B, needs about 600 KB; 4 per kv head, as in Llama-8B, about 300 KB).  Nothing is allocated: the first call on a device looks up
+ * the array's device address (cudaGetSymbolAddress) and caches it, so make that
+ * first call before any stream capture.  Each call first clears the counters
+ * with cudaMemsetAsync on `stream`.  All calls share the one array, so calls
+ * whose work overlaps on the GPU (different streams, or another thread) race:
+ * serialise them.  Arguments, layouts and errors as for ntx_attn_decode. */
+ntx_status ntx_attn_decode_noalloc(const float* q, const void* k_cache, const void* v_cache, float* out,
+                                   int n_q_heads, int n_kv_heads, int head_dim, int32_t n_ctx, int32_t max_ctx,
+                                   void* stream);
+
 /* SwiGLU (listed in "Arquitectura y estructura del código"):
  * out_i = gate_i / (1 + e^-gate_i) * up_i, fp32 [n]. */
 ntx_status ntx_swiglu(const float* gate, const float* up, float* out, int64_t n, void* stream);

@@ -22,7 +22,7 @@ STATUS_NAMES = {0: "NTX_OK", 1: "NTX_EINVAL", 2: "NTX_EUNSUPPORTED", 3: "NTX_ENO
 
 # Every symbol of include/ntx.h.
 EXPORTS = ("ntx_last_error", "ntx_version", "ntx_row_bytes", "ntx_block_elems", "ntx_device_error", "ntx_gemv_q",
-           "ntx_dequant_q", "ntx_repack_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_workspace_bytes", "ntx_swiglu",
+           "ntx_dequant_q", "ntx_repack_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_decode_noalloc", "ntx_attn_workspace_bytes", "ntx_swiglu",
            "ntx_softmax", "ntx_argmax", "ntx_embed", "ntx_model_create", "ntx_model_destroy", "ntx_decode_step",
            "ntx_stream_layers", "ntx_stream_stats")
 
@@ -73,6 +73,7 @@ def lib() -> ctypes.CDLL:
             "ntx_rope": ([vp, vp, ci, ci, ci, i32, cf, vp], ci),
             "ntx_attn_decode": ([vp, vp, vp, vp, ci, ci, ci, i32, i32, vp, sz, vp], ci),
             "ntx_attn_workspace_bytes": ([ci, ci, ci, i32], sz),
+            "ntx_attn_decode_noalloc": ([vp, vp, vp, vp, ci, ci, ci, i32, i32, vp], ci),
             "ntx_swiglu": ([vp, vp, vp, i64, vp], ci),
             "ntx_softmax": ([vp, vp, i64, vp], ci),
             "ntx_argmax": ([vp, i64, vp, vp], ci),
@@ -163,6 +164,12 @@ def ntx_attn_decode(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, n
                     workspace_bytes, stream=None) -> None:
     check(lib().ntx_attn_decode(_p(q), _p(k_cache), _p(v_cache), _p(out), n_q_heads, n_kv_heads, head_dim, n_ctx,
                                 max_ctx, _p(workspace), workspace_bytes, _s(stream)))
+
+
+def ntx_attn_decode_noalloc(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, n_ctx, max_ctx,
+                            stream=None) -> None:
+    check(lib().ntx_attn_decode_noalloc(_p(q), _p(k_cache), _p(v_cache), _p(out), n_q_heads, n_kv_heads, head_dim,
+                                        n_ctx, max_ctx, _s(stream)))
 
 
 def ntx_swiglu(gate, up, out, n, stream=None) -> None:

@@ -31,7 +31,7 @@ constexpr int kThreads = kConsumers + 32;
 constexpr int kSub = 64;                          // positions per stage
 constexpr int kStageBytes = kSub * HD * 2 * 2;    // K and V rows
 constexpr int kStages = 4;
-constexpr int kCounterBytes = 256;                // ticket counters at the start of the workspace
+constexpr int kCounterBytes = kAttnCounterBytes;  // ticket counters at the start of the workspace
 constexpr int kPartFloats = 4 + HD;               // m, l, 2 pad, acc[128]: 528-byte records
 constexpr int kMaxSplit = 128;
 constexpr uint32_t kPolls = 1u << 22;
@@ -388,23 +388,37 @@ NTX_EXPORT size_t ntx_attn_workspace_bytes(int n_q_heads, int n_kv_heads, int he
     return attn_workspace_bytes_for(n_q_heads, n_kv_heads, head_dim, attn_split_for(n_q_heads, n_kv_heads, max_ctx));
 }
 
+namespace ntx {
+
+ntx_status attn_check(const void* q, const void* k_cache, const void* v_cache, const void* out, int n_q_heads,
+                      int n_kv_heads, int head_dim, int32_t n_ctx, int32_t max_ctx, const char* who)
+{
+    const std::string w(who);
+    if (!q || !k_cache || !v_cache || !out) return fail(NTX_EINVAL, w + ": null pointer");
+    if (head_dim != HD) return fail(NTX_EUNSUPPORTED, w + ": head_dim must be 128");
+    if (n_kv_heads < 1 || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads)
+        return fail(NTX_EINVAL, w + ": n_q_heads must be a positive multiple of n_kv_heads");
+    const int G = n_q_heads / n_kv_heads;
+    if (G != 1 && G != 2 && G != 4 && G != 8)
+        return fail(NTX_EUNSUPPORTED, w + ": q heads per kv head must be 1, 2, 4 or 8");
+    if (n_kv_heads > 64) return fail(NTX_EUNSUPPORTED, w + ": at most 64 kv heads");
+    if (max_ctx < 1 || n_ctx < 1 || n_ctx > max_ctx) return fail(NTX_EINVAL, w + ": need 1 <= n_ctx <= max_ctx");
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+        return fail(NTX_EINVAL, w + ": q, out and the caches must be 16-byte aligned");
+    return NTX_OK;
+}
+
+}  // namespace ntx
+
 NTX_EXPORT ntx_status ntx_attn_decode(const float* q, const void* k_cache, const void* v_cache, float* out,
                                       int n_q_heads, int n_kv_heads, int head_dim, int32_t n_ctx, int32_t max_ctx,
                                       void* workspace, size_t workspace_bytes, void* stream)
 {
-    if (!q || !k_cache || !v_cache || !out || !workspace) return fail(NTX_EINVAL, "ntx_attn_decode: null pointer");
-    if (head_dim != HD) return fail(NTX_EUNSUPPORTED, "ntx_attn_decode: head_dim must be 128");
-    if (n_kv_heads < 1 || n_q_heads < n_kv_heads || n_q_heads % n_kv_heads)
-        return fail(NTX_EINVAL, "ntx_attn_decode: n_q_heads must be a positive multiple of n_kv_heads");
-    const int G = n_q_heads / n_kv_heads;
-    if (G != 1 && G != 2 && G != 4 && G != 8)
-        return fail(NTX_EUNSUPPORTED, "ntx_attn_decode: q heads per kv head must be 1, 2, 4 or 8");
-    if (n_kv_heads > 64) return fail(NTX_EUNSUPPORTED, "ntx_attn_decode: at most 64 kv heads");
-    if (max_ctx < 1 || n_ctx < 1 || n_ctx > max_ctx)
-        return fail(NTX_EINVAL, "ntx_attn_decode: need 1 <= n_ctx <= max_ctx");
-    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
-        !aligned(workspace, 16))
-        return fail(NTX_EINVAL, "ntx_attn_decode: q, out, caches and workspace must be 16-byte aligned");
+    ntx_status st = attn_check(q, k_cache, v_cache, out, n_q_heads, n_kv_heads, head_dim, n_ctx, max_ctx,
+                               "ntx_attn_decode");
+    if (st != NTX_OK) return st;
+    if (!workspace || !aligned(workspace, 16))
+        return fail(NTX_EINVAL, "ntx_attn_decode: workspace must be non-null and 16-byte aligned");
     const int n_split = attn_split_for(n_q_heads, n_kv_heads, max_ctx);
     if (workspace_bytes < attn_workspace_bytes_for(n_q_heads, n_kv_heads, head_dim, n_split))
         return fail(NTX_EINVAL, "ntx_attn_decode: workspace smaller than ntx_attn_workspace_bytes()");

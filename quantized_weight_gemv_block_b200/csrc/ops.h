@@ -25,6 +25,9 @@ struct AttnArgs {
     int n_split;                // CTAs per kv head
     bool pdl;
 };
+constexpr int kAttnCounterBytes = 256;   // ticket counters at the start of an attention workspace
+ntx_status attn_check(const void* q, const void* k_cache, const void* v_cache, const void* out, int n_q_heads,
+                      int n_kv_heads, int head_dim, int32_t n_ctx, int32_t max_ctx, const char* who);
 int attn_split_for(int n_q_heads, int n_kv_heads, int32_t max_ctx);
 size_t attn_workspace_bytes_for(int n_q_heads, int n_kv_heads, int head_dim, int n_split);
 ntx_status attn_launch(const AttnArgs& a, cudaStream_t s);
