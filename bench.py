@@ -172,13 +172,15 @@ def gemv_shapes(spec):
 
 def measure_gemv_roofline(ntx, model, spec, stream, iters=3):
     """Time every decode GEMV of one step on its own (same weights, same shapes, same
-    stream) with CUDA events: the dominant kernel's achieved HBM bandwidth."""
+    stream) with CUDA events: the dominant kernel's achieved HBM bandwidth.  Only
+    HBM-resident layers count; streamed layers are bound by the host link, which is
+    reported on its own."""
     import torch
     import synth
     x = torch.randn(max(spec.hidden, spec.ffn, spec.q_dim), device="cuda")
     y = torch.empty(max(spec.vocab, spec.ffn, spec.qkv_rows), device="cuda")
     launches = []
-    for t in model.layers:
+    for t in model.layers[:model.n_resident]:
         launches.append((t["w_qkv"], spec.qkv_rows, spec.hidden))
         launches.append((t["w_o"], spec.hidden, spec.q_dim))
         launches.append((t["w_gate"], spec.ffn, spec.hidden))

@@ -102,8 +102,11 @@ size_t ntx_row_bytes(int qtype, int64_t cols);
 /* Elements per block of qtype (32 or 256), 0 if unknown. */
 int ntx_block_elems(int qtype);
 
-/* Error code recorded by a kernel on the current device whose bounded wait ran
- * out (0 = none), and reset it.  Synchronises the current device. */
+/* Error code recorded by a kernel on the current device (0 = none), and reset
+ * it: bit 0 a consumer's wait for a filled stage ran out, bit 1 a producer's
+ * wait for a drained stage, bit 2 a producer's final drain, bit 3 shared memory
+ * was not aligned as the copies need (the kernel did nothing).  Bits of several
+ * kernels are OR-ed.  Synchronises the current device. */
 ntx_status ntx_device_error(uint32_t* code);
 
 /* ---------------------------------------------------------------- quantized GEMV
@@ -151,8 +154,9 @@ ntx_status ntx_rope(float* q, float* k, int n_q_heads, int n_kv_heads, int head_
  *   k_cache, v_cache  device fp16 [n_kv_heads, max_ctx, head_dim]
  *   out     device fp32 [n_q_heads, head_dim]
  *   workspace / workspace_bytes: device scratch of at least
- *           ntx_attn_workspace_bytes(...) bytes, 16-byte aligned; zero-initialised
- *           by the caller once before first use (the kernel leaves it zeroed).
+ *           ntx_attn_workspace_bytes(...) bytes, 16-byte aligned, for the partial
+ *           results of the context splits; it needs no initialisation.
+ * Two kernels run on `stream`: the split kernel, then the merge of the splits.
  * head_dim == 128, n_q_heads a multiple of n_kv_heads with at most 8 q heads per
  * kv head, 1 <= n_ctx <= max_ctx.  Calls sharing a workspace must not overlap. */
 ntx_status ntx_attn_decode(const float* q, const void* k_cache, const void* v_cache, float* out, int n_q_heads,
@@ -164,14 +168,13 @@ size_t ntx_attn_workspace_bytes(int n_q_heads, int n_kv_heads, int head_dim, int
  * memory: code that runs under a fixed, pre-planned memory budget or inside a
  * host framework whose allocator hands out no scratch, and so has no workspace
  * to pass.  (The pages have no counterpart; this is an addition of this library.)
- * The split partials and counters live in a device array of 512 KiB that the
+ * The split partials live in a device array of 512 KiB that the
  * library holds on every GPU that loads it, until the process exits.  Shapes
  * whose workspace (ntx_attn_workspace_bytes) exceeds 512 KiB are rejected with
  * NTX_EUNSUPPORTED (on a 148-SM B200: 8 q heads per kv head with 8 kv heads, as
  * in Llama-70B, needs about 600 KB; 4 per kv head, as in Llama-8B, about 300 KB).  Nothing is allocated: the first call on a device looks up
  * the array's device address (cudaGetSymbolAddress) and caches it, so make that
- * first call before any stream capture.  Each call first clears the counters
- * with cudaMemsetAsync on `stream`.  All calls share the one array, so calls
+ * first call before any stream capture.  All calls share the one array, so calls
  * whose work overlaps on the GPU (different streams, or another thread) race:
  * serialise them.  Arguments, layouts and errors as for ntx_attn_decode. */
 ntx_status ntx_attn_decode_noalloc(const float* q, const void* k_cache, const void* v_cache, float* out,

@@ -6,18 +6,29 @@
 // [s P, s P + P) of kv head g together with the G = n_q / n_kv query heads that
 // read it, so every K / V row is fetched from HBM once:
 //  * a producer warp streams the range in stages of 64 positions (K rows and V
-//    rows, 32 KB) with 1-D bulk copies into a ring of shared-memory stages;
-//  * 16 consumer warps: scores (lanes own 4 dims of a K row, the G partial dot
-//    products are reduced across the warp with a transposed butterfly), an
-//    online softmax per query head (running max m and sum l), then P.V with
-//    paired fp32 FMAs;
-//  * the partial (m, l, acc[128]) of each query head goes to the workspace; the
-//    last CTA of kv head g (ticket counter, reset after use) bulk-copies all
-//    partials of its head into shared memory and merges them with the
-//    log-sum-exp rule in a fixed order, so the result is deterministic.
+//    rows, 32 KB) into a ring of shared-memory stages with TMA tensor copies of
+//    64 x 64 fp16 boxes in the 128-byte swizzle, so the tensor-core operand loads
+//    (ldmatrix, 8 rows of one column) hit 8 different bank groups;
+//  * both contractions run on the tensor cores (mma.sync m16n8k16, fp16
+//    operands, fp32 accumulation), in two warp roles that overlap across stages:
+//    4 score warps form S^T = K q^T (q split into an fp16 high part and an fp16
+//    remainder, two products, so q keeps ~22 bits) and run the online softmax
+//    (running max m per query head, per-lane shares of the running sum l), and
+//    hand P and the rescale factors of stage i through a double buffer to 8 P.V
+//    warps, which form O^T = V^T P^T (P split the same way) while the score warps
+//    move on to stage i + 1.  K and V are fp16 already, so every product is exact
+//    and only the fp32 accumulation rounds;
+//  * the partial (m, l, acc[128]) of each query head goes to the workspace, and a
+//    second kernel (one CTA per query head, launched as a programmatic dependent)
+//    merges the splits with the log-sum-exp rule in a fixed order, so the result
+//    is deterministic.
 // Every wait is bounded; a wait that runs out records an error and the CTA still
 // finishes.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
 #include <algorithm>
+#include <mutex>
 
 #include "ops.h"
 
@@ -25,23 +36,22 @@ namespace ntx {
 namespace {
 
 constexpr int HD = 128;
-constexpr int kConsumerWarps = 16;
-constexpr int kConsumers = kConsumerWarps * 32;
-constexpr int kThreads = kConsumers + 32;
+constexpr int kSWarps = 4;                        // score + softmax warps, 16 positions each
+constexpr int kPVWarps = 8;                       // P.V warps, 16 dims each
+constexpr int kProducerWarp = kSWarps + kPVWarps;
+constexpr int kThreads = (kProducerWarp + 1) * 32;
 constexpr int kSub = 64;                          // positions per stage
-constexpr int kStageBytes = kSub * HD * 2 * 2;    // K and V rows
+constexpr int kBoxBytes = kSub * 128;             // 64 rows x 64 dims fp16, swizzled 128 B rows
+constexpr int kStageBytes = 4 * kBoxBytes;        // K dims 0-63, 64-127, then V the same
 constexpr int kStages = 4;
-constexpr int kCounterBytes = kAttnCounterBytes;  // ticket counters at the start of the workspace
 constexpr int kPartFloats = 4 + HD;               // m, l, 2 pad, acc[128]: 528-byte records
 constexpr int kMaxSplit = 128;
 constexpr uint32_t kPolls = 1u << 22;
 
 struct KArgs {
+    CUtensorMap tk, tv;         // K and V caches as [n_kv][max_ctx][128] fp16, 64 x 64 boxes
     const float* q;
-    const __half* kc;
-    const __half* vc;
     float* out;
-    uint32_t* cnt;
     float* part;
     int max_ctx, n_split;
     int32_t n_ctx;
@@ -49,42 +59,98 @@ struct KArgs {
     int use_pdl;
 };
 
+// Tensor-core helpers (mma.sync m16n8k16, fp16 in, fp32 accumulate).
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2])
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_addr(p)));
+}
+
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t (&r)[4], const void* p)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(smem_addr(p)));
+}
+
+// (x, y) as an fp16 pair (element x in the low half) plus the fp16 pair of what
+// that rounding left out; hi + lo carries ~22 significant bits of each value.
+__device__ __forceinline__ void split_f16x2(float x, float y, uint32_t& hi, uint32_t& lo)
+{
+    const __half2 h = __floats2half2_rn(x, y);
+    const float2 hf = __half22float2(h);
+    const __half2 l = __floats2half2_rn(x - hf.x, y - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 // shared-memory layout (bytes)
-constexpr int kOffBars = 0;                             // full[4], empty[4], merge barrier
-constexpr int kOffFlag = 80;
-constexpr int kOffStat = 128;                           // m[8], l[8], alpha[8]
-constexpr int kOffScore = 256;                          // s[8][64] floats
-constexpr int kOffRed = kOffScore + 8 * kSub * 4;       // [16][128] floats
-constexpr int kOffRing = kOffRed + kConsumerWarps * HD * 4;
+constexpr int kOffBars = 0;      // full[4], empty[4], pfull[2], pempty[2]
+constexpr int kOffWMax = 256;    // [2][4 warps][8 heads] stage maxima of the score warps
+constexpr int kOffWSum = 512;    // [4 warps][8 heads] final sums
+constexpr int kOffAlpha = 640;   // [2][8] rescale factors of the running accumulators
+constexpr int kScStride = kSub + 8;                     // floats per head row of P (bank spread)
+constexpr int kOffP = 1024;                             // P[2][8 heads][72] floats
+constexpr int kOffRing = (kOffP + 2 * 8 * kScStride * 4 + 1023) & ~1023;   // the swizzle repeats every 1024 B
 constexpr int kSmem = kOffRing + kStages * kStageBytes;
 
-template <int G>
-__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const KArgs a)
+// Byte offset of 16-byte chunk c (dims 8c .. 8c + 7) of row r inside a swizzled
+// 64 x 64 box: chunk index XOR (row mod 8), as the 128-byte TMA swizzle stores it.
+__device__ __forceinline__ uint32_t swz(int r, int c) { return (uint32_t)(r * 128 + (((c ^ r) & 7) << 4)); }
+
+__device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int x, int y, int z, uint64_t* bar,
+                                        uint64_t policy)
 {
-    extern __shared__ __align__(128) uint8_t sm[];
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint "
+        "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+template <int G>
+__global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant__ KArgs a)
+{
+    extern __shared__ __align__(1024) uint8_t sm[];
     uint64_t* full = reinterpret_cast<uint64_t*>(sm + kOffBars);
     uint64_t* empty = full + kStages;
-    uint64_t* mbar = empty + kStages;
-    int* flag = reinterpret_cast<int*>(sm + kOffFlag);
-    float* s_m = reinterpret_cast<float*>(sm + kOffStat);
-    float* s_l = s_m + 8;
-    float* s_alpha = s_l + 8;
-    float* sc = reinterpret_cast<float*>(sm + kOffScore);
-    float* red = reinterpret_cast<float*>(sm + kOffRed);
+    uint64_t* pfull = empty + kStages;
+    uint64_t* pempty = pfull + 2;
+    float* wmax = reinterpret_cast<float*>(sm + kOffWMax);
+    float* wsum = reinterpret_cast<float*>(sm + kOffWSum);
+    float* s_alpha = reinterpret_cast<float*>(sm + kOffAlpha);
+    float* Pbuf = reinterpret_cast<float*>(sm + kOffP);
     uint8_t* ring = sm + kOffRing;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (warp == kProducerWarp && lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&a.tk)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&a.tv)) : "memory");
+    }
+    if (smem_addr(ring) & 1023u) {
+        // the swizzled boxes need a 1024-byte aligned ring; never issue a copy otherwise
+        if (tid == 0) record_device_error(DEVERR_SMEM_ALIGN);
+        return;
+    }
     if (tid == 0) {
         for (int i = 0; i < kStages; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kConsumerWarps);
+            mbar_init(&empty[i], kSWarps + kPVWarps);
         }
-        mbar_init(mbar, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&pfull[b], kSWarps);
+            mbar_init(&pempty[b], kPVWarps);
+        }
         fence_mbar_init();
-    }
-    if (tid < 8) {
-        s_m[tid] = -INFINITY;
-        s_l[tid] = 0.f;
     }
     __syncthreads();
     if (a.use_pdl) {
@@ -97,225 +163,319 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const KArgs a)
     const int t0 = sp * P;
     const int np = max(0, min(n_ctx, t0 + P) - t0);
     const int nsub = (np + kSub - 1) / kSub;
+    const int gid = lane >> 2, tig = lane & 3;
+    float* part = a.part + (size_t)(g * a.n_split + sp) * G * kPartFloats;
 
-    if (warp == kConsumerWarps) {
+    if (warp == kProducerWarp) {
         // ------------------------------------------------------------ producer
-        if (lane == 0) {
-            const uint64_t pol = policy_evict_first();
-            const __half* kb = a.kc + ((int64_t)g * a.max_ctx + t0) * HD;
-            const __half* vb = a.vc + ((int64_t)g * a.max_ctx + t0) * HD;
-            int s = 0;
-            uint32_t ph = 0;
-            for (int i = 0; i < nsub; ++i) {
-                if (!mbar_wait(&empty[s], ph ^ 1u, kPolls)) {
-                    record_device_error(DEVERR_EMPTY_WAIT);
-                    // the stages issued last must land before the CTA may exit
-                    for (int k = 1; k <= kStages && k <= i; ++k) {
-                        const int j = i - k;
-                        mbar_wait(&full[j % kStages], (uint32_t)(j / kStages) & 1u, 1u << 20);
-                    }
-                    break;
-                }
-                const int cnt = min(kSub, np - i * kSub);
-                const uint32_t bytes = (uint32_t)cnt * HD * 2;
-                uint8_t* st = ring + s * kStageBytes;
-                mbar_arrive_expect_tx(&full[s], 2 * bytes);
-                bulk_g2s(st, kb + (int64_t)i * kSub * HD, bytes, &full[s], pol);
-                bulk_g2s(st + kSub * HD * 2, vb + (int64_t)i * kSub * HD, bytes, &full[s], pol);
-                if (++s == kStages) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-            }
-        }
-    } else {
-        // ----------------------------------------------------------- consumers
-        // q of the G heads, pre-scaled by 1/sqrt(128); lane owns dims 4 lane .. +3
-        uint64_t q2[G][2];
-        const float scale = 0.08838834764831845f;
-#pragma unroll
-        for (int h = 0; h < G; ++h) {
-            const float4 v = *reinterpret_cast<const float4*>(a.q + (int64_t)(g * G + h) * HD + 4 * lane);
-            q2[h][0] = pack2(__float_as_uint(v.x * scale), __float_as_uint(v.y * scale));
-            q2[h][1] = pack2(__float_as_uint(v.z * scale), __float_as_uint(v.w * scale));
-        }
-        // P.V ownership: WPH = 16 / G warps per head, positions interleaved over them
-        constexpr int WPH = kConsumerWarps / G;
-        const int pv_head = warp / WPH, pv_sub = warp % WPH;
-        uint64_t acc2[2] = {0, 0};
-        bool dead = false;
+        const uint64_t pol = policy_evict_first();
         int s = 0;
         uint32_t ph = 0;
-        for (int i = 0; i < nsub; ++i) {
-            const int cnt = min(kSub, np - i * kSub);
-            if (!dead && !mbar_wait(&full[s], ph, kPolls)) {
-                record_device_error(DEVERR_FULL_WAIT);
-                dead = true;
-            }
-            const __half* Ks = reinterpret_cast<const __half*>(ring + s * kStageBytes);
-            const __half* Vs = Ks + kSub * HD;
-            // scores: warp w takes positions w, w + 16, ...
-#pragma unroll
-            for (int t = warp; t < kSub; t += kConsumerWarps) {
-                float part[G];
-                if (t < cnt && !dead) {
-                    const uint2 raw = *reinterpret_cast<const uint2*>(Ks + t * HD + 4 * lane);
-                    const float2 k01 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-                    const float2 k23 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-                    const uint64_t ka = pack2(__float_as_uint(k01.x), __float_as_uint(k01.y));
-                    const uint64_t kb2 = pack2(__float_as_uint(k23.x), __float_as_uint(k23.y));
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        uint64_t d2 = 0;
-                        fma2(d2, q2[h][0], ka);
-                        fma2(d2, q2[h][1], kb2);
-                        const f2 d = f2_from(d2);
-                        part[h] = d.x + d.y;
-                    }
-                } else {
-#pragma unroll
-                    for (int h = 0; h < G; ++h) part[h] = 0.f;
+        for (int i = 0; i < nsub && lane == 0; ++i) {
+            if (!mbar_wait(&empty[s], ph ^ 1u, kPolls)) {
+                record_device_error(DEVERR_EMPTY_WAIT);
+                // the stages issued last must land before the CTA may exit
+                for (int k = 1; k <= kStages && k <= i; ++k) {
+                    const int jj = i - k;
+                    mbar_wait(&full[jj % kStages], (uint32_t)(jj / kStages) & 1u, 1u << 20);
                 }
-                // transposed butterfly: halving rounds leave one head per lane group
-                int head = 0;
-#pragma unroll
-                for (int n = G, sh = 16; n > 1; n >>= 1, sh >>= 1) {
-                    const bool hi = (lane & sh) != 0;
-#pragma unroll
-                    for (int k = 0; k < n / 2; ++k) {
-                        const float send = hi ? part[k] : part[k + n / 2];
-                        const float keep = hi ? part[k + n / 2] : part[k];
-                        part[k] = keep + __shfl_xor_sync(0xffffffffu, send, sh);
-                    }
-                    head += hi ? n / 2 : 0;
-                }
-                float v = part[0];
-#pragma unroll
-                for (int sh = 16 / G; sh > 0; sh >>= 1) v += __shfl_xor_sync(0xffffffffu, v, sh);
-                if ((lane & (32 / G - 1)) == 0) sc[head * kSub + t] = v;
+                break;
             }
-            named_bar_sync(1, kConsumers);
-            // online softmax: warp h updates head h
-            if (warp < G) {
-                const int h = warp;
-                const float x0 = lane < cnt ? sc[h * kSub + lane] : -INFINITY;
-                const float x1 = lane + 32 < cnt ? sc[h * kSub + lane + 32] : -INFINITY;
-                const float mx = gemv::warp_max(fmaxf(x0, x1));
-                const float m_old = s_m[h];
-                const float m_new = fmaxf(m_old, mx);
-                const float e0 = lane < cnt ? expf(x0 - m_new) : 0.f;
-                const float e1 = lane + 32 < cnt ? expf(x1 - m_new) : 0.f;
-                sc[h * kSub + lane] = e0;
-                sc[h * kSub + lane + 32] = e1;
-                const float sum = gemv::warp_sum(e0 + e1);
-                if (lane == 0) {
-                    const float alpha = m_old == -INFINITY ? 0.f : expf(m_old - m_new);
-                    s_alpha[h] = alpha;
-                    s_m[h] = m_new;
-                    s_l[h] = s_l[h] * alpha + sum;
-                }
-            }
-            named_bar_sync(1, kConsumers);
-            // P.V: this thread's 4 dims of head pv_head, positions pv_sub, pv_sub + WPH, ...
-            {
-                const float alpha = s_alpha[pv_head];
-                const uint64_t al2 = pack2(__float_as_uint(alpha), __float_as_uint(alpha));
-                acc2[0] = mul2(acc2[0], al2);
-                acc2[1] = mul2(acc2[1], al2);
-                if (!dead) {
-#pragma unroll 4
-                    for (int t = pv_sub; t < cnt; t += WPH) {
-                        const float p = sc[pv_head * kSub + t];
-                        const uint64_t p2 = pack2(__float_as_uint(p), __float_as_uint(p));
-                        const uint2 raw = *reinterpret_cast<const uint2*>(Vs + t * HD + 4 * lane);
-                        const float2 v01 = __half22float2(*reinterpret_cast<const __half2*>(&raw.x));
-                        const float2 v23 = __half22float2(*reinterpret_cast<const __half2*>(&raw.y));
-                        fma2(acc2[0], p2, pack2(__float_as_uint(v01.x), __float_as_uint(v01.y)));
-                        fma2(acc2[1], p2, pack2(__float_as_uint(v23.x), __float_as_uint(v23.y)));
-                    }
-                }
-            }
-            // the next stage's scores overwrite sc: every consumer must be done reading it
-            named_bar_sync(1, kConsumers);
-            if (lane == 0) mbar_arrive(&empty[s]);
+            // whole boxes always arrive: rows past the context are zero-filled or masked later
+            uint8_t* st = ring + s * kStageBytes;
+            const int y = t0 + i * kSub;
+            mbar_arrive_expect_tx(&full[s], (uint32_t)kStageBytes);
+            tma_box(st, &a.tk, 0, y, g, &full[s], pol);
+            tma_box(st + kBoxBytes, &a.tk, 64, y, g, &full[s], pol);
+            tma_box(st + 2 * kBoxBytes, &a.tv, 0, y, g, &full[s], pol);
+            tma_box(st + 3 * kBoxBytes, &a.tv, 64, y, g, &full[s], pol);
             if (++s == kStages) {
                 s = 0;
                 ph ^= 1u;
             }
         }
-        // combine the WPH warps of each head, write this split's partial
-        const f2 a01 = f2_from(acc2[0]), a23 = f2_from(acc2[1]);
-        *reinterpret_cast<float4*>(red + warp * HD + 4 * lane) = make_float4(a01.x, a01.y, a23.x, a23.y);
-        named_bar_sync(1, kConsumers);
-        if (pv_sub == 0) {
-            float4 o = *reinterpret_cast<const float4*>(red + warp * HD + 4 * lane);
-            for (int w = 1; w < WPH; ++w) {
-                const float4 r = *reinterpret_cast<const float4*>(red + (warp + w) * HD + 4 * lane);
-                o.x += r.x;
-                o.y += r.y;
-                o.z += r.z;
-                o.w += r.w;
+    } else if (warp < kSWarps) {
+        // ------------------------------------------- score and softmax warps
+        // S^T[position][head] = K q^T for positions 16 warp .. +15 of each stage.  q^T is
+        // the B operand (k = dim, n = head): each head is brought to max |q| in [1, 2)
+        // by a power of two (undone on the scores, exactly), then split into an fp16
+        // high part and an fp16 remainder; heads >= G are zero.  The four lanes of a
+        // quad (same gid) hold the 128 dims of head gid.
+        uint32_t qh[8][2], ql[8][2];
+        float mul0, mul1;   // score multipliers of heads 2 tig and 2 tig + 1
+        {
+            const float* qrow = a.q + (int64_t)(g * G + gid) * HD;
+            float2 v[8][2];
+            float mx = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    v[ks][half] = make_float2(0.f, 0.f);
+                    if (gid < G) v[ks][half] = *reinterpret_cast<const float2*>(qrow + 16 * ks + 8 * half + 2 * tig);
+                    mx = fmaxf(mx, fmaxf(fabsf(v[ks][half].x), fabsf(v[ks][half].y)));
+                }
             }
-            float* pp = a.part + ((size_t)(g * a.n_split + sp) * G + pv_head) * kPartFloats;
-            *reinterpret_cast<float4*>(pp + 4 + 4 * lane) = o;
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            // e = floor(log2 mx) from the bit pattern (mx normal); zero or subnormal heads keep e = 0
+            int e = 0;
+            if (mx >= 1.17549435e-38f && mx <= 3.4e38f) e = (int)((__float_as_uint(mx) >> 23) & 0xffu) - 127;
+            e = max(-100, min(100, e));
+            const float down = __uint_as_float((uint32_t)(127 - e) << 23);
+            // scores carry 1/sqrt(128) = 2^-3.5: 2^-4 goes into the exponent, sqrt(2) stays a multiply
+            const float up = __uint_as_float((uint32_t)(127 + e - 4) << 23) * 1.41421356237309515f;
+            mul0 = __shfl_sync(0xffffffffu, up, (2 * tig) << 2);
+            mul1 = __shfl_sync(0xffffffffu, up, (2 * tig + 1) << 2);
+#pragma unroll
+            for (int ks = 0; ks < 8; ++ks)
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+                    split_f16x2(v[ks][half].x * down, v[ks][half].y * down, qh[ks][half], ql[ks][half]);
+        }
+        // running max of heads 2 tig, 2 tig + 1 (identical in every lane with this tig)
+        // and this lane's share of the running sums
+        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+        const int m0w = 16 * warp;
+        const int j = lane >> 3, r = m0w + ((j & 1) << 3) + (lane & 7);
+        int s = 0;
+        uint32_t ph = 0;
+        for (int i = 0; i < nsub; ++i) {
+            const int cnt = min(kSub, np - i * kSub);
+            const int b = i & 1;
+            const bool ok_full = mbar_wait(&full[s], ph, kPolls);
+            const bool ok_p = mbar_wait(&pempty[b], ((uint32_t)(i >> 1) & 1u) ^ 1u, kPolls);
+            if (!ok_full || !ok_p) record_device_error(DEVERR_FULL_WAIT);
+            const uint8_t* Ks = ring + s * kStageBytes;
+            // ldmatrix: lane -> matrix j = lane / 8 (rows +8 if j odd, dims +8 if j >= 2), row lane % 8;
+            // four accumulation chains (dims 0-63 / 64-127, high / low part of q)
+            float c[4][4] = {};
+            if (m0w < cnt) {
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {
+                    uint32_t av[4];
+                    ldsm_x4(av, Ks + (ks >> 2) * kBoxBytes + swz(r, 2 * ks + (j >> 1)));
+                    mma_f16(c[(ks >> 2) * 2], av, qh[ks]);
+                    mma_f16(c[(ks >> 2) * 2 + 1], av, ql[ks]);
+                }
+            }
+            // K of this stage is no longer needed by this warp
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);
+            // sc[q]: q = 0 position gid, head 2 tig; 1 same position, head 2 tig + 1; 2, 3 position gid + 8
+            const bool v0 = m0w + gid < cnt, v1 = m0w + gid + 8 < cnt;
+            float sc[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) sc[q] = ((c[0][q] + c[1][q]) + (c[2][q] + c[3][q])) * ((q & 1) ? mul1 : mul0);
+            if (!v0) sc[0] = sc[1] = -INFINITY;
+            if (!v1) sc[2] = sc[3] = -INFINITY;
+            // stage maximum per head: this warp's 16 positions, then the four warps'
+            float x0 = fmaxf(sc[0], sc[2]), x1 = fmaxf(sc[1], sc[3]);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, o));
+                x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, o));
+            }
+            float* wm = wmax + b * (kSWarps * 8);
+            if (gid == 0) {
+                wm[warp * 8 + 2 * tig] = x0;
+                wm[warp * 8 + 2 * tig + 1] = x1;
+            }
+            named_bar_sync(2, kSWarps * 32);
+#pragma unroll
+            for (int w = 0; w < kSWarps; ++w) {
+                x0 = fmaxf(x0, wm[w * 8 + 2 * tig]);
+                x1 = fmaxf(x1, wm[w * 8 + 2 * tig + 1]);
+            }
+            const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
+            const float al0 = m0 == -INFINITY ? 0.f : expf(m0 - n0);
+            const float al1 = m1 == -INFINITY ? 0.f : expf(m1 - n1);
+            m0 = n0;
+            m1 = n1;
+            float p[4];
+            p[0] = v0 ? expf(sc[0] - n0) : 0.f;
+            p[1] = v0 ? expf(sc[1] - n1) : 0.f;
+            p[2] = v1 ? expf(sc[2] - n0) : 0.f;
+            p[3] = v1 ? expf(sc[3] - n1) : 0.f;
+            l0 = l0 * al0 + (p[0] + p[2]);
+            l1 = l1 * al1 + (p[1] + p[3]);
+            // P[head][position] for the P.V warps (masked positions are 0)
+            float* Pb = Pbuf + b * (8 * kScStride);
+            if (m0w < cnt) {
+                Pb[(2 * tig) * kScStride + m0w + gid] = p[0];
+                Pb[(2 * tig + 1) * kScStride + m0w + gid] = p[1];
+                Pb[(2 * tig) * kScStride + m0w + gid + 8] = p[2];
+                Pb[(2 * tig + 1) * kScStride + m0w + gid + 8] = p[3];
+            }
+            if (warp == 0 && gid == 0) {
+                s_alpha[b * 8 + 2 * tig] = al0;
+                s_alpha[b * 8 + 2 * tig + 1] = al1;
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pfull[b]);
+            if (++s == kStages) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+        // sums over the 16 positions of each warp, then over the warps
+#pragma unroll
+        for (int o = 4; o < 32; o <<= 1) {
+            l0 += __shfl_xor_sync(0xffffffffu, l0, o);
+            l1 += __shfl_xor_sync(0xffffffffu, l1, o);
+        }
+        if (gid == 0) {
+            wsum[warp * 8 + 2 * tig] = l0;
+            wsum[warp * 8 + 2 * tig + 1] = l1;
+        }
+        named_bar_sync(2, kSWarps * 32);
+        if (warp == 0 && gid == 0) {
+            float L0 = 0.f, L1 = 0.f;
+            for (int w = 0; w < kSWarps; ++w) {
+                L0 += wsum[w * 8 + 2 * tig];
+                L1 += wsum[w * 8 + 2 * tig + 1];
+            }
+            if (2 * tig < G) {
+                part[(2 * tig) * kPartFloats] = m0;
+                part[(2 * tig) * kPartFloats + 1] = L0;
+            }
+            if (2 * tig + 1 < G) {
+                part[(2 * tig + 1) * kPartFloats] = m1;
+                part[(2 * tig + 1) * kPartFloats + 1] = L1;
+            }
+        }
+    } else {
+        // ------------------------------------------------------ P.V warps
+        // O^T[dim][head] += V^T[dim][t] P^T[t][head] for dims 16 pw .. +15; the high and
+        // low fp16 parts of P accumulate in separate chains
+        const int pw = warp - kSWarps;
+        const int j = lane >> 3;
+        float acc[2][4] = {};
+        int s = 0;
+        uint32_t ph = 0;
+        for (int i = 0; i < nsub; ++i) {
+            const int cnt = min(kSub, np - i * kSub);
+            const int b = i & 1;
+            const bool ok_full = mbar_wait(&full[s], ph, kPolls);
+            const bool ok_p = mbar_wait(&pfull[b], (uint32_t)(i >> 1) & 1u, kPolls);
+            if (!ok_full || !ok_p) record_device_error(DEVERR_FULL_WAIT);
+            uint8_t* Vs = ring + s * kStageBytes + 2 * kBoxBytes + (pw >> 2) * kBoxBytes;
+            const int r_end = (cnt + 15) & ~15;
+            if (cnt < r_end) {
+                // rows cnt .. r_end - 1 were not part of the context: zero this warp's 16 dims of
+                // them (two 16-byte chunks per row) so 0 * garbage cannot reach the sums
+                for (int idx = lane; idx < 2 * (r_end - cnt); idx += 32) {
+                    const int rr = cnt + (idx >> 1);
+                    *reinterpret_cast<uint4*>(Vs + swz(rr, 2 * pw + (idx & 1))) = make_uint4(0u, 0u, 0u, 0u);
+                }
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                __syncwarp();
+            }
+            const float* Pb = Pbuf + b * (8 * kScStride);
+            const float a0 = s_alpha[b * 8 + 2 * tig], a1 = s_alpha[b * 8 + 2 * tig + 1];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                acc[h][0] *= a0;
+                acc[h][1] *= a1;
+                acc[h][2] *= a0;
+                acc[h][3] *= a1;
+            }
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {
+                const int k0 = 16 * kk;
+                if (k0 < cnt) {
+                    // matrix j: positions +8 if j >= 2, dims +8 if j odd
+                    uint32_t av[4];
+                    ldsm_x4_trans(av, Vs + swz(k0 + ((j >> 1) << 3) + (lane & 7), 2 * pw + (j & 1)));
+                    const float2 p0 = *reinterpret_cast<const float2*>(Pb + gid * kScStride + k0 + 2 * tig);
+                    const float2 p1 = *reinterpret_cast<const float2*>(Pb + gid * kScStride + k0 + 8 + 2 * tig);
+                    uint32_t bh[2], bl[2];
+                    split_f16x2(p0.x, p0.y, bh[0], bl[0]);
+                    split_f16x2(p1.x, p1.y, bh[1], bl[1]);
+                    mma_f16(acc[0], av, bh);
+                    mma_f16(acc[1], av, bl);
+                }
+            }
+            __syncwarp();
             if (lane == 0) {
-                pp[0] = s_m[pv_head];
-                pp[1] = s_l[pv_head];
+                mbar_arrive(&pempty[b]);
+                mbar_arrive(&empty[s]);
             }
+            if (++s == kStages) {
+                s = 0;
+                ph ^= 1u;
+            }
+        }
+        // acc[.][0]: dim 16 pw + gid, head 2 tig; [1] head 2 tig + 1; [2], [3] the same for dim + 8
+        const int d0 = 16 * pw + gid;
+        if (2 * tig < G) {
+            part[(2 * tig) * kPartFloats + 4 + d0] = acc[0][0] + acc[1][0];
+            part[(2 * tig) * kPartFloats + 4 + d0 + 8] = acc[0][2] + acc[1][2];
+        }
+        if (2 * tig + 1 < G) {
+            part[(2 * tig + 1) * kPartFloats + 4 + d0] = acc[0][1] + acc[1][1];
+            part[(2 * tig + 1) * kPartFloats + 4 + d0 + 8] = acc[0][3] + acc[1][3];
         }
     }
 
-    // ---- the last CTA of kv head g merges the splits (fixed order)
-    __threadfence();
-    __syncthreads();
-    if (tid == 0) {
-        const uint32_t ticket = atomicAdd(&a.cnt[g], 1u);
-        *flag = (ticket == (uint32_t)a.n_split - 1u) ? 1 : 0;
+}
+
+// Merge of the splits, one CTA per query head and one thread per dim: with
+// M = max_s m_s over splits that saw a position, w_s = e^(m_s - M) and
+// L = sum_s l_s w_s, out[d] = sum_s (w_s / L) acc_s[d], summed in split order.
+template <int G>
+__global__ void __launch_bounds__(HD) attn_merge_kernel(const float* part, float* out, int n_split, int use_pdl)
+{
+    constexpr int B = 32;   // splits whose partial dims are loaded together
+    __shared__ float wn[kMaxSplit];
+    if (use_pdl) {
+        pdl_launch_dependents();
+        pdl_wait();
     }
-    __syncthreads();
-    if (*flag) {
-        __threadfence();
-        // all partials of this kv head in one bulk copy (the ring is free now)
-        const float* base = a.part + (size_t)g * a.n_split * G * kPartFloats;
-        const uint32_t bytes = (uint32_t)(a.n_split * G * kPartFloats * 4);
-        float* pm = reinterpret_cast<float*>(ring);
-        if (tid == 0) {
-            asm volatile("fence.proxy.async.global;" ::: "memory");
-            mbar_arrive_expect_tx(mbar, bytes);
-            bulk_g2s(pm, base, bytes, mbar, policy_evict_first());
-        }
-        const bool ok = mbar_wait(mbar, 0, kPolls);
-        if (!ok && tid == 0) record_device_error(DEVERR_FULL_WAIT);
-        for (int idx = tid; ok && idx < G * HD; idx += kThreads) {
-            const int hh = idx / HD, d = idx % HD;
-            float M = -INFINITY;
-            for (int s2 = 0; s2 < a.n_split; ++s2) {
-                const float* ps = pm + ((size_t)s2 * G + hh) * kPartFloats;
-                if (ps[1] > 0.f) M = fmaxf(M, ps[0]);
-            }
-            float L = 0.f, o = 0.f;
-            for (int s2 = 0; s2 < a.n_split; ++s2) {
-                const float* ps = pm + ((size_t)s2 * G + hh) * kPartFloats;
-                if (ps[1] > 0.f) {
-                    const float w = expf(ps[0] - M);
-                    L = fmaf(ps[1], w, L);
-                    o = fmaf(ps[4 + d], w, o);
+    const int qh = blockIdx.x, g = qh / G, h = qh % G, d = threadIdx.x, lane = d & 31;
+    const size_t rec = (size_t)G * kPartFloats;   // floats from one split's record of this head to the next
+    const float* base = part + ((size_t)g * n_split * G + h) * kPartFloats;
+    float o = 0.f;
+    for (int s0 = 0; s0 < n_split; s0 += B) {
+        float v[B];
+#pragma unroll
+        for (int k = 0; k < B; ++k) v[k] = s0 + k < n_split ? __ldcg(base + (s0 + k) * rec + 4 + d) : 0.f;
+        if (s0 == 0) {
+            if (d < 32) {
+                float M = -INFINITY;
+                for (int s2 = lane; s2 < n_split; s2 += 32)
+                    if (__ldcg(base + s2 * rec + 1) > 0.f) M = fmaxf(M, __ldcg(base + s2 * rec));
+                M = gemv::warp_max(M);
+                float L = 0.f;
+                for (int s2 = lane; s2 < n_split; s2 += 32) {
+                    const float l = __ldcg(base + s2 * rec + 1);
+                    const float w = l > 0.f ? expf(__ldcg(base + s2 * rec) - M) : 0.f;
+                    wn[s2] = w;
+                    L = fmaf(l, w, L);
                 }
+                L = gemv::warp_sum(L);
+                const float inv = 1.f / L;
+                __syncwarp();
+                for (int s2 = lane; s2 < n_split; s2 += 32) wn[s2] *= inv;
             }
-            a.out[(int64_t)(g * G + hh) * HD + d] = o / L;
+            __syncthreads();
         }
-        if (tid == 0) a.cnt[g] = 0u;
+#pragma unroll
+        for (int k = 0; k < B; ++k)
+            if (s0 + k < n_split) o = fmaf(wn[s0 + k], v[k], o);
     }
+    out[(size_t)qh * HD + d] = o;
 }
 
 template <int G>
-ntx_status launch_g(const KArgs& k, int grid, cudaStream_t s, bool pdl)
+ntx_status launch_g(const KArgs& k, int n_q_heads, cudaStream_t s, bool pdl)
 {
     static bool configured = false;
     if (!configured) {
         cudaFuncSetAttribute(attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         configured = true;
     }
+    const int grid = (n_q_heads / G) * k.n_split;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kThreads);
@@ -328,6 +488,47 @@ ntx_status launch_g(const KArgs& k, int grid, cudaStream_t s, bool pdl)
     cfg.numAttrs = pdl ? 1 : 0;
     cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G>, k);
     if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("attention launch: ") + cudaGetErrorString(e));
+    // the merge always waits for the split kernel through the programmatic dependency
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3(n_q_heads);
+    mc.blockDim = dim3(HD);
+    mc.stream = s;
+    mc.attrs = attr;
+    mc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&mc, attn_merge_kernel<G>, (const float*)k.part, k.out, k.n_split, 1);
+    if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("attention merge launch: ") + cudaGetErrorString(e));
+    return NTX_OK;
+}
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder()
+{
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// A KV cache [n_kv][max_ctx][128] fp16 as a 3-D tensor map read in 64 x 64 boxes
+// with the 128-byte swizzle; boxes past max_ctx are zero-filled.
+ntx_status encode_kv_map(CUtensorMap* m, const __half* cache, int n_kv, int max_ctx)
+{
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tmap_encoder();
+    if (!enc) return fail(NTX_ECUDA, "attention: cuTensorMapEncodeTiled is not available from the driver");
+    const cuuint64_t dims[3] = {(cuuint64_t)HD, (cuuint64_t)max_ctx, (cuuint64_t)n_kv};
+    const cuuint64_t strides[2] = {(cuuint64_t)HD * 2, (cuuint64_t)max_ctx * HD * 2};
+    const cuuint32_t box[3] = {64, (cuuint32_t)kSub, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<__half*>(cache), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(NTX_ECUDA, "attention: KV tensor map encoding failed (" + std::to_string(r) + ")");
     return NTX_OK;
 }
 
@@ -338,42 +539,40 @@ cudaError_t take_device_error_attn(uint32_t* out) { return take_tu_device_error(
 int attn_split_for(int n_q_heads, int n_kv_heads, int32_t max_ctx)
 {
     (void)max_ctx;
-    const int G = n_q_heads / n_kv_heads;
-    // one CTA per SM, and every split's partial must fit the merge buffer
-    const int by_merge = (kStages * kStageBytes) / (G * kPartFloats * 4);
-    return std::min(std::min(kMaxSplit, by_merge), std::max(1, num_sms() / n_kv_heads));
+    (void)n_q_heads;
+    // one CTA per SM
+    return std::min(kMaxSplit, std::max(1, num_sms() / n_kv_heads));
 }
 
 size_t attn_workspace_bytes_for(int n_q_heads, int n_kv_heads, int head_dim, int n_split)
 {
     (void)head_dim;
     const int G = n_q_heads / n_kv_heads;
-    return (size_t)kCounterBytes + (size_t)n_kv_heads * n_split * G * kPartFloats * sizeof(float);
+    return (size_t)n_kv_heads * n_split * G * kPartFloats * sizeof(float);
 }
 
 ntx_status attn_launch(const AttnArgs& a, cudaStream_t s)
 {
     const int G = a.n_q_heads / a.n_kv_heads;
-    if ((size_t)a.n_split * G * kPartFloats * 4 > (size_t)kStages * kStageBytes)
-        return fail(NTX_EUNSUPPORTED, "attention: too many splits for the merge buffer");
+    if (a.n_split < 1 || a.n_split > kMaxSplit || G * a.n_split * 4 > 2 * 8 * kScStride * 4)
+        return fail(NTX_EUNSUPPORTED, "attention: split count out of range");
     KArgs k{};
+    ntx_status st = encode_kv_map(&k.tk, a.k_cache, a.n_kv_heads, a.max_ctx);
+    if (st != NTX_OK) return st;
+    if ((st = encode_kv_map(&k.tv, a.v_cache, a.n_kv_heads, a.max_ctx)) != NTX_OK) return st;
     k.q = a.q;
-    k.kc = a.k_cache;
-    k.vc = a.v_cache;
     k.out = a.out;
-    k.cnt = reinterpret_cast<uint32_t*>(a.workspace);
-    k.part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.workspace) + kCounterBytes);
+    k.part = reinterpret_cast<float*>(a.workspace);
     k.max_ctx = a.max_ctx;
     k.n_split = a.n_split;
     k.n_ctx = a.n_ctx;
     k.pos_dev = a.pos_dev;
     k.use_pdl = a.pdl ? 1 : 0;
-    const int grid = a.n_kv_heads * a.n_split;
     switch (G) {
-    case 1: return launch_g<1>(k, grid, s, a.pdl);
-    case 2: return launch_g<2>(k, grid, s, a.pdl);
-    case 4: return launch_g<4>(k, grid, s, a.pdl);
-    case 8: return launch_g<8>(k, grid, s, a.pdl);
+    case 1: return launch_g<1>(k, a.n_q_heads, s, a.pdl);
+    case 2: return launch_g<2>(k, a.n_q_heads, s, a.pdl);
+    case 4: return launch_g<4>(k, a.n_q_heads, s, a.pdl);
+    case 8: return launch_g<8>(k, a.n_q_heads, s, a.pdl);
     default: return fail(NTX_EUNSUPPORTED, "attention: q heads per kv head must be 1, 2, 4 or 8");
     }
 }

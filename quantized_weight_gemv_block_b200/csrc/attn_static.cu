@@ -1,8 +1,8 @@
 // attn_static.cu - decode attention whose scratch is a fixed device array owned
 // by this library, for callers that cannot allocate device memory themselves.
 //
-// The split partials and ticket counters of the attention kernel normally live
-// in a workspace the caller allocates.  Here they live in g_attn_scratch, a
+// The split partials of the attention kernel normally live in a workspace the
+// caller allocates.  Here they live in g_attn_scratch, a
 // file-scope device array of kStaticScratchBytes that exists on every GPU that
 // loads the library, for as long as the process runs.  In host code the array's
 // name only stands for the symbol; its device address is looked up once per
@@ -60,8 +60,8 @@ NTX_EXPORT ntx_status ntx_attn_decode_noalloc(const float* q, const void* k_cach
     void* ws = nullptr;
     if ((st = static_scratch(&ws)) != NTX_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    // the ticket counters must start at zero; the partials are overwritten before use
-    NTX_CUDA_TRY(cudaMemsetAsync(ws, 0, kAttnCounterBytes, s));
+    // nothing in the scratch carries over between calls: every split's partial is
+    // written before the merge reads it, so it needs no clearing
     AttnArgs a{};
     a.q = q;
     a.k_cache = (const __half*)k_cache;

@@ -33,6 +33,7 @@ enum : uint32_t {
     DEVERR_FULL_WAIT = 1u,     // consumer waited too long for a stage to fill
     DEVERR_EMPTY_WAIT = 2u,    // producer waited too long for a stage to drain
     DEVERR_DRAIN_WAIT = 4u,    // producer gave up draining its copies on exit
+    DEVERR_SMEM_ALIGN = 8u,    // shared memory not aligned as the copies need; nothing was done
 };
 
 // One flag per translation unit; ntx_device_error() collects them all.

@@ -21,11 +21,10 @@ struct AttnArgs {
     int n_q_heads, n_kv_heads, head_dim, max_ctx;
     int32_t n_ctx;              // used when n_ctx_from_pos is null
     const int32_t* pos_dev;     // if set: n_ctx = *pos_dev + 1 (read on the device)
-    void* workspace;            // counters + partials, zeroed once
+    void* workspace;            // split partials (no initialisation needed)
     int n_split;                // CTAs per kv head
     bool pdl;
 };
-constexpr int kAttnCounterBytes = 256;   // ticket counters at the start of an attention workspace
 ntx_status attn_check(const void* q, const void* k_cache, const void* v_cache, const void* out, int n_q_heads,
                       int n_kv_heads, int head_dim, int32_t n_ctx, int32_t max_ctx, const char* who);
 int attn_split_for(int n_q_heads, int n_kv_heads, int32_t max_ctx);

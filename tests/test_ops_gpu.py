@@ -108,12 +108,16 @@ def test_attention(ntx, orc, syn, nq, nkv, n_ctx, max_ctx):
     vc = syn.normal_f16_host(6, 3, nkv * max_ctx * hd)
     out = torch.full((nq * hd,), float("nan"), dtype=torch.float32, device="cuda")
     wsb = ntx.ntx_attn_workspace_bytes(nq, nkv, hd, max_ctx)
-    ws = torch.zeros(wsb, dtype=torch.uint8, device="cuda")
+    ws = torch.full((wsb,), 0xFF, dtype=torch.uint8, device="cuda")     # NaN bytes: it needs no initialisation
     kd, vd = dev(kc.view(np.float16)), dev(vc.view(np.float16))
-    for _ in range(2):       # the workspace counters must come back to zero for the next call
+    o = orc.attn_decode(q, kc.reshape(nkv, max_ctx, hd), vc.reshape(nkv, max_ctx, hd), nq, nkv, hd, n_ctx, max_ctx)
+    first = None
+    for _ in range(2):       # a second call on the used workspace gives the same bits
         ntx.ntx_attn_decode(dev(q), kd, vd, out, nq, nkv, hd, n_ctx, max_ctx, ws, wsb)
         torch.cuda.synchronize()
-        o = orc.attn_decode(q, kc.reshape(nkv, max_ctx, hd), vc.reshape(nkv, max_ctx, hd), nq, nkv, hd, n_ctx,
-                            max_ctx)
-        assert rel_err(out.cpu().numpy(), o) <= 1e-4
-    assert int(ws[:256].view(torch.int32).abs().sum()) == 0
+        got = out.cpu().numpy().copy()
+        assert rel_err(got, o) <= 1e-4
+        if first is None:
+            first = got
+        else:
+            assert np.array_equal(first, got)
