@@ -69,18 +69,24 @@ typedef enum ntx_qtype {
     NTX_Q4_0 = 1,
     NTX_Q4_K = 2,
     NTX_Q6_K = 3,
-    /* Tiled layouts (flag NTX_TILED): the same blocks, the same bytes per row,
-     * regrouped inside fixed tiles so every code run starts on a 16-byte boundary.
-     * Produced from the GGUF-style layout by ntx_repack_q, lossless.
-     *   NTX_Q8_0_T tile = 8 blocks (256 weights, 272 B): 256 int8 codes in element
-     *              order | the 8 fp16 d
-     *   NTX_Q4_0_T tile = 8 blocks (256 weights, 144 B): the 8 blocks' 16 code bytes
-     *              (nibble order unchanged) | the 8 fp16 d
-     *   NTX_Q4_K_T tile = 1 superblock: identical to NTX_Q4_K
-     *   NTX_Q6_K_T tile = 8 superblocks (2048 weights, 1680 B): 8 x 128 B low code
-     *              bits | 8 x 64 B high code bits | 8 x 16 int8 scales | 8 fp16 d
-     * A row of a tiled tensor must hold whole tiles (cols a multiple of 256, 2048
-     * for Q6_K). */
+    /* Tiled layouts (flag NTX_TILED): the same information in the same bytes per
+     * row, reordered for the tensor-core GEMV.  Produced from the GGUF-style
+     * layout by ntx_repack_q, lossless.  Rows come in groups of 16 (a tiled
+     * tensor has a multiple of 16 rows); a group is a run of units along the
+     * row, unit u covering columns [u UK, (u + 1) UK) of the group's 16 rows in
+     * 16 x the GGUF-style bytes of UK columns (UK = 32 for Q8_0 / Q4_0: one
+     * block; 256 for Q4_K / Q6_K: one superblock).  Inside a unit the codes of
+     * each 32-column step sit in the order in which lane 4 gid + tig of a warp
+     * takes them as the A operand of one m16n8k32 integer MMA (rows gid and
+     * gid + 8, columns 4 tig .. 4 tig + 3 and 16 + 4 tig .. 16 + 4 tig + 3),
+     * followed by the unit's scales:
+     *   NTX_Q8_0_T  unit 544 B: 32 lanes x 16 int8 codes | 8 x (d[r], d[r+8])
+     *   NTX_Q4_0_T  unit 288 B: 32 lanes x 8 B (two 4-bit codes per byte) | 8 x (d[r], d[r+8])
+     *   NTX_Q6_K_T  unit 3360 B: 8 steps x 32 lanes x 12 B (four 6-bit codes per 3
+     *               bytes) | 256 B int8 sub-block scales | 8 x (d[r], d[r+8])
+     *   NTX_Q4_K_T  unit 2304 B: 8 steps x 32 lanes x 8 B | 8 x 24 B of 6-bit scales
+     *               and mins | 8 x (d[r], d[r+8], dmin[r], dmin[r+8])
+     * A row of a tiled tensor must hold whole units. */
     NTX_TILED = 16,
     NTX_Q8_0_T = 16,
     NTX_Q4_0_T = 17,
@@ -95,8 +101,8 @@ const char* ntx_last_error(void);
 int ntx_version(void);
 
 /* Bytes of one packed row of `cols` elements; 0 if qtype is unknown or cols is
- * not a positive multiple of the format's block size (32 or 256; for a tiled
- * qtype, of the tile size).  Tiled and GGUF-style rows have the same length. */
+ * not a positive multiple of the format's block size (32 or 256).  Tiled and
+ * GGUF-style rows have the same length. */
 size_t ntx_row_bytes(int qtype, int64_t cols);
 
 /* Elements per block of qtype (32 or 256), 0 if unknown. */
@@ -115,16 +121,18 @@ ntx_status ntx_device_error(uint32_t* code);
  *   W    device, packed [rows, cols] in `qtype`; 16-byte aligned
  *   x    device fp32 [cols];  y  device fp32 [rows] (must not overlap x or W)
  * Accumulation is fp32; results match the exact dot product to a normwise
- * relative error far below 2e-3.  rows >= 1; cols a multiple of the block size.
- * Rows whose byte length is a multiple of 16 take the bulk-copy pipeline; other
- * shapes take a simpler kernel. */
+ * relative error far below 2e-3.  rows >= 1 (a multiple of 16 for a tiled
+ * qtype); cols a multiple of the block size.  Tiled layouts run on the integer
+ * tensor cores (x taken as 24-bit fixed point relative to max |x|); GGUF-style
+ * rows whose byte length is a multiple of 16 take the bulk-copy CUDA-core
+ * pipeline; other shapes take a simpler kernel. */
 ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t cols, const float* x, float* y,
                       void* stream);
 
 /* Repack W [rows, cols] from the GGUF-style layout of `qtype` (NTX_Q8_0 ..
  * NTX_Q6_K) into the tiled layout qtype | NTX_TILED, device to device: W_tiled
  * receives rows * ntx_row_bytes(qtype, cols) bytes and must not overlap W.
- * cols must be a multiple of the tile size.  A pure byte permutation. */
+ * rows must be a multiple of 16.  A lossless reordering of the bits. */
 ntx_status ntx_repack_q(int qtype, const void* W, void* W_tiled, int64_t rows, int64_t cols, void* stream);
 
 /* Dequantize W [rows, cols] to fp32 out [rows, cols] (row-major).  The result

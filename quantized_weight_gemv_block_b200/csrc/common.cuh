@@ -67,12 +67,12 @@ struct QTraits {
 inline bool is_tiled(int qtype) { return (qtype & NTX_TILED) != 0; }
 inline int base_qtype(int qtype) { return qtype & ~NTX_TILED; }
 
-// Elements per tile of a tiled layout (8 blocks, one Q4_K superblock, 8 Q6_K superblocks).
+// Columns per unit of a tiled layout (one block, or one superblock).
 inline int tile_elems(int qtype)
 {
     switch (base_qtype(qtype)) {
-    case NTX_Q8_0: case NTX_Q4_0: case NTX_Q4_K: return 256;
-    case NTX_Q6_K: return 2048;
+    case NTX_Q8_0: case NTX_Q4_0: return 32;
+    case NTX_Q4_K: case NTX_Q6_K: return 256;
     default: return 0;
     }
 }

@@ -1,11 +1,13 @@
-// gemv.cu - host side of the quantized GEMV (launch shaping, C ABI), the simple
-// kernel for rows that are not 16-byte multiples, and the dequantization kernel.
+// gemv.cu - host side of the quantized GEMV (launch shaping, C ABI; the tiled
+// layouts go to the tensor-core kernel of qmma.cu), the simple kernel for rows
+// that are not 16-byte multiples, and the dequantization kernel.
 #include <algorithm>
 #include <mutex>
 
 #include "blocks.cuh"
 #include "gemv_kernel.cuh"
 #include "launch.h"
+#include "ops.h"
 
 namespace ntx {
 namespace gemv {
@@ -16,7 +18,7 @@ __global__ void dequant_kernel(const uint8_t* W, int64_t rows, int64_t cols, int
     const int64_t total = rows * cols;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t r = i / cols, e = i % cols;
-        out[i] = weight_in_row<QT>(W + r * rb, e);
+        out[i] = weight_at<QT>(W, r, e, rb);
     }
 }
 
@@ -27,35 +29,10 @@ __global__ void gemv_simple_kernel(const uint8_t* W, int rows, int cols, int64_t
     const int warps = blockDim.x >> 5;
     const int lane = threadIdx.x & 31;
     for (int r = blockIdx.x * warps + (threadIdx.x >> 5); r < rows; r += gridDim.x * warps) {
-        const uint8_t* row = W + (int64_t)r * rb;
         float acc = 0.f;
-        for (int i = lane; i < cols; i += 32) acc = fmaf(weight_in_row<QT>(row, i), x[i], acc);
+        for (int i = lane; i < cols; i += 32) acc = fmaf(weight_at<QT>(W, r, i, rb), x[i], acc);
         acc = warp_sum(acc);
         if (lane == 0) y[r] = acc;
-    }
-}
-
-// GGUF-style -> tiled: out byte o of a tile comes from byte src(o) of the same
-// tile in the GGUF-style layout.
-template <int B>
-__device__ __forceinline__ int repack_src(int o)
-{
-    if (B == NTX_Q8_0) return o < 256 ? 34 * (o >> 5) + 2 + (o & 31) : 34 * ((o - 256) >> 1) + ((o - 256) & 1);
-    if (B == NTX_Q4_0) return o < 128 ? 18 * (o >> 4) + 2 + (o & 15) : 18 * ((o - 128) >> 1) + ((o - 128) & 1);
-    if (B == NTX_Q4_K) return o;
-    if (o < 1024) return 210 * (o >> 7) + (o & 127);
-    if (o < 1536) return 210 * ((o - 1024) >> 6) + 128 + ((o - 1024) & 63);
-    if (o < 1664) return 210 * ((o - 1536) >> 4) + 192 + ((o - 1536) & 15);
-    return 210 * ((o - 1664) >> 1) + 208 + ((o - 1664) & 1);
-}
-
-template <int B>
-__global__ void repack_kernel(const uint8_t* in, uint8_t* out, int64_t n_bytes, int tile_bytes)
-{
-    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_bytes; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t tile = i / tile_bytes;
-        const int o = (int)(i - tile * tile_bytes);
-        out[i] = in[tile * tile_bytes + repack_src<B>(o)];
     }
 }
 
@@ -92,14 +69,6 @@ ntx_status launch_t(Params P, cudaStream_t s, int grid_cap)
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     });
     P.m24 = 1u << 24;
-    P.m28 = 1u << 28;
-    P.m30 = 1u << 30;
-    P.m16 = 16u;
-    for (int i = 0; i < 3; ++i) {
-        P.kb[i] = 0xFFu << (8 * i);
-        P.ks[i] = 0x80u << (8 * i);
-    }
-    P.k0f = 0x0F0F0F0Fu;
     const int outs = Outs<QT, EPI>::value;
     int grid = std::min(grid_cap, (P.M + outs - 1) / outs);
     grid = std::max(grid, 1);
@@ -114,10 +83,6 @@ ntx_status launch_q(int qtype, const Params& P, cudaStream_t s, int grid_cap)
     case NTX_Q4_0: return launch_t<NTX_Q4_0, EPI, PRO>(P, s, grid_cap);
     case NTX_Q4_K: return launch_t<NTX_Q4_K, EPI, PRO>(P, s, grid_cap);
     case NTX_Q6_K: return launch_t<NTX_Q6_K, EPI, PRO>(P, s, grid_cap);
-    case NTX_Q8_0_T: return launch_t<NTX_Q8_0_T, EPI, PRO>(P, s, grid_cap);
-    case NTX_Q4_0_T: return launch_t<NTX_Q4_0_T, EPI, PRO>(P, s, grid_cap);
-    case NTX_Q4_K_T: return launch_t<NTX_Q4_K, EPI, PRO>(P, s, grid_cap);
-    case NTX_Q6_K_T: return launch_t<NTX_Q6_K_T, EPI, PRO>(P, s, grid_cap);
     default: return fail(NTX_EINVAL, "unknown qtype");
     }
 }
@@ -127,6 +92,7 @@ ntx_status launch_q(int qtype, const Params& P, cudaStream_t s, int grid_cap)
 ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s)
 {
     using namespace gemv;
+    if (is_tiled(qtype)) return qmma_launch(qtype, epi, pro, P, s);
     const int cap = num_sms();
     if (epi == EPI_STORE && pro == PRO_X) return launch_q<EPI_STORE, PRO_X>(qtype, P, s, cap);
     if (epi == EPI_ADD && pro == PRO_X) return launch_q<EPI_ADD, PRO_X>(qtype, P, s, cap);
@@ -140,7 +106,8 @@ cudaError_t take_device_error_gemv(uint32_t* out) { return take_tu_device_error(
 
 bool gemv_fast_path_ok(int qtype, const void* W, int64_t cols)
 {
-    return aligned(W, 16) && row_bytes(qtype, cols) % 16 == 0;
+    // the tiled layouts need only a 16-byte aligned base (their 16-row groups are 16-byte multiples)
+    return aligned(W, 16) && (is_tiled(qtype) || row_bytes(qtype, cols) % 16 == 0);
 }
 
 }  // namespace ntx
@@ -153,6 +120,7 @@ NTX_EXPORT ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t
     if (qtraits(qtype).block_elems == 0) return fail(NTX_EINVAL, "ntx_gemv_q: unknown qtype");
     if (!W || !x || !y) return fail(NTX_EINVAL, "ntx_gemv_q: null pointer");
     if (rows < 1 || rows > (1 << 30)) return fail(NTX_EINVAL, "ntx_gemv_q: rows out of range");
+    if (is_tiled(qtype) && rows % 16) return fail(NTX_EINVAL, "ntx_gemv_q: tiled layouts need a multiple of 16 rows");
     if (row_bytes(qtype, cols) == 0 || cols > (1 << 28))
         return fail(NTX_EINVAL, "ntx_gemv_q: cols must be a positive multiple of the block size");
     if (!aligned(x, 4) || !aligned(y, 4)) return fail(NTX_EINVAL, "ntx_gemv_q: x / y must be 4-byte aligned");
@@ -175,10 +143,11 @@ NTX_EXPORT ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t
     switch (qtype) {
     case NTX_Q8_0: NTX_SIMPLE(NTX_Q8_0); break;
     case NTX_Q4_0: NTX_SIMPLE(NTX_Q4_0); break;
-    case NTX_Q4_K: case NTX_Q4_K_T: NTX_SIMPLE(NTX_Q4_K); break;
+    case NTX_Q4_K: NTX_SIMPLE(NTX_Q4_K); break;
     case NTX_Q6_K: NTX_SIMPLE(NTX_Q6_K); break;
     case NTX_Q8_0_T: NTX_SIMPLE(NTX_Q8_0_T); break;
     case NTX_Q4_0_T: NTX_SIMPLE(NTX_Q4_0_T); break;
+    case NTX_Q4_K_T: NTX_SIMPLE(NTX_Q4_K_T); break;
     case NTX_Q6_K_T: NTX_SIMPLE(NTX_Q6_K_T); break;
     }
 #undef NTX_SIMPLE
@@ -190,6 +159,7 @@ NTX_EXPORT ntx_status ntx_dequant_q(int qtype, const void* W, int64_t rows, int6
     if (qtraits(qtype).block_elems == 0) return fail(NTX_EINVAL, "ntx_dequant_q: unknown qtype");
     if (!W || !out) return fail(NTX_EINVAL, "ntx_dequant_q: null pointer");
     if (rows < 1 || row_bytes(qtype, cols) == 0) return fail(NTX_EINVAL, "ntx_dequant_q: bad shape");
+    if (is_tiled(qtype) && rows % 16) return fail(NTX_EINVAL, "ntx_dequant_q: tiled layouts need a multiple of 16 rows");
     if (!aligned(out, 4)) return fail(NTX_EINVAL, "ntx_dequant_q: out must be 4-byte aligned");
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t rb = row_bytes(qtype, cols);
@@ -200,10 +170,11 @@ NTX_EXPORT ntx_status ntx_dequant_q(int qtype, const void* W, int64_t rows, int6
     switch (qtype) {
     case NTX_Q8_0: NTX_DQ(NTX_Q8_0); break;
     case NTX_Q4_0: NTX_DQ(NTX_Q4_0); break;
-    case NTX_Q4_K: case NTX_Q4_K_T: NTX_DQ(NTX_Q4_K); break;
+    case NTX_Q4_K: NTX_DQ(NTX_Q4_K); break;
     case NTX_Q6_K: NTX_DQ(NTX_Q6_K); break;
     case NTX_Q8_0_T: NTX_DQ(NTX_Q8_0_T); break;
     case NTX_Q4_0_T: NTX_DQ(NTX_Q4_0_T); break;
+    case NTX_Q4_K_T: NTX_DQ(NTX_Q4_K_T); break;
     case NTX_Q6_K_T: NTX_DQ(NTX_Q6_K_T); break;
     }
 #undef NTX_DQ
@@ -216,20 +187,10 @@ NTX_EXPORT ntx_status ntx_repack_q(int qtype, const void* W, void* W_tiled, int6
     if (!W || !W_tiled) return fail(NTX_EINVAL, "ntx_repack_q: null pointer");
     if (rows < 1 || row_bytes(qtype | NTX_TILED, cols) == 0)
         return fail(NTX_EINVAL, "ntx_repack_q: cols must be a positive multiple of the tile size");
+    if (rows % 16) return fail(NTX_EINVAL, "ntx_repack_q: tiled layouts need a multiple of 16 rows");
     const int64_t n = rows * row_bytes(qtype, cols);
     const char* a = (const char*)W;
     const char* b = (const char*)W_tiled;
     if (a < b + n && b < a + n) return fail(NTX_EINVAL, "ntx_repack_q: W and W_tiled overlap");
-    cudaStream_t s = (cudaStream_t)stream;
-    const int threads = 256;
-    const int grid = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)num_sms() * 32);
-    const uint8_t* in = (const uint8_t*)W;
-    uint8_t* out = (uint8_t*)W_tiled;
-    switch (qtype) {
-    case NTX_Q8_0: gemv::repack_kernel<NTX_Q8_0><<<grid, threads, 0, s>>>(in, out, n, 272); break;
-    case NTX_Q4_0: gemv::repack_kernel<NTX_Q4_0><<<grid, threads, 0, s>>>(in, out, n, 144); break;
-    case NTX_Q4_K: gemv::repack_kernel<NTX_Q4_K><<<grid, threads, 0, s>>>(in, out, n, 144); break;
-    case NTX_Q6_K: gemv::repack_kernel<NTX_Q6_K><<<grid, threads, 0, s>>>(in, out, n, 1680); break;
-    }
-    return check_launch("ntx_repack_q");
+    return repack_launch(qtype, W, W_tiled, rows, cols, (cudaStream_t)stream);
 }

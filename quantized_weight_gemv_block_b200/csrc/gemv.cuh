@@ -1,4 +1,5 @@
-// gemv.cuh - block-quantized GEMV for sm_100a (batch 1), with optional fused
+// gemv.cuh - block-quantized GEMV for sm_100a (batch 1) on the GGUF-style
+// layouts (the tiled layouts run on the tensor cores, qmma.cuh), with optional fused
 // prologue (RMSNorm of the input) and epilogues (residual add, SwiGLU of a
 // gate/up row pair, RoPE + fp16 KV-cache append for a fused QKV projection).
 //
@@ -70,12 +71,9 @@ struct Params {
     int stage_bytes;
     int x_bytes;
     int use_pdl;
-    // multipliers that let shifts run as integer multiplies on the FMA pipe
-    // (v >> 8 == umulhi(v, 2^24) etc.); passed in so they stay multiplies
-    uint32_t m24, m28, m30, m16;
-    // logic constants passed in registers, so a mask-and-flip or mask-and-merge is
-    // one three-input logic op: kb[i] = 0xFF << 8i, ks[i] = 0x80 << 8i, k0f = 0x0F0F0F0F
-    uint32_t kb[3], ks[3], k0f;
+    // multiplier that lets a shift run as an integer multiply on the FMA pipe
+    // (v >> 8 == umulhi(v, 2^24)); passed in so it stays a multiply
+    uint32_t m24;
 };
 
 template <int QT>
@@ -108,14 +106,6 @@ template <>
 struct Fmt<NTX_Q6_K> {
     static constexpr int E = 32, BE = 256, BB = 210;
 };
-template <>
-struct Fmt<NTX_Q8_0_T> : Fmt<NTX_Q8_0> {};
-template <>
-struct Fmt<NTX_Q4_0_T> : Fmt<NTX_Q4_0> {};
-template <>
-struct Fmt<NTX_Q4_K_T> : Fmt<NTX_Q4_K> {};
-template <>
-struct Fmt<NTX_Q6_K_T> : Fmt<NTX_Q6_K> {};
 
 // ------------------------------------------------------------------ element maps
 // chunk-local element index and code-field bit position of value (piece j, lane k)
@@ -357,170 +347,19 @@ struct Dot<NTX_Q6_K> {
 };
 
 
-// ------------------------------------------------------------------ tiled layouts
-// Same element ownership as the GGUF-style kernels; code runs are 8- or 16-byte
-// aligned, so each is one shared-memory load, and the right shifts run as
-// umulhi on the FMA pipe (the logic pipe is the scarce one).
-
-// Per-thread byte offsets inside a row chunk (constant for the whole kernel).
-template <int QT>
-struct TOff {
-    __device__ __forceinline__ explicit TOff(int) {}
-};
-
-template <>
-struct TOff<NTX_Q8_0_T> {
-    int code, d;
-    __device__ __forceinline__ explicit TOff(int t)
-    {
-        const int tile = 272 * (t >> 4), hb = t & 15;             // 16 threads per tile, half a block each
-        code = tile + 16 * hb;
-        d = tile + 256 + 2 * (hb >> 1);
-    }
-};
-
-template <>
-struct TOff<NTX_Q4_0_T> {
-    int code, d;
-    __device__ __forceinline__ explicit TOff(int t)
-    {
-        const int b = t >> 1, tile = 144 * (b >> 3);
-        code = tile + 16 * (b & 7) + 8 * (t & 1);
-        d = tile + 128 + 2 * (b & 7);
-    }
-};
-
-template <>
-struct TOff<NTX_Q6_K_T> {
-    int qa, qh, sc, d;
-    uint32_t sel0, sel1;      // byte selectors of this thread's two scales in each scale word
-    __device__ __forceinline__ explicit TOff(int t)
-    {
-        const int sb = t >> 3, s = sb & 7, hh = (t & 7) >> 2, u = t & 3;
-        const int tile = 1680 * (sb >> 3);
-        qa = tile + 128 * s + 64 * hh + 8 * u;
-        qh = tile + 1024 + 64 * s + 32 * hh + 8 * u;
-        sc = tile + 1536 + 16 * s + 8 * hh;
-        d = tile + 1664 + 2 * s;
-        // scale of group qq is byte 2 qq + (u >> 1) of the 8 scale bytes; build 0x4B0000bb
-        const uint32_t k = (uint32_t)(u >> 1);
-        sel0 = 0x7540u | k;
-        sel1 = 0x7540u | (k + 2);
-    }
-};
-
-template <>
-struct Dot<NTX_Q8_0_T> {
-    static __device__ __forceinline__ float row(const uint8_t* row, const TOff<NTX_Q8_0_T>& o,
-                                                const uint64_t (&x)[8], float off, const Params& P)
-    {
-        const uint4 c = *reinterpret_cast<const uint4*>(row + o.code);
-        const float d = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(row + o.d));
-        const uint32_t w[4] = {c.x, c.y, c.z, c.w};
-        uint64_t a = 0, b = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const uint32_t v = w[j], v8 = __umulhi(v, P.m24);
-            // code byte ^ 0x80 = code + 128, masked in place: value (code + 128) * 2^(p - 149)
-            fma2(a, pack2((v & P.kb[0]) ^ P.ks[0], (v & P.kb[1]) ^ P.ks[1]), x[2 * j]);
-            fma2(b, pack2((v & P.kb[2]) ^ P.ks[2], (v8 & P.kb[2]) ^ P.ks[2]), x[2 * j + 1]);
-        }
-        const f2 s2 = f2_from(add2(a, b));
-        return d * ((s2.x + s2.y) - off);
-    }
-};
-
-template <>
-struct Dot<NTX_Q4_0_T> {
-    static __device__ __forceinline__ float row(const uint8_t* row, const TOff<NTX_Q4_0_T>& o,
-                                                const uint64_t (&x)[8], float off, uint32_t m24)
-    {
-        const uint2 c = *reinterpret_cast<const uint2*>(row + o.code);
-        const float d = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(row + o.d));
-        uint64_t a0 = 0, a1 = 0;
-        const uint32_t w2[2] = {c.x, c.y};
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            const uint32_t v = w2[w], v8 = __umulhi(v, m24);
-            fma2(a0, pack2(v & 0xFu, v & 0xF00u), x[2 * w]);
-            fma2(a1, pack2(v & 0xF0000u, v8 & 0xF0000u), x[2 * w + 1]);
-            fma2(a0, pack2(v & 0xF0u, v & 0xF000u), x[4 + 2 * w]);
-            fma2(a1, pack2(v & 0xF00000u, v8 & 0xF00000u), x[4 + 2 * w + 1]);
-        }
-        const f2 s2 = f2_from(add2(a0, a1));
-        return d * ((s2.x + s2.y) - off);
-    }
-};
-
-template <>
-struct Dot<NTX_Q6_K_T> {
-    static __device__ __forceinline__ float row(const uint8_t* row, const TOff<NTX_Q6_K_T>& o,
-                                                const uint64_t (&x)[16], const float (&off)[4], const Params& P)
-    {
-        const uint32_t m24 = P.m24, m28 = P.m28, m30 = P.m30, m16 = P.m16, M = P.k0f;
-        const uint2 qa = *reinterpret_cast<const uint2*>(row + o.qa);
-        const uint2 qb = *reinterpret_cast<const uint2*>(row + o.qa + 32);
-        const uint2 qh = *reinterpret_cast<const uint2*>(row + o.qh);
-        const uint2 sc = *reinterpret_cast<const uint2*>(row + o.sc);
-        const float d = f16_bits_to_f32(*reinterpret_cast<const uint16_t*>(row + o.d));
-        // int8 scale s -> fp32 without a conversion unit: the byte s ^ 0x80 = s + 128 in the
-        // mantissa of 2^23 gives 2^23 + 128 + s exactly
-        const uint32_t sx = sc.x ^ 0x80808080u, sy = sc.y ^ 0x80808080u;
-        const float C = 8388736.0f;   // 2^23 + 128
-        float ds[4];
-        ds[0] = d * (__uint_as_float(__byte_perm(sx, 0x4B000000u, o.sel0)) - C);
-        ds[1] = d * (__uint_as_float(__byte_perm(sx, 0x4B000000u, o.sel1)) - C);
-        ds[2] = d * (__uint_as_float(__byte_perm(sy, 0x4B000000u, o.sel0)) - C);
-        ds[3] = d * (__uint_as_float(__byte_perm(sy, 0x4B000000u, o.sel1)) - C);
-        uint64_t acc[4] = {0, 0, 0, 0};
-        const uint32_t qaw[2] = {qa.x, qa.y}, qbw[2] = {qb.x, qb.y}, qhw[2] = {qh.x, qh.y};
-#pragma unroll
-        for (int w = 0; w < 2; ++w) {
-            const uint32_t hA = qhw[w] & 0x33333333u;                    // high bits of qq 0 and 2
-            const uint32_t hB = __umulhi(qhw[w], m30) & 0x33333333u;     // of qq 1 and 3
-            uint32_t code[4];
-            // (a & M) | (b & ~M): one three-input logic op with M in a register
-            code[0] = (qaw[w] & M) | ((hA * m16) & ~M);
-            code[1] = (qbw[w] & M) | ((hB * m16) & ~M);
-            code[2] = (__umulhi(qaw[w], m28) & M) | (hA & ~M);
-            code[3] = (__umulhi(qbw[w], m28) & M) | (hB & ~M);
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-                const uint32_t v = code[qq], v8 = __umulhi(v, m24);
-                fma2(acc[qq], pack2(v & 0xFFu, v & 0xFF00u), x[2 * (2 * qq + w)]);
-                fma2(acc[qq], pack2(v & 0xFF0000u, v8 & 0xFF0000u), x[2 * (2 * qq + w) + 1]);
-            }
-        }
-        float res = 0.f;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-            const f2 a = f2_from(acc[qq]);
-            res = fmaf(ds[qq], (a.x + a.y) - off[qq], res);
-        }
-        return res;
-    }
-};
-
 // One row of one stage for this thread, in units of 2^(S-149).
 template <int QT>
-__device__ __forceinline__ float dot_row(const uint8_t* row, const TOff<QT>& o, int lt,
-                                         const uint64_t (&xr)[2 * (Fmt<QT>::E / 4)], const float (&offs)[4],
-                                         const Params& P)
+__device__ __forceinline__ float dot_row(const uint8_t* row, int lt, const uint64_t (&xr)[2 * (Fmt<QT>::E / 4)],
+                                         const float (&offs)[4], const Params& P)
 {
     if constexpr (QT == NTX_Q8_0) {
         return Dot<NTX_Q8_0>::row(row, lt, xr, offs[0]);
     } else if constexpr (QT == NTX_Q4_0) {
         return Dot<NTX_Q4_0>::row(row, lt, xr, offs[0]);
-    } else if constexpr ((QT & 3) == NTX_Q4_K) {
+    } else if constexpr (QT == NTX_Q4_K) {
         return Dot<NTX_Q4_K>::row(row, lt, xr, offs[0], offs[1], P.m24);
-    } else if constexpr (QT == NTX_Q6_K) {
-        return Dot<NTX_Q6_K>::row(row, lt, xr, offs);
-    } else if constexpr (QT == NTX_Q8_0_T) {
-        return Dot<NTX_Q8_0_T>::row(row, o, xr, offs[0], P);
-    } else if constexpr (QT == NTX_Q4_0_T) {
-        return Dot<NTX_Q4_0_T>::row(row, o, xr, offs[0], P.m24);
     } else {
-        return Dot<NTX_Q6_K_T>::row(row, o, xr, offs, P);
+        return Dot<NTX_Q6_K>::row(row, lt, xr, offs);
     }
 }
 

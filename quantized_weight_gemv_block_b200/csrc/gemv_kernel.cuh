@@ -222,13 +222,13 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params P)
 #pragma unroll
             for (int j = 0; j < NP; ++j) {
                 int e, p;
-                elem_of<(QT & 3)>(lt, j, 0, e, p);
+                elem_of<QT>(lt, j, 0, e, p);
                 const float4 v = *reinterpret_cast<const float4*>(base + e);
                 const float vv[4] = {v.x, v.y, v.z, v.w};
                 float o[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    elem_of<(QT & 3)>(lt, j, k, e, p);
+                    elem_of<QT>(lt, j, k, e, p);
                     o[k] = scale2(vv[k], S - p);
                 }
                 piece[j] = make_float4(o[0], o[1], o[2], o[3]);
@@ -268,9 +268,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params P)
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
                 int e, p;
-                elem_of<(QT & 3)>(lt, j, k, e, p);
+                elem_of<QT>(lt, j, k, e, p);
                 // offset code at bit p as an fp32 bit pattern (value code * 2^(p-149))
-                constexpr int B = QT & 3;
+                constexpr int B = QT;
                 const uint32_t code = B == NTX_Q8_0 ? 128u : B == NTX_Q4_0 ? 8u : B == NTX_Q6_K ? 32u : 1u;
                 const float unit = __uint_as_float(code << p);
                 const int og = B == NTX_Q4_K ? (j >> 2) : B == NTX_Q6_K ? (j >> 1) : 0;
@@ -282,7 +282,6 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params P)
     const int CB = P.chunk_bytes, SB = P.stage_bytes;
     const bool one_chunk = NCH == 1;
     if (one_chunk && lt < K / E) load_x(0, K / E);
-    const TOff<QT> toff(lt);
     const uint8_t* my_stage0 = stages + (size_t)(grp * R) * CB;
     int s = 0;
     uint32_t ph = 0;
@@ -306,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params P)
                 // rows past the end of a partial group hold stale bytes; their sums are never stored
 #pragma unroll
                 for (int r = 0; r < R; ++r)
-                    acc[r] += dot_row<QT>(b + (size_t)r * CB, toff, lt, xr, offs, P);
+                    acc[r] += dot_row<QT>(b + (size_t)r * CB, lt, xr, offs, P);
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);

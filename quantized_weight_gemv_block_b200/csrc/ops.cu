@@ -133,9 +133,8 @@ __global__ void embed_kernel(const uint8_t* E, int64_t rb, int64_t hidden, const
         pdl_wait();
     }
     const int32_t token = *token_dev;
-    const uint8_t* row = E + (int64_t)token * rb;
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < hidden; i += (int64_t)gridDim.x * blockDim.x)
-        h[i] = gemv::weight_in_row<QT>(row, i);
+        h[i] = gemv::weight_at<QT>(E, token, i, rb);
 }
 
 __global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos)
@@ -171,7 +170,7 @@ ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t*
     case NTX_Q6_K: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q6_K>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q8_0_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q8_0_T>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q4_0_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q4_0_T>, e, rb, hidden, token_dev, h, p); break;
-    case NTX_Q4_K_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q4_K>, e, rb, hidden, token_dev, h, p); break;
+    case NTX_Q4_K_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q4_K_T>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q6_K_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q6_K_T>, e, rb, hidden, token_dev, h, p); break;
     }
     if (err != cudaSuccess) return fail(NTX_ECUDA, std::string("embedding launch: ") + cudaGetErrorString(err));

@@ -10,6 +10,8 @@ ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t*
                         bool pdl);
 ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, cudaStream_t s);
 ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
+ntx_status qmma_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
+ntx_status repack_launch(int qtype, const void* W, void* W_tiled, int64_t rows, int64_t cols, cudaStream_t s);
 bool gemv_fast_path_ok(int qtype, const void* W, int64_t cols);
 
 // Split-KV decode attention (attn.cu).

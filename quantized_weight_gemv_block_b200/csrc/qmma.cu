@@ -1,0 +1,207 @@
+// qmma.cu - host side of the tensor-core GEMV for the tiled layouts (launch
+// shaping) and the repack kernel GGUF-style -> tiled.
+#include <algorithm>
+#include <mutex>
+
+#include "launch.h"
+#include "qmma.cuh"
+
+namespace ntx {
+namespace qmma {
+
+// ------------------------------------------------------------------ repack
+// Readers of the GGUF-style source row (the codes as the formats store them).
+
+__device__ __forceinline__ int src_q4_0(const uint8_t* row, int64_t e)
+{
+    const uint8_t* blk = row + (e >> 5) * 18 + 2;
+    const int i = (int)(e & 31);
+    return i < 16 ? (blk[i] & 15) : (blk[i - 16] >> 4);
+}
+
+__device__ __forceinline__ int src_q6_k(const uint8_t* row, int64_t e)
+{
+    const uint8_t* b = row + (e >> 8) * 210;
+    const int r256 = (int)(e & 255), h = r256 >> 7, t = r256 & 127;
+    const int lo = t < 64 ? (b[64 * h + t] & 15) : (b[64 * h + t - 64] >> 4);
+    const int hi = (b[128 + 32 * h + (t & 31)] >> (2 * (t >> 5))) & 3;
+    return lo | (hi << 4);
+}
+
+__device__ __forceinline__ int src_q4_k(const uint8_t* row, int64_t e)
+{
+    const uint8_t* b = row + (e >> 8) * 144;
+    const int r256 = (int)(e & 255), c = r256 >> 6, r = r256 & 63;
+    const int byte = b[16 + 32 * c + (r & 31)];
+    return r < 32 ? (byte & 15) : (byte >> 4);
+}
+
+// Q4_K 6-bit value V(m, b) of the tiled layout for rows (gid, gid + 8) of group W16.
+__device__ __forceinline__ int src_q4_k_v(const uint8_t* W16, int64_t rb, int64_t sb, int gid, int m, int b)
+{
+    const uint8_t* blk = W16 + (int64_t)(gid + 8 * (b & 1)) * rb + sb * 144;
+    int sc, mn;
+    gemv::q4k_sm(blk + 4, m, sc, mn);
+    return (b & 2) ? mn : sc;
+}
+
+// Byte `o` of unit u of the 16-row group that starts at GGUF row pointer W16.
+template <int QT>
+__device__ __forceinline__ uint8_t tiled_byte(const uint8_t* W16, int64_t rb, int64_t u, int o)
+{
+    if constexpr (QT == NTX_Q8_0_T) {
+        if (o < 512) {
+            const int lane = o >> 4, reg = (o >> 2) & 3, j = o & 3;
+            const int row = (lane >> 2) + 8 * (reg & 1);
+            const int col = 16 * (reg >> 1) + 4 * (lane & 3) + j;
+            return W16[row * rb + u * 34 + 2 + col];
+        }
+        const int p = o - 512, row = (p >> 2) + 8 * ((p >> 1) & 1);
+        return W16[row * rb + u * 34 + (p & 1)];
+    } else if constexpr (QT == NTX_Q4_0_T) {
+        if (o < 256) {
+            const int lane = o >> 3, hi = (o >> 2) & 1, j = o & 3;
+            const uint8_t* row = W16 + (int64_t)((lane >> 2) + 8 * hi) * rb;
+            const int64_t e = 32 * u + 4 * (lane & 3) + j;
+            return (uint8_t)(src_q4_0(row, e) | (src_q4_0(row, e + 16) << 4));
+        }
+        const int p = o - 256, row = (p >> 2) + 8 * ((p >> 1) & 1);
+        return W16[row * rb + u * 18 + (p & 1)];
+    } else if constexpr (QT == NTX_Q6_K_T) {
+        if (o < 3072) {
+            const int m = o / 384, r = o % 384, lane = r / 12, wi = (r % 12) >> 2, j = r & 3;
+            const int gid = lane >> 2, tig = lane & 3;
+            const int64_t e0 = 256 * u + 32 * m + 4 * tig + j;
+            // A: row gid col c; B: row gid+8 col c; C: row gid col c+16; a3: row gid+8 col c+16
+            const uint8_t* rowA = W16 + (int64_t)(gid + (wi == 1 ? 8 : 0)) * rb;
+            const int q = src_q6_k(rowA, e0 + (wi == 2 ? 16 : 0));
+            const int q3 = src_q6_k(W16 + (int64_t)(gid + 8) * rb, e0 + 16);
+            return (uint8_t)(q | (((q3 >> (2 * wi)) & 3) << 6));
+        }
+        if (o < 3328) {
+            const int p = o - 3072, vec = p >> 4, bi = p & 15;
+            const int gid = vec >> 1, par = vec & 1, hi = bi >> 3, mm = bi & 7;
+            return W16[(int64_t)(gid + 8 * hi) * rb + u * 210 + 192 + 2 * mm + par];
+        }
+        const int p = o - 3328, row = (p >> 2) + 8 * ((p >> 1) & 1);
+        return W16[row * rb + u * 210 + 208 + (p & 1)];
+    } else {
+        if (o < 2048) {
+            const int m = o >> 8, r = o & 255, lane = r >> 3, hi = (r >> 2) & 1, j = r & 3;
+            const uint8_t* row = W16 + (int64_t)((lane >> 2) + 8 * hi) * rb;
+            const int64_t e = 256 * u + 32 * m + 4 * (lane & 3) + j;
+            return (uint8_t)(src_q4_k(row, e) | (src_q4_k(row, e + 16) << 4));
+        }
+        if (o < 2240) {
+            const int p = o - 2048, gid = p / 24, r = p % 24;
+            if (r < 16) {
+                const int wn = r >> 2, b = r & 3;
+                return (uint8_t)((src_q4_k_v(W16, rb, u, gid, 2 * wn, b) & 15) |
+                                 ((src_q4_k_v(W16, rb, u, gid, 2 * wn + 1, b) & 15) << 4));
+            }
+            const int wh = (r - 16) >> 2, b = r & 3;
+            int v = 0;
+            for (int t = 0; t < 4; ++t) v |= ((src_q4_k_v(W16, rb, u, gid, 4 * wh + t, b) >> 4) & 3) << (2 * t);
+            return (uint8_t)v;
+        }
+        const int p = o - 2240, gid = p >> 3, k = (p >> 1) & 3;
+        // k: 0 d(gid), 1 d(gid+8), 2 dmin(gid), 3 dmin(gid+8)
+        const int row = gid + 8 * (k & 1);
+        return W16[(int64_t)row * rb + u * 144 + 2 * (k >> 1) + (p & 1)];
+    }
+}
+
+template <int QT>
+__global__ void repack_kernel(const uint8_t* in, uint8_t* out, int64_t n_bytes, int64_t rb)
+{
+    using T = gemv::Tiled<QT>;
+    const int64_t gb = 16 * rb;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_bytes; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t grp = i / gb, o = i - grp * gb;
+        const int64_t u = o / T::UB;
+        out[i] = tiled_byte<QT>(in + grp * gb, rb, u, (int)(o - u * T::UB));
+    }
+}
+
+// ------------------------------------------------------------------ launch shaping
+
+template <int QT>
+bool shape(Params& P)
+{
+    using T = gemv::Tiled<QT>;
+    P.x_bytes = P.K * 4;   // 32 words per 32-column step
+    const int avail = kSmemLimit - kHeader - P.x_bytes - 128;
+    // chunks of up to 2048 columns (whole units), shrunk until at least 3 stages fit
+    int ce = std::min(P.K, 2048) / T::UK * T::UK;
+    while (ce > T::UK && avail / (ce / T::UK * T::UB) < 3) ce = std::max(T::UK, ce / 2 / T::UK * T::UK);
+    if (ce < T::UK) return false;
+    P.chunk_elems = ce;
+    P.n_chunks = (P.K + ce - 1) / ce;
+    P.chunk_bytes = ce / T::UK * T::UB;
+    P.stage_bytes = P.chunk_bytes;
+    const int ns = std::min(kMaxStages, avail / P.stage_bytes);
+    if (ns < 2) return false;
+    P.n_stages = ns;
+    return true;
+}
+
+template <int QT, int EPI, int PRO>
+ntx_status launch_t(Params P, cudaStream_t s, int grid_cap)
+{
+    if (!shape<QT>(P)) return fail(NTX_EUNSUPPORTED, "gemv: row too long for the shared-memory pipeline");
+    auto kern = qmma_kernel<QT, EPI, PRO>;
+    const int smem = kHeader + P.x_bytes + P.n_stages * P.stage_bytes + 128;
+    static std::once_flag once[4][4][2];
+    std::call_once(once[QT & 3][EPI][PRO], [&] {
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
+    });
+    const int grid = std::max(1, std::min(grid_cap, P.M / 16));
+    return launch_kernel(kern, dim3(grid), dim3(kThreads), smem, s, P.use_pdl != 0, P);
+}
+
+template <int EPI, int PRO>
+ntx_status launch_q(int qtype, const Params& P, cudaStream_t s, int grid_cap)
+{
+    switch (qtype) {
+    case NTX_Q8_0_T: return launch_t<NTX_Q8_0_T, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q4_0_T: return launch_t<NTX_Q4_0_T, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q4_K_T: return launch_t<NTX_Q4_K_T, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q6_K_T: return launch_t<NTX_Q6_K_T, EPI, PRO>(P, s, grid_cap);
+    default: return fail(NTX_EINVAL, "unknown tiled qtype");
+    }
+}
+
+}  // namespace qmma
+
+ntx_status qmma_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s)
+{
+    using namespace gemv;
+    if (P.M % 16) return fail(NTX_EINVAL, "gemv: tiled layouts need a multiple of 16 rows");
+    const int cap = num_sms();
+    if (epi == EPI_STORE && pro == PRO_X) return qmma::launch_q<EPI_STORE, PRO_X>(qtype, P, s, cap);
+    if (epi == EPI_ADD && pro == PRO_X) return qmma::launch_q<EPI_ADD, PRO_X>(qtype, P, s, cap);
+    if (epi == EPI_SWIGLU && pro == PRO_RMSNORM) return qmma::launch_q<EPI_SWIGLU, PRO_RMSNORM>(qtype, P, s, cap);
+    if (epi == EPI_QKV && pro == PRO_RMSNORM) return qmma::launch_q<EPI_QKV, PRO_RMSNORM>(qtype, P, s, cap);
+    if (epi == EPI_STORE && pro == PRO_RMSNORM) return qmma::launch_q<EPI_STORE, PRO_RMSNORM>(qtype, P, s, cap);
+    return fail(NTX_EUNSUPPORTED, "gemv: unsupported prologue / epilogue combination");
+}
+
+ntx_status repack_launch(int qtype, const void* W, void* W_tiled, int64_t rows, int64_t cols, cudaStream_t s)
+{
+    const int64_t rb = row_bytes(qtype, cols);
+    const int64_t n = rows * rb;
+    const int threads = 256;
+    const int grid = (int)std::min<int64_t>((n + threads - 1) / threads, (int64_t)num_sms() * 32);
+    const uint8_t* in = (const uint8_t*)W;
+    uint8_t* out = (uint8_t*)W_tiled;
+    switch (qtype) {
+    case NTX_Q8_0: qmma::repack_kernel<NTX_Q8_0_T><<<grid, threads, 0, s>>>(in, out, n, rb); break;
+    case NTX_Q4_0: qmma::repack_kernel<NTX_Q4_0_T><<<grid, threads, 0, s>>>(in, out, n, rb); break;
+    case NTX_Q4_K: qmma::repack_kernel<NTX_Q4_K_T><<<grid, threads, 0, s>>>(in, out, n, rb); break;
+    case NTX_Q6_K: qmma::repack_kernel<NTX_Q6_K_T><<<grid, threads, 0, s>>>(in, out, n, rb); break;
+    default: return fail(NTX_EINVAL, "ntx_repack_q: qtype must be a GGUF-style format");
+    }
+    return check_launch("ntx_repack_q");
+}
+
+}  // namespace ntx

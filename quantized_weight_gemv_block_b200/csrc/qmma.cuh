@@ -1,0 +1,583 @@
+// qmma.cuh - block-quantized GEMV for the tiled layouts on the integer tensor
+// cores (batch 1).
+//
+// The GEMV kernel of the ntransformer news summary ("Arquitectura y estructura
+// del código": cuda/ holds the GEMV kernels) for B200.  Batch-1 GEMV streams every
+// weight once, so the work per weight must stay far below the SM's issue rate to
+// keep HBM busy.  Dequantizing each weight to fp32 and multiplying costs several
+// instructions per weight; here the packed codes go to the tensor cores as they are:
+//  * the input vector x is turned once per CTA into 24-bit fixed point,
+//    x_int = rint(x 2^S) with |x_int| < 2^22, written as three balanced signed
+//    8-bit limbs, x_int = l0 + 2^8 l1 + 2^16 l2 (S from max |x|, a power of two);
+//  * one m16n8k32 integer MMA takes a 16-row x 32-column block of codes (int8 for
+//    Q8_0, unsigned 4- or 6-bit codes for the others) as its A operand and the
+//    limbs of x as its B operand: the 8 columns of B hold limb l of x's 32 values
+//    (or, for Q6_K, of the 16 values of one 16-column sub-block each), so each C
+//    column is an exact integer partial dot product of one limb;
+//  * the format's per-block scale (fp16 d, int8 or 6-bit sub-block scales, the
+//    Q4_K mins, the code offsets 8 and 32) is applied to those integers, in
+//    integer arithmetic where it is exact, in fp32 once per block otherwise;
+//  * the limbs are recombined (weights 1, 2^8, 2^16) and the row total is scaled
+//    by 2^-S, exactly.
+// The products are exact; x carries 23 bits (relative to max |x|) where fp32
+// carries 24; sums round at fp32 once per block or superblock.
+//
+// Structure (one CTA per SM, 8 consumer warps + 1 producer warp):
+//  * the CTA owns a contiguous range of 16-row groups; a stage is one group x one
+//    chunk of KC columns, contiguous in the tiled layout, streamed by the producer
+//    warp with one 1-D bulk copy (cp.async.bulk, L2 evict-first) into a ring of
+//    shared-memory stages guarded by mbarriers;
+//  * each consumer warp takes every 8th unit (32 or 256 columns) of a stage; per
+//    32-column step a lane loads its two rows' codes with one shared-memory load,
+//    unpacks 4-/6-bit codes into bytes with a few logic ops, issues one MMA and
+//    folds the step's integers into its row accumulators;
+//  * row totals are reduced over the 4 lanes of a quad (limb weights) and over the
+//    warps through shared memory, then the fused epilogue runs (store, residual
+//    add, SwiGLU of a gate / up group pair, RoPE + fp16 KV-cache append).
+#pragma once
+
+#include "blocks.cuh"
+
+namespace ntx {
+namespace qmma {
+
+using gemv::Params;
+
+constexpr int kWarps = 8;                  // consumer warps
+constexpr int kCons = kWarps * 32;
+constexpr int kThreads = kCons + 32;       // + the producer warp
+constexpr int kMaxStages = 8;
+constexpr int kHeader = 3072;              // barriers, reduction scratch, RoPE table
+constexpr int kOffRed = 256;               // [2][kWarps][2 mats][16] floats
+constexpr int kOffRope = 2304;             // [64][cos, sin]
+constexpr int kSmemLimit = 227 * 1024;
+constexpr uint32_t kWaitPolls = 1u << 22;
+
+// ------------------------------------------------------------------ MMA helpers
+
+// C = A B for A 16 x 32 int8 (row), B 32 x 8 int8 (col), int32 accumulation from 0.
+__device__ __forceinline__ void mma_s8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
+
+// The same with A unsigned 8-bit.
+__device__ __forceinline__ void mma_u8(int (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=r"(c[0]), "=r"(c[1]), "=r"(c[2]), "=r"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
+
+// Byte k of w, sign-extended (prmt with the sign-replicate selector).
+template <int k>
+__device__ __forceinline__ int sbyte(uint32_t w)
+{
+    constexpr uint32_t sel = k | ((8 | k) << 4) | ((8 | k) << 8) | ((8 | k) << 12);
+    uint32_t r;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "n"(sel));
+    return (int)r;
+}
+
+// Byte k of w, zero-extended.
+template <int k>
+__device__ __forceinline__ int ubyte(uint32_t w)
+{
+    return (int)__byte_perm(w, 0u, 0x4440u | k);
+}
+
+// ------------------------------------------------------------------ x staging
+// Step u (columns 32u .. 32u + 31) of x occupies 32 words at xq + 32u:
+//  words 8l + w (l = 0..2, w = 0..7): limb l of columns 32u + 4w .. + 3, one byte each;
+//  words 24..31: per-column sums of the limbs over what one C column covers
+//    (Q6_K: words 24 + 4h + l = sum of limb l over the 16 columns of half h, words
+//    27 and 31 zero; other formats: word 24 + l = sum of limb l over the 32 columns,
+//    words 27..31 zero).  Lane tig reads its two C columns' sums at 24 + 2 tig.
+
+template <bool HALVES>
+__device__ __forceinline__ void stage_x_step(uint32_t* xs, int w, bool ok, float4 v, float two_s)
+{
+    // z = x_int + 0x8080: bytes 0 and 1 of z are the low limbs + 128, z >> 16 the top limb
+    const float mag = 12582912.0f;   // 1.5 * 2^23: fmaf rounds x 2^S to an integer in its low bits
+    const int bias = 0x8080 - 0x4B400000;
+    const int z0 = __float_as_int(fmaf(v.x, two_s, mag)) + bias;
+    const int z1 = __float_as_int(fmaf(v.y, two_s, mag)) + bias;
+    const int z2 = __float_as_int(fmaf(v.z, two_s, mag)) + bias;
+    const int z3 = __float_as_int(fmaf(v.w, two_s, mag)) + bias;
+    const uint32_t lo01 = __byte_perm(z0, z1, 0x5410), lo23 = __byte_perm(z2, z3, 0x5410);
+    const uint32_t w0 = __byte_perm(lo01, lo23, 0x6420) ^ 0x80808080u;
+    const uint32_t w1 = __byte_perm(lo01, lo23, 0x7531) ^ 0x80808080u;
+    const uint32_t w2 = __byte_perm(__byte_perm(z0, z1, 0x0062), __byte_perm(z2, z3, 0x0062), 0x5410);
+    // column sums of the four values (byte sums of the signed limbs)
+    int s0 = __dp4a((int)w0, 0x01010101, 0), s1 = __dp4a((int)w1, 0x01010101, 0), s2 = __dp4a((int)w2, 0x01010101, 0);
+#pragma unroll
+    for (int o = 1; o < (HALVES ? 4 : 8); o <<= 1) {
+        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
+        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
+        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+    }
+    __syncwarp();   // every lane of the step has read its floats before any limb word lands
+    if (ok) {
+        xs[w] = w0;
+        xs[8 + w] = w1;
+        xs[16 + w] = w2;
+        if (HALVES) {
+            if ((w & 3) == 0) {
+                const int h = w >> 2;
+                xs[24 + 4 * h] = (uint32_t)s0;
+                xs[25 + 4 * h] = (uint32_t)s1;
+                xs[26 + 4 * h] = (uint32_t)s2;
+                xs[27 + 4 * h] = 0u;
+            }
+        } else {
+            if (w == 0) {
+                xs[24] = (uint32_t)s0;
+                xs[25] = (uint32_t)s1;
+                xs[26] = (uint32_t)s2;
+            } else if (w == 1) {
+                xs[27] = 0u;
+                xs[28] = 0u;
+                xs[29] = 0u;
+                xs[30] = 0u;
+                xs[31] = 0u;
+            }
+        }
+    }
+}
+
+// ------------------------------------------------------------------ lane constants
+
+struct Lane {
+    int lane, gid, tig;
+    int boff;        // word of this lane's B value in a step
+    bool bval;       // lane's B column is a limb column (not a zero column)
+    bool b_hi;       // Q6_K: the column belongs to the second 16-column half (B word b1)
+};
+
+template <int QT>
+__device__ __forceinline__ Lane make_lane(int lane)
+{
+    Lane L;
+    L.lane = lane;
+    L.gid = lane >> 2;
+    L.tig = lane & 3;
+    if constexpr (QT == NTX_Q6_K_T) {
+        // column n = gid: half g = n / 4, limb l = n % 4 (limb 3 is a zero column)
+        const int g = L.gid >> 2, l = L.gid & 3;
+        L.boff = 8 * l + 4 * g + L.tig;
+        L.bval = l < 3;
+        L.b_hi = g == 1;
+    } else {
+        // column n = gid: limb n for n < 3, zero columns after
+        L.boff = 8 * L.gid + L.tig;
+        L.bval = L.gid < 3;
+        L.b_hi = false;
+    }
+    return L;
+}
+
+// B operand of one step: b0 covers columns 0-15 of the step, b1 columns 16-31.
+template <int QT>
+__device__ __forceinline__ void b_frag(const uint32_t* xs, const Lane& L, uint32_t& b0, uint32_t& b1)
+{
+    if constexpr (QT == NTX_Q6_K_T) {
+        const uint32_t w = L.bval ? xs[L.boff] : 0u;
+        b0 = L.b_hi ? 0u : w;
+        b1 = L.b_hi ? w : 0u;
+    } else {
+        b0 = L.bval ? xs[L.boff] : 0u;
+        b1 = L.bval ? xs[L.boff + 4] : 0u;
+    }
+}
+
+__device__ __forceinline__ float2 d_pair(const uint8_t* p)
+{
+    return __half22float2(*reinterpret_cast<const __half2*>(p));
+}
+
+// ------------------------------------------------------------------ units
+// acc0 / acc1: this lane's running fp32 sums for rows gid / gid + 8, in units of
+// its C columns' limb (the quad reduction applies the limb weights).
+
+template <int QT>
+struct Unit;
+
+template <>
+struct Unit<NTX_Q8_0_T> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
+                                               float& acc1)
+    {
+        const uint4 a4 = *reinterpret_cast<const uint4*>(U + 16 * L.lane);
+        const uint32_t a[4] = {a4.x, a4.y, a4.z, a4.w};
+        uint32_t b0, b1;
+        b_frag<NTX_Q8_0_T>(xs, L, b0, b1);
+        int c[4];
+        mma_s8(c, a, b0, b1);
+        const float2 d = d_pair(U + 512 + 4 * L.gid);
+        acc0 = fmaf((float)(c[0] + 256 * c[1]), d.x, acc0);
+        acc1 = fmaf((float)(c[2] + 256 * c[3]), d.y, acc1);
+    }
+};
+
+template <>
+struct Unit<NTX_Q4_0_T> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
+                                               float& acc1)
+    {
+        const uint2 pq = *reinterpret_cast<const uint2*>(U + 8 * L.lane);
+        const uint32_t M = 0x0F0F0F0Fu;
+        const uint32_t a[4] = {pq.x & M, pq.y & M, (pq.x >> 4) & M, (pq.y >> 4) & M};
+        uint32_t b0, b1;
+        b_frag<NTX_Q4_0_T>(xs, L, b0, b1);
+        int c[4];
+        mma_u8(c, a, b0, b1);
+        // codes carry +8: subtract 8 x (this lane's two columns' limb sums)
+        const int2 X = *reinterpret_cast<const int2*>(xs + 24 + 2 * L.tig);
+        const int off = -8 * (X.x + 256 * X.y);
+        const float2 d = d_pair(U + 256 + 4 * L.gid);
+        acc0 = fmaf((float)(c[0] + 256 * c[1] + off), d.x, acc0);
+        acc1 = fmaf((float)(c[2] + 256 * c[3] + off), d.y, acc1);
+    }
+};
+
+template <>
+struct Unit<NTX_Q6_K_T> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
+                                               float& acc1)
+    {
+        // this lane's scales: sub-blocks 2m + (tig / 2) of rows gid (bytes 0-7) and gid + 8 (8-15)
+        const uint4 sv = *reinterpret_cast<const uint4*>(U + 3072 + 16 * (2 * L.gid + (L.tig >> 1)));
+        // per row: s * (limb-0 column), s * (limb-1 column), s * (the columns' limb sums)
+        int p0 = 0, p1 = 0, q0 = 0, q1 = 0, o0 = 0, o1 = 0, r0 = 0, r1 = 0;
+        const uint32_t M6 = 0x3F3F3F3Fu;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const uint8_t* w = U + 384 * m + 12 * L.lane;
+            const uint32_t A = *reinterpret_cast<const uint32_t*>(w);
+            const uint32_t B = *reinterpret_cast<const uint32_t*>(w + 4);
+            const uint32_t C = *reinterpret_cast<const uint32_t*>(w + 8);
+            uint32_t a[4];
+            a[0] = A & M6;
+            a[1] = B & M6;
+            a[2] = C & M6;
+            a[3] = ((A >> 6) & 0x03030303u) | ((B >> 4) & 0x0C0C0C0Cu) | ((C >> 2) & 0x30303030u);
+            const uint32_t* x = xs + 32 * m;
+            uint32_t b0, b1;
+            b_frag<NTX_Q6_K_T>(x, L, b0, b1);
+            int c[4];
+            mma_u8(c, a, b0, b1);
+            const int2 X = *reinterpret_cast<const int2*>(x + 24 + 2 * L.tig);
+            int s0, s1;
+            if (m < 4) {
+                s0 = m == 0 ? sbyte<0>(sv.x) : m == 1 ? sbyte<1>(sv.x) : m == 2 ? sbyte<2>(sv.x) : sbyte<3>(sv.x);
+                s1 = m == 0 ? sbyte<0>(sv.z) : m == 1 ? sbyte<1>(sv.z) : m == 2 ? sbyte<2>(sv.z) : sbyte<3>(sv.z);
+            } else {
+                s0 = m == 4 ? sbyte<0>(sv.y) : m == 5 ? sbyte<1>(sv.y) : m == 6 ? sbyte<2>(sv.y) : sbyte<3>(sv.y);
+                s1 = m == 4 ? sbyte<0>(sv.w) : m == 5 ? sbyte<1>(sv.w) : m == 6 ? sbyte<2>(sv.w) : sbyte<3>(sv.w);
+            }
+            p0 += s0 * c[0];
+            p1 += s0 * c[1];
+            o0 += s0 * X.x;
+            o1 += s0 * X.y;
+            q0 += s1 * c[2];
+            q1 += s1 * c[3];
+            r0 += s1 * X.x;
+            r1 += s1 * X.y;
+        }
+        // codes carry +32; every column's integer total is exact before the fp32 step
+        const float2 d = d_pair(U + 3328 + 4 * L.gid);
+        acc0 = fmaf(d.x, fmaf(256.f, (float)(p1 - 32 * o1), (float)(p0 - 32 * o0)), acc0);
+        acc1 = fmaf(d.y, fmaf(256.f, (float)(q1 - 32 * r1), (float)(q0 - 32 * r0)), acc1);
+    }
+};
+
+template <>
+struct Unit<NTX_Q4_K_T> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
+                                               float& acc1)
+    {
+        // the 32 six-bit scales / mins of this lane's two rows, one word per step:
+        // byte 0 scale row gid, 1 scale row gid + 8, 2 min row gid, 3 min row gid + 8
+        const uint8_t* v = U + 2048 + 24 * L.gid;    // 8-byte aligned
+        const uint2 na = *reinterpret_cast<const uint2*>(v);
+        const uint2 nb = *reinterpret_cast<const uint2*>(v + 8);
+        const uint2 hw = *reinterpret_cast<const uint2*>(v + 16);
+        uint32_t S[8];
+        const uint32_t n4[4] = {na.x, na.y, nb.x, nb.y};
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const uint32_t lo = (m & 1 ? (n4[m >> 1] >> 4) : n4[m >> 1]) & 0x0F0F0F0Fu;
+            const uint32_t h = m < 4 ? hw.x : hw.y;
+            const int sh = 2 * (m & 3);
+            const uint32_t hi = (sh <= 4 ? (h << (4 - sh)) : (h >> (sh - 4))) & 0x30303030u;
+            S[m] = lo | hi;
+        }
+        int p0 = 0, p1 = 0, q0 = 0, q1 = 0, o0 = 0, r0 = 0;
+        const uint32_t M = 0x0F0F0F0Fu;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const uint2 pq = *reinterpret_cast<const uint2*>(U + 256 * m + 8 * L.lane);
+            const uint32_t a[4] = {pq.x & M, pq.y & M, (pq.x >> 4) & M, (pq.y >> 4) & M};
+            const uint32_t* x = xs + 32 * m;
+            uint32_t b0, b1;
+            b_frag<NTX_Q4_K_T>(x, L, b0, b1);
+            int c[4];
+            mma_u8(c, a, b0, b1);
+            const int2 X = *reinterpret_cast<const int2*>(x + 24 + 2 * L.tig);
+            const int xp = X.x + 256 * X.y;
+            const int sc0 = ubyte<0>(S[m]), sc1 = ubyte<1>(S[m]), mn0 = ubyte<2>(S[m]), mn1 = ubyte<3>(S[m]);
+            p0 += sc0 * c[0];
+            p1 += sc0 * c[1];
+            q0 += sc1 * c[2];
+            q1 += sc1 * c[3];
+            o0 += mn0 * xp;
+            r0 += mn1 * xp;
+        }
+        const uint2 dd = *reinterpret_cast<const uint2*>(U + 2240 + 8 * L.gid);
+        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+        acc0 = fmaf(d.x, fmaf(256.f, (float)p1, (float)p0), fmaf(-dm.x, (float)o0, acc0));
+        acc1 = fmaf(d.y, fmaf(256.f, (float)q1, (float)q0), fmaf(-dm.y, (float)r0, acc1));
+    }
+};
+
+// ------------------------------------------------------------------ epilogue
+
+// Output row `row` (thread r of warp 0 holds rows r of the group; t = row total).
+template <int EPI>
+__device__ __forceinline__ void epilogue(const Params& P, int row, float t, float t_up, int32_t pos,
+                                         const float* rope_cs)
+{
+    using namespace gemv;
+    if (EPI == EPI_STORE) {
+        P.y[row] = t;
+    } else if (EPI == EPI_ADD) {
+        P.y[row] = P.y[row] + t;
+    } else if (EPI == EPI_SWIGLU) {
+        P.y[row] = t / (1.0f + expf(-t)) * t_up;
+    } else if (EPI == EPI_QKV) {
+        // rows: q [0, q_rows), k [q_rows, q_rows + kv_rows), v after; RoPE on (2i, 2i+1)
+        const float other = __shfl_xor_sync(0x0000ffffu, t, 1);
+        float v = t;
+        const int hd = P.head_dim;
+        if (row < P.q_rows + P.kv_rows) {
+            const int pi = (row % hd) / 2;
+            const float cf = rope_cs[2 * pi], sf = rope_cs[2 * pi + 1];
+            v = (row & 1) ? (other * sf + t * cf) : (t * cf - other * sf);
+        }
+        if (row < P.q_rows) {
+            P.q_out[row] = v;
+        } else {
+            const int kvr = row - P.q_rows;
+            const bool is_v = kvr >= P.kv_rows;
+            const int j = is_v ? kvr - P.kv_rows : kvr;
+            const int g = j / hd, dd = j % hd;
+            __half* cache = is_v ? P.v_cache : P.k_cache;
+            cache[((int64_t)g * P.max_ctx + pos) * hd + dd] = __float2half_rn(v);
+        }
+    }
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int QT, int EPI, int PRO>
+__global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
+{
+    using T = gemv::Tiled<QT>;
+    constexpr int NM = EPI == gemv::EPI_SWIGLU ? 2 : 1;    // matrices per group (gate, up)
+    constexpr int SPU = T::UK / 32;                         // steps per unit
+
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* empty = full + kMaxStages;
+    float* red = reinterpret_cast<float*>(smem + kOffRed);
+    float* rope_cs = reinterpret_cast<float*>(smem + kOffRope);
+    uint32_t* xq = reinterpret_cast<uint32_t*>(smem + kHeader);
+    uint8_t* stages = smem + kHeader + P.x_bytes;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int n_groups = P.M / 16;
+    const int g_begin = (int)((long long)n_groups * blockIdx.x / gridDim.x);
+    const int g_end = (int)((long long)n_groups * (blockIdx.x + 1) / gridDim.x);
+    const int64_t group_bytes = 16 * P.row_bytes;
+
+    if (tid == 0) {
+        for (int s = 0; s < P.n_stages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], kWarps);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (P.use_pdl) pdl_launch_dependents();
+
+    if (warp == kWarps) {
+        // ------------------------------------------------------------- producer
+        // (weights do not depend on earlier kernels, so streaming starts at once)
+        if (lane == 0) {
+            const uint64_t pol = policy_evict_first();
+            const int NS = P.n_stages, NCH = P.n_chunks, CE = P.chunk_elems, K = P.K;
+            int s = 0, issued = 0;
+            uint32_t ph = 0;
+            bool okay = true;
+            for (int gi = g_begin; gi < g_end && okay; ++gi) {
+                for (int mat = 0; mat < NM && okay; ++mat) {
+                    const uint8_t* base = (mat ? P.W2 : P.W) + (int64_t)gi * group_bytes;
+                    for (int c = 0; c < NCH; ++c) {
+                        if (!mbar_wait(&empty[s], ph ^ 1u, kWaitPolls)) {
+                            record_device_error(DEVERR_EMPTY_WAIT);
+                            okay = false;
+                            break;
+                        }
+                        const uint32_t bytes = (uint32_t)(min(CE, K - c * CE) / T::UK * T::UB);
+                        mbar_arrive_expect_tx(&full[s], bytes);
+                        bulk_g2s(stages + (size_t)s * P.stage_bytes, base + (int64_t)c * P.chunk_bytes, bytes,
+                                 &full[s], pol);
+                        ++issued;
+                        if (++s == NS) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                    }
+                }
+            }
+            // Drain: the stages issued last must complete before the CTA may exit.
+            if (!okay) {
+                for (int k = 1; k <= NS && k <= issued; ++k) {
+                    const int j = issued - k;
+                    mbar_wait(&full[j % NS], (uint32_t)(j / NS) & 1u, 1u << 20);
+                }
+            }
+        }
+        return;
+    }
+
+    // ----------------------------------------------------------------- consumers
+    if (P.use_pdl) pdl_wait();
+    float* rs = red;   // scratch for the prologue reductions
+    // (1) x into shared memory as fp32 (RMSNorm applied), gathering max |x|
+    const int K4 = P.K / 4;
+    float4* xf = reinterpret_cast<float4*>(xq);
+    const float4* x4 = reinterpret_cast<const float4*>(P.x);
+    float mx = 0.f;
+    if (PRO == gemv::PRO_RMSNORM) {
+        float ss = 0.f;
+        for (int i = tid; i < K4; i += kCons) {
+            const float4 v = x4[i];
+            xf[i] = v;
+            ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+        }
+        ss = gemv::warp_sum(ss);
+        if (lane == 0) rs[warp] = ss;
+        named_bar_sync(1, kCons);
+        float tot = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) tot += rs[w];
+        const float inv = 1.0f / sqrtf(tot / (float)P.K + P.eps);
+        const float4* w4 = reinterpret_cast<const float4*>(P.norm_w);
+        for (int i = tid; i < K4; i += kCons) {
+            const float4 a = xf[i], w = w4[i];
+            const float4 v = make_float4(a.x * inv * w.x, a.y * inv * w.y, a.z * inv * w.z, a.w * inv * w.w);
+            xf[i] = v;
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+    } else {
+        for (int i = tid; i < K4; i += kCons) {
+            const float4 v = x4[i];
+            xf[i] = v;
+            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        }
+    }
+    mx = gemv::warp_max(mx);
+    if (lane == 0) rs[kWarps + warp] = mx;
+    named_bar_sync(1, kCons);   // also orders every fp32 store before the limb conversion
+    mx = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, rs[kWarps + w]);
+    // |x| 2^S < 2^22; a zero vector keeps S = 0 (all limbs zero)
+    const int S = (mx > 0.f && mx <= 3.4e38f) ? max(-100, min(127, 21 - ilogbf(mx))) : 0;
+    const float two_s = __uint_as_float((uint32_t)(127 + S) << 23);
+    // (2) fp32 -> limbs, in place: 8 lanes per 32-column step
+    {
+        const int n_steps = P.K / 32, sub = lane >> 3, w = lane & 7;
+        for (int base = warp * 4; base < n_steps; base += kWarps * 4) {
+            const int u = base + sub;
+            const bool ok = u < n_steps;
+            const float4 v = ok ? xf[u * 8 + w] : make_float4(0.f, 0.f, 0.f, 0.f);
+            stage_x_step<QT == NTX_Q6_K_T>(xq + 32 * u, w, ok, v, two_s);
+        }
+    }
+    const int32_t pos = (EPI == gemv::EPI_QKV) ? (P.pos_dev ? *P.pos_dev : P.pos) : 0;
+    if (EPI == gemv::EPI_QKV && tid < P.head_dim / 2) {
+        // RoPE angles of this position, pos * theta^(-2i/head_dim), in double; read by the epilogue
+        const double ang = (double)pos * pow((double)P.theta, -(2.0 * tid) / (double)P.head_dim);
+        double sn, cs;
+        sincos(ang, &sn, &cs);
+        rope_cs[2 * tid] = (float)cs;
+        rope_cs[2 * tid + 1] = (float)sn;
+    }
+    named_bar_sync(1, kCons);   // limbs and the RoPE table complete
+
+    const Lane L = make_lane<QT>(lane);
+    const float limb_w = (L.tig & 1) ? 65536.f : 1.f;   // this lane's C columns: limbs 0,1 or limb 2
+    const int NS = P.n_stages, NCH = P.n_chunks, CE = P.chunk_elems, K = P.K;
+    int s = 0;
+    uint32_t ph = 0;
+    bool dead = false;
+    int gcount = 0;
+    for (int gi = g_begin; gi < g_end; ++gi, ++gcount) {
+        float* rg = red + (gcount & 1) * (kWarps * 32);   // [warp][mat][16]
+#pragma unroll 1
+        for (int mat = 0; mat < NM; ++mat) {
+            float acc0 = 0.f, acc1 = 0.f;
+            for (int c = 0; c < NCH; ++c) {
+                const int n_units = min(CE, K - c * CE) / T::UK;
+                if (!dead && !mbar_wait(&full[s], ph, kWaitPolls)) {
+                    record_device_error(DEVERR_FULL_WAIT);
+                    dead = true;    // keep taking part in every barrier so the CTA still finishes
+                }
+                const uint8_t* st = stages + (size_t)s * P.stage_bytes;
+                if (!dead) {
+                    const uint32_t* xc = xq + 32 * (c * CE / 32);
+                    for (int un = warp; un < n_units; un += kWarps)
+                        Unit<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, L, acc0, acc1);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);
+                if (++s == NS) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            // quad reduction with the limb weights: lane tig 0 ends with rows gid, gid + 8
+            acc0 *= limb_w;
+            acc1 *= limb_w;
+            acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+            acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+            acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+            acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
+            if (L.tig == 0) {
+                rg[warp * 32 + mat * 16 + L.gid] = acc0;
+                rg[warp * 32 + mat * 16 + L.gid + 8] = acc1;
+            }
+        }
+        named_bar_sync(1, kCons);
+        if (tid < 16) {
+            float t[2] = {0.f, 0.f};
+#pragma unroll
+            for (int mat = 0; mat < NM; ++mat)
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) t[mat] += rg[w * 32 + mat * 16 + tid];
+            t[0] = gemv::scale2(t[0], -S);
+            t[1] = gemv::scale2(t[1], -S);
+            epilogue<EPI>(P, gi * 16 + tid, t[0], t[1], pos, rope_cs);
+        }
+    }
+}
+
+}  // namespace qmma
+}  // namespace ntx

@@ -122,12 +122,14 @@ def test_decode_entry_points_reject_null_model(ntx):
 def test_repack_rejects_bad_arguments(ntx):
     p = 0x10000
     f = ntx.lib().ntx_repack_q
-    assert f(ntx.NTX_Q8_0_T, p, p * 4, 2, 256, None) == ntx.NTX_EINVAL      # already tiled
-    assert f(ntx.NTX_Q8_0, p, p * 4, 2, 224, None) == ntx.NTX_EINVAL        # not whole tiles
-    assert f(ntx.NTX_Q6_K, p, p * 4, 2, 1024, None) == ntx.NTX_EINVAL       # Q6_K tile = 2048
-    assert f(ntx.NTX_Q4_0, p, p + 100, 2, 256, None) == ntx.NTX_EINVAL      # overlap
-    assert f(ntx.NTX_Q4_0, None, p, 2, 256, None) == ntx.NTX_EINVAL
+    assert f(ntx.NTX_Q8_0_T, p, p * 4, 16, 256, None) == ntx.NTX_EINVAL     # already tiled
+    assert f(ntx.NTX_Q8_0, p, p * 4, 16, 48, None) == ntx.NTX_EINVAL        # not whole blocks
+    assert f(ntx.NTX_Q6_K, p, p * 4, 16, 128, None) == ntx.NTX_EINVAL       # Q6_K unit = 256
+    assert f(ntx.NTX_Q8_0, p, p * 4, 8, 256, None) == ntx.NTX_EINVAL        # rows not a multiple of 16
+    assert f(ntx.NTX_Q4_0, p, p + 100, 16, 256, None) == ntx.NTX_EINVAL     # overlap
+    assert f(ntx.NTX_Q4_0, None, p, 16, 256, None) == ntx.NTX_EINVAL
     assert ntx.ntx_row_bytes(ntx.NTX_Q6_K_T, 2048) == 1680
-    assert ntx.ntx_row_bytes(ntx.NTX_Q6_K_T, 256) == 0
-    assert ntx.ntx_row_bytes(ntx.NTX_Q8_0_T, 256) == 272
+    assert ntx.ntx_row_bytes(ntx.NTX_Q6_K_T, 256) == 210
+    assert ntx.ntx_row_bytes(ntx.NTX_Q6_K_T, 128) == 0
+    assert ntx.ntx_row_bytes(ntx.NTX_Q8_0_T, 32) == 34
     assert ntx.ntx_block_elems(ntx.NTX_Q4_K_T) == 256

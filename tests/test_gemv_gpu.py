@@ -176,8 +176,11 @@ def make_tiled(ntx, syn, qtype, rows, cols, seed=1):
     return host, tiled
 
 
-TILED_FAST = [(Q8_0, 37, 4096 + 256), (Q4_0, 37, 4096 + 256), (Q4_K, 37, 8192 + 256), (Q6_K, 37, 8192 + 2048),
-              (Q8_0, 150, 4096), (Q6_K, 2, 2048), (Q4_0, 300, 1024), (Q8_0, 1, 256)]
+# 16-row groups: one group, fewer groups than SMs, several per SM; several 2048-column
+# chunks and a partial one; a row shorter than one chunk
+TILED_FAST = [(Q8_0, 48, 4096 + 256), (Q4_0, 48, 4096 + 256), (Q4_K, 48, 8192 + 256), (Q6_K, 48, 8192 + 256),
+              (Q8_0, 4096, 4096), (Q6_K, 16, 2048), (Q4_0, 304, 1024), (Q8_0, 16, 32), (Q4_K, 16, 256),
+              (Q6_K, 4096, 1024 + 256), (Q4_0, 32, 96)]
 
 
 @pytest.mark.parametrize("qtype,rows,cols", TILED_FAST, ids=[f"{NAMES[q]}_t-{r}x{c}" for q, r, c in TILED_FAST])
@@ -190,7 +193,7 @@ def test_gemv_tiled(ntx, orc, syn, qtype, rows, cols):
 
 @pytest.mark.parametrize("qtype", [Q8_0, Q4_0, Q4_K, Q6_K], ids=list(NAMES.values()))
 def test_tiled_dequant_bit_exact_and_simple_path(ntx, orc, syn, qtype):
-    rows, cols = 19, 4096 if qtype != Q6_K else 6144
+    rows, cols = 32, 4096 if qtype != Q6_K else 6144
     host, W = make_tiled(ntx, syn, qtype, rows, cols)
     out = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
     ntx.ntx_dequant_q(qtype | T, W, rows, cols, out)
@@ -228,11 +231,11 @@ def test_gemv_tiled_full_shapes(ntx, orc, syn, qtype, rows, cols):
     assert rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)) <= GEMV_TIGHT
 
 
-def test_repack_is_a_byte_permutation(ntx, syn):
-    for qtype, cols in ((Q8_0, 512), (Q4_0, 512), (Q4_K, 512), (Q6_K, 4096)):
-        host, W = make_tiled(ntx, syn, qtype, 3, cols)
-        a = np.sort(host.ravel())
-        b = np.sort(W.cpu().numpy())
-        assert np.array_equal(a, b)
-        if qtype == Q4_K:
-            assert np.array_equal(host.ravel(), W.cpu().numpy())
+@pytest.mark.parametrize("qtype,rows,cols", [(Q8_0, 32, 512), (Q4_0, 16, 256), (Q4_K, 32, 512), (Q6_K, 16, 768)],
+                         ids=["q8_0", "q4_0", "q4_k", "q6_k"])
+def test_repack_matches_documented_layout(ntx, syn, qtype, rows, cols):
+    """The repack kernel's bytes equal the layout the header documents (an independent
+    numpy model of it)."""
+    import tiling
+    host, W = make_tiled(ntx, syn, qtype, rows, cols)
+    assert np.array_equal(W.cpu().numpy(), tiling.tile(qtype, host, rows, cols))
