@@ -387,6 +387,39 @@ def profile_gemv(what, launches):
     print(json.dumps({"gemv": what, "bytes": W.numel(), "us": us, "gbs": W.numel() / (us * 1e-6) / 1e9}))
 
 
+def profile_attn(what, launches):
+    """A few launches of the split-KV decode attention on one shape (random fp16 KV
+    cache, L2 flushed between launches), nothing else: the case that profiler
+    captures of the attention kernel run.  what = QHEADS:KVHEADS:CONTEXT."""
+    import torch
+    import quantized_weight_gemv_block_b200 as ntx
+    from quantized_weight_gemv_block_b200 import build
+    build.build()
+    nq, nkv, ctx = (int(v) for v in what.split(":"))
+    hd = 128
+    g = torch.Generator(device="cuda").manual_seed(7)
+    q = torch.randn(nq * hd, device="cuda", generator=g)
+    k = torch.randn(nkv * ctx * hd, device="cuda", generator=g).half()
+    v = torch.randn(nkv * ctx * hd, device="cuda", generator=g).half()
+    out = torch.empty(nq * hd, device="cuda")
+    wsb = ntx.ntx_attn_workspace_bytes(nq, nkv, hd, ctx)
+    ws = torch.empty(wsb, dtype=torch.uint8, device="cuda")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    times = []
+    for i in range(launches + 1):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        ntx.ntx_attn_decode(q, k, v, out, nq, nkv, hd, ctx, ctx, ws, wsb)
+        e1.record()
+        torch.cuda.synchronize()
+        if i:
+            times.append(e0.elapsed_time(e1) * 1e3)
+    us = sorted(times)[len(times) // 2]
+    kv = 2 * nkv * ctx * hd * 2
+    print(json.dumps({"attn": what, "kv_bytes": kv, "us_median": us, "gbs": kv / (us * 1e-6) / 1e9}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -401,9 +434,13 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--profile-gemv", default=None, metavar="FMT:ROWSxCOLS",
                     help="only run the GEMV kernel on one matrix (for profilers), e.g. q6_k:28672x8192")
+    ap.add_argument("--profile-attn", default=None, metavar="QHEADS:KVHEADS:CONTEXT",
+                    help="only run the decode attention on one shape (for profilers), e.g. 64:8:8193")
     args = ap.parse_args()
     if args.profile_gemv:
         return profile_gemv(args.profile_gemv, args.steps)
+    if args.profile_attn:
+        return profile_attn(args.profile_attn, args.steps)
     if args.warmup < 3:
         args.warmup = 3
 
