@@ -71,6 +71,7 @@ struct Params {
     int stage_bytes;
     int x_bytes;
     int use_pdl;
+    int recv_bytes;       // tensor-core GEMV: bytes of the per-group row sums of a CTA pair
     // multiplier that lets a shift run as an integer multiply on the FMA pipe
     // (v >> 8 == umulhi(v, 2^24)); passed in so it stays a multiply
     uint32_t m24;

@@ -1,9 +1,9 @@
 // qmma.cu - host side of the tensor-core GEMV for the tiled layouts (launch
 // shaping) and the repack kernel GGUF-style -> tiled.
 #include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
-#include "launch.h"
 #include "qmma.cuh"
 
 namespace ntx {
@@ -125,18 +125,29 @@ __global__ void repack_kernel(const uint8_t* in, uint8_t* out, int64_t n_bytes, 
 
 // ------------------------------------------------------------------ launch shaping
 
+// Columns a CTA takes: the whole row, or the larger half when CTA pairs split it.
 template <int QT>
-bool shape(Params& P)
+int cta_cols(int K, int csize)
 {
     using T = gemv::Tiled<QT>;
-    P.x_bytes = P.K * 4;   // 32 words per 32-column step
-    const int avail = kSmemLimit - kHeader - P.x_bytes - 128;
+    return csize == 2 ? (K / T::UK + 1) / 2 * T::UK : K;
+}
+
+template <int QT>
+bool shape(Params& P, int n_clusters, int csize, int n_mats)
+{
+    using T = gemv::Tiled<QT>;
+    const int kh = cta_cols<QT>(P.K, csize);
+    P.x_bytes = kh * 4;   // 32 words per 32-column step of the half
+    const int max_groups = (P.M / 16 + n_clusters - 1) / n_clusters;
+    P.recv_bytes = max_groups * n_mats * 16 * 4;
+    const int avail = kSmemLimit - kHeader - P.x_bytes - P.recv_bytes - 128;
     // chunks of up to 2048 columns (whole units), shrunk until at least 3 stages fit
-    int ce = std::min(P.K, 2048) / T::UK * T::UK;
+    int ce = std::min(kh, 2048) / T::UK * T::UK;
     while (ce > T::UK && avail / (ce / T::UK * T::UB) < 3) ce = std::max(T::UK, ce / 2 / T::UK * T::UK);
-    if (ce < T::UK) return false;
+    if (ce < T::UK || avail <= 0) return false;
     P.chunk_elems = ce;
-    P.n_chunks = (P.K + ce - 1) / ce;
+    P.n_chunks = (kh + ce - 1) / ce;
     P.chunk_bytes = ce / T::UK * T::UB;
     P.stage_bytes = P.chunk_bytes;
     const int ns = std::min(kMaxStages, avail / P.stage_bytes);
@@ -145,28 +156,88 @@ bool shape(Params& P)
     return true;
 }
 
+// Clusters of `csize` CTAs (one per SM) that fit on the device at once, per kernel.
 template <int QT, int EPI, int PRO>
-ntx_status launch_t(Params P, cudaStream_t s, int grid_cap)
+int max_clusters(int csize)
 {
-    if (!shape<QT>(P)) return fail(NTX_EUNSUPPORTED, "gemv: row too long for the shared-memory pipeline");
+    static std::once_flag once[3];
+    static int n[3] = {0, 0, 0};
+    std::call_once(once[csize], [csize] {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(csize * 256);
+        cfg.blockDim = dim3(kThreads);
+        cfg.dynamicSmemBytes = kSmemLimit;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = csize;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int c = 0;
+        if (cudaOccupancyMaxActiveClusters(&c, qmma_kernel<QT, EPI, PRO>, &cfg) != cudaSuccess || c < 1) {
+            cudaGetLastError();
+            c = std::max(1, num_sms() / csize);
+        }
+        n[csize] = c;
+    });
+    return n[csize];
+}
+
+// Whether CTA pairs split the columns: when whole rows would leave the last round of
+// 16-row groups unbalanced (fewer than 6 groups per SM) and the rows are long
+// (16384 columns or more) so half a row still amortises a group's fixed costs.
+// Measured on B200: 8192 x 28672 Q6_K 4.84 TB/s split against 4.39 whole; at 8192
+// columns the two are even, at 4096 the split loses.  NTX_GEMV_SPLIT=0 / 1
+// overrides the choice (a tuning override).
+inline int pick_cluster_size(int M, int K)
+{
+    const char* env = std::getenv("NTX_GEMV_SPLIT");
+    if (env && env[0] == '0') return 1;
+    if (env && env[0] == '1') return 2;
+    return (M / 16 < 6 * num_sms() && K >= 16384) ? 2 : 1;
+}
+
+template <int QT, int EPI, int PRO>
+ntx_status launch_t(Params P, cudaStream_t s)
+{
     auto kern = qmma_kernel<QT, EPI, PRO>;
-    const int smem = kHeader + P.x_bytes + P.n_stages * P.stage_bytes + 128;
     static std::once_flag once[4][4][2];
     std::call_once(once[QT & 3][EPI][PRO], [&] {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     });
-    const int grid = std::max(1, std::min(grid_cap, P.M / 16));
-    return launch_kernel(kern, dim3(grid), dim3(kThreads), smem, s, P.use_pdl != 0, P);
+    const int csize = pick_cluster_size(P.M, P.K);
+    const int n_clusters = std::max(1, std::min(max_clusters<QT, EPI, PRO>(csize), P.M / 16));
+    if (!shape<QT>(P, n_clusters, csize, EPI == gemv::EPI_SWIGLU ? 2 : 1))
+        return fail(NTX_EUNSUPPORTED, "gemv: row too long for the shared-memory pipeline");
+    const int smem = kHeader + P.x_bytes + P.n_stages * P.stage_bytes + P.recv_bytes + 128;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize * n_clusters);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = P.use_pdl ? 2 : 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, P);
+    if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("gemv (tensor cores) launch: ") + cudaGetErrorString(e));
+    return NTX_OK;
 }
 
 template <int EPI, int PRO>
-ntx_status launch_q(int qtype, const Params& P, cudaStream_t s, int grid_cap)
+ntx_status launch_q(int qtype, const Params& P, cudaStream_t s)
 {
     switch (qtype) {
-    case NTX_Q8_0_T: return launch_t<NTX_Q8_0_T, EPI, PRO>(P, s, grid_cap);
-    case NTX_Q4_0_T: return launch_t<NTX_Q4_0_T, EPI, PRO>(P, s, grid_cap);
-    case NTX_Q4_K_T: return launch_t<NTX_Q4_K_T, EPI, PRO>(P, s, grid_cap);
-    case NTX_Q6_K_T: return launch_t<NTX_Q6_K_T, EPI, PRO>(P, s, grid_cap);
+    case NTX_Q8_0_T: return launch_t<NTX_Q8_0_T, EPI, PRO>(P, s);
+    case NTX_Q4_0_T: return launch_t<NTX_Q4_0_T, EPI, PRO>(P, s);
+    case NTX_Q4_K_T: return launch_t<NTX_Q4_K_T, EPI, PRO>(P, s);
+    case NTX_Q6_K_T: return launch_t<NTX_Q6_K_T, EPI, PRO>(P, s);
     default: return fail(NTX_EINVAL, "unknown tiled qtype");
     }
 }
@@ -177,12 +248,11 @@ ntx_status qmma_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaS
 {
     using namespace gemv;
     if (P.M % 16) return fail(NTX_EINVAL, "gemv: tiled layouts need a multiple of 16 rows");
-    const int cap = num_sms();
-    if (epi == EPI_STORE && pro == PRO_X) return qmma::launch_q<EPI_STORE, PRO_X>(qtype, P, s, cap);
-    if (epi == EPI_ADD && pro == PRO_X) return qmma::launch_q<EPI_ADD, PRO_X>(qtype, P, s, cap);
-    if (epi == EPI_SWIGLU && pro == PRO_RMSNORM) return qmma::launch_q<EPI_SWIGLU, PRO_RMSNORM>(qtype, P, s, cap);
-    if (epi == EPI_QKV && pro == PRO_RMSNORM) return qmma::launch_q<EPI_QKV, PRO_RMSNORM>(qtype, P, s, cap);
-    if (epi == EPI_STORE && pro == PRO_RMSNORM) return qmma::launch_q<EPI_STORE, PRO_RMSNORM>(qtype, P, s, cap);
+    if (epi == EPI_STORE && pro == PRO_X) return qmma::launch_q<EPI_STORE, PRO_X>(qtype, P, s);
+    if (epi == EPI_ADD && pro == PRO_X) return qmma::launch_q<EPI_ADD, PRO_X>(qtype, P, s);
+    if (epi == EPI_SWIGLU && pro == PRO_RMSNORM) return qmma::launch_q<EPI_SWIGLU, PRO_RMSNORM>(qtype, P, s);
+    if (epi == EPI_QKV && pro == PRO_RMSNORM) return qmma::launch_q<EPI_QKV, PRO_RMSNORM>(qtype, P, s);
+    if (epi == EPI_STORE && pro == PRO_RMSNORM) return qmma::launch_q<EPI_STORE, PRO_RMSNORM>(qtype, P, s);
     return fail(NTX_EUNSUPPORTED, "gemv: unsupported prologue / epilogue combination");
 }
 

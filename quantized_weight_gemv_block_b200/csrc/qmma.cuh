@@ -22,18 +22,30 @@
 // The products are exact; x carries 23 bits (relative to max |x|) where fp32
 // carries 24; sums round at fp32 once per block or superblock.
 //
-// Structure (one CTA per SM, 8 consumer warps + 1 producer warp):
-//  * the CTA owns a contiguous range of 16-row groups; a stage is one group x one
-//    chunk of KC columns, contiguous in the tiled layout, streamed by the producer
-//    warp with one 1-D bulk copy (cp.async.bulk, L2 evict-first) into a ring of
-//    shared-memory stages guarded by mbarriers;
+// Structure (one CTA per SM, 8 consumer warps, a producer and a reducer warp):
+//  * the grid is made of clusters of 1 or 2 CTAs; a cluster owns a contiguous
+//    range of 16-row groups.  For matrices with few groups per SM the two CTAs of
+//    a pair split the columns in halves (so the groups spread over 74 pairs
+//    instead of 148 CTAs, which evens out the last round, and each CTA stages
+//    only its half of x); both CTAs add each group's partial
+//    row sums into a zeroed buffer in the first CTA's shared memory (the second
+//    through distributed shared memory), and after a cluster barrier the first
+//    CTA runs the epilogue of all its rows (with two addends the sum does not
+//    depend on their order);
+//  * a stage is one group x one chunk of KC columns of the CTA's half, contiguous
+//    in the tiled layout, streamed by the producer warp with one 1-D bulk copy
+//    (cp.async.bulk, L2 evict-first) into a ring of shared-memory stages guarded
+//    by mbarriers;
 //  * each consumer warp takes every 8th unit (32 or 256 columns) of a stage; per
 //    32-column step a lane loads its two rows' codes with one shared-memory load,
 //    unpacks 4-/6-bit codes into bytes with a few logic ops, issues one MMA and
 //    folds the step's integers into its row accumulators;
 //  * row totals are reduced over the 4 lanes of a quad (limb weights) and over the
-//    warps through shared memory, then the fused epilogue runs (store, residual
-//    add, SwiGLU of a gate / up group pair, RoPE + fp16 KV-cache append).
+//    8 warps through shared memory in a fixed order (a barrier of the consumer
+//    warps per group: measured faster on B200 than handing the sums to a separate
+//    reducer warp through mbarriers) into the pair's sums; after the cluster
+//    barrier the fused epilogue runs (store, residual add, SwiGLU of a gate / up
+//    group pair, RoPE + fp16 KV-cache append).
 #pragma once
 
 #include "blocks.cuh"
@@ -45,11 +57,12 @@ using gemv::Params;
 
 constexpr int kWarps = 8;                  // consumer warps
 constexpr int kCons = kWarps * 32;
-constexpr int kThreads = kCons + 32;       // + the producer warp
+constexpr int kProducer = kWarps;          // warp index of the producer
+constexpr int kThreads = kCons + 32;
 constexpr int kMaxStages = 8;
-constexpr int kHeader = 3072;              // barriers, reduction scratch, RoPE table
 constexpr int kOffRed = 256;               // [2][kWarps][2 mats][16] floats
-constexpr int kOffRope = 2304;             // [64][cos, sin]
+constexpr int kOffRope = kOffRed + 2 * kWarps * 32 * 4;   // [64][cos, sin]
+constexpr int kHeader = kOffRope + 512 + 256;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr uint32_t kWaitPolls = 1u << 22;
 
@@ -88,6 +101,47 @@ template <int k>
 __device__ __forceinline__ int ubyte(uint32_t w)
 {
     return (int)__byte_perm(w, 0u, 0x4440u | k);
+}
+
+// ------------------------------------------------------------------ cluster helpers
+
+__device__ __forceinline__ uint32_t cluster_rank()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_size()
+{
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+    return r;
+}
+
+// Barrier of all threads of the cluster (of the CTA alone when the cluster is one CTA).
+__device__ __forceinline__ void cluster_sync(uint32_t csize)
+{
+    if (csize == 1)
+        __syncthreads();
+    else
+        asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
+
+
+// Address of `p` (this CTA's shared memory) in the shared memory of cluster CTA `rank`.
+__device__ __forceinline__ uint32_t peer_addr(const void* p, uint32_t rank)
+{
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_addr(p)), "r"(rank));
+    return r;
+}
+
+// Atomic add of v to the fp32 at shared::cluster address addr.
+__device__ __forceinline__ void red_add_cluster(uint32_t addr, float v)
+{
+    asm volatile("red.relaxed.cluster.shared::cluster.add.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
 // ------------------------------------------------------------------ x staging
@@ -347,21 +401,23 @@ struct Unit<NTX_Q4_K_T> {
 
 // ------------------------------------------------------------------ epilogue
 
-// Output row `row` (thread r of warp 0 holds rows r of the group; t = row total).
+// Output row `row` (t = row total, t_up the up-projection total for SwiGLU).  Called
+// by whole warps; `ok` is false for lanes past the last row.
 template <int EPI>
-__device__ __forceinline__ void epilogue(const Params& P, int row, float t, float t_up, int32_t pos,
+__device__ __forceinline__ void epilogue(const Params& P, int row, bool ok, float t, float t_up, int32_t pos,
                                          const float* rope_cs)
 {
     using namespace gemv;
     if (EPI == EPI_STORE) {
-        P.y[row] = t;
+        if (ok) P.y[row] = t;
     } else if (EPI == EPI_ADD) {
-        P.y[row] = P.y[row] + t;
+        if (ok) P.y[row] = P.y[row] + t;
     } else if (EPI == EPI_SWIGLU) {
-        P.y[row] = t / (1.0f + expf(-t)) * t_up;
+        if (ok) P.y[row] = t / (1.0f + expf(-t)) * t_up;
     } else if (EPI == EPI_QKV) {
         // rows: q [0, q_rows), k [q_rows, q_rows + kv_rows), v after; RoPE on (2i, 2i+1)
-        const float other = __shfl_xor_sync(0x0000ffffu, t, 1);
+        const float other = __shfl_xor_sync(0xffffffffu, t, 1);
+        if (!ok) return;
         float v = t;
         const int hd = P.head_dim;
         if (row < P.q_rows + P.kv_rows) {
@@ -398,12 +454,21 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
     float* rope_cs = reinterpret_cast<float*>(smem + kOffRope);
     uint32_t* xq = reinterpret_cast<uint32_t*>(smem + kHeader);
     uint8_t* stages = smem + kHeader + P.x_bytes;
+    float* sums = reinterpret_cast<float*>(stages + (size_t)P.n_stages * P.stage_bytes);   // [group][mat][16]
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // clusters of 1 CTA (whole rows) or 2 CTAs (each takes one half of the columns)
+    const uint32_t rank = cluster_rank(), csize = cluster_size();
+    const int n_clusters = gridDim.x / csize, cluster = blockIdx.x / csize;
     const int n_groups = P.M / 16;
-    const int g_begin = (int)((long long)n_groups * blockIdx.x / gridDim.x);
-    const int g_end = (int)((long long)n_groups * (blockIdx.x + 1) / gridDim.x);
+    const int g_begin = (int)((long long)n_groups * cluster / n_clusters);
+    const int g_end = (int)((long long)n_groups * (cluster + 1) / n_clusters);
     const int64_t group_bytes = 16 * P.row_bytes;
+    // this CTA's columns: units [u0, u1) of the row (rank 0 takes the larger half)
+    const int n_units_row = P.K / T::UK, half = csize == 2 ? (n_units_row + 1) / 2 : n_units_row;
+    const int u0 = rank ? half : 0, u1 = rank ? n_units_row : half;
+    const int k0 = u0 * T::UK, KR = (u1 - u0) * T::UK;
+    const int CE = P.chunk_elems, NCH = (KR + CE - 1) / CE;
 
     if (tid == 0) {
         for (int s = 0; s < P.n_stages; ++s) {
@@ -412,28 +477,30 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
         }
         fence_mbar_init();
     }
-    __syncthreads();
+    for (int i = tid; i < P.recv_bytes / 4; i += kThreads) sums[i] = 0.f;
+    // both CTAs initialised before either touches the other's shared memory
+    cluster_sync(csize);
     if (P.use_pdl) pdl_launch_dependents();
 
-    if (warp == kWarps) {
+    if (warp == kProducer) {
         // ------------------------------------------------------------- producer
         // (weights do not depend on earlier kernels, so streaming starts at once)
         if (lane == 0) {
             const uint64_t pol = policy_evict_first();
-            const int NS = P.n_stages, NCH = P.n_chunks, CE = P.chunk_elems, K = P.K;
+            const int NS = P.n_stages;
             int s = 0, issued = 0;
             uint32_t ph = 0;
             bool okay = true;
             for (int gi = g_begin; gi < g_end && okay; ++gi) {
                 for (int mat = 0; mat < NM && okay; ++mat) {
-                    const uint8_t* base = (mat ? P.W2 : P.W) + (int64_t)gi * group_bytes;
+                    const uint8_t* base = (mat ? P.W2 : P.W) + (int64_t)gi * group_bytes + (int64_t)u0 * T::UB;
                     for (int c = 0; c < NCH; ++c) {
                         if (!mbar_wait(&empty[s], ph ^ 1u, kWaitPolls)) {
                             record_device_error(DEVERR_EMPTY_WAIT);
                             okay = false;
                             break;
                         }
-                        const uint32_t bytes = (uint32_t)(min(CE, K - c * CE) / T::UK * T::UB);
+                        const uint32_t bytes = (uint32_t)(min(CE, KR - c * CE) / T::UK * T::UB);
                         mbar_arrive_expect_tx(&full[s], bytes);
                         bulk_g2s(stages + (size_t)s * P.stage_bytes, base + (int64_t)c * P.chunk_bytes, bytes,
                                  &full[s], pol);
@@ -453,130 +520,152 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                 }
             }
         }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------- consumers
+        if (P.use_pdl) pdl_wait();
+        float* rs = red;   // scratch for the prologue reductions
+        // (1) this CTA's columns of x into shared memory as fp32 (RMSNorm applied: the
+        // sum of squares runs over the whole vector), gathering max |x| of the half
+        const int K4 = P.K / 4, h0 = k0 / 4, h1 = (k0 + KR) / 4;
+        float4* xf = reinterpret_cast<float4*>(xq);
+        const float4* x4 = reinterpret_cast<const float4*>(P.x);
+        float mx = 0.f;
+        if (PRO == gemv::PRO_RMSNORM) {
+            float ss = 0.f;
+            for (int i = tid; i < K4; i += kCons) {
+                const float4 v = x4[i];
+                if (i >= h0 && i < h1) xf[i - h0] = v;
+                ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+            }
+            ss = gemv::warp_sum(ss);
+            if (lane == 0) rs[warp] = ss;
+            named_bar_sync(1, kCons);
+            float tot = 0.f;
+#pragma unroll
+            for (int w = 0; w < kWarps; ++w) tot += rs[w];
+            const float inv = 1.0f / sqrtf(tot / (float)P.K + P.eps);
+            const float4* w4 = reinterpret_cast<const float4*>(P.norm_w) + h0;
+            for (int i = tid; i < h1 - h0; i += kCons) {
+                const float4 a = xf[i], w = w4[i];
+                const float4 v = make_float4(a.x * inv * w.x, a.y * inv * w.y, a.z * inv * w.z, a.w * inv * w.w);
+                xf[i] = v;
+                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+            }
+        } else {
+            for (int i = tid; i < h1 - h0; i += kCons) {
+                const float4 v = x4[h0 + i];
+                xf[i] = v;
+                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+            }
+        }
+        mx = gemv::warp_max(mx);
+        if (lane == 0) rs[kWarps + warp] = mx;
+        named_bar_sync(1, kCons);   // also orders every fp32 store before the limb conversion
+        mx = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, rs[kWarps + w]);
+        // |x| 2^S < 2^22; a zero half keeps S = 0 (all limbs zero)
+        const int S = (mx > 0.f && mx <= 3.4e38f) ? max(-100, min(127, 21 - ilogbf(mx))) : 0;
+        const float two_s = __uint_as_float((uint32_t)(127 + S) << 23);
+        // (2) fp32 -> limbs, in place: 8 lanes per 32-column step
+        {
+            const int n_steps = KR / 32, sub = lane >> 3, w = lane & 7;
+            for (int base = warp * 4; base < n_steps; base += kWarps * 4) {
+                const int u = base + sub;
+                const bool ok = u < n_steps;
+                const float4 v = ok ? xf[u * 8 + w] : make_float4(0.f, 0.f, 0.f, 0.f);
+                stage_x_step<QT == NTX_Q6_K_T>(xq + 32 * u, w, ok, v, two_s);
+            }
+        }
+        const int32_t pos = (EPI == gemv::EPI_QKV) ? (P.pos_dev ? *P.pos_dev : P.pos) : 0;
+        if (EPI == gemv::EPI_QKV && tid < P.head_dim / 2) {
+            // RoPE angles of this position, pos * theta^(-2i/head_dim), in double; read by the epilogue
+            const double ang = (double)pos * pow((double)P.theta, -(2.0 * tid) / (double)P.head_dim);
+            double sn, cs;
+            sincos(ang, &sn, &cs);
+            rope_cs[2 * tid] = (float)cs;
+            rope_cs[2 * tid + 1] = (float)sn;
+        }
+        named_bar_sync(1, kCons);   // limbs and the RoPE table complete
+
+        const Lane L = make_lane<QT>(lane);
+        const float limb_w = (L.tig & 1) ? 65536.f : 1.f;   // this lane's C columns: limbs 0,1 or limb 2
+        const int NS = P.n_stages;
+        int s = 0;
+        uint32_t ph = 0;
+        bool dead = false;
+        int gl = 0;
+        const uint32_t sums0 = peer_addr(sums, 0);   // the pair's sums, in the first CTA
+        for (int gi = g_begin; gi < g_end; ++gi, ++gl) {
+            float* rg = red + (gl & 1) * (kWarps * 32);   // [warp][mat][16]
+#pragma unroll 1
+            for (int mat = 0; mat < NM; ++mat) {
+                float acc0 = 0.f, acc1 = 0.f;
+                for (int c = 0; c < NCH; ++c) {
+                    const int n_units = min(CE, KR - c * CE) / T::UK;
+                    if (!dead && !mbar_wait(&full[s], ph, kWaitPolls)) {
+                        record_device_error(DEVERR_FULL_WAIT);
+                        dead = true;    // keep taking part in every barrier so the CTA still finishes
+                    }
+                    const uint8_t* st = stages + (size_t)s * P.stage_bytes;
+                    if (!dead) {
+                        const uint32_t* xc = xq + 32 * (c * CE / 32);
+                        for (int un = warp; un < n_units; un += kWarps)
+                            Unit<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, L, acc0, acc1);
+                    }
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[s]);
+                    if (++s == NS) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                // quad reduction with the limb weights: lane tig 0 ends with rows gid, gid + 8
+                acc0 *= limb_w;
+                acc1 *= limb_w;
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
+                if (L.tig == 0) {
+                    rg[warp * 32 + mat * 16 + L.gid] = acc0;
+                    rg[warp * 32 + mat * 16 + L.gid + 8] = acc1;
+                }
+            }
+            named_bar_sync(1, kCons);
+            if (tid < 16 * NM) {
+                // the 8 warps' sums in warp order, scaled by 2^-S, into the pair's sums
+                const int row = tid & 15, mat = tid >> 4;
+                float t = 0.f;
+#pragma unroll
+                for (int w = 0; w < kWarps; ++w) t += rg[w * 32 + mat * 16 + row];
+                t = gemv::scale2(t, -S);
+                const int slot = (gl * NM + mat) * 16 + row;
+                if (csize == 1)
+                    sums[slot] = t;
+                else
+                    red_add_cluster(sums0 + 4u * slot, t);
+            }
+        }
+        // every addend of the pair has landed once both CTAs pass the cluster barrier
+        cluster_sync(csize);
+        if (rank == 0) {
+            // epilogue of all rows of the pair's groups; RoPE partners (2i, 2i + 1) sit in adjacent lanes
+            const int n_rows = (g_end - g_begin) * 16;
+            for (int base = 0; base < n_rows; base += kCons) {
+                const int r = base + tid;
+                const bool ok = r < n_rows;
+                const int gl2 = ok ? r >> 4 : 0, rr = r & 15;
+                const float a = ok ? sums[(gl2 * NM) * 16 + rr] : 0.f;
+                const float b = (ok && NM == 2) ? sums[(gl2 * NM + 1) * 16 + rr] : 0.f;
+                epilogue<EPI>(P, g_begin * 16 + r, ok, a, b, pos, rope_cs);
+            }
+        }
         return;
     }
-
-    // ----------------------------------------------------------------- consumers
-    if (P.use_pdl) pdl_wait();
-    float* rs = red;   // scratch for the prologue reductions
-    // (1) x into shared memory as fp32 (RMSNorm applied), gathering max |x|
-    const int K4 = P.K / 4;
-    float4* xf = reinterpret_cast<float4*>(xq);
-    const float4* x4 = reinterpret_cast<const float4*>(P.x);
-    float mx = 0.f;
-    if (PRO == gemv::PRO_RMSNORM) {
-        float ss = 0.f;
-        for (int i = tid; i < K4; i += kCons) {
-            const float4 v = x4[i];
-            xf[i] = v;
-            ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
-        }
-        ss = gemv::warp_sum(ss);
-        if (lane == 0) rs[warp] = ss;
-        named_bar_sync(1, kCons);
-        float tot = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) tot += rs[w];
-        const float inv = 1.0f / sqrtf(tot / (float)P.K + P.eps);
-        const float4* w4 = reinterpret_cast<const float4*>(P.norm_w);
-        for (int i = tid; i < K4; i += kCons) {
-            const float4 a = xf[i], w = w4[i];
-            const float4 v = make_float4(a.x * inv * w.x, a.y * inv * w.y, a.z * inv * w.z, a.w * inv * w.w);
-            xf[i] = v;
-            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-        }
-    } else {
-        for (int i = tid; i < K4; i += kCons) {
-            const float4 v = x4[i];
-            xf[i] = v;
-            mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-        }
-    }
-    mx = gemv::warp_max(mx);
-    if (lane == 0) rs[kWarps + warp] = mx;
-    named_bar_sync(1, kCons);   // also orders every fp32 store before the limb conversion
-    mx = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, rs[kWarps + w]);
-    // |x| 2^S < 2^22; a zero vector keeps S = 0 (all limbs zero)
-    const int S = (mx > 0.f && mx <= 3.4e38f) ? max(-100, min(127, 21 - ilogbf(mx))) : 0;
-    const float two_s = __uint_as_float((uint32_t)(127 + S) << 23);
-    // (2) fp32 -> limbs, in place: 8 lanes per 32-column step
-    {
-        const int n_steps = P.K / 32, sub = lane >> 3, w = lane & 7;
-        for (int base = warp * 4; base < n_steps; base += kWarps * 4) {
-            const int u = base + sub;
-            const bool ok = u < n_steps;
-            const float4 v = ok ? xf[u * 8 + w] : make_float4(0.f, 0.f, 0.f, 0.f);
-            stage_x_step<QT == NTX_Q6_K_T>(xq + 32 * u, w, ok, v, two_s);
-        }
-    }
-    const int32_t pos = (EPI == gemv::EPI_QKV) ? (P.pos_dev ? *P.pos_dev : P.pos) : 0;
-    if (EPI == gemv::EPI_QKV && tid < P.head_dim / 2) {
-        // RoPE angles of this position, pos * theta^(-2i/head_dim), in double; read by the epilogue
-        const double ang = (double)pos * pow((double)P.theta, -(2.0 * tid) / (double)P.head_dim);
-        double sn, cs;
-        sincos(ang, &sn, &cs);
-        rope_cs[2 * tid] = (float)cs;
-        rope_cs[2 * tid + 1] = (float)sn;
-    }
-    named_bar_sync(1, kCons);   // limbs and the RoPE table complete
-
-    const Lane L = make_lane<QT>(lane);
-    const float limb_w = (L.tig & 1) ? 65536.f : 1.f;   // this lane's C columns: limbs 0,1 or limb 2
-    const int NS = P.n_stages, NCH = P.n_chunks, CE = P.chunk_elems, K = P.K;
-    int s = 0;
-    uint32_t ph = 0;
-    bool dead = false;
-    int gcount = 0;
-    for (int gi = g_begin; gi < g_end; ++gi, ++gcount) {
-        float* rg = red + (gcount & 1) * (kWarps * 32);   // [warp][mat][16]
-#pragma unroll 1
-        for (int mat = 0; mat < NM; ++mat) {
-            float acc0 = 0.f, acc1 = 0.f;
-            for (int c = 0; c < NCH; ++c) {
-                const int n_units = min(CE, K - c * CE) / T::UK;
-                if (!dead && !mbar_wait(&full[s], ph, kWaitPolls)) {
-                    record_device_error(DEVERR_FULL_WAIT);
-                    dead = true;    // keep taking part in every barrier so the CTA still finishes
-                }
-                const uint8_t* st = stages + (size_t)s * P.stage_bytes;
-                if (!dead) {
-                    const uint32_t* xc = xq + 32 * (c * CE / 32);
-                    for (int un = warp; un < n_units; un += kWarps)
-                        Unit<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, L, acc0, acc1);
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[s]);
-                if (++s == NS) {
-                    s = 0;
-                    ph ^= 1u;
-                }
-            }
-            // quad reduction with the limb weights: lane tig 0 ends with rows gid, gid + 8
-            acc0 *= limb_w;
-            acc1 *= limb_w;
-            acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
-            acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
-            acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
-            acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
-            if (L.tig == 0) {
-                rg[warp * 32 + mat * 16 + L.gid] = acc0;
-                rg[warp * 32 + mat * 16 + L.gid + 8] = acc1;
-            }
-        }
-        named_bar_sync(1, kCons);
-        if (tid < 16) {
-            float t[2] = {0.f, 0.f};
-#pragma unroll
-            for (int mat = 0; mat < NM; ++mat)
-#pragma unroll
-                for (int w = 0; w < kWarps; ++w) t[mat] += rg[w * 32 + mat * 16 + tid];
-            t[0] = gemv::scale2(t[0], -S);
-            t[1] = gemv::scale2(t[1], -S);
-            epilogue<EPI>(P, gi * 16 + tid, t[0], t[1], pos, rope_cs);
-        }
-    }
+    // the producer warp meets the consumers at the cluster barrier
+    cluster_sync(csize);
 }
 
 }  // namespace qmma

@@ -239,3 +239,15 @@ def test_repack_matches_documented_layout(ntx, syn, qtype, rows, cols):
     import tiling
     host, W = make_tiled(ntx, syn, qtype, rows, cols)
     assert np.array_equal(W.cpu().numpy(), tiling.tile(qtype, host, rows, cols))
+
+
+@pytest.mark.parametrize("split", ["0", "1"], ids=["whole-rows", "column-halves"])
+@pytest.mark.parametrize("qtype,rows,cols", [(Q6_K, 1024, 8192 + 256), (Q8_0, 2048, 4096 + 32), (Q4_K, 160, 2304),
+                                             (Q4_0, 32, 64)], ids=["q6_k", "q8_0", "q4_k", "q4_0"])
+def test_gemv_tiled_both_cluster_shapes(ntx, orc, syn, monkeypatch, split, qtype, rows, cols):
+    """Whole rows per CTA and CTA pairs that split the columns (forced either way): both
+    match the oracle, including an odd number of units per row."""
+    monkeypatch.setenv("NTX_GEMV_SPLIT", split)
+    host, W = make_tiled(ntx, syn, qtype, rows, cols)
+    x = syn.normal_f32_host(7, 12, cols)
+    assert rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)) <= GEMV_TIGHT
