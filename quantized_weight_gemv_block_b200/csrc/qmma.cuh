@@ -60,6 +60,7 @@ constexpr int kCons = kWarps * 32;
 constexpr int kProducer = kWarps;          // warp index of the producer
 constexpr int kThreads = kCons + 32;
 constexpr int kMaxStages = 8;
+constexpr int kOffXBar = 128;              // mbarrier of the bulk copy of x
 constexpr int kOffRed = 256;               // [2][kWarps][2 mats][16] floats
 constexpr int kOffRope = kOffRed + 2 * kWarps * 32 * 4;   // [64][cos, sin]
 constexpr int kHeader = kOffRope + 512 + 256;
@@ -450,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
     uint64_t* empty = full + kMaxStages;
+    uint64_t* xbar = reinterpret_cast<uint64_t*>(smem + kOffXBar);
     float* red = reinterpret_cast<float*>(smem + kOffRed);
     float* rope_cs = reinterpret_cast<float*>(smem + kOffRope);
     uint32_t* xq = reinterpret_cast<uint32_t*>(smem + kHeader);
@@ -475,6 +477,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], kWarps);
         }
+        mbar_init(xbar, 1);
         fence_mbar_init();
     }
     for (int i = tid; i < P.recv_bytes / 4; i += kThreads) sums[i] = 0.f;
@@ -525,18 +528,35 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
         // ------------------------------------------------------------- consumers
         if (P.use_pdl) pdl_wait();
         float* rs = red;   // scratch for the prologue reductions
-        // (1) this CTA's columns of x into shared memory as fp32 (RMSNorm applied: the
-        // sum of squares runs over the whole vector), gathering max |x| of the half
-        const int K4 = P.K / 4, h0 = k0 / 4, h1 = (k0 + KR) / 4;
+        // (1) this CTA's columns of x into shared memory with one bulk copy (x is
+        // 16-byte aligned and the half starts on a 32-column step), then RMSNorm (its sum
+        // of squares runs over the whole vector) and max |x| of the CTA's columns
+        const int K4 = P.K / 4, h0 = k0 / 4, h1 = (k0 + KR) / 4, nh = h1 - h0;
         float4* xf = reinterpret_cast<float4*>(xq);
         const float4* x4 = reinterpret_cast<const float4*>(P.x);
+        if (tid == 0 && KR > 0) {
+            mbar_arrive_expect_tx(xbar, (uint32_t)KR * 4u);
+            bulk_g2s(xf, P.x + k0, (uint32_t)KR * 4u, xbar, policy_evict_last());
+        }
+        if (KR > 0 && !mbar_wait(xbar, 0, kWaitPolls) && tid == 0) record_device_error(DEVERR_FULL_WAIT);
         float mx = 0.f;
         if (PRO == gemv::PRO_RMSNORM) {
             float ss = 0.f;
-            for (int i = tid; i < K4; i += kCons) {
-                const float4 v = x4[i];
-                if (i >= h0 && i < h1) xf[i - h0] = v;
+            for (int i = tid; i < nh; i += kCons) {
+                const float4 v = xf[i];
                 ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+            }
+            // the other CTA's columns, from global memory, 8 loads in flight per thread
+            for (int j0 = tid; j0 < K4 - nh; j0 += 8 * kCons) {
+                float4 v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int jj = j0 + j * kCons;
+                    v[j] = jj < K4 - nh ? x4[jj < h0 ? jj : jj + nh] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    ss = fmaf(v[j].x, v[j].x, fmaf(v[j].y, v[j].y, fmaf(v[j].z, v[j].z, fmaf(v[j].w, v[j].w, ss))));
             }
             ss = gemv::warp_sum(ss);
             if (lane == 0) rs[warp] = ss;
@@ -546,16 +566,28 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
             for (int w = 0; w < kWarps; ++w) tot += rs[w];
             const float inv = 1.0f / sqrtf(tot / (float)P.K + P.eps);
             const float4* w4 = reinterpret_cast<const float4*>(P.norm_w) + h0;
-            for (int i = tid; i < h1 - h0; i += kCons) {
-                const float4 a = xf[i], w = w4[i];
-                const float4 v = make_float4(a.x * inv * w.x, a.y * inv * w.y, a.z * inv * w.z, a.w * inv * w.w);
-                xf[i] = v;
-                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+            for (int i0 = tid; i0 < nh; i0 += 8 * kCons) {
+                float4 w[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i = i0 + j * kCons;
+                    w[j] = i < nh ? w4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int i = i0 + j * kCons;
+                    if (i < nh) {
+                        const float4 a = xf[i];
+                        const float4 v = make_float4(a.x * inv * w[j].x, a.y * inv * w[j].y, a.z * inv * w[j].z,
+                                                     a.w * inv * w[j].w);
+                        xf[i] = v;
+                        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+                    }
+                }
             }
         } else {
-            for (int i = tid; i < h1 - h0; i += kCons) {
-                const float4 v = x4[h0 + i];
-                xf[i] = v;
+            for (int i = tid; i < nh; i += kCons) {
+                const float4 v = xf[i];
                 mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
             }
         }
