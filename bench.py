@@ -170,39 +170,74 @@ def gemv_shapes(spec):
             (spec.vocab, spec.hidden, 1)]
 
 
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture per
+# shape, bytes per launch) of the tiled tensor-core GEMV, and a hash of the kernel
+# sources it was taken with: a changed kernel reports traffic as unknown (null).
+GEMV_TRAFFIC_SRC_SHA = "e485a694e121188f"
+GEMV_TRAFFIC = {"q6_k_t:10240x8192": 69004032, "q6_k_t:8192x8192": 55123200, "q6_k_t:28672x8192": 196366848,
+                "q6_k_t:8192x28672": 195896320, "q6_k_t:128256x8192": 865172480, "q8_0_t:6144x4096": 26791424,
+                "q8_0_t:4096x4096": 17878528, "q8_0_t:14336x4096": 62471680, "q8_0_t:4096x14336": 62529280,
+                "q8_0_t:128256x4096": 561447936}
+
+
+def gemv_sources_sha():
+    import hashlib
+    h = hashlib.sha256()
+    d = os.path.join(os.path.dirname(os.path.abspath(__file__)), "quantized_weight_gemv_block_b200", "csrc")
+    for f in ("qmma.cuh", "qmma.cu", "blocks.cuh", "common.cuh", "gemv.cuh"):
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def measure_gemv_roofline(ntx, model, spec, stream, iters=3):
-    """Time every decode GEMV of one step on its own (same weights, same shapes, same
-    stream) with CUDA events: the dominant kernel's achieved HBM bandwidth.  Only
-    HBM-resident layers count; streamed layers are bound by the host link, which is
-    reported on its own."""
+    """Time every decode GEMV of one step on its own (the same weights and shapes as
+    the step, plain store epilogue, same stream) with CUDA events.  Per shape: bytes
+    per launch (packed weights + x + y) and the average launch time, cycling over the
+    layers so no launch finds its weights in L2.  The aggregate over a step's launches
+    is the dominant kernel's achieved HBM bandwidth.  Only HBM-resident layers count;
+    streamed layers are bound by the host link, which is reported on its own."""
     import torch
     import synth
     x = torch.randn(max(spec.hidden, spec.ffn, spec.q_dim), device="cuda")
     y = torch.empty(max(spec.vocab, spec.ffn, spec.qkv_rows), device="cuda")
-    launches = []
-    for t in model.layers[:model.n_resident]:
-        launches.append((t["w_qkv"], spec.qkv_rows, spec.hidden))
-        launches.append((t["w_o"], spec.hidden, spec.q_dim))
-        launches.append((t["w_gate"], spec.ffn, spec.hidden))
-        launches.append((t["w_up"], spec.ffn, spec.hidden))
-        launches.append((t["w_down"], spec.hidden, spec.ffn))
-    launches.append((model.output, spec.vocab, spec.hidden))
-    nbytes = sum(r * synth.row_bytes(spec.qtype, c) + 4 * (c + r) for _, r, c in launches)
+    res = model.layers[:model.n_resident]
+    shapes = [("qkv", [t["w_qkv"] for t in res], spec.qkv_rows, spec.hidden),
+              ("o", [t["w_o"] for t in res], spec.hidden, spec.q_dim),
+              ("gate_up", [t[k] for t in res for k in ("w_gate", "w_up")], spec.ffn, spec.hidden),
+              ("down", [t["w_down"] for t in res], spec.hidden, spec.ffn),
+              ("lm_head", [model.output], spec.vocab, spec.hidden)]
     q = lib_qtype(spec)
+    fmt = {0: "q8_0", 1: "q4_0", 2: "q4_k", 3: "q6_k"}[spec.qtype] + ("_t" if spec.tiled else "")
+    sha = gemv_sources_sha()
+    out, tot_bytes, tot_ms, tot_launch, tot_traffic = {}, 0.0, 0.0, 0, 0.0
     with torch.cuda.stream(stream):
-        for W, r, c in launches[:20]:
-            ntx.ntx_gemv_q(q, W, r, c, x, y, stream.cuda_stream)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        e0.record(stream)
-        for _ in range(iters):
-            for W, r, c in launches:
+        for name, mats, r, c in shapes:
+            per = r * synth.row_bytes(spec.qtype, c) + 4 * (c + r)
+            n = max(len(mats) * iters, 4)
+            for W in mats[:4]:
                 ntx.ntx_gemv_q(q, W, r, c, x, y, stream.cuda_stream)
-        e1.record(stream)
-        torch.cuda.synchronize()
-    ms = e0.elapsed_time(e1) / (iters * len(launches))
-    per_launch = nbytes / len(launches)
-    return per_launch / (ms * 1e-3) / 1e9, per_launch, ms
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for i in range(n):
+                ntx.ntx_gemv_q(q, mats[i % len(mats)], r, c, x, y, stream.cuda_stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / n
+            launches = len(mats)    # launches of this shape in one decode step
+            tr = GEMV_TRAFFIC.get(f"{fmt}:{r}x{c}") if sha == GEMV_TRAFFIC_SRC_SHA else None
+            out[name] = {"shape": f"{fmt}:{r}x{c}", "bytes_per_launch": per, "avg_launch_us": ms * 1e3,
+                         "achieved_gbs": per / (ms * 1e-3) / 1e9, "launches_per_step": launches,
+                         "traffic_per_launch": tr}
+            tot_bytes += per * launches
+            tot_ms += ms * launches
+            tot_launch += launches
+            tot_traffic = None if (tr is None or tot_traffic is None) else tot_traffic + tr * launches
+    agg = {"achieved": tot_bytes / (tot_ms * 1e-3) / 1e9, "bytes_per_launch": tot_bytes / tot_launch,
+           "avg_launch_us": tot_ms * 1e3 / tot_launch,
+           "traffic": None if tot_traffic is None else tot_traffic / tot_launch}
+    return agg, out
 
 
 def run_decode_bench(args, rank, world, local):
@@ -494,10 +529,12 @@ def main():
         line["host_link"] = {"h2d_bytes_per_step": r["h2d_bytes"], "achieved_gbs": r["h2d_gbs"],
                              "measured_pinned_h2d_gbs": r["h2d_peak_gbs"], "frac": r["h2d_gbs"] / r["h2d_peak_gbs"]}
     if rank == 0:
-        gbs, per_launch, ms = measure_gemv_roofline(ntx, model, spec, stream)
-        line["roofline"] = {"bound": "hbm", "kernel": "gemv_kernel<%s>" % config["format"], "achieved": gbs,
-                            "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": gbs / peak,
-                            "traffic": None, "bytes_per_launch": per_launch, "avg_launch_us": ms * 1e3}
+        agg, per_shape = measure_gemv_roofline(ntx, model, spec, stream)
+        line["roofline"] = {"bound": "hbm", "kernel": "qmma_kernel<%s> (all GEMV launches of one step)" % config["format"],
+                            "achieved": agg["achieved"], "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
+                            "frac": agg["achieved"] / peak, "traffic": agg["traffic"],
+                            "bytes_per_launch": agg["bytes_per_launch"], "avg_launch_us": agg["avg_launch_us"]}
+        line["gemv_shapes"] = per_shape
         if not args.no_extras:
             line["gemv_q8_0_4096x4096"] = {"tiled": gemv_bench(ntx, tiled=True), "gguf": gemv_bench(ntx, tiled=False)}
         if not args.no_cpu_baseline:

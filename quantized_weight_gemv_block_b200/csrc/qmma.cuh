@@ -120,6 +120,22 @@ __device__ __forceinline__ uint32_t cluster_size()
     return r;
 }
 
+__device__ __forceinline__ void cluster_arrive()
+{
+    asm volatile("barrier.cluster.arrive.release;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_wait()
+{
+    asm volatile("barrier.cluster.wait.acquire;" ::: "memory");
+}
+
+// Arrive on named barrier `id` without waiting (the waiting side uses named_bar_sync).
+__device__ __forceinline__ void named_bar_arrive(int id, int threads)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
 // Barrier of all threads of the cluster (of the CTA alone when the cluster is one CTA).
 __device__ __forceinline__ void cluster_sync(uint32_t csize)
 {
@@ -472,20 +488,23 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
     const int k0 = u0 * T::UK, KR = (u1 - u0) * T::UK;
     const int CE = P.chunk_elems, NCH = (KR + CE - 1) / CE;
 
-    if (tid == 0) {
-        for (int s = 0; s < P.n_stages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kWarps);
-        }
-        mbar_init(xbar, 1);
-        fence_mbar_init();
-    }
-    for (int i = tid; i < P.recv_bytes / 4; i += kThreads) sums[i] = 0.f;
-    // both CTAs initialised before either touches the other's shared memory
-    cluster_sync(csize);
-    if (P.use_pdl) pdl_launch_dependents();
-
+    // Start-up: the producer warp initialises the barriers and starts streaming at once;
+    // the consumers zero the pair's sums and wait for the barriers (and, in a pair, for
+    // both CTAs: cluster barrier phase 0, which the producer joins without waiting).
     if (warp == kProducer) {
+        if (lane == 0) {
+            for (int s = 0; s < P.n_stages; ++s) {
+                mbar_init(&full[s], 1);
+                mbar_init(&empty[s], kWarps);
+            }
+            mbar_init(xbar, 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+        if (csize == 1)
+            named_bar_arrive(2, kThreads);
+        else
+            cluster_arrive();
         // ------------------------------------------------------------- producer
         // (weights do not depend on earlier kernels, so streaming starts at once)
         if (lane == 0) {
@@ -524,9 +543,21 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
             }
         }
         __syncwarp();
+        if (csize == 2) cluster_wait();   // phase 0, joined at the start
     } else {
         // ------------------------------------------------------------- consumers
-        if (P.use_pdl) pdl_wait();
+        for (int i = tid; i < P.recv_bytes / 4; i += kCons) sums[i] = 0.f;
+        if (csize == 1) {
+            named_bar_sync(2, kThreads);
+        } else {
+            // both CTAs initialised before either touches the other's shared memory
+            cluster_arrive();
+            cluster_wait();
+        }
+        if (P.use_pdl) {
+            pdl_launch_dependents();
+            pdl_wait();
+        }
         float* rs = red;   // scratch for the prologue reductions
         // (1) this CTA's columns of x into shared memory with one bulk copy (x is
         // 16-byte aligned and the half starts on a 32-column step), then RMSNorm (its sum
