@@ -153,9 +153,14 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         fence_mbar_init();
     }
     __syncthreads();
+    // Programmatic dependent launch: the consumers wait for the previous kernel (which
+    // writes q and the K / V row at the new position) before reading anything; the
+    // producer waits only before the first stage that holds that row, since older rows
+    // were written by earlier steps (the step word was written before the first kernel
+    // that launches early).
     if (a.use_pdl) {
         pdl_launch_dependents();
-        pdl_wait();
+        if (warp != kProducerWarp) pdl_wait();
     }
     const int g = blockIdx.x / a.n_split, sp = blockIdx.x % a.n_split;
     const int n_ctx = a.pos_dev ? (*a.pos_dev + 1) : a.n_ctx;
@@ -171,7 +176,12 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         const uint64_t pol = policy_evict_first();
         int s = 0;
         uint32_t ph = 0;
+        bool waited = !a.use_pdl;
         for (int i = 0; i < nsub && lane == 0; ++i) {
+            if (!waited && t0 + (i + 1) * kSub > n_ctx - 1) {
+                pdl_wait();
+                waited = true;
+            }
             if (!mbar_wait(&empty[s], ph ^ 1u, kPolls)) {
                 record_device_error(DEVERR_EMPTY_WAIT);
                 // the stages issued last must land before the CTA may exit
