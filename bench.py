@@ -171,7 +171,7 @@ def gemv_shapes(spec):
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture per
-# shape, bytes per launch) of the tiled tensor-core GEMV, and a hash of the kernel
+# shape, bytes per launch) of the tiled GEMV, and a hash of the kernel
 # sources it was taken with: a changed kernel reports traffic as unknown (null).
 GEMV_TRAFFIC_SRC_SHA = "e485a694e121188f"
 GEMV_TRAFFIC = {"q6_k_t:10240x8192": 69004032, "q6_k_t:8192x8192": 55123200, "q6_k_t:28672x8192": 196366848,

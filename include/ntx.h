@@ -70,15 +70,16 @@ typedef enum ntx_qtype {
     NTX_Q4_K = 2,
     NTX_Q6_K = 3,
     /* Tiled layouts (flag NTX_TILED): the same information in the same bytes per
-     * row, reordered for the tensor-core GEMV.  Produced from the GGUF-style
+     * row, reordered for the streaming GEMV.  Produced from the GGUF-style
      * layout by ntx_repack_q, lossless.  Rows come in groups of 16 (a tiled
      * tensor has a multiple of 16 rows); a group is a run of units along the
      * row, unit u covering columns [u UK, (u + 1) UK) of the group's 16 rows in
      * 16 x the GGUF-style bytes of UK columns (UK = 32 for Q8_0 / Q4_0: one
      * block; 256 for Q4_K / Q6_K: one superblock).  Inside a unit the codes of
-     * each 32-column step sit in the order in which lane 4 gid + tig of a warp
-     * takes them as the A operand of one m16n8k32 integer MMA (rows gid and
-     * gid + 8, columns 4 tig .. 4 tig + 3 and 16 + 4 tig .. 16 + 4 tig + 3),
+     * each 32-column step sit in "lane" order: lane 4 gid + tig holds rows gid
+     * and gid + 8 at columns 4 tig .. 4 tig + 3 and 16 + 4 tig .. 16 + 4 tig + 3
+     * (the A fragment of an m16n8k32 integer MMA; the four lanes of a gid are
+     * adjacent, so one gid's two rows over the whole step are contiguous bytes),
      * followed by the unit's scales:
      *   NTX_Q8_0_T  unit 544 B: 32 lanes x 16 int8 codes | 8 x (d[r], d[r+8])
      *   NTX_Q4_0_T  unit 288 B: 32 lanes x 8 B (two 4-bit codes per byte) | 8 x (d[r], d[r+8])
@@ -122,10 +123,11 @@ ntx_status ntx_device_error(uint32_t* code);
  *   x    device fp32 [cols];  y  device fp32 [rows] (must not overlap x or W)
  * Accumulation is fp32; results match the exact dot product to a normwise
  * relative error far below 2e-3.  rows >= 1 (a multiple of 16 for a tiled
- * qtype); cols a multiple of the block size.  Tiled layouts run on the integer
- * tensor cores (x taken as 24-bit fixed point relative to max |x|); GGUF-style
- * rows whose byte length is a multiple of 16 take the bulk-copy CUDA-core
- * pipeline; other shapes take a simpler kernel. */
+ * qtype); cols a multiple of the block size.  Tiled layouts take integer dots
+ * of the codes with x as 24-bit fixed point (relative to max |x|) by dp4a on the
+ * CUDA cores (NTX_GEMV_CORE=tc selects integer MMAs instead; same results up to
+ * fp32 rounding order); GGUF-style rows whose byte length is a multiple of 16
+ * take the bulk-copy fp32 CUDA-core pipeline; other shapes a simpler kernel. */
 ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t cols, const float* x, float* y,
                       void* stream);
 

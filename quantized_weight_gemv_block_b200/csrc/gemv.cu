@@ -1,5 +1,5 @@
 // gemv.cu - host side of the quantized GEMV (launch shaping, C ABI; the tiled
-// layouts go to the tensor-core kernel of qmma.cu), the simple kernel for rows
+// layouts go to the integer-dot kernel of qmma.cu), the simple kernel for rows
 // that are not 16-byte multiples, and the dequantization kernel.
 #include <algorithm>
 #include <mutex>

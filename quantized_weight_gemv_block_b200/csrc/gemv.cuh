@@ -1,5 +1,5 @@
 // gemv.cuh - block-quantized GEMV for sm_100a (batch 1) on the GGUF-style
-// layouts (the tiled layouts run on the tensor cores, qmma.cuh), with optional fused
+// layouts (the tiled layouts take integer dots, qmma.cuh), with optional fused
 // prologue (RMSNorm of the input) and epilogues (residual add, SwiGLU of a
 // gate/up row pair, RoPE + fp16 KV-cache append for a fused QKV projection).
 //
@@ -71,7 +71,7 @@ struct Params {
     int stage_bytes;
     int x_bytes;
     int use_pdl;
-    int recv_bytes;       // tensor-core GEMV: bytes of the per-group row sums of a CTA pair
+    int recv_bytes;       // tiled GEMV: bytes of the per-group row sums of a CTA pair
     // multiplier that lets a shift run as an integer multiply on the FMA pipe
     // (v >> 8 == umulhi(v, 2^24)); passed in so it stays a multiply
     uint32_t m24;

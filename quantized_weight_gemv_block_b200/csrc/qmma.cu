@@ -1,5 +1,5 @@
-// qmma.cu - host side of the tensor-core GEMV for the tiled layouts (launch
-// shaping) and the repack kernel GGUF-style -> tiled.
+// qmma.cu - host side of the GEMV for the tiled layouts (launch shaping, the choice
+// of CUDA-core or tensor-core units) and the repack kernel GGUF-style -> tiled.
 #include <algorithm>
 #include <cstdlib>
 #include <mutex>
@@ -157,7 +157,7 @@ bool shape(Params& P, int n_clusters, int csize, int n_mats)
 }
 
 // Clusters of `csize` CTAs (one per SM) that fit on the device at once, per kernel.
-template <int QT, int EPI, int PRO>
+template <int QT, int EPI, int PRO, int CORE>
 int max_clusters(int csize)
 {
     static std::once_flag once[3];
@@ -175,7 +175,7 @@ int max_clusters(int csize)
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         int c = 0;
-        if (cudaOccupancyMaxActiveClusters(&c, qmma_kernel<QT, EPI, PRO>, &cfg) != cudaSuccess || c < 1) {
+        if (cudaOccupancyMaxActiveClusters(&c, qmma_kernel<QT, EPI, PRO, CORE>, &cfg) != cudaSuccess || c < 1) {
             cudaGetLastError();
             c = std::max(1, num_sms() / csize);
         }
@@ -198,16 +198,16 @@ inline int pick_cluster_size(int M, int K)
     return (M / 16 < 6 * num_sms() && K >= 16384) ? 2 : 1;
 }
 
-template <int QT, int EPI, int PRO>
+template <int QT, int EPI, int PRO, int CORE>
 ntx_status launch_t(Params P, cudaStream_t s)
 {
-    auto kern = qmma_kernel<QT, EPI, PRO>;
+    auto kern = qmma_kernel<QT, EPI, PRO, CORE>;
     static std::once_flag once[4][4][2];
     std::call_once(once[QT & 3][EPI][PRO], [&] {
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
     });
     const int csize = pick_cluster_size(P.M, P.K);
-    const int n_clusters = std::max(1, std::min(max_clusters<QT, EPI, PRO>(csize), P.M / 16));
+    const int n_clusters = std::max(1, std::min(max_clusters<QT, EPI, PRO, CORE>(csize), P.M / 16));
     if (!shape<QT>(P, n_clusters, csize, EPI == gemv::EPI_SWIGLU ? 2 : 1))
         return fail(NTX_EUNSUPPORTED, "gemv: row too long for the shared-memory pipeline");
     const int smem = kHeader + P.x_bytes + P.n_stages * P.stage_bytes + P.recv_bytes + 128;
@@ -226,18 +226,37 @@ ntx_status launch_t(Params P, cudaStream_t s)
     cfg.attrs = attr;
     cfg.numAttrs = P.use_pdl ? 2 : 1;
     const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, P);
-    if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("gemv (tensor cores) launch: ") + cudaGetErrorString(e));
+    if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("gemv (tiled) launch: ") + cudaGetErrorString(e));
     return NTX_OK;
+}
+
+// Which units reduce the codes: dp4a on the CUDA cores (1, the default) or the integer
+// tensor cores (0).  Measured on B200 (event-timed, inputs larger than L2): Q6_K
+// 28672 x 8192 5.10 TB/s dp4a against 5.11 MMA, 8192 x 28672 5.11 against 5.05, Q8_0
+// 32768 x 4096 5.07 against 5.18, Q4_0 57344 x 4096 3.48 against 2.87, Q4_K 3.50 against
+// 3.69.  NTX_GEMV_CORE=tc / dp4a overrides the choice (a tuning override).
+inline int pick_core()
+{
+    const char* env = std::getenv("NTX_GEMV_CORE");
+    if (env && env[0] == 't') return 0;
+    if (env && env[0] == 'd') return 1;
+    return 1;
+}
+
+template <int QT, int EPI, int PRO>
+ntx_status launch_c(const Params& P, cudaStream_t s)
+{
+    return pick_core() == 0 ? launch_t<QT, EPI, PRO, 0>(P, s) : launch_t<QT, EPI, PRO, 1>(P, s);
 }
 
 template <int EPI, int PRO>
 ntx_status launch_q(int qtype, const Params& P, cudaStream_t s)
 {
     switch (qtype) {
-    case NTX_Q8_0_T: return launch_t<NTX_Q8_0_T, EPI, PRO>(P, s);
-    case NTX_Q4_0_T: return launch_t<NTX_Q4_0_T, EPI, PRO>(P, s);
-    case NTX_Q4_K_T: return launch_t<NTX_Q4_K_T, EPI, PRO>(P, s);
-    case NTX_Q6_K_T: return launch_t<NTX_Q6_K_T, EPI, PRO>(P, s);
+    case NTX_Q8_0_T: return launch_c<NTX_Q8_0_T, EPI, PRO>(P, s);
+    case NTX_Q4_0_T: return launch_c<NTX_Q4_0_T, EPI, PRO>(P, s);
+    case NTX_Q4_K_T: return launch_c<NTX_Q4_K_T, EPI, PRO>(P, s);
+    case NTX_Q6_K_T: return launch_c<NTX_Q6_K_T, EPI, PRO>(P, s);
     default: return fail(NTX_EINVAL, "unknown tiled qtype");
     }
 }

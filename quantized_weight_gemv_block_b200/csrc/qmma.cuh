@@ -1,19 +1,17 @@
-// qmma.cuh - block-quantized GEMV for the tiled layouts on the integer tensor
-// cores (batch 1).
+// qmma.cuh - block-quantized GEMV for the tiled layouts (batch 1).
 //
 // The GEMV kernel of the ntransformer news summary ("Arquitectura y estructura
 // del código": cuda/ holds the GEMV kernels) for B200.  Batch-1 GEMV streams every
 // weight once, so the work per weight must stay far below the SM's issue rate to
 // keep HBM busy.  Dequantizing each weight to fp32 and multiplying costs several
-// instructions per weight; here the packed codes go to the tensor cores as they are:
+// instructions per weight; here the packed codes are multiplied as integers:
 //  * the input vector x is turned once per CTA into 24-bit fixed point,
 //    x_int = rint(x 2^S) with |x_int| < 2^22, written as three balanced signed
 //    8-bit limbs, x_int = l0 + 2^8 l1 + 2^16 l2 (S from max |x|, a power of two);
-//  * one m16n8k32 integer MMA takes a 16-row x 32-column block of codes (int8 for
-//    Q8_0, unsigned 4- or 6-bit codes for the others) as its A operand and the
-//    limbs of x as its B operand: the 8 columns of B hold limb l of x's 32 values
-//    (or, for Q6_K, of the 16 values of one 16-column sub-block each), so each C
-//    column is an exact integer partial dot product of one limb;
+//  * the codes (int8 for Q8_0, unsigned 4- or 6-bit codes for the others, unpacked
+//    to bytes with a few logic ops per word) are dotted with each limb, four bytes
+//    at a time, by dp4a on the CUDA cores (CORE 1, the default): every partial sum is
+//    an exact integer;
 //  * the format's per-block scale (fp16 d, int8 or 6-bit sub-block scales, the
 //    Q4_K mins, the code offsets 8 and 32) is applied to those integers, in
 //    integer arithmetic where it is exact, in fp32 once per block otherwise;
@@ -21,8 +19,12 @@
 //    by 2^-S, exactly.
 // The products are exact; x carries 23 bits (relative to max |x|) where fp32
 // carries 24; sums round at fp32 once per block or superblock.
+// CORE 0 does the same integer dots with one m16n8k32 integer MMA per 16 x 32 block
+// (codes as A, the limbs as the 8 columns of B); it is kept as a measured
+// alternative (NTX_GEMV_CORE=tc): on B200 the dp4a path streams as fast or faster on
+// every decode shape, so no tensor core is needed for batch 1.
 //
-// Structure (one CTA per SM, 8 consumer warps, a producer and a reducer warp):
+// Structure (one CTA per SM, 8 consumer warps and a producer warp):
 //  * the grid is made of clusters of 1 or 2 CTAs; a cluster owns a contiguous
 //    range of 16-row groups.  For matrices with few groups per SM the two CTAs of
 //    a pair split the columns in halves (so the groups spread over 74 pairs
@@ -36,11 +38,10 @@
 //    in the tiled layout, streamed by the producer warp with one 1-D bulk copy
 //    (cp.async.bulk, L2 evict-first) into a ring of shared-memory stages guarded
 //    by mbarriers;
-//  * each consumer warp takes every 8th unit (32 or 256 columns) of a stage; per
-//    32-column step a lane loads its two rows' codes with one shared-memory load,
-//    unpacks 4-/6-bit codes into bytes with a few logic ops, issues one MMA and
-//    folds the step's integers into its row accumulators;
-//  * row totals are reduced over the 4 lanes of a quad (limb weights) and over the
+//  * each consumer warp takes every 8th unit (32 or 256 columns) of a stage; the
+//    shared-memory reads of a warp are contiguous or spread over distinct banks
+//    (lane units for Q8_0, row-pair units for the others, below);
+//  * row totals are reduced over the threads of a warp that share rows and over the
 //    8 warps through shared memory in a fixed order (a barrier of the consumer
 //    warps per group: measured faster on B200 than handing the sums to a separate
 //    reducer warp through mbarriers) into the pair's sums; after the cluster
@@ -163,14 +164,19 @@ __device__ __forceinline__ void red_add_cluster(uint32_t addr, float v)
 
 // ------------------------------------------------------------------ x staging
 // Step u (columns 32u .. 32u + 31) of x occupies 32 words at xq + 32u:
-//  words 8l + w (l = 0..2, w = 0..7): limb l of columns 32u + 4w .. + 3, one byte each;
+//  words 8l + w (l = 0..2, w = 0..7): limb l of columns 32u + 4w .. + 3, one byte each
+//    (PAIRED, the CUDA-core lane units: word 8l + 2(w mod 4) + w / 4 instead, so the two
+//    words a lane needs, columns 4 tig.. and 16 + 4 tig.., are adjacent);
 //  words 24..31: per-column sums of the limbs over what one C column covers
 //    (Q6_K: words 24 + 4h + l = sum of limb l over the 16 columns of half h, words
 //    27 and 31 zero; other formats: word 24 + l = sum of limb l over the 32 columns,
 //    words 27..31 zero).  Lane tig reads its two C columns' sums at 24 + 2 tig.
+// For the CUDA-core row-pair units every word index i of step u is stored at
+// i XOR 8 (u mod 4) (sx below): the four quarter-warps of a warp read the same words
+// of four consecutive steps, which then fall in four different bank groups.
 
-template <bool HALVES>
-__device__ __forceinline__ void stage_x_step(uint32_t* xs, int w, bool ok, float4 v, float two_s)
+template <bool HALVES, bool PAIRED>
+__device__ __forceinline__ void stage_x_step(uint32_t* xs, int w, bool ok, float4 v, float two_s, int sx)
 {
     // z = x_int + 0x8080: bytes 0 and 1 of z are the low limbs + 128, z >> 16 the top limb
     const float mag = 12582912.0f;   // 1.5 * 2^23: fmaf rounds x 2^S to an integer in its low bits
@@ -193,28 +199,29 @@ __device__ __forceinline__ void stage_x_step(uint32_t* xs, int w, bool ok, float
     }
     __syncwarp();   // every lane of the step has read its floats before any limb word lands
     if (ok) {
-        xs[w] = w0;
-        xs[8 + w] = w1;
-        xs[16 + w] = w2;
+        const int wp = PAIRED ? 2 * (w & 3) + (w >> 2) : w;
+        xs[wp ^ sx] = w0;
+        xs[(8 + wp) ^ sx] = w1;
+        xs[(16 + wp) ^ sx] = w2;
         if (HALVES) {
             if ((w & 3) == 0) {
                 const int h = w >> 2;
-                xs[24 + 4 * h] = (uint32_t)s0;
-                xs[25 + 4 * h] = (uint32_t)s1;
-                xs[26 + 4 * h] = (uint32_t)s2;
-                xs[27 + 4 * h] = 0u;
+                xs[(24 + 4 * h) ^ sx] = (uint32_t)s0;
+                xs[(25 + 4 * h) ^ sx] = (uint32_t)s1;
+                xs[(26 + 4 * h) ^ sx] = (uint32_t)s2;
+                xs[(27 + 4 * h) ^ sx] = 0u;
             }
         } else {
             if (w == 0) {
-                xs[24] = (uint32_t)s0;
-                xs[25] = (uint32_t)s1;
-                xs[26] = (uint32_t)s2;
+                xs[24 ^ sx] = (uint32_t)s0;
+                xs[25 ^ sx] = (uint32_t)s1;
+                xs[26 ^ sx] = (uint32_t)s2;
             } else if (w == 1) {
-                xs[27] = 0u;
-                xs[28] = 0u;
-                xs[29] = 0u;
-                xs[30] = 0u;
-                xs[31] = 0u;
+                xs[27 ^ sx] = 0u;
+                xs[28 ^ sx] = 0u;
+                xs[29 ^ sx] = 0u;
+                xs[30 ^ sx] = 0u;
+                xs[31 ^ sx] = 0u;
             }
         }
     }
@@ -268,6 +275,25 @@ __device__ __forceinline__ void b_frag(const uint32_t* xs, const Lane& L, uint32
 __device__ __forceinline__ float2 d_pair(const uint8_t* p)
 {
     return __half22float2(*reinterpret_cast<const __half2*>(p));
+}
+
+// Q4_K: the 32 six-bit scales / mins of rows gid and gid + 8 of a unit, one word per
+// step m: byte 0 scale row gid, 1 scale row gid + 8, 2 min row gid, 3 min row gid + 8.
+__device__ __forceinline__ void q4k_scale_words(const uint8_t* U, int gid, uint32_t (&S)[8])
+{
+    const uint8_t* v = U + 2048 + 24 * gid;    // 8-byte aligned
+    const uint2 na = *reinterpret_cast<const uint2*>(v);
+    const uint2 nb = *reinterpret_cast<const uint2*>(v + 8);
+    const uint2 hw = *reinterpret_cast<const uint2*>(v + 16);
+    const uint32_t n4[4] = {na.x, na.y, nb.x, nb.y};
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const uint32_t lo = (m & 1 ? (n4[m >> 1] >> 4) : n4[m >> 1]) & 0x0F0F0F0Fu;
+        const uint32_t h = m < 4 ? hw.x : hw.y;
+        const int sh = 2 * (m & 3);
+        const uint32_t hi = (sh <= 4 ? (h << (4 - sh)) : (h >> (sh - 4))) & 0x30303030u;
+        S[m] = lo | hi;
+    }
 }
 
 // ------------------------------------------------------------------ units
@@ -371,22 +397,8 @@ struct Unit<NTX_Q4_K_T> {
     static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
                                                float& acc1)
     {
-        // the 32 six-bit scales / mins of this lane's two rows, one word per step:
-        // byte 0 scale row gid, 1 scale row gid + 8, 2 min row gid, 3 min row gid + 8
-        const uint8_t* v = U + 2048 + 24 * L.gid;    // 8-byte aligned
-        const uint2 na = *reinterpret_cast<const uint2*>(v);
-        const uint2 nb = *reinterpret_cast<const uint2*>(v + 8);
-        const uint2 hw = *reinterpret_cast<const uint2*>(v + 16);
         uint32_t S[8];
-        const uint32_t n4[4] = {na.x, na.y, nb.x, nb.y};
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const uint32_t lo = (m & 1 ? (n4[m >> 1] >> 4) : n4[m >> 1]) & 0x0F0F0F0Fu;
-            const uint32_t h = m < 4 ? hw.x : hw.y;
-            const int sh = 2 * (m & 3);
-            const uint32_t hi = (sh <= 4 ? (h << (4 - sh)) : (h >> (sh - 4))) & 0x30303030u;
-            S[m] = lo | hi;
-        }
+        q4k_scale_words(U, L.gid, S);
         int p0 = 0, p1 = 0, q0 = 0, q1 = 0, o0 = 0, r0 = 0;
         const uint32_t M = 0x0F0F0F0Fu;
 #pragma unroll
@@ -413,6 +425,238 @@ struct Unit<NTX_Q4_K_T> {
         const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
         acc0 = fmaf(d.x, fmaf(256.f, (float)p1, (float)p0), fmaf(-dm.x, (float)o0, acc0));
         acc1 = fmaf(d.y, fmaf(256.f, (float)q1, (float)q0), fmaf(-dm.y, (float)r0, acc1));
+    }
+};
+
+// ------------------------------------------------------------------ CUDA-core units
+// The same tiled bytes, reduced on the CUDA cores with dp4a (four 8-bit products and
+// an int32 add per instruction).  Integer partial sums (exact) are weighted by the
+// sub-block scales in int32 and recombined over the limbs (1, 2^8, 2^16) in fp32 once
+// per block or superblock.
+//
+// Lane units (Q8_0): each lane takes the 16 bytes the MMA would give it as its A
+// fragment (a warp's loads are contiguous and conflict-free): row gid at columns
+// 4 tig .. + 3 and 16 + 4 tig .. + 3 and the same columns of row gid + 8, dotted with
+// its 8 columns of each of the three limbs.  The lane's two limb words of a step sit
+// side by side (the PAIRED x layout).  acc0 / acc1 end as this lane's share of rows
+// gid / gid + 8 in units of x_int, summed over the quad afterwards.
+
+// dot of one code word with one limb word, added to c
+__device__ __forceinline__ int dp4(uint32_t a, uint32_t x, int c)
+{
+    return __dp4a((int)a, (int)x, c);
+}
+
+// the limbs' integer sums c0 + 2^8 c1 + 2^16 c2 in fp32
+__device__ __forceinline__ float limbs_f(int c0, int c1, int c2)
+{
+    return fmaf((float)c2, 65536.f, fmaf((float)c1, 256.f, (float)c0));
+}
+
+// limb words of a step for lane tig: X[l].x = columns 4 tig.., X[l].y = 16 + 4 tig..
+__device__ __forceinline__ void x_words(const uint32_t* xs, int tig, uint2 (&X)[3])
+{
+#pragma unroll
+    for (int l = 0; l < 3; ++l) X[l] = *reinterpret_cast<const uint2*>(xs + 8 * l + 2 * tig);
+}
+
+template <int QT>
+struct Dot;
+
+template <>
+struct Dot<NTX_Q8_0_T> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
+                                               float& acc1)
+    {
+        const uint4 a = *reinterpret_cast<const uint4*>(U + 16 * L.lane);
+        uint2 X[3];
+        x_words(xs, L.tig, X);
+        int c0[3], c1[3];
+#pragma unroll
+        for (int l = 0; l < 3; ++l) {
+            c0[l] = dp4(a.z, X[l].y, dp4(a.x, X[l].x, 0));
+            c1[l] = dp4(a.w, X[l].y, dp4(a.y, X[l].x, 0));
+        }
+        const float2 d = d_pair(U + 512 + 4 * L.gid);
+        acc0 = fmaf(d.x, limbs_f(c0[0], c0[1], c0[2]), acc0);
+        acc1 = fmaf(d.y, limbs_f(c1[0], c1[1], c1[2]), acc1);
+    }
+};
+
+// Row-pair units (Q4_0, Q4_K, Q6_K): a thread takes the bytes of the four lanes of
+// one gid in one step, i.e. rows gid and gid + 8 over all 32 columns of the step, so
+// each sub-block's dp4a chain runs over its 16 or 32 columns before the one scale
+// multiply, and the x words of the step are shared by the whole chain.  Threads
+// 8j .. 8j + 7 of a warp take gids 0..7 of the same step (their x loads are one
+// broadcast; their code loads start 32 or 48 bytes apart).  g = lane mod 8,
+// j = lane / 8; acc0 / acc1 end as this thread's share of rows g / g + 8 in units of
+// x_int, summed over j afterwards.
+
+// Byte `sel & 3` of w, sign-extended; sel from sbyte_sel(k).
+__device__ __forceinline__ uint32_t sbyte_sel(int k)
+{
+    return (uint32_t)k | ((uint32_t)(8 | k) * 0x1110u);
+}
+__device__ __forceinline__ int sbyte_r(uint32_t w, uint32_t sel)
+{
+    uint32_t r;
+    asm("prmt.b32 %0, %1, 0, %2;" : "=r"(r) : "r"(w), "r"(sel));
+    return (int)r;
+}
+
+// limb words of a step (word i at i XOR sx): X[l][h] = limb l of columns 16h .. 16h + 15
+__device__ __forceinline__ void x_step(const uint32_t* xs, int sx, uint4 (&X)[3][2])
+{
+#pragma unroll
+    for (int l = 0; l < 3; ++l)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) X[l][h] = *reinterpret_cast<const uint4*>(xs + ((8 * l + 4 * h) ^ sx));
+}
+
+// component t of a uint4 (t a compile-time index after unrolling)
+__device__ __forceinline__ uint32_t comp(const uint4& v, int t)
+{
+    return t == 0 ? v.x : t == 1 ? v.y : t == 2 ? v.z : v.w;
+}
+
+template <int QT>
+struct Row;
+
+template <>
+struct Row<NTX_Q4_0_T> {
+    // U: the unit (one step), xs: its x words, sx: the step's x swizzle
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, int sx, int g, float& acc0,
+                                               float& acc1)
+    {
+        const uint4* L = reinterpret_cast<const uint4*>(U + 32 * g);   // (P, Q) of lanes tig 0..3
+        const uint4 u0 = L[0], u1 = L[1];
+        const uint32_t Pw[4] = {u0.x, u0.z, u1.x, u1.z}, Qw[4] = {u0.y, u0.w, u1.y, u1.w};
+        uint4 X[3][2];
+        x_step(xs, sx, X);
+        const uint4 xsum = *reinterpret_cast<const uint4*>(xs + (24 ^ sx));
+        const uint32_t M = 0x0F0F0F0Fu;
+        int c0[3], c1[3];
+#pragma unroll
+        for (int l = 0; l < 3; ++l) {
+            // codes carry +8: start at -8 x (the limb's sum over the step)
+            c0[l] = c1[l] = -8 * (int)comp(xsum, l);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                c0[l] = dp4((Pw[t] >> 4) & M, comp(X[l][1], t), dp4(Pw[t] & M, comp(X[l][0], t), c0[l]));
+                c1[l] = dp4((Qw[t] >> 4) & M, comp(X[l][1], t), dp4(Qw[t] & M, comp(X[l][0], t), c1[l]));
+            }
+        }
+        const float2 d = d_pair(U + 256 + 4 * g);
+        acc0 = fmaf(d.x, limbs_f(c0[0], c0[1], c0[2]), acc0);
+        acc1 = fmaf(d.y, limbs_f(c1[0], c1[1], c1[2]), acc1);
+    }
+};
+
+template <>
+struct Row<NTX_Q6_K_T> {
+    // U: the superblock unit, xs: its x words; the thread takes steps j and j + 4
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, int g, int j, float& acc0,
+                                               float& acc1)
+    {
+        // int8 scales: vector (g, parity) holds row g at bytes 0-7 and row g + 8 at bytes
+        // 8-15, byte m of each = sub-block 2m + parity (se: parity 0, so: parity 1)
+        const uint4 se = *reinterpret_cast<const uint4*>(U + 3072 + 32 * g);
+        const uint4 so = *reinterpret_cast<const uint4*>(U + 3072 + 32 * g + 16);
+        const uint32_t sel = sbyte_sel(j);   // byte m mod 4 = j
+        const uint32_t M6 = 0x3F3F3F3Fu;
+        int p0[3] = {0, 0, 0}, p1[3] = {0, 0, 0};   // per limb: rows g, g + 8
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int m = j + 4 * k;
+            // lanes tig 0..3 of gid g: words A, B, C of each
+            const uint4* L = reinterpret_cast<const uint4*>(U + 384 * m + 48 * g);
+            const uint4 v0 = L[0], v1 = L[1], v2 = L[2];
+            const uint32_t A[4] = {v0.x, v0.w, v1.z, v2.y}, B[4] = {v0.y, v1.x, v1.w, v2.z},
+                           C[4] = {v0.z, v1.y, v2.x, v2.w};
+            const uint32_t* x = xs + 32 * m;
+            const int sx = 8 * j;   // step m mod 4 = j (a unit starts on a multiple of 8 steps)
+            uint4 X[3][2];
+            x_step(x, sx, X);
+            const uint4 h0 = *reinterpret_cast<const uint4*>(x + (24 ^ sx));   // limb sums of half 0
+            const uint4 h1 = *reinterpret_cast<const uint4*>(x + (28 ^ sx));   // and of half 1
+            // sub-blocks 2m (e) and 2m + 1 (o) of rows g (0) and g + 8 (1)
+            const int s_e0 = sbyte_r(k ? se.y : se.x, sel), s_e1 = sbyte_r(k ? se.w : se.z, sel);
+            const int s_o0 = sbyte_r(k ? so.y : so.x, sel), s_o1 = sbyte_r(k ? so.w : so.z, sel);
+            // 6-bit codes of rows g / g + 8, sub-blocks 2m / 2m + 1, per lane tig
+            uint32_t a0[4], a1[4], a2[4], a3[4];
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                a0[t] = A[t] & M6;
+                a1[t] = B[t] & M6;
+                a2[t] = C[t] & M6;
+                a3[t] = ((A[t] >> 6) & 0x03030303u) | ((B[t] >> 4) & 0x0C0C0C0Cu) | ((C[t] >> 2) & 0x30303030u);
+            }
+#pragma unroll
+            for (int l = 0; l < 3; ++l) {
+                // codes carry +32: each chain starts at -32 x (the limb's sum over its half)
+                int e0 = -32 * (int)comp(h0, l), e1 = e0, o0 = -32 * (int)comp(h1, l), o1 = o0;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    e0 = dp4(a0[t], comp(X[l][0], t), e0);
+                    e1 = dp4(a1[t], comp(X[l][0], t), e1);
+                    o0 = dp4(a2[t], comp(X[l][1], t), o0);
+                    o1 = dp4(a3[t], comp(X[l][1], t), o1);
+                }
+                p0[l] += s_e0 * e0 + s_o0 * o0;
+                p1[l] += s_e1 * e1 + s_o1 * o1;
+            }
+        }
+        const float2 d = d_pair(U + 3328 + 4 * g);
+        acc0 = fmaf(d.x, limbs_f(p0[0], p0[1], p0[2]), acc0);
+        acc1 = fmaf(d.y, limbs_f(p1[0], p1[1], p1[2]), acc1);
+    }
+};
+
+template <>
+struct Row<NTX_Q4_K_T> {
+    // U: the superblock unit, xs: its x words; the thread takes steps (= sub-blocks) j and j + 4
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, int g, int j, float& acc0,
+                                               float& acc1)
+    {
+        const uint8_t* v = U + 2048 + 24 * g;   // packed 6-bit scales / mins of rows g, g + 8
+        const uint32_t M = 0x0F0F0F0Fu;
+        int p0[3] = {0, 0, 0}, p1[3] = {0, 0, 0};   // per limb: rows g, g + 8
+        int n0[3] = {0, 0, 0}, n1[3] = {0, 0, 0};   // mins x limb sums
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int m = j + 4 * k;
+            // sub-block m: byte 0 scale row g, 1 scale row g + 8, 2 min row g, 3 min row g + 8
+            const uint32_t nw = *reinterpret_cast<const uint32_t*>(v + 4 * (m >> 1));
+            const uint32_t hw = *reinterpret_cast<const uint32_t*>(v + 16 + 4 * k);
+            const uint32_t S = ((nw >> (4 * (m & 1))) & 0x0F0F0F0Fu) | (((hw >> (2 * j)) & 0x03030303u) << 4);
+            const uint4* L = reinterpret_cast<const uint4*>(U + 256 * m + 32 * g);
+            const uint4 u0 = L[0], u1 = L[1];
+            const uint32_t Pw[4] = {u0.x, u0.z, u1.x, u1.z}, Qw[4] = {u0.y, u0.w, u1.y, u1.w};
+            const uint32_t* x = xs + 32 * m;
+            const int sx = 8 * j;   // step m mod 4 = j (a unit starts on a multiple of 8 steps)
+            uint4 X[3][2];
+            x_step(x, sx, X);
+            const uint4 xsum = *reinterpret_cast<const uint4*>(x + (24 ^ sx));
+            const int sc0 = ubyte<0>(S), sc1 = ubyte<1>(S), mn0 = ubyte<2>(S), mn1 = ubyte<3>(S);
+#pragma unroll
+            for (int l = 0; l < 3; ++l) {
+                int c0 = 0, c1 = 0;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    c0 = dp4((Pw[t] >> 4) & M, comp(X[l][1], t), dp4(Pw[t] & M, comp(X[l][0], t), c0));
+                    c1 = dp4((Qw[t] >> 4) & M, comp(X[l][1], t), dp4(Qw[t] & M, comp(X[l][0], t), c1));
+                }
+                p0[l] += sc0 * c0;
+                p1[l] += sc1 * c1;
+                n0[l] += mn0 * (int)comp(xsum, l);
+                n1[l] += mn1 * (int)comp(xsum, l);
+            }
+        }
+        const uint2 dd = *reinterpret_cast<const uint2*>(U + 2240 + 8 * g);
+        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+        acc0 = fmaf(d.x, limbs_f(p0[0], p0[1], p0[2]), fmaf(-dm.x, limbs_f(n0[0], n0[1], n0[2]), acc0));
+        acc1 = fmaf(d.y, limbs_f(p1[0], p1[1], p1[2]), fmaf(-dm.y, limbs_f(n1[0], n1[1], n1[2]), acc1));
     }
 };
 
@@ -457,12 +701,15 @@ __device__ __forceinline__ void epilogue(const Params& P, int row, bool ok, floa
 
 // ------------------------------------------------------------------ kernel
 
-template <int QT, int EPI, int PRO>
+// CORE 0: the per-step sums on the tensor cores (Unit); CORE 1: on the CUDA cores (Dot, Row).
+template <int QT, int EPI, int PRO, int CORE>
 __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
 {
     using T = gemv::Tiled<QT>;
     constexpr int NM = EPI == gemv::EPI_SWIGLU ? 2 : 1;    // matrices per group (gate, up)
     constexpr int SPU = T::UK / 32;                         // steps per unit
+    // CUDA-core path: lane units (the MMA's fragments) for Q8_0, row-pair units otherwise
+    constexpr bool ROWS = CORE == 1 && QT != NTX_Q8_0_T;
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -638,7 +885,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                 const int u = base + sub;
                 const bool ok = u < n_steps;
                 const float4 v = ok ? xf[u * 8 + w] : make_float4(0.f, 0.f, 0.f, 0.f);
-                stage_x_step<QT == NTX_Q6_K_T>(xq + 32 * u, w, ok, v, two_s);
+                stage_x_step<QT == NTX_Q6_K_T, CORE == 1 && QT == NTX_Q8_0_T>(xq + 32 * u, w, ok, v, two_s,
+                                                                          ROWS ? 8 * (u & 3) : 0);
             }
         }
         const int32_t pos = (EPI == gemv::EPI_QKV) ? (P.pos_dev ? *P.pos_dev : P.pos) : 0;
@@ -653,7 +901,9 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
         named_bar_sync(1, kCons);   // limbs and the RoPE table complete
 
         const Lane L = make_lane<QT>(lane);
-        const float limb_w = (L.tig & 1) ? 65536.f : 1.f;   // this lane's C columns: limbs 0,1 or limb 2
+        // CORE 0: this lane's C columns hold limbs 0, 1 or limb 2; CORE 1 sums are whole
+        const float limb_w = (CORE == 0 && (L.tig & 1)) ? 65536.f : 1.f;
+        const int rgid = lane & 7, rj = lane >> 3;   // row-pair units: gid, step slot
         const int NS = P.n_stages;
         int s = 0;
         uint32_t ph = 0;
@@ -664,7 +914,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
             float* rg = red + (gl & 1) * (kWarps * 32);   // [warp][mat][16]
 #pragma unroll 1
             for (int mat = 0; mat < NM; ++mat) {
-                float acc0 = 0.f, acc1 = 0.f;
+                float acc0 = 0.f, acc1 = 0.f;   // this lane's shares of rows gid, gid + 8
                 for (int c = 0; c < NCH; ++c) {
                     const int n_units = min(CE, KR - c * CE) / T::UK;
                     if (!dead && !mbar_wait(&full[s], ph, kWaitPolls)) {
@@ -674,8 +924,24 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                     const uint8_t* st = stages + (size_t)s * P.stage_bytes;
                     if (!dead) {
                         const uint32_t* xc = xq + 32 * (c * CE / 32);
-                        for (int un = warp; un < n_units; un += kWarps)
-                            Unit<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, L, acc0, acc1);
+                        if (CORE == 0) {
+                            for (int un = warp; un < n_units; un += kWarps)
+                                Unit<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, L, acc0, acc1);
+                        } else if constexpr (QT == NTX_Q8_0_T) {
+                            for (int un = warp; un < n_units; un += kWarps)
+                                Dot<QT>::run(st + (size_t)un * T::UB, xc + 32 * un, L, acc0, acc1);
+                        } else if constexpr (QT == NTX_Q4_0_T) {
+                            // a warp takes 4 units (steps) at a time, one per 8 threads
+                            const int sx = 8 * ((c * CE / 32 + rj) & 3);
+                            for (int u4 = 4 * warp; u4 < n_units; u4 += 4 * kWarps) {
+                                const int un = u4 + rj;
+                                if (un < n_units)
+                                    Row<QT>::run(st + (size_t)un * T::UB, xc + 32 * un, sx, rgid, acc0, acc1);
+                            }
+                        } else {
+                            for (int un = warp; un < n_units; un += kWarps)
+                                Row<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, rgid, rj, acc0, acc1);
+                        }
                     }
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&empty[s]);
@@ -684,16 +950,29 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                         ph ^= 1u;
                     }
                 }
-                // quad reduction with the limb weights: lane tig 0 ends with rows gid, gid + 8
-                acc0 *= limb_w;
-                acc1 *= limb_w;
-                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
-                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
-                acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
-                acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
-                if (L.tig == 0) {
-                    rg[warp * 32 + mat * 16 + L.gid] = acc0;
-                    rg[warp * 32 + mat * 16 + L.gid + 8] = acc1;
+                if constexpr (ROWS) {
+                    // sum over the 4 threads of each gid: lane g < 8 ends with rows g, g + 8
+                    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 8);
+                    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 8);
+                    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 16);
+                    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 16);
+                    if (lane < 8) {
+                        rg[warp * 32 + mat * 16 + lane] = acc0;
+                        rg[warp * 32 + mat * 16 + lane + 8] = acc1;
+                    }
+                } else {
+                    // quad reduction (with the limb weights of the MMA's C columns): lane tig 0
+                    // ends with rows gid, gid + 8
+                    acc0 *= limb_w;
+                    acc1 *= limb_w;
+                    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 1);
+                    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 1);
+                    acc0 += __shfl_xor_sync(0xffffffffu, acc0, 2);
+                    acc1 += __shfl_xor_sync(0xffffffffu, acc1, 2);
+                    if (L.tig == 0) {
+                        rg[warp * 32 + mat * 16 + L.gid] = acc0;
+                        rg[warp * 32 + mat * 16 + L.gid + 8] = acc1;
+                    }
                 }
             }
             named_bar_sync(1, kCons);

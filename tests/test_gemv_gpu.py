@@ -241,13 +241,51 @@ def test_repack_matches_documented_layout(ntx, syn, qtype, rows, cols):
     assert np.array_equal(W.cpu().numpy(), tiling.tile(qtype, host, rows, cols))
 
 
+@pytest.mark.parametrize("core", ["tc", "dp4a"], ids=["tensor-cores", "cuda-cores"])
 @pytest.mark.parametrize("split", ["0", "1"], ids=["whole-rows", "column-halves"])
 @pytest.mark.parametrize("qtype,rows,cols", [(Q6_K, 1024, 8192 + 256), (Q8_0, 2048, 4096 + 32), (Q4_K, 160, 2304),
                                              (Q4_0, 32, 64)], ids=["q6_k", "q8_0", "q4_k", "q4_0"])
-def test_gemv_tiled_both_cluster_shapes(ntx, orc, syn, monkeypatch, split, qtype, rows, cols):
-    """Whole rows per CTA and CTA pairs that split the columns (forced either way): both
-    match the oracle, including an odd number of units per row."""
+def test_gemv_tiled_both_cluster_shapes(ntx, orc, syn, monkeypatch, core, split, qtype, rows, cols):
+    """Whole rows per CTA and CTA pairs that split the columns (forced either way), with
+    the per-step sums on the tensor cores or on the CUDA cores: all match the oracle,
+    including an odd number of units per row."""
     monkeypatch.setenv("NTX_GEMV_SPLIT", split)
+    monkeypatch.setenv("NTX_GEMV_CORE", core)
     host, W = make_tiled(ntx, syn, qtype, rows, cols)
     x = syn.normal_f32_host(7, 12, cols)
     assert rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)) <= GEMV_TIGHT
+
+
+@pytest.mark.parametrize("core", ["tc", "dp4a"], ids=["tensor-cores", "cuda-cores"])
+@pytest.mark.parametrize("qtype", [Q8_0, Q4_0, Q4_K, Q6_K], ids=list(NAMES.values()))
+def test_tiled_one_hot_both_cores(ntx, syn, monkeypatch, core, qtype):
+    """A one-hot x returns the dequantized column bit for bit on either unit."""
+    monkeypatch.setenv("NTX_GEMV_CORE", core)
+    rows, cols = 32, 4096 + (256 if qtype in (Q4_K, Q6_K) else 32)
+    host, W = make_tiled(ntx, syn, qtype, rows, cols)
+    dq = torch.empty((rows, cols), dtype=torch.float32, device="cuda")
+    ntx.ntx_dequant_q(qtype | T, W, rows, cols, dq)
+    for k in (0, 17, cols // 2 + 3, cols - 1):
+        x = np.zeros(cols, dtype=np.float32)
+        x[k] = 1.0
+        assert np.array_equal(gpu_gemv(ntx, qtype | T, W, rows, cols, x), dq[:, k].cpu().numpy()), (core, k)
+
+
+@pytest.mark.parametrize("core", ["tc", "dp4a"], ids=["tensor-cores", "cuda-cores"])
+@pytest.mark.parametrize("qtype", [Q8_0, Q4_0, Q4_K, Q6_K], ids=list(NAMES.values()))
+def test_tiled_input_edge_cases(ntx, orc, syn, monkeypatch, core, qtype):
+    """The tiled path takes x as 24-bit fixed point relative to max |x|: a zero x gives
+    exact zeros, and very small, very large and mixed-magnitude inputs stay within the
+    tolerance (values far below max |x| round to zero, which the normwise error allows)."""
+    monkeypatch.setenv("NTX_GEMV_CORE", core)
+    rows, cols = 48, 8192 + 256
+    host, W = make_tiled(ntx, syn, qtype, rows, cols)
+    zero = np.zeros(cols, dtype=np.float32)
+    assert np.array_equal(gpu_gemv(ntx, qtype | T, W, rows, cols, zero), np.zeros(rows, dtype=np.float32))
+    x = syn.normal_f32_host(3, 12, cols)
+    x[::7] *= 1e20
+    x[1::7] *= 1e-20
+    assert rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)) <= GEMV_TIGHT
+    for scale in (1e-30, 1e25):
+        xs = (syn.normal_f32_host(4, 12, cols) * np.float32(scale)).astype(np.float32)
+        assert rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, xs), orc.gemv(qtype, host, rows, cols, xs)) <= GEMV_TIGHT
