@@ -432,49 +432,49 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
 
 // Merge of the splits, one CTA per query head and one thread per dim: with
 // M = max_s m_s over splits that saw a position, w_s = e^(m_s - M) and
-// L = sum_s l_s w_s, out[d] = sum_s (w_s / L) acc_s[d], summed in split order.
+// L = sum_s l_s w_s, out[d] = (sum_s w_s acc_s[d]) / L.  Each thread reads every
+// split's (m, l) (the same addresses across the CTA) and its dim of every split's
+// accumulator, 32 splits per round of loads, and merges the rounds online (the
+// running sums rescaled when the maximum grows), so one round trip to L2 serves up
+// to 32 splits and no barrier is needed.
 template <int G>
 __global__ void __launch_bounds__(HD) attn_merge_kernel(const float* part, float* out, int n_split, int use_pdl)
 {
-    constexpr int B = 32;   // splits whose partial dims are loaded together
-    __shared__ float wn[kMaxSplit];
+    constexpr int B = 32;   // splits whose records are loaded together
     if (use_pdl) {
         pdl_launch_dependents();
         pdl_wait();
     }
-    const int qh = blockIdx.x, g = qh / G, h = qh % G, d = threadIdx.x, lane = d & 31;
+    const int qh = blockIdx.x, g = qh / G, h = qh % G, d = threadIdx.x;
     const size_t rec = (size_t)G * kPartFloats;   // floats from one split's record of this head to the next
     const float* base = part + ((size_t)g * n_split * G + h) * kPartFloats;
-    float o = 0.f;
+    float M = -INFINITY, L = 0.f, o = 0.f;
     for (int s0 = 0; s0 < n_split; s0 += B) {
+        float2 ml[B];
         float v[B];
 #pragma unroll
-        for (int k = 0; k < B; ++k) v[k] = s0 + k < n_split ? __ldcg(base + (s0 + k) * rec + 4 + d) : 0.f;
-        if (s0 == 0) {
-            if (d < 32) {
-                float M = -INFINITY;
-                for (int s2 = lane; s2 < n_split; s2 += 32)
-                    if (__ldcg(base + s2 * rec + 1) > 0.f) M = fmaxf(M, __ldcg(base + s2 * rec));
-                M = gemv::warp_max(M);
-                float L = 0.f;
-                for (int s2 = lane; s2 < n_split; s2 += 32) {
-                    const float l = __ldcg(base + s2 * rec + 1);
-                    const float w = l > 0.f ? expf(__ldcg(base + s2 * rec) - M) : 0.f;
-                    wn[s2] = w;
-                    L = fmaf(l, w, L);
-                }
-                L = gemv::warp_sum(L);
-                const float inv = 1.f / L;
-                __syncwarp();
-                for (int s2 = lane; s2 < n_split; s2 += 32) wn[s2] *= inv;
-            }
-            __syncthreads();
+        for (int k = 0; k < B; ++k) {
+            const bool ok = s0 + k < n_split;
+            ml[k] = ok ? __ldcg(reinterpret_cast<const float2*>(base + (s0 + k) * rec)) : make_float2(0.f, 0.f);
+            v[k] = ok ? __ldcg(base + (s0 + k) * rec + 4 + d) : 0.f;
         }
+        float Mb = M;
 #pragma unroll
         for (int k = 0; k < B; ++k)
-            if (s0 + k < n_split) o = fmaf(wn[s0 + k], v[k], o);
+            if (ml[k].y > 0.f) Mb = fmaxf(Mb, ml[k].x);
+        if (Mb == -INFINITY) continue;   // no split of this round saw a position
+        const float r = M == -INFINITY ? 0.f : expf(M - Mb);
+        L *= r;
+        o *= r;
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+            const float w = ml[k].y > 0.f ? expf(ml[k].x - Mb) : 0.f;
+            L = fmaf(ml[k].y, w, L);
+            o = fmaf(w, v[k], o);
+        }
+        M = Mb;
     }
-    out[(size_t)qh * HD + d] = o;
+    out[(size_t)qh * HD + d] = o / L;
 }
 
 template <int G>

@@ -33,6 +33,7 @@ struct ntx_model {
     float* att = nullptr;
     float* act = nullptr;
     int32_t* step = nullptr;
+    float* rope = nullptr;   // the step's RoPE table [head_dim / 2][cos, sin]
     void* attn_ws = nullptr;
     int n_split = 1;
     bool pdl = true;
@@ -82,7 +83,7 @@ ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, b
         P.head_dim = d.head_dim;
         P.max_ctx = d.max_ctx;
         P.pos_dev = m->step + 1;
-        P.theta = d.rope_theta;
+        P.rope_cs = m->rope;
         P.k_cache = (__half*)L.k_cache;
         P.v_cache = (__half*)L.v_cache;
         P.q_out = m->q;
@@ -229,6 +230,7 @@ void free_model(ntx_model* m)
     cudaFree(m->att);
     cudaFree(m->act);
     cudaFree(m->step);
+    cudaFree(m->rope);
     cudaFree(m->attn_ws);
     cudaFree(m->ring);
     delete m;
@@ -271,6 +273,7 @@ NTX_EXPORT ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** m
     alloc((void**)&m->att, (size_t)qd * 4);
     alloc((void**)&m->act, (size_t)d.ffn * 4);
     alloc((void**)&m->step, 16);
+    alloc((void**)&m->rope, (size_t)d.head_dim * 4);
     alloc(&m->attn_ws, ws);
     if (e == cudaSuccess) e = cudaMemset(m->attn_ws, 0, ws);
     if (e == cudaSuccess) e = cudaMemset(m->step, 0, 16);
@@ -320,7 +323,7 @@ NTX_EXPORT ntx_status ntx_decode_step(ntx_model* m, int32_t token, int32_t pos, 
     if (pos < 0 || pos >= m->d.max_ctx) return fail(NTX_EINVAL, "ntx_decode_step: pos out of range");
     if (!aligned(logits, 4)) return fail(NTX_EINVAL, "ntx_decode_step: logits must be 4-byte aligned");
     cudaStream_t s = (cudaStream_t)stream;
-    ntx_status st = set_step_launch(m->step, token, pos, s);
+    ntx_status st = set_step_launch(m->step, token, pos, m->rope, m->d.rope_theta, m->d.head_dim, s);
     if (st != NTX_OK) return st;
     if (!m->use_graph) return enqueue_resident(m, m->d.n_layers, logits, s, true);
     if (!m->graph || m->graph_logits != logits) {
@@ -369,7 +372,7 @@ NTX_EXPORT ntx_status ntx_stream_layers(ntx_model* m, int32_t token, int32_t pos
     const ntx_model_desc& d = m->d;
     const int nres = d.n_resident;
     NTX_CUDA_TRY(cudaEventRecord(m->ev_start, cs));
-    ntx_status st = set_step_launch(m->step, token, pos, cs);
+    ntx_status st = set_step_launch(m->step, token, pos, m->rope, d.rope_theta, d.head_dim, cs);
     if (st != NTX_OK) return st;
     int64_t h2d = 0;
     // copies of streamed layer j into slot (j - nres) % 2; the slot is free once

@@ -92,6 +92,8 @@ ntx_status launch_q(int qtype, const Params& P, cudaStream_t s, int grid_cap)
 ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s)
 {
     using namespace gemv;
+    if (epi == EPI_QKV && (!P.rope_cs || P.head_dim > 128))
+        return fail(NTX_EINVAL, "gemv: the fused QKV epilogue needs the step's RoPE table (head_dim <= 128)");
     if (is_tiled(qtype)) return qmma_launch(qtype, epi, pro, P, s);
     const int cap = num_sms();
     if (epi == EPI_STORE && pro == PRO_X) return launch_q<EPI_STORE, PRO_X>(qtype, P, s, cap);

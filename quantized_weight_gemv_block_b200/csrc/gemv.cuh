@@ -59,7 +59,7 @@ struct Params {
     int q_rows, kv_rows, head_dim, max_ctx;
     const int32_t* pos_dev;
     int32_t pos;
-    float theta;
+    const float* rope_cs; // [head_dim / 2][cos, sin] of pos theta^(-2i/head_dim), written before the kernel
     __half* k_cache;
     __half* v_cache;
     float* q_out;

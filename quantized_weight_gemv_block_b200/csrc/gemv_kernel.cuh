@@ -244,14 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemv_kernel(const Params P)
     }
 
     const int32_t pos = (EPI == EPI_QKV) ? (P.pos_dev ? *P.pos_dev : P.pos) : 0;
-    if (EPI == EPI_QKV && tid < P.head_dim / 2) {
-        // RoPE angles of this position, pos * theta^(-2i/head_dim), in double; read by the epilogue
-        const double ang = (double)pos * pow((double)P.theta, -(2.0 * tid) / (double)P.head_dim);
-        double sn, cs;
-        sincos(ang, &sn, &cs);
-        rope_cs[2 * tid] = (float)cs;
-        rope_cs[2 * tid + 1] = (float)sn;
-    }
+    if (EPI == EPI_QKV && tid < P.head_dim) rope_cs[tid] = P.rope_cs[tid];   // the step's RoPE table
     bool dead = false;
     // this thread's x pieces of a chunk, and the offset / min sums of its elements
     uint64_t xr[2 * NP];

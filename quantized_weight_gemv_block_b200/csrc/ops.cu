@@ -137,10 +137,24 @@ __global__ void embed_kernel(const uint8_t* E, int64_t rb, int64_t hidden, const
         h[i] = gemv::weight_at<QT>(E, token, i, rb);
 }
 
-__global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos)
+// The step word (token, position) and the RoPE table of the position: rope[2i] and
+// rope[2i + 1] = cos and sin of pos theta^(-2i/head_dim), computed in double, for
+// i < head_dim / 2 (the rotation of "RoPE" in the ntransformer news summary's kernel
+// list).  Later kernels of the step read both.
+__global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim)
 {
-    step[0] = token;
-    step[1] = pos;
+    const int i = threadIdx.x;
+    if (i == 0) {
+        step[0] = token;
+        step[1] = pos;
+    }
+    if (rope && i < head_dim / 2) {
+        const double ang = (double)pos * pow((double)theta, -(2.0 * i) / (double)head_dim);
+        double sn, cs;
+        sincos(ang, &sn, &cs);
+        rope[2 * i] = (float)cs;
+        rope[2 * i + 1] = (float)sn;
+    }
 }
 
 }  // namespace
@@ -177,9 +191,10 @@ ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t*
     return NTX_OK;
 }
 
-ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, cudaStream_t s)
+ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
+                           cudaStream_t s)
 {
-    set_step_kernel<<<1, 1, 0, s>>>(step, token, pos);
+    set_step_kernel<<<1, std::max(32, head_dim / 2), 0, s>>>(step, token, pos, rope, theta, head_dim);
     return check_launch("step counter");
 }
 

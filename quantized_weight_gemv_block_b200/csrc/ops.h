@@ -8,7 +8,10 @@ namespace ntx {
 
 ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t* token_dev, float* h, cudaStream_t s,
                         bool pdl);
-ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, cudaStream_t s);
+// Writes the step word (token, pos) and, if rope is not null, the RoPE table of pos
+// ([head_dim / 2][cos, sin] floats) for the kernels of the step.
+ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
+                           cudaStream_t s);
 ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
 ntx_status qmma_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
 ntx_status repack_launch(int qtype, const void* W, void* W_tiled, int64_t rows, int64_t cols, cudaStream_t s);

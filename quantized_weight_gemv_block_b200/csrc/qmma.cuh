@@ -175,8 +175,15 @@ __device__ __forceinline__ void red_add_cluster(uint32_t addr, float v)
 // i XOR 8 (u mod 4) (sx below): the four quarter-warps of a warp read the same words
 // of four consecutive steps, which then fall in four different bank groups.
 
-template <bool HALVES, bool PAIRED>
-__device__ __forceinline__ void stage_x_step(uint32_t* xs, int w, bool ok, float4 v, float two_s, int sx)
+// The limb words and column sums of the 4 columns a lane holds (lane w of the 8 lanes
+// of a step); the sums are already reduced over the step's lanes (or each half's).
+struct XLimbs {
+    uint32_t w0, w1, w2;
+    int s0, s1, s2;
+};
+
+template <bool HALVES>
+__device__ __forceinline__ XLimbs x_limbs(float4 v, float two_s)
 {
     // z = x_int + 0x8080: bytes 0 and 1 of z are the low limbs + 128, z >> 16 the top limb
     const float mag = 12582912.0f;   // 1.5 * 2^23: fmaf rounds x 2^S to an integer in its low bits
@@ -186,43 +193,50 @@ __device__ __forceinline__ void stage_x_step(uint32_t* xs, int w, bool ok, float
     const int z2 = __float_as_int(fmaf(v.z, two_s, mag)) + bias;
     const int z3 = __float_as_int(fmaf(v.w, two_s, mag)) + bias;
     const uint32_t lo01 = __byte_perm(z0, z1, 0x5410), lo23 = __byte_perm(z2, z3, 0x5410);
-    const uint32_t w0 = __byte_perm(lo01, lo23, 0x6420) ^ 0x80808080u;
-    const uint32_t w1 = __byte_perm(lo01, lo23, 0x7531) ^ 0x80808080u;
-    const uint32_t w2 = __byte_perm(__byte_perm(z0, z1, 0x0062), __byte_perm(z2, z3, 0x0062), 0x5410);
+    XLimbs r;
+    r.w0 = __byte_perm(lo01, lo23, 0x6420) ^ 0x80808080u;
+    r.w1 = __byte_perm(lo01, lo23, 0x7531) ^ 0x80808080u;
+    r.w2 = __byte_perm(__byte_perm(z0, z1, 0x0062), __byte_perm(z2, z3, 0x0062), 0x5410);
     // column sums of the four values (byte sums of the signed limbs)
-    int s0 = __dp4a((int)w0, 0x01010101, 0), s1 = __dp4a((int)w1, 0x01010101, 0), s2 = __dp4a((int)w2, 0x01010101, 0);
+    r.s0 = __dp4a((int)r.w0, 0x01010101, 0);
+    r.s1 = __dp4a((int)r.w1, 0x01010101, 0);
+    r.s2 = __dp4a((int)r.w2, 0x01010101, 0);
 #pragma unroll
     for (int o = 1; o < (HALVES ? 4 : 8); o <<= 1) {
-        s0 += __shfl_xor_sync(0xffffffffu, s0, o);
-        s1 += __shfl_xor_sync(0xffffffffu, s1, o);
-        s2 += __shfl_xor_sync(0xffffffffu, s2, o);
+        r.s0 += __shfl_xor_sync(0xffffffffu, r.s0, o);
+        r.s1 += __shfl_xor_sync(0xffffffffu, r.s1, o);
+        r.s2 += __shfl_xor_sync(0xffffffffu, r.s2, o);
     }
-    __syncwarp();   // every lane of the step has read its floats before any limb word lands
-    if (ok) {
-        const int wp = PAIRED ? 2 * (w & 3) + (w >> 2) : w;
-        xs[wp ^ sx] = w0;
-        xs[(8 + wp) ^ sx] = w1;
-        xs[(16 + wp) ^ sx] = w2;
-        if (HALVES) {
-            if ((w & 3) == 0) {
-                const int h = w >> 2;
-                xs[(24 + 4 * h) ^ sx] = (uint32_t)s0;
-                xs[(25 + 4 * h) ^ sx] = (uint32_t)s1;
-                xs[(26 + 4 * h) ^ sx] = (uint32_t)s2;
-                xs[(27 + 4 * h) ^ sx] = 0u;
-            }
-        } else {
-            if (w == 0) {
-                xs[24 ^ sx] = (uint32_t)s0;
-                xs[25 ^ sx] = (uint32_t)s1;
-                xs[26 ^ sx] = (uint32_t)s2;
-            } else if (w == 1) {
-                xs[27 ^ sx] = 0u;
-                xs[28 ^ sx] = 0u;
-                xs[29 ^ sx] = 0u;
-                xs[30 ^ sx] = 0u;
-                xs[31 ^ sx] = 0u;
-            }
+    return r;
+}
+
+// Store lane w's limb words (and, from the lanes that hold them, the sums) of step xs.
+template <bool HALVES, bool PAIRED>
+__device__ __forceinline__ void x_store(uint32_t* xs, int w, const XLimbs& r, int sx)
+{
+    const int wp = PAIRED ? 2 * (w & 3) + (w >> 2) : w;
+    xs[wp ^ sx] = r.w0;
+    xs[(8 + wp) ^ sx] = r.w1;
+    xs[(16 + wp) ^ sx] = r.w2;
+    if (HALVES) {
+        if ((w & 3) == 0) {
+            const int h = w >> 2;
+            xs[(24 + 4 * h) ^ sx] = (uint32_t)r.s0;
+            xs[(25 + 4 * h) ^ sx] = (uint32_t)r.s1;
+            xs[(26 + 4 * h) ^ sx] = (uint32_t)r.s2;
+            xs[(27 + 4 * h) ^ sx] = 0u;
+        }
+    } else {
+        if (w == 0) {
+            xs[24 ^ sx] = (uint32_t)r.s0;
+            xs[25 ^ sx] = (uint32_t)r.s1;
+            xs[26 ^ sx] = (uint32_t)r.s2;
+        } else if (w == 1) {
+            xs[27 ^ sx] = 0u;
+            xs[28 ^ sx] = 0u;
+            xs[29 ^ sx] = 0u;
+            xs[30 ^ sx] = 0u;
+            xs[31 ^ sx] = 0u;
         }
     }
 }
@@ -801,29 +815,51 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
             cluster_arrive();
             cluster_wait();
         }
+        float* rs = red;   // scratch for the prologue reductions
+        const int K4 = P.K / 4, h0 = k0 / 4, h1 = (k0 + KR) / 4, nh = h1 - h0;
+        float4* xf = reinterpret_cast<float4*>(xq);
+        const float4* x4 = reinterpret_cast<const float4*>(P.x);
+        const float4* w4 = reinterpret_cast<const float4*>(P.norm_w) + h0;
+        // (0) Before the programmatic wait, what needs nothing from the previous kernel:
+        // the RMSNorm weights of this thread's first NW float4 of x (float4 i = tid + j kCons,
+        // the same float4 the passes below take) into registers, and the step's RoPE table
+        // (written with the position word before the first kernel of a step that launches
+        // early) into shared memory for the epilogue.
+        const float rope_v = (EPI == gemv::EPI_QKV && tid < P.head_dim) ? P.rope_cs[tid] : 0.f;
+        constexpr bool RMS = PRO == gemv::PRO_RMSNORM;
+        constexpr int NW = RMS ? 8 : 4;
+        float4 wr[NW];
+#pragma unroll
+        for (int j = 0; j < NW; ++j) {
+            const int i = tid + j * kCons;
+            wr[j] = (RMS && i < nh) ? w4[i] : make_float4(1.f, 1.f, 1.f, 1.f);
+        }
         if (P.use_pdl) {
             pdl_launch_dependents();
             pdl_wait();
         }
-        float* rs = red;   // scratch for the prologue reductions
         // (1) this CTA's columns of x into shared memory with one bulk copy (x is
-        // 16-byte aligned and the half starts on a 32-column step), then RMSNorm (its sum
-        // of squares runs over the whole vector) and max |x| of the CTA's columns
-        const int K4 = P.K / 4, h0 = k0 / 4, h1 = (k0 + KR) / 4, nh = h1 - h0;
-        float4* xf = reinterpret_cast<float4*>(xq);
-        const float4* x4 = reinterpret_cast<const float4*>(P.x);
+        // 16-byte aligned and the half starts on a 32-column step)
         if (tid == 0 && KR > 0) {
             mbar_arrive_expect_tx(xbar, (uint32_t)KR * 4u);
             bulk_g2s(xf, P.x + k0, (uint32_t)KR * 4u, xbar, policy_evict_last());
         }
         if (KR > 0 && !mbar_wait(xbar, 0, kWaitPolls) && tid == 0) record_device_error(DEVERR_FULL_WAIT);
-        float mx = 0.f;
-        if (PRO == gemv::PRO_RMSNORM) {
-            float ss = 0.f;
-            for (int i = tid; i < nh; i += kCons) {
-                const float4 v = xf[i];
-                ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
-            }
+        // (2) one pass: the sum of squares (RMSNorm; it runs over the whole vector) and
+        // max |x w| (w = 1 without RMSNorm) over the CTA's columns
+        float ss = 0.f, mw = 0.f;
+        auto pass1 = [&](const float4& v, const float4& w) {
+            if (RMS) ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+            mw = fmaxf(mw, fmaxf(fmaxf(fabsf(v.x * w.x), fabsf(v.y * w.y)), fmaxf(fabsf(v.z * w.z), fabsf(v.w * w.w))));
+        };
+#pragma unroll
+        for (int j = 0; j < NW; ++j) {
+            const int i = tid + j * kCons;
+            if (i < nh) pass1(xf[i], wr[j]);
+        }
+        for (int i = tid + NW * kCons; i < nh; i += kCons)
+            pass1(xf[i], RMS ? w4[i] : make_float4(1.f, 1.f, 1.f, 1.f));
+        if (RMS) {
             // the other CTA's columns, from global memory, 8 loads in flight per thread
             for (int j0 = tid; j0 < K4 - nh; j0 += 8 * kCons) {
                 float4 v[8];
@@ -837,67 +873,66 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                     ss = fmaf(v[j].x, v[j].x, fmaf(v[j].y, v[j].y, fmaf(v[j].z, v[j].z, fmaf(v[j].w, v[j].w, ss))));
             }
             ss = gemv::warp_sum(ss);
-            if (lane == 0) rs[warp] = ss;
-            named_bar_sync(1, kCons);
-            float tot = 0.f;
-#pragma unroll
-            for (int w = 0; w < kWarps; ++w) tot += rs[w];
-            const float inv = 1.0f / sqrtf(tot / (float)P.K + P.eps);
-            const float4* w4 = reinterpret_cast<const float4*>(P.norm_w) + h0;
-            for (int i0 = tid; i0 < nh; i0 += 8 * kCons) {
-                float4 w[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int i = i0 + j * kCons;
-                    w[j] = i < nh ? w4[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int i = i0 + j * kCons;
-                    if (i < nh) {
-                        const float4 a = xf[i];
-                        const float4 v = make_float4(a.x * inv * w[j].x, a.y * inv * w[j].y, a.z * inv * w[j].z,
-                                                     a.w * inv * w[j].w);
-                        xf[i] = v;
-                        mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-                    }
-                }
-            }
-        } else {
-            for (int i = tid; i < nh; i += kCons) {
-                const float4 v = xf[i];
-                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
-            }
         }
-        mx = gemv::warp_max(mx);
-        if (lane == 0) rs[kWarps + warp] = mx;
-        named_bar_sync(1, kCons);   // also orders every fp32 store before the limb conversion
-        mx = 0.f;
+        mw = gemv::warp_max(mw);
+        if (lane == 0) {
+            rs[warp] = ss;
+            rs[kWarps + warp] = mw;
+        }
+        named_bar_sync(1, kCons);
+        float tot = 0.f, mx = 0.f;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, rs[kWarps + w]);
+        for (int w = 0; w < kWarps; ++w) {
+            tot += rs[w];
+            mx = fmaxf(mx, rs[kWarps + w]);
+        }
+        // the normalised value is fl(fl(x w) inv): its largest magnitude is fl(max |x w| inv)
+        const float inv = RMS ? 1.0f / sqrtf(tot / (float)P.K + P.eps) : 1.f;
+        if (RMS) mx *= inv;
         // |x| 2^S < 2^22; a zero half keeps S = 0 (all limbs zero)
         const int S = (mx > 0.f && mx <= 3.4e38f) ? max(-100, min(127, 21 - ilogbf(mx))) : 0;
         const float two_s = __uint_as_float((uint32_t)(127 + S) << 23);
-        // (2) fp32 -> limbs, in place: 8 lanes per 32-column step
+        // (3) normalised fp32 -> limbs, in place: 8 lanes per 32-column step, float4
+        // i = tid + j kCons; 4 rounds at a time, all reads of a round before its stores
         {
-            const int n_steps = KR / 32, sub = lane >> 3, w = lane & 7;
-            for (int base = warp * 4; base < n_steps; base += kWarps * 4) {
-                const int u = base + sub;
-                const bool ok = u < n_steps;
-                const float4 v = ok ? xf[u * 8 + w] : make_float4(0.f, 0.f, 0.f, 0.f);
-                stage_x_step<QT == NTX_Q6_K_T, CORE == 1 && QT == NTX_Q8_0_T>(xq + 32 * u, w, ok, v, two_s,
-                                                                          ROWS ? 8 * (u & 3) : 0);
+            const int n_steps = KR / 32, n_rounds = (n_steps + 31) / 32, wl = lane & 7;
+            auto convert4 = [&](int j0, const float4 (&w)[4]) {
+                XLimbs r[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = tid + (j0 + k) * kCons;
+                    float4 v = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (RMS)
+                        v = make_float4(v.x * w[k].x * inv, v.y * w[k].y * inv, v.z * w[k].z * inv, v.w * w[k].w * inv);
+                    r[k] = x_limbs<QT == NTX_Q6_K_T>(v, two_s);
+                }
+                __syncwarp();   // every lane of a step has read its floats before any limb word lands
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int u = (tid + (j0 + k) * kCons) >> 3;
+                    if (u < n_steps)
+                        x_store<QT == NTX_Q6_K_T, CORE == 1 && QT == NTX_Q8_0_T>(xq + 32 * u, wl, r[k],
+                                                                               ROWS ? 8 * (u & 3) : 0);
+                }
+            };
+#pragma unroll
+            for (int j0 = 0; j0 < NW; j0 += 4) {
+                if (j0 < n_rounds) {
+                    const float4 w[4] = {wr[j0], wr[j0 + 1], wr[j0 + 2], wr[j0 + 3]};
+                    convert4(j0, w);
+                }
+            }
+            for (int j0 = NW; j0 < n_rounds; j0 += 4) {
+                float4 w[4];
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = tid + (j0 + k) * kCons;
+                    w[k] = (RMS && i < nh) ? w4[i] : make_float4(1.f, 1.f, 1.f, 1.f);
+                }
+                convert4(j0, w);
             }
         }
-        const int32_t pos = (EPI == gemv::EPI_QKV) ? (P.pos_dev ? *P.pos_dev : P.pos) : 0;
-        if (EPI == gemv::EPI_QKV && tid < P.head_dim / 2) {
-            // RoPE angles of this position, pos * theta^(-2i/head_dim), in double; read by the epilogue
-            const double ang = (double)pos * pow((double)P.theta, -(2.0 * tid) / (double)P.head_dim);
-            double sn, cs;
-            sincos(ang, &sn, &cs);
-            rope_cs[2 * tid] = (float)cs;
-            rope_cs[2 * tid + 1] = (float)sn;
-        }
+        if (EPI == gemv::EPI_QKV && tid < P.head_dim) rope_cs[tid] = rope_v;   // read by the epilogue
         named_bar_sync(1, kCons);   // limbs and the RoPE table complete
 
         const Lane L = make_lane<QT>(lane);
@@ -994,6 +1029,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
         cluster_sync(csize);
         if (rank == 0) {
             // epilogue of all rows of the pair's groups; RoPE partners (2i, 2i + 1) sit in adjacent lanes
+            const int32_t pos = (EPI == gemv::EPI_QKV) ? (P.pos_dev ? *P.pos_dev : P.pos) : 0;
             const int n_rows = (g_end - g_begin) * 16;
             for (int base = 0; base < n_rows; base += kCons) {
                 const int r = base + tid;
