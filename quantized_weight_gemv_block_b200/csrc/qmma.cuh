@@ -172,8 +172,10 @@ __device__ __forceinline__ void red_add_cluster(uint32_t addr, float v)
 //    27 and 31 zero; other formats: word 24 + l = sum of limb l over the 32 columns,
 //    words 27..31 zero).  Lane tig reads its two C columns' sums at 24 + 2 tig.
 // For the CUDA-core row-pair units every word index i of step u is stored at
-// i XOR 8 (u mod 4) (sx below): the four quarter-warps of a warp read the same words
-// of four consecutive steps, which then fall in four different bank groups.
+// i XOR 8 (u mod 4) (sx below): the four quarter-warps of a warp read the same words of
+// four consecutive steps, and a warp converting x writes four consecutive steps, which
+// then fall in four different bank groups.  The Q8_0 lane units read no sums (words
+// 24..31 hold no data there); only the tensor-core units read the zero words.
 
 // The limb words and column sums of the 4 columns a lane holds (lane w of the 8 lanes
 // of a step); the sums are already reduced over the step's lanes (or each half's).
@@ -182,7 +184,7 @@ struct XLimbs {
     int s0, s1, s2;
 };
 
-template <bool HALVES>
+template <bool HALVES, bool SUMS>
 __device__ __forceinline__ XLimbs x_limbs(float4 v, float two_s)
 {
     // z = x_int + 0x8080: bytes 0 and 1 of z are the low limbs + 128, z >> 16 the top limb
@@ -197,41 +199,47 @@ __device__ __forceinline__ XLimbs x_limbs(float4 v, float two_s)
     r.w0 = __byte_perm(lo01, lo23, 0x6420) ^ 0x80808080u;
     r.w1 = __byte_perm(lo01, lo23, 0x7531) ^ 0x80808080u;
     r.w2 = __byte_perm(__byte_perm(z0, z1, 0x0062), __byte_perm(z2, z3, 0x0062), 0x5410);
-    // column sums of the four values (byte sums of the signed limbs)
-    r.s0 = __dp4a((int)r.w0, 0x01010101, 0);
-    r.s1 = __dp4a((int)r.w1, 0x01010101, 0);
-    r.s2 = __dp4a((int)r.w2, 0x01010101, 0);
+    r.s0 = r.s1 = r.s2 = 0;
+    if (SUMS) {
+        // column sums of the four values (byte sums of the signed limbs)
+        r.s0 = __dp4a((int)r.w0, 0x01010101, 0);
+        r.s1 = __dp4a((int)r.w1, 0x01010101, 0);
+        r.s2 = __dp4a((int)r.w2, 0x01010101, 0);
 #pragma unroll
-    for (int o = 1; o < (HALVES ? 4 : 8); o <<= 1) {
-        r.s0 += __shfl_xor_sync(0xffffffffu, r.s0, o);
-        r.s1 += __shfl_xor_sync(0xffffffffu, r.s1, o);
-        r.s2 += __shfl_xor_sync(0xffffffffu, r.s2, o);
+        for (int o = 1; o < (HALVES ? 4 : 8); o <<= 1) {
+            r.s0 += __shfl_xor_sync(0xffffffffu, r.s0, o);
+            r.s1 += __shfl_xor_sync(0xffffffffu, r.s1, o);
+            r.s2 += __shfl_xor_sync(0xffffffffu, r.s2, o);
+        }
     }
     return r;
 }
 
-// Store lane w's limb words (and, from the lanes that hold them, the sums) of step xs.
-template <bool HALVES, bool PAIRED>
+// Store lane w's limb words of step xs and, from the lanes that hold them, the sums
+// (SUMS) and the zero words (ZEROS: words 27..31, or 27 and 31 with HALVES, which the
+// tensor-core units read; the CUDA-core units leave them unread).
+template <bool HALVES, bool PAIRED, bool SUMS, bool ZEROS>
 __device__ __forceinline__ void x_store(uint32_t* xs, int w, const XLimbs& r, int sx)
 {
     const int wp = PAIRED ? 2 * (w & 3) + (w >> 2) : w;
     xs[wp ^ sx] = r.w0;
     xs[(8 + wp) ^ sx] = r.w1;
     xs[(16 + wp) ^ sx] = r.w2;
+    if (!SUMS) return;
     if (HALVES) {
         if ((w & 3) == 0) {
             const int h = w >> 2;
             xs[(24 + 4 * h) ^ sx] = (uint32_t)r.s0;
             xs[(25 + 4 * h) ^ sx] = (uint32_t)r.s1;
             xs[(26 + 4 * h) ^ sx] = (uint32_t)r.s2;
-            xs[(27 + 4 * h) ^ sx] = 0u;
+            if (ZEROS) xs[(27 + 4 * h) ^ sx] = 0u;
         }
     } else {
         if (w == 0) {
             xs[24 ^ sx] = (uint32_t)r.s0;
             xs[25 ^ sx] = (uint32_t)r.s1;
             xs[26 ^ sx] = (uint32_t)r.s2;
-        } else if (w == 1) {
+        } else if (ZEROS && w == 1) {
             xs[27 ^ sx] = 0u;
             xs[28 ^ sx] = 0u;
             xs[29 ^ sx] = 0u;
@@ -724,6 +732,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
     constexpr int SPU = T::UK / 32;                         // steps per unit
     // CUDA-core path: lane units (the MMA's fragments) for Q8_0, row-pair units otherwise
     constexpr bool ROWS = CORE == 1 && QT != NTX_Q8_0_T;
+    // the x limb sums are read by every unit but the Q8_0 lane units (no code offset)
+    constexpr bool XSUMS = !(CORE == 1 && QT == NTX_Q8_0_T);
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t* full = reinterpret_cast<uint64_t*>(smem);
@@ -904,15 +914,15 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                     float4 v = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
                     if (RMS)
                         v = make_float4(v.x * w[k].x * inv, v.y * w[k].y * inv, v.z * w[k].z * inv, v.w * w[k].w * inv);
-                    r[k] = x_limbs<QT == NTX_Q6_K_T>(v, two_s);
+                    r[k] = x_limbs<QT == NTX_Q6_K_T, XSUMS>(v, two_s);
                 }
                 __syncwarp();   // every lane of a step has read its floats before any limb word lands
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int u = (tid + (j0 + k) * kCons) >> 3;
                     if (u < n_steps)
-                        x_store<QT == NTX_Q6_K_T, CORE == 1 && QT == NTX_Q8_0_T>(xq + 32 * u, wl, r[k],
-                                                                               ROWS ? 8 * (u & 3) : 0);
+                        x_store<QT == NTX_Q6_K_T, CORE == 1 && QT == NTX_Q8_0_T, XSUMS, CORE == 0>(
+                            xq + 32 * u, wl, r[k], ROWS ? 8 * (u & 3) : 0);
                 }
             };
 #pragma unroll
