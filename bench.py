@@ -217,13 +217,21 @@ def measure_gemv_roofline(ntx, model, spec, stream, iters=3):
             n = max(len(mats) * iters, 4)
             for W in mats[:4]:
                 ntx.ntx_gemv_q(q, W, r, c, x, y, stream.cuda_stream)
+            torch.cuda.synchronize()
+            # the n launches back to back in a CUDA graph, so the host's launch rate does
+            # not bound the small shapes
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n):
+                    ntx.ntx_gemv_q(q, mats[i % len(mats)], r, c, x, y, stream.cuda_stream)
+            g.replay()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
             e0.record(stream)
-            for i in range(n):
-                ntx.ntx_gemv_q(q, mats[i % len(mats)], r, c, x, y, stream.cuda_stream)
+            g.replay()
             e1.record(stream)
             torch.cuda.synchronize()
+            del g
             ms = e0.elapsed_time(e1) / n
             launches = len(mats)    # launches of this shape in one decode step
             tr = GEMV_TRAFFIC.get(f"{fmt}:{r}x{c}") if sha == GEMV_TRAFFIC_SRC_SHA else None
@@ -388,38 +396,43 @@ def gemv_bench(ntx, iters=50, tiled=True):
 
 
 def profile_gemv(what, launches):
-    """A few launches of one GEMV (weights larger than L2), nothing else: the case
-    that profiler captures of the GEMV kernel run."""
+    """A few launches of each listed GEMV (what = FMT:ROWSxCOLS[,FMT:ROWSxCOLS...],
+    weights larger than L2 or ncu's cache flush between captured launches), nothing
+    else: the case that profiler captures of the GEMV kernel run.  Per shape: one
+    warm-up launch, then `launches` launches timed together with CUDA events."""
     import torch
     import synth
     import quantized_weight_gemv_block_b200 as ntx
     from quantized_weight_gemv_block_b200 import build
     build.build()
     synth.build_dev()
-    fmt, shape = what.split(":")
-    rows, cols = (int(v) for v in shape.split("x"))
-    tiled = fmt.endswith("_t")
-    q = synth.qtype_of(fmt[:-2] if tiled else fmt)
-    W = torch.empty(rows * synth.row_bytes(q, cols), dtype=torch.uint8, device="cuda")
-    synth.blocks_dev(W, q, 0, 1, rows, cols, synth.sweep_qparams(q))
-    if tiled:
-        Wt = torch.empty_like(W)
-        ntx.ntx_repack_q(q, W, Wt, rows, cols)
-        W = Wt
-        q |= 16
-    x = torch.empty(cols, device="cuda")
-    synth.normal_f32_dev(x, 0, 2)
-    y = torch.empty(rows, device="cuda")
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    ntx.ntx_gemv_q(q, W, rows, cols, x, y)
-    torch.cuda.synchronize()
-    e0.record()
-    for _ in range(launches):
+    for one in what.split(","):
+        fmt, shape = one.split(":")
+        rows, cols = (int(v) for v in shape.split("x"))
+        tiled = fmt.endswith("_t")
+        q = synth.qtype_of(fmt[:-2] if tiled else fmt)
+        W = torch.empty(rows * synth.row_bytes(q, cols), dtype=torch.uint8, device="cuda")
+        synth.blocks_dev(W, q, 0, 1, rows, cols, synth.sweep_qparams(q))
+        if tiled:
+            Wt = torch.empty_like(W)
+            ntx.ntx_repack_q(q, W, Wt, rows, cols)
+            W = Wt
+            q |= 16
+        x = torch.empty(cols, device="cuda")
+        synth.normal_f32_dev(x, 0, 2)
+        y = torch.empty(rows, device="cuda")
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ntx.ntx_gemv_q(q, W, rows, cols, x, y)
-    e1.record()
-    torch.cuda.synchronize()
-    us = e0.elapsed_time(e1) * 1e3 / launches
-    print(json.dumps({"gemv": what, "bytes": W.numel(), "us": us, "gbs": W.numel() / (us * 1e-6) / 1e9}))
+        torch.cuda.synchronize()
+        e0.record()
+        for _ in range(launches):
+            ntx.ntx_gemv_q(q, W, rows, cols, x, y)
+        e1.record()
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / launches
+        print(json.dumps({"gemv": one, "bytes": W.numel(), "us": us, "gbs": W.numel() / (us * 1e-6) / 1e9}))
+        del W, x, y
+        torch.cuda.empty_cache()
 
 
 def profile_attn(what, launches):
@@ -467,7 +480,7 @@ def main():
                     help="weights handed to the library as tiled (repacked once at load) or GGUF-style blocks")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
-    ap.add_argument("--profile-gemv", default=None, metavar="FMT:ROWSxCOLS",
+    ap.add_argument("--profile-gemv", default=None, metavar="FMT:ROWSxCOLS[,...]",
                     help="only run the GEMV kernel on one matrix (for profilers), e.g. q6_k:28672x8192")
     ap.add_argument("--profile-attn", default=None, metavar="QHEADS:KVHEADS:CONTEXT",
                     help="only run the decode attention on one shape (for profilers), e.g. 64:8:8193")
