@@ -173,11 +173,11 @@ def gemv_shapes(spec):
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture per
 # shape, bytes per launch) of the tiled GEMV, and a hash of the kernel
 # sources it was taken with: a changed kernel reports traffic as unknown (null).
-GEMV_TRAFFIC_SRC_SHA = "e485a694e121188f"
-GEMV_TRAFFIC = {"q6_k_t:10240x8192": 69004032, "q6_k_t:8192x8192": 55123200, "q6_k_t:28672x8192": 196366848,
-                "q6_k_t:8192x28672": 195896320, "q6_k_t:128256x8192": 865172480, "q8_0_t:6144x4096": 26791424,
-                "q8_0_t:4096x4096": 17878528, "q8_0_t:14336x4096": 62471680, "q8_0_t:4096x14336": 62529280,
-                "q8_0_t:128256x4096": 561447936}
+GEMV_TRAFFIC_SRC_SHA = "ef8754e57a60e05a"
+GEMV_TRAFFIC = {"q6_k_t:10240x8192": 68894464, "q6_k_t:8192x8192": 55124736, "q6_k_t:28672x8192": 193633536,
+                "q6_k_t:8192x28672": 192967680, "q6_k_t:128256x8192": 862197504, "q8_0_t:6144x4096": 26788864,
+                "q8_0_t:4096x4096": 17875968, "q8_0_t:14336x4096": 62442240, "q8_0_t:4096x14336": 62483456,
+                "q8_0_t:128256x4096": 558348032}
 
 
 def gemv_sources_sha():
