@@ -173,11 +173,11 @@ def gemv_shapes(spec):
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture per
 # shape, bytes per launch) of the tiled GEMV, and a hash of the kernel
 # sources it was taken with: a changed kernel reports traffic as unknown (null).
-GEMV_TRAFFIC_SRC_SHA = "ef8754e57a60e05a"
-GEMV_TRAFFIC = {"q6_k_t:10240x8192": 68894464, "q6_k_t:8192x8192": 55124736, "q6_k_t:28672x8192": 193633536,
-                "q6_k_t:8192x28672": 192967680, "q6_k_t:128256x8192": 862197504, "q8_0_t:6144x4096": 26788864,
-                "q8_0_t:4096x4096": 17875968, "q8_0_t:14336x4096": 62442240, "q8_0_t:4096x14336": 62483456,
-                "q8_0_t:128256x4096": 558348032}
+GEMV_TRAFFIC_SRC_SHA = "d118f419951f3ecf"
+GEMV_TRAFFIC = {"q6_k_t:10240x8192": 68896512, "q6_k_t:8192x8192": 55124992, "q6_k_t:28672x8192": 192979200,
+                "q6_k_t:8192x28672": 192954624, "q6_k_t:128256x8192": 862085888, "q8_0_t:6144x4096": 26788864,
+                "q8_0_t:4096x4096": 17875968, "q8_0_t:14336x4096": 62440448, "q8_0_t:4096x14336": 62481664,
+                "q8_0_t:128256x4096": 558824960}
 
 
 def gemv_sources_sha():
@@ -380,19 +380,49 @@ def gemv_bench(ntx, iters=50, tiled=True):
     x = torch.empty(cols, device="cuda")
     synth.normal_f32_dev(x, 0, 2)
     y = torch.empty(rows, device="cuda")
-    s = torch.cuda.current_stream()
+    s = torch.cuda.Stream()
     for c in copies:
-        ntx.ntx_gemv_q(q, c, rows, cols, x, y)
+        ntx.ntx_gemv_q(q, c, rows, cols, x, y, s.cuda_stream)
+    torch.cuda.synchronize()
+    # back to back from a CUDA graph, so the host's launch rate does not bound them
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        for i in range(iters):
+            ntx.ntx_gemv_q(q, copies[i % 16], rows, cols, x, y, s.cuda_stream)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(s):   # replay() launches on the current stream
+        g.replay()
+        torch.cuda.synchronize()
+        e0.record(s)
+        g.replay()
+        e1.record(s)
     torch.cuda.synchronize()
-    e0.record(s)
-    for i in range(iters):
-        ntx.ntx_gemv_q(q, copies[i % 16], rows, cols, x, y)
-    e1.record(s)
-    torch.cuda.synchronize()
+    del g
     us = e0.elapsed_time(e1) * 1e3 / iters
     nbytes = rows * rb + 4 * (rows + cols)
     return {"us": us, "gbs": nbytes / (us * 1e-6) / 1e9}
+
+
+def measure_read_ceiling(ntx, stream, nbytes=4 << 30, iters=10):
+    """The practical HBM ceiling of the GEMV's data path: ntx_stream_read_probe (one CTA
+    per SM, 1-D bulk copies into a shared-memory ring, no arithmetic) over a buffer much
+    larger than L2, timed with CUDA events on the bench stream."""
+    import torch
+    buf = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    buf.fill_(1)
+    for _ in range(3):
+        ntx.ntx_stream_read_probe(buf, nbytes, stream.cuda_stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(iters):
+        ntx.ntx_stream_read_probe(buf, nbytes, stream.cuda_stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / iters
+    del buf
+    torch.cuda.empty_cache()
+    return nbytes / (ms * 1e-3) / 1e9
 
 
 def profile_gemv(what, launches):
@@ -548,6 +578,10 @@ def main():
                             "frac": agg["achieved"] / peak, "traffic": agg["traffic"],
                             "bytes_per_launch": agg["bytes_per_launch"], "avg_launch_us": agg["avg_launch_us"]}
         line["gemv_shapes"] = per_shape
+        ceil_gbs = measure_read_ceiling(ntx, stream)
+        line["read_ceiling"] = {"kernel": "ntx_stream_read_probe (bulk-copy ring, one CTA per SM, no arithmetic)",
+                                "gbs": ceil_gbs, "frac_of_%s" % peak_kind: ceil_gbs / peak}
+        line["roofline"]["frac_of_read_ceiling"] = agg["achieved"] / ceil_gbs
         if not args.no_extras:
             line["gemv_q8_0_4096x4096"] = {"tiled": gemv_bench(ntx, tiled=True), "gguf": gemv_bench(ntx, tiled=False)}
         if not args.no_cpu_baseline:

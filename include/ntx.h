@@ -127,9 +127,20 @@ ntx_status ntx_device_error(uint32_t* code);
  * of the codes with x as 24-bit fixed point (relative to max |x|) by dp4a on the
  * CUDA cores (NTX_GEMV_CORE=tc selects integer MMAs instead; same results up to
  * fp32 rounding order); GGUF-style rows whose byte length is a multiple of 16
- * take the bulk-copy fp32 CUDA-core pipeline; other shapes a simpler kernel. */
+ * take the bulk-copy fp32 CUDA-core pipeline; other shapes a simpler kernel.
+ * The two pipelines launch as programmatic dependents: when the previous kernel
+ * on the stream is one of this library's, they start streaming W before it has
+ * finished (x is read and y written only after it completed), so W must not be
+ * written by that previous kernel (no kernel of this library writes weights). */
 ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t cols, const float* x, float* y,
                       void* stream);
+
+/* Measurement helper, not part of the decode path: streams `bytes` bytes of src
+ * (device, 16-byte aligned, a multiple of 16 bytes) from HBM into shared memory the
+ * way the tiled GEMV streams its weights (one CTA per SM, 1-D bulk copies, L2
+ * evict-first, a ring of 24 KB stages) and does nothing else; its bytes per second
+ * are the practical ceiling of the GEMV's data path.  Asynchronous on `stream`. */
+ntx_status ntx_stream_read_probe(const void* src, size_t bytes, void* stream);
 
 /* Repack W [rows, cols] from the GGUF-style layout of `qtype` (NTX_Q8_0 ..
  * NTX_Q6_K) into the tiled layout qtype | NTX_TILED, device to device: W_tiled

@@ -22,6 +22,7 @@ STATUS_NAMES = {0: "NTX_OK", 1: "NTX_EINVAL", 2: "NTX_EUNSUPPORTED", 3: "NTX_ENO
 
 # Every symbol of include/ntx.h.
 EXPORTS = ("ntx_last_error", "ntx_version", "ntx_row_bytes", "ntx_block_elems", "ntx_device_error", "ntx_gemv_q",
+           "ntx_stream_read_probe",
            "ntx_dequant_q", "ntx_repack_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_decode_noalloc", "ntx_attn_workspace_bytes", "ntx_swiglu",
            "ntx_softmax", "ntx_argmax", "ntx_embed", "ntx_model_create", "ntx_model_destroy", "ntx_decode_step",
            "ntx_stream_layers", "ntx_stream_stats")
@@ -67,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "ntx_block_elems": ([ci], ci),
             "ntx_device_error": ([ctypes.POINTER(ctypes.c_uint32)], ci),
             "ntx_gemv_q": ([ci, vp, i64, i64, vp, vp, vp], ci),
+            "ntx_stream_read_probe": ([vp, sz, vp], ci),
             "ntx_dequant_q": ([ci, vp, i64, i64, vp, vp], ci),
             "ntx_repack_q": ([ci, vp, vp, i64, i64, vp], ci),
             "ntx_rmsnorm": ([vp, vp, vp, i64, cf, vp], ci),
@@ -138,6 +140,10 @@ def ntx_device_error() -> int:
 
 def ntx_gemv_q(qtype, W, rows, cols, x, y, stream=None) -> None:
     check(lib().ntx_gemv_q(qtype, _p(W), rows, cols, _p(x), _p(y), _s(stream)))
+
+
+def ntx_stream_read_probe(src, nbytes, stream=None) -> None:
+    check(lib().ntx_stream_read_probe(_p(src), nbytes, _s(stream)))
 
 
 def ntx_dequant_q(qtype, W, rows, cols, out, stream=None) -> None:

@@ -53,10 +53,12 @@ NTX_EXPORT ntx_status ntx_device_error(uint32_t* code)
 {
     if (!code) return fail(NTX_EINVAL, "ntx_device_error: null pointer");
     NTX_CUDA_TRY(cudaDeviceSynchronize());
-    uint32_t a = 0, b = 0, c = 0;
+    uint32_t a = 0, b = 0, c = 0, d = 0, e = 0;
     NTX_CUDA_TRY(take_device_error_gemv(&a));
     NTX_CUDA_TRY(take_device_error_attn(&b));
     NTX_CUDA_TRY(take_device_error_decode(&c));
-    *code = a | b | c;
+    NTX_CUDA_TRY(take_device_error_qmma(&d));
+    NTX_CUDA_TRY(take_device_error_probe(&e));
+    *code = a | b | c | d | e;
     return NTX_OK;
 }

@@ -54,6 +54,8 @@ static inline cudaError_t take_tu_device_error(uint32_t* out)
 cudaError_t take_device_error_gemv(uint32_t* out);
 cudaError_t take_device_error_attn(uint32_t* out);
 cudaError_t take_device_error_decode(uint32_t* out);
+cudaError_t take_device_error_qmma(uint32_t* out);
+cudaError_t take_device_error_probe(uint32_t* out);
 
 int num_sms();
 

@@ -137,6 +137,9 @@ NTX_EXPORT ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t
         P.K = (int)cols;
         P.x = x;
         P.y = y;
+        // programmatic dependent launch: the weight stream may start while the previous
+        // kernel of the stream finishes; x is read and y written only after it completed
+        P.use_pdl = true;
         return gemv_launch(qtype, gemv::EPI_STORE, gemv::PRO_X, P, s);
     }
     const int threads = 256, warps = threads / 32;

@@ -293,4 +293,7 @@ ntx_status repack_launch(int qtype, const void* W, void* W_tiled, int64_t rows, 
     return check_launch("ntx_repack_q");
 }
 
+// The tiled GEMV's device error flag (this translation unit's).
+cudaError_t take_device_error_qmma(uint32_t* out) { return take_tu_device_error(out); }
+
 }  // namespace ntx

@@ -289,3 +289,40 @@ def test_tiled_input_edge_cases(ntx, orc, syn, monkeypatch, core, qtype):
     for scale in (1e-30, 1e25):
         xs = (syn.normal_f32_host(4, 12, cols) * np.float32(scale)).astype(np.float32)
         assert rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, xs), orc.gemv(qtype, host, rows, cols, xs)) <= GEMV_TIGHT
+
+
+@pytest.mark.parametrize("qtype", [Q8_0 | T, Q6_K | T, Q8_0], ids=["q8_0_t", "q6_k_t", "q8_0"])
+def test_gemv_chain_without_sync(ntx, orc, syn, qtype):
+    """Back-to-back GEMVs on one stream (programmatic dependent launch): the second
+    reads the first's output, and a third overwrites the first's input; each matches the
+    oracle on the values it actually read."""
+    base = qtype & ~T
+    K1, M1 = (8192 + 256, 512) if base == Q6_K else (4096 + 32, 512)
+    M2 = M1
+    h1, W1 = (make_tiled(ntx, syn, base, M1, K1, seed=3) if qtype & T else make(syn, base, M1, K1, 3))
+    K2 = M1 if base != Q6_K else 512
+    h2, W2 = (make_tiled(ntx, syn, base, M2, K2, seed=4) if qtype & T else make(syn, base, M2, K2, 4))
+    h3, W3 = (make_tiled(ntx, syn, base, K1, M2, seed=5) if qtype & T else make(syn, base, K1, M2, 5))
+    x = torch.from_numpy(syn.normal_f32_host(6, 12, K1)).cuda()
+    x0 = x.cpu().numpy().copy()
+    a = torch.empty(M1, dtype=torch.float32, device="cuda")
+    b = torch.empty(M2, dtype=torch.float32, device="cuda")
+    ntx.ntx_gemv_q(qtype, W1, M1, K1, x, a)      # a = W1 x
+    ntx.ntx_gemv_q(qtype, W2, M2, K2, a, b)      # b = W2 a (reads the previous output)
+    ntx.ntx_gemv_q(qtype, W3, K1, M2, b, x)      # x = W3 b (overwrites the first input)
+    torch.cuda.synchronize()
+    an, bn, xn = a.cpu().numpy(), b.cpu().numpy(), x.cpu().numpy()
+    assert rel_err(an, orc.gemv(base, h1, M1, K1, x0)) <= GEMV_TIGHT
+    assert rel_err(bn, orc.gemv(base, h2, M2, K2, an)) <= GEMV_TIGHT
+    assert rel_err(xn, orc.gemv(base, h3, K1, M2, bn)) <= GEMV_TIGHT
+
+
+def test_stream_read_probe(ntx):
+    """The HBM read probe streams a buffer (larger than L2, with a ragged tail slice)
+    without a device error."""
+    buf = torch.empty((256 << 20) + 48, dtype=torch.uint8, device="cuda")
+    ntx.ntx_stream_read_probe(buf, buf.numel())
+    torch.cuda.synchronize()
+    assert ntx.ntx_device_error() == 0
+    with pytest.raises(ntx.NtxError):
+        ntx.ntx_stream_read_probe(buf, 100)
