@@ -79,7 +79,8 @@ ORC_EXPORT int orc_block_elems(int qtype)
 {
     switch (qtype) {
     case ORC_Q8_0: case ORC_Q4_0: return 32;
-    case ORC_Q4_K: case ORC_Q6_K: return 256;
+    case ORC_Q4_K: case ORC_Q6_K: case ORC_Q5_K: return 256;
+    case ORC_F16: case ORC_F32: return 1;
     default: return 0;
     }
 }
@@ -91,6 +92,9 @@ ORC_EXPORT int orc_block_bytes(int qtype)
     case ORC_Q4_0: return 18;
     case ORC_Q4_K: return 144;
     case ORC_Q6_K: return 210;
+    case ORC_Q5_K: return 176;
+    case ORC_F16: return 2;
+    case ORC_F32: return 4;
     default: return 0;
     }
 }
@@ -174,6 +178,38 @@ static void dq_q6_k(const uint8_t* b, float* w)
     }
 }
 
+/* Q5_K (176 B / 256 weights): fp16 d, fp16 dmin, 12 bytes of scales/mins packed
+ * as in Q4_K, 32 bytes qh of fifth code bits, 128 bytes qs of low 4 code bits.
+ * (Format named with the K-quants in "Descripción general de NTransformer"; the
+ * pages print no layout, so this is the GGUF convention as best known.)  Element
+ * 64c + l (c = 0..3, l = 0..31): low 4 bits = low nibble of qs[32c + l], fifth bit =
+ * bit 2c of qh[l]; element 64c + 32 + l: high nibble of qs[32c + l] and bit 2c + 1 of
+ * qh[l].  q in 0..31, sub-block j = e / 32, w = d * scale_j * q - dmin * min_j. */
+static void dq_q5_k(const uint8_t* b, float* w)
+{
+    float d = f16_at(b), dmin = f16_at(b + 2);
+    const uint8_t* s = b + 4;
+    const uint8_t* qh = b + 16;
+    const uint8_t* qs = b + 48;
+    for (int e = 0; e < 256; ++e) {
+        int c = e / 64, r = e % 64, l = r % 32, upper = r >= 32;
+        int lo = upper ? (qs[32 * c + l] >> 4) : (qs[32 * c + l] & 15);
+        int hi = (qh[l] >> (2 * c + upper)) & 1;
+        int q = lo + 16 * hi;
+        int sc, m;
+        q4k_scale_min(s, e / 32, &sc, &m);
+        float a = (d * (float)sc) * (float)q;   /* exact: at most 22 significant bits */
+        float z = dmin * (float)m;              /* exact */
+        w[e] = a - z;                           /* the one rounding */
+    }
+}
+
+/* F16: one IEEE binary16 value per weight (little-endian); F32: one binary32.
+ * (Formats named in "Descripción general de NTransformer".) */
+static void dq_f16(const uint8_t* b, float* w) { *w = f16_at(b); }
+
+static void dq_f32(const uint8_t* b, float* w) { memcpy(w, b, 4); }
+
 static int dequant_block(int qtype, const uint8_t* b, float* w)
 {
     switch (qtype) {
@@ -181,6 +217,9 @@ static int dequant_block(int qtype, const uint8_t* b, float* w)
     case ORC_Q4_0: dq_q4_0(b, w); return 0;
     case ORC_Q4_K: dq_q4_k(b, w); return 0;
     case ORC_Q6_K: dq_q6_k(b, w); return 0;
+    case ORC_Q5_K: dq_q5_k(b, w); return 0;
+    case ORC_F16: dq_f16(b, w); return 0;
+    case ORC_F32: dq_f32(b, w); return 0;
     default: return -1;
     }
 }

@@ -29,7 +29,7 @@
 extern "C" {
 #endif
 
-enum { ORC_Q8_0 = 0, ORC_Q4_0 = 1, ORC_Q4_K = 2, ORC_Q6_K = 3 };
+enum { ORC_Q8_0 = 0, ORC_Q4_0 = 1, ORC_Q4_K = 2, ORC_Q6_K = 3, ORC_Q5_K = 4, ORC_F16 = 5, ORC_F32 = 6 };
 
 float orc_f16_to_f32(uint16_t h);
 uint16_t orc_f32_to_f16(float f);

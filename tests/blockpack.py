@@ -60,6 +60,30 @@ def pack_q6_k(d_bits: int, sc, q) -> bytes:
     return bytes(ql + qh + [v & 0xFF for v in sc] + [d_bits & 0xFF, d_bits >> 8])
 
 
+def pack_q5_k(d_bits: int, dmin_bits: int, sc, m, q) -> bytes:
+    sc, m, q = [int(v) for v in sc], [int(v) for v in m], [int(v) for v in q]
+    assert len(sc) == 8 and len(m) == 8 and len(q) == 256
+    assert all(0 <= v < 64 for v in sc + m) and all(0 <= v < 32 for v in q)
+    # scales and mins exactly as Q4_K: reuse that packer's 12 bytes
+    s = list(pack_q4_k(0, 0, sc, m, [0] * 256)[4:16])
+    qh = [0] * 32
+    qs = [0] * 128
+    for e in range(256):
+        chunk, r = divmod(e, 64)
+        upper, lane = divmod(r, 32)
+        qs[32 * chunk + lane] |= (q[e] & 15) << (4 * upper)
+        qh[lane] |= (q[e] >> 4) << (2 * chunk + upper)
+    return bytes([d_bits & 0xFF, d_bits >> 8, dmin_bits & 0xFF, dmin_bits >> 8] + s + qh + qs)
+
+
+def pack_f16(bits) -> bytes:
+    return b"".join(bytes([int(v) & 0xFF, int(v) >> 8]) for v in bits)
+
+
+def pack_f32(values) -> bytes:
+    return np.array(values, dtype=np.float32).tobytes()
+
+
 def logical_weights(qtype: int, fields: dict) -> list:
     """Exact (Fraction) weights of one block from its logical fields."""
     from fractions import Fraction as Fr
@@ -79,6 +103,13 @@ def logical_weights(qtype: int, fields: dict) -> list:
     if qtype == 3:
         d = f16(fields["d"])
         return [d * fields["sc"][e // 16] * (fields["q"][e] - 32) for e in range(256)]
+    if qtype == 4:
+        d, dmin = f16(fields["d"]), f16(fields["dmin"])
+        return [d * fields["sc"][e // 32] * fields["q"][e] - dmin * fields["m"][e // 32] for e in range(256)]
+    if qtype == 5:
+        return [f16(b) for b in fields["bits"]]
+    if qtype == 6:
+        return [Fr(float(v)) for v in np.array(fields["values"], dtype=np.float32)]
     raise ValueError(qtype)
 
 
@@ -93,6 +124,15 @@ def random_fields(qtype: int, rng: np.random.Generator, d_range=(1e-3, 1e-2)) ->
                 "m": rng.integers(0, 64, 8), "q": rng.integers(0, 16, 256)}
     if qtype == 3:
         return {"d": d, "sc": rng.integers(-127, 128, 16), "q": rng.integers(0, 64, 256)}
+    if qtype == 4:
+        return {"d": d, "dmin": f16_bits(rng.uniform(*d_range)), "sc": rng.integers(0, 64, 8),
+                "m": rng.integers(0, 64, 8), "q": rng.integers(0, 32, 256)}
+    if qtype == 5:
+        # finite binary16 patterns of both signs, subnormals included
+        bits = rng.integers(0, 0x7C00, 1) | (rng.integers(0, 2, 1) << 15)
+        return {"bits": bits}
+    if qtype == 6:
+        return {"values": rng.standard_normal(1).astype(np.float32) * np.float32(10.0) ** rng.integers(-30, 30)}
     raise ValueError(qtype)
 
 
@@ -103,7 +143,15 @@ def pack(qtype: int, f: dict) -> bytes:
         return pack_q4_0(f["d"], f["q"])
     if qtype == 2:
         return pack_q4_k(f["d"], f["dmin"], f["sc"], f["m"], f["q"])
-    return pack_q6_k(f["d"], f["sc"], f["q"])
+    if qtype == 3:
+        return pack_q6_k(f["d"], f["sc"], f["q"])
+    if qtype == 4:
+        return pack_q5_k(f["d"], f["dmin"], f["sc"], f["m"], f["q"])
+    if qtype == 5:
+        return pack_f16(f["bits"])
+    if qtype == 6:
+        return pack_f32(f["values"])
+    raise ValueError(qtype)
 
 
 def parse_golden(path: str):

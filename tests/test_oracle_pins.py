@@ -16,8 +16,22 @@ import pytest
 import blockpack as bp
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
-QT = {"q8_0": 0, "q4_0": 1, "q4_k": 2, "q6_k": 3}
-BLOCK = {0: (32, 34), 1: (32, 18), 2: (256, 144), 3: (256, 210)}
+QT = {"q8_0": 0, "q4_0": 1, "q4_k": 2, "q6_k": 3, "q5_k": 4, "f16": 5, "f32": 6}
+BLOCK = {0: (32, 34), 1: (32, 18), 2: (256, 144), 3: (256, 210), 4: (256, 176), 5: (1, 2), 6: (1, 4)}
+ALL = [0, 1, 2, 3, 4, 5, 6]
+
+
+def integer_fields(qtype, rng):
+    """Random fields whose weights are all integers (d = dmin = 1, or integer values)."""
+    if qtype == 5:
+        return {"bits": [bp.f16_bits(float(rng.integers(-50, 51)))]}
+    if qtype == 6:
+        return {"values": [float(rng.integers(-50, 51))]}
+    f = bp.random_fields(qtype, rng)
+    f["d"] = bp.f16_bits(1.0)
+    if qtype in (2, 4):
+        f["dmin"] = bp.f16_bits(1.0)
+    return f
 
 
 # ------------------------------------------------------------------ fp16
@@ -70,12 +84,12 @@ def test_golden_blocks(orc, path):
 
 # -------------------------------------------------- round trip of random blocks
 
-@pytest.mark.parametrize("qtype", [0, 1, 2, 3])
+@pytest.mark.parametrize("qtype", ALL)
 def test_dequant_round_trip(orc, qtype):
     """pack(logical fields) -> oracle dequant == exact value of d/scale/min/code, bit for bit."""
     rng = np.random.default_rng(10 + qtype)
     be, bb = BLOCK[qtype]
-    nblk = 24
+    nblk = 24 if be > 1 else 4096
     fields = [bp.random_fields(qtype, rng) for _ in range(nblk)]
     # plus extreme fields: largest codes and scales, subnormal d
     ext = bp.random_fields(qtype, rng)
@@ -87,6 +101,16 @@ def test_dequant_round_trip(orc, qtype):
     if qtype == 3:
         ext["sc"][:] = -128
         ext["q"][:] = 0
+    if qtype == 4:
+        ext["sc"][:] = 63
+        ext["m"][:] = 63
+        ext["q"][:] = 31
+    if qtype == 5:
+        ext = {"bits": [0x0001]}            # smallest subnormal
+        fields.append({"bits": [0x7BFF]})   # largest finite
+        fields.append({"bits": [0x8000]})   # negative zero
+    if qtype == 6:
+        ext = {"values": [np.float32(1e-45)]}   # smallest fp32 subnormal
     fields.append(ext)
     raw = b"".join(bp.pack(qtype, f) for f in fields)
     got = orc.dequant(qtype, np.frombuffer(raw, dtype=np.uint8), 1, be * len(fields))[0]
@@ -96,22 +120,18 @@ def test_dequant_round_trip(orc, qtype):
 
 # ------------------------------------------------------------------ GEMV
 
-@pytest.mark.parametrize("qtype", [0, 1, 2, 3])
+@pytest.mark.parametrize("qtype", ALL)
 def test_gemv_exact_integers(orc, qtype):
     """d = dmin = 1 and integer x: every product and sum is an integer, so y is exact."""
     rng = np.random.default_rng(20 + qtype)
     be, bb = BLOCK[qtype]
-    rows, nb = 5, 3
+    rows, nb = 5, (3 if be > 1 else 96)
     cols = nb * be
-    one = bp.f16_bits(1.0)
     W = np.zeros((rows, nb * bb), dtype=np.uint8)
     wint = np.zeros((rows, cols), dtype=np.int64)
     for r in range(rows):
         for b in range(nb):
-            f = bp.random_fields(qtype, rng)
-            f["d"] = one
-            if qtype == 2:
-                f["dmin"] = one
+            f = integer_fields(qtype, rng)
             W[r, b * bb:(b + 1) * bb] = np.frombuffer(bp.pack(qtype, f), dtype=np.uint8)
             wint[r, b * be:(b + 1) * be] = [int(v) for v in bp.logical_weights(qtype, f)]
     x = rng.integers(-9, 10, cols)
@@ -134,12 +154,12 @@ def test_gemv_one_hot_picks_column(orc):
         assert np.array_equal(orc.gemv(0, W, rows, cols, x), dense[:, k].astype(np.float32))
 
 
-@pytest.mark.parametrize("qtype", [0, 1, 2, 3])
+@pytest.mark.parametrize("qtype", ALL)
 def test_gemv_matches_exact_rational(orc, qtype):
     """Double accumulation of exact products: result is the exact dot product to ~1 ulp of fp32."""
     rng = np.random.default_rng(30 + qtype)
     be, bb = BLOCK[qtype]
-    rows, nb = 3, 2
+    rows, nb = 3, (2 if be > 1 else 64)
     cols = nb * be
     fields = [[bp.random_fields(qtype, rng) for _ in range(nb)] for _ in range(rows)]
     W = np.frombuffer(b"".join(bp.pack(qtype, f) for rf in fields for f in rf), dtype=np.uint8)
