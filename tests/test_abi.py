@@ -57,6 +57,12 @@ def test_gemv_rejects_bad_arguments(ntx):
     assert _status(ntx, "ntx_gemv_q", 0, p, 4, 256, p + 2, p, None) == ntx.NTX_EINVAL
     assert "aligned" in ntx.ntx_last_error()
     assert _status(ntx, "ntx_dequant_q", 3, p, 1, 100, p, None) == ntx.NTX_EINVAL
+    # tiled layouts take whole 16-row groups
+    assert _status(ntx, "ntx_gemv_q", 16, p, 40, 256, p, p, None) == ntx.NTX_EINVAL
+    # formats without GPU kernels yet (Q5_K, F16, F32 codes) are rejected, not misread
+    for q in (4, 5, 6, 20):
+        assert _status(ntx, "ntx_gemv_q", q, p, 16, 256, p, p, None) == ntx.NTX_EINVAL
+    assert ntx.lib().ntx_row_bytes(4, 256) == 0
 
 
 def test_ops_reject_bad_arguments(ntx):
@@ -117,6 +123,13 @@ def test_decode_entry_points_reject_null_model(ntx):
     assert ntx.lib().ntx_stream_layers(None, 0, 0, 0x10000, None, None, 0) == ntx.NTX_EINVAL
     assert ntx.lib().ntx_model_destroy(None) == ntx.NTX_EINVAL
     assert ntx.lib().ntx_device_error(None) == ntx.NTX_EINVAL
+
+
+def test_read_probe_rejects_bad_arguments(ntx):
+    p = 1 << 20
+    assert _status(ntx, "ntx_stream_read_probe", None, 256, None) == ntx.NTX_EINVAL
+    assert _status(ntx, "ntx_stream_read_probe", p, 100, None) == ntx.NTX_EINVAL       # not a multiple of 16
+    assert _status(ntx, "ntx_stream_read_probe", p + 8, 256, None) == ntx.NTX_EINVAL   # not 16-byte aligned
 
 
 def test_repack_rejects_bad_arguments(ntx):
