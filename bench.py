@@ -124,11 +124,14 @@ def barrier(world):
 
 
 def max_over_ranks(v, world):
+    """The largest of the ranks' values (step times: the job is as slow as its slowest
+    replica); NCCL reduces a device tensor, gloo a host one."""
     if world == 1:
         return v
     import torch
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
@@ -522,7 +525,11 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    rank, world, local = dist_setup(args.gpus)
+    if args.impl == "reference":
+        # the CPU oracle needs no process group: rank 0 alone runs it, the others exit
+        rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
+    else:
+        rank, world, local = dist_setup(args.gpus)
     spec = spec_for(args.workload, args.layout)
     config = {"workload": args.workload, "layers": spec.n_layers, "hidden": spec.hidden, "ffn": spec.ffn,
               "q_heads": spec.n_q_heads, "kv_heads": spec.n_kv_heads, "vocab": spec.vocab, "format": ["q8_0", "q4_0",
