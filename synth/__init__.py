@@ -36,10 +36,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 HOST_LIB = os.path.join(_HERE, "libsynth_host.so")
 DEV_LIB = os.path.join(_HERE, "libsynth_dev.so")
 
-Q8_0, Q4_0, Q4_K, Q6_K = 0, 1, 2, 3
-QTYPE_NAMES = {"q8_0": Q8_0, "q4_0": Q4_0, "q4_k": Q4_K, "q6_k": Q6_K}
+Q8_0, Q4_0, Q4_K, Q6_K, Q5_K = 0, 1, 2, 3, 4
+QTYPE_NAMES = {"q8_0": Q8_0, "q4_0": Q4_0, "q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K}
 # (elements per block, bytes per block)
-BLOCK = {Q8_0: (32, 34), Q4_0: (32, 18), Q4_K: (256, 144), Q6_K: (256, 210)}
+BLOCK = {Q8_0: (32, 34), Q4_0: (32, 18), Q4_K: (256, 144), Q6_K: (256, 210), Q5_K: (256, 176)}
 
 
 def qtype_of(name) -> int:
@@ -83,6 +83,12 @@ def _code_mean_square(qtype: int) -> float:
         for s in range(1, 9):
             m = (15 * s + 1) // 2
             acc.append(np.mean((s * np.arange(16, dtype=np.float64) - m) ** 2))
+        return float(np.mean(acc))
+    if qtype == Q5_K:
+        acc = []
+        for s in range(1, 5):
+            m = (31 * s + 1) // 2
+            acc.append(np.mean((s * np.arange(32, dtype=np.float64) - m) ** 2))
         return float(np.mean(acc))
     if qtype == Q6_K:
         sc2 = np.mean(np.arange(1, 17, dtype=np.float64) ** 2)

@@ -18,6 +18,9 @@
  *                               scales and mins | [16,144) 4-bit codes
  *   Q6_K (210 B / 256 weights): [0,128) low 4 code bits | [128,192) high 2 code bits
  *                               | [192,208) int8 sub-block scales | [208,210) fp16 d
+ *   Q5_K (176 B / 256 weights): [0,2) fp16 d | [2,4) fp16 dmin | [4,16) packed 6-bit
+ *                               scales and mins (as Q4_K) | [16,48) fifth code bits |
+ *                               [48,176) low 4 code bits
  * Codes are random bytes; only the scale fields are shaped (see syn_fill_block).
  */
 #ifndef SYNTH_H
@@ -36,14 +39,16 @@
 #define SYN_Q4_0 1
 #define SYN_Q4_K 2
 #define SYN_Q6_K 3
+#define SYN_Q5_K 4
 
 /* Scale-field distribution of one tensor.
  *   d = fp16(k * 2^d_exp) with k uniform in [d_lo, d_hi]
  *   mode 0: the sweep distribution: Q4_K 6-bit scales/mins uniform in 0..63 and
  *           dmin drawn like d; Q6_K sub-scales uniform in -127..127.
  *   mode 1: the decode distribution: Q4_K scales uniform in 1..8, mins =
- *           round(7.5 * scale) (so weights are centred), dmin = d; Q6_K sub-scales
- *           uniform in 1..16.
+ *           round(7.5 * scale) (so weights are centred), dmin = d; Q5_K scales
+ *           uniform in 1..4, mins = round(15.5 * scale); Q6_K sub-scales uniform in
+ *           1..16.  (Q5_K uses the sweep rule of Q4_K in mode 0.)
  * Q8_0 codes are uniform in -127..127 and Q4_0 / Q4_K / Q6_K codes are uniform
  * over their full range in both modes. */
 typedef struct syn_qparams {
@@ -135,18 +140,33 @@ SYN_HD uint16_t syn_scale_bits(uint32_t r, const syn_qparams* P)
 
 SYN_HD int syn_block_bytes(int qtype)
 {
-    return qtype == SYN_Q8_0 ? 34 : qtype == SYN_Q4_0 ? 18 : qtype == SYN_Q4_K ? 144 : qtype == SYN_Q6_K ? 210 : 0;
+    return qtype == SYN_Q8_0 ? 34 : qtype == SYN_Q4_0 ? 18 : qtype == SYN_Q4_K ? 144 : qtype == SYN_Q6_K ? 210
+         : qtype == SYN_Q5_K ? 176 : 0;
 }
 
 SYN_HD int syn_block_elems(int qtype)
 {
-    return (qtype == SYN_Q8_0 || qtype == SYN_Q4_0) ? 32 : (qtype == SYN_Q4_K || qtype == SYN_Q6_K) ? 256 : 0;
+    return (qtype == SYN_Q8_0 || qtype == SYN_Q4_0) ? 32
+         : (qtype == SYN_Q4_K || qtype == SYN_Q6_K || qtype == SYN_Q5_K) ? 256 : 0;
 }
 
 /* Draws consumed per block (block b uses draws [b*D, b*D + D)). */
 SYN_HD uint64_t syn_block_draws(int qtype)
 {
-    return qtype == SYN_Q8_0 ? 17 : qtype == SYN_Q4_0 ? 3 : qtype == SYN_Q4_K ? 19 : 33;
+    return qtype == SYN_Q8_0 ? 17 : qtype == SYN_Q4_0 ? 3 : qtype == SYN_Q4_K ? 19 : qtype == SYN_Q5_K ? 23 : 33;
+}
+
+/* 6-bit scale / min packing of the K-quants: sub-blocks 0..3 whole in bytes 0..3 (scale)
+ * and 4..7 (min); sub-blocks 4..7 keep their low 4 bits in bytes 8..11 (scale low nibble,
+ * min high nibble) and their top 2 bits in the top bits of bytes 0..3 (scale) and 4..7
+ * (min). */
+SYN_HD void syn_pack_k_scales(const uint8_t* s6, const uint8_t* m6, uint8_t* sc)
+{
+    for (int j = 0; j < 4; ++j) {
+        sc[j] = (uint8_t)(s6[j] | ((s6[j + 4] >> 4) << 6));
+        sc[j + 4] = (uint8_t)(m6[j] | ((m6[j + 4] >> 4) << 6));
+        sc[j + 8] = (uint8_t)((s6[j + 4] & 0xF) | ((m6[j + 4] & 0xF) << 4));
+    }
 }
 
 /* Write block number `b` of the tensor with stream key `key` to out[0 .. block_bytes). */
@@ -182,17 +202,31 @@ SYN_HD void syn_fill_block(int qtype, uint64_t key, uint64_t b, const syn_qparam
                 s6[j] = (uint8_t)(1 + ((r1 >> (3 * j)) & 7));
                 m6[j] = (uint8_t)((15 * s6[j] + 1) / 2);
             }
-            /* 6-bit packing: sub-blocks 0..3 whole in bytes 0..3 (scale) and 4..7
-             * (min); sub-blocks 4..7 keep their low 4 bits in bytes 8..11 (scale low
-             * nibble, min high nibble) and their top 2 bits in the top bits of
-             * bytes 0..3 (scale) and 4..7 (min). */
-            for (int j = 0; j < 4; ++j) {
-                sc[j] = (uint8_t)(s6[j] | ((s6[j + 4] >> 4) << 6));
-                sc[j + 4] = (uint8_t)(m6[j] | ((m6[j + 4] >> 4) << 6));
-                sc[j + 8] = (uint8_t)((s6[j + 4] & 0xF) | ((m6[j + 4] & 0xF) << 4));
-            }
+            syn_pack_k_scales(s6, m6, sc);
         }
         for (int i = 0; i < 16; ++i) syn_put_u64(out + 16 + 8 * i, syn_draw(key, n0 + 3 + i));
+    } else if (qtype == SYN_Q5_K) {
+        uint64_t r0 = syn_draw(key, n0);
+        uint16_t d = syn_scale_bits((uint32_t)r0, P);
+        syn_put_u16(out, d);
+        uint8_t* sc = out + 4;
+        if (P->mode == 0) {
+            syn_put_u16(out + 2, syn_scale_bits((uint32_t)(r0 >> 32), P));
+            uint64_t r1 = syn_draw(key, n0 + 1), r2 = syn_draw(key, n0 + 2);
+            for (int i = 0; i < 8; ++i) sc[i] = (uint8_t)(r1 >> (8 * i));
+            for (int i = 0; i < 4; ++i) sc[8 + i] = (uint8_t)(r2 >> (8 * i));
+        } else {
+            syn_put_u16(out + 2, d);
+            uint64_t r1 = syn_draw(key, n0 + 1);
+            uint8_t s6[8], m6[8];
+            for (int j = 0; j < 8; ++j) {
+                s6[j] = (uint8_t)(1 + ((r1 >> (2 * j)) & 3));
+                m6[j] = (uint8_t)((31 * s6[j] + 1) / 2);
+            }
+            syn_pack_k_scales(s6, m6, sc);
+        }
+        for (int i = 0; i < 4; ++i) syn_put_u64(out + 16 + 8 * i, syn_draw(key, n0 + 3 + i));
+        for (int i = 0; i < 16; ++i) syn_put_u64(out + 48 + 8 * i, syn_draw(key, n0 + 7 + i));
     } else if (qtype == SYN_Q6_K) {
         for (int i = 0; i < 24; ++i) syn_put_u64(out + 8 * i, syn_draw(key, n0 + 1 + i));
         int8_t* sc = (int8_t*)(out + 192);

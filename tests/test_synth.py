@@ -26,13 +26,13 @@ def test_generator_f16_conversion_matches_ieee(syn):
         assert syn.host().syn_f16_bits_of_scaled(int(k), int(e)) == want
 
 
-@pytest.mark.parametrize("qtype", [0, 1, 2, 3])
+@pytest.mark.parametrize("qtype", [0, 1, 2, 3, 4])
 def test_sweep_distribution(orc, syn, qtype):
     qp = syn.sweep_qparams(qtype)
     W = syn.blocks_host(qtype, 1, 1, 64, 1024, qp)
     be, bb = syn.BLOCK[qtype]
     blocks = W.reshape(-1, bb)
-    d_off = {0: 0, 1: 0, 2: 0, 3: 208}[qtype]
+    d_off = {0: 0, 1: 0, 2: 0, 3: 208, 4: 0}[qtype]
     d = blocks[:, d_off:d_off + 2].copy().view(np.float16).astype(np.float64).ravel()
     assert d.min() >= 0.999e-3 and d.max() <= 1.0001e-2
     if qtype == 0:
@@ -42,7 +42,7 @@ def test_sweep_distribution(orc, syn, qtype):
     assert np.all(np.isfinite(dense))
 
 
-@pytest.mark.parametrize("qtype", [0, 1, 2, 3])
+@pytest.mark.parametrize("qtype", [0, 1, 2, 3, 4])
 def test_decode_recipe_is_unit_gain(orc, syn, qtype):
     """Decode tensors map a unit-RMS input to a roughly unit-RMS output."""
     K = 2048
