@@ -9,7 +9,9 @@ workloads, random weights of the Llama architecture):
                                  Q8_0 weights, KV cache prefilled to 4096 positions
   llama70b_q4k_stream            70B shape in Q4_K, layers 0-35 resident, 36-79 streamed
                                  from pinned host memory through the two-slot HBM ring
-  gemv_q8_0_4096                 Q8_0 GEMV 4096 x 4096 (rotating over weight copies)
+  gemv_sweep                     the quantized GEMV sweep at the Llama-8B layer shapes in Q4_0
+                                 and Q4_K (both layouts) and the single Q8_0 4096 x 4096 GEMV,
+                                 weights rotated over copies larger than 2 x L2; metric GB/s
 
 One step = one decode step (one token); the metric is tokens per second.
 `--impl reference` times the CPU oracle (as it stands) on a bounded sample of
@@ -138,16 +140,16 @@ def max_over_ranks(v, world):
 
 # --------------------------------------------------------------------------- workloads
 
-def spec_for(name, layout="tiled"):
+def spec_for(name, layout="tiled", layers=None):
+    """The workload's model; `layers` shortens it (profiler captures only)."""
     import synth
     tiled = layout == "tiled"
-    if name == "llama70b_q6k_decode":
-        return synth.ModelSpec(**synth.LLAMA_70B_Q6_K, tiled=tiled)
-    if name == "llama8b_q8_0_decode":
-        return synth.ModelSpec(**synth.LLAMA_8B_Q8_0, tiled=tiled)
-    if name == "llama70b_q4k_stream":
-        return synth.ModelSpec(**synth.LLAMA_70B_Q4_K, tiled=tiled)
-    raise ValueError(name)
+    base = {"llama70b_q6k_decode": synth.LLAMA_70B_Q6_K, "llama8b_q8_0_decode": synth.LLAMA_8B_Q8_0,
+            "llama70b_q4k_stream": synth.LLAMA_70B_Q4_K}[name]
+    kw = dict(base)
+    if layers:
+        kw["n_layers"] = layers
+    return synth.ModelSpec(**kw, tiled=tiled)
 
 
 def lib_qtype(spec):
@@ -166,21 +168,26 @@ def step_bytes(spec):
     return w + kv_read_bytes(spec) + synth.row_bytes(spec.qtype, spec.hidden)
 
 
-def gemv_shapes(spec):
-    """(rows, cols, launches per step) of the decode GEMVs."""
-    return [(spec.qkv_rows, spec.hidden, spec.n_layers), (spec.hidden, spec.q_dim, spec.n_layers),
-            (spec.ffn, spec.hidden, 2 * spec.n_layers), (spec.hidden, spec.ffn, spec.n_layers),
-            (spec.vocab, spec.hidden, 1)]
+def gemv_kinds(spec):
+    """The step's fused GEMV launches per kind: (name, replay kind, rows, cols, matrices per
+    launch, launches per step, algorithmic bytes per launch).  Bytes = packed weights read +
+    the fp32 vectors read and written (+ the fp16 K / V rows the QKV epilogue appends)."""
+    import synth
+    h, f, qd, L = spec.hidden, spec.ffn, spec.q_dim, spec.n_layers
+    rb = lambda c: synth.row_bytes(spec.qtype, c)
+    kvd = spec.n_kv_heads * spec.head_dim
+    return [("qkv", 0, spec.qkv_rows, h, 1, L, spec.qkv_rows * rb(h) + 4 * (2 * h + qd) + 2 * 2 * kvd),
+            ("o", 1, h, qd, 1, L, h * rb(qd) + 4 * (qd + 2 * h)),
+            ("gate_up", 2, f, h, 2, L, 2 * f * rb(h) + 4 * (2 * h + f)),
+            ("down", 3, h, f, 1, L, h * rb(f) + 4 * (f + 2 * h)),
+            ("lm_head", 4, spec.vocab, h, 1, 1, spec.vocab * rb(h) + 4 * (2 * h + spec.vocab))]
 
 
-# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture per
-# shape, bytes per launch) of the tiled GEMV, and a hash of the kernel
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture of the step's
+# fused launch of each kind, bytes per launch) of the tiled GEMV, and a hash of the kernel
 # sources it was taken with: a changed kernel reports traffic as unknown (null).
-GEMV_TRAFFIC_SRC_SHA = "d118f419951f3ecf"
-GEMV_TRAFFIC = {"q6_k_t:10240x8192": 68896512, "q6_k_t:8192x8192": 55124992, "q6_k_t:28672x8192": 192979200,
-                "q6_k_t:8192x28672": 192954624, "q6_k_t:128256x8192": 862085888, "q8_0_t:6144x4096": 26788864,
-                "q8_0_t:4096x4096": 17875968, "q8_0_t:14336x4096": 62440448, "q8_0_t:4096x14336": 62481664,
-                "q8_0_t:128256x4096": 558824960}
+GEMV_TRAFFIC_SRC_SHA = None
+GEMV_TRAFFIC = {}
 
 
 def gemv_sources_sha():
@@ -193,60 +200,59 @@ def gemv_sources_sha():
     return h.hexdigest()[:16]
 
 
-def measure_gemv_roofline(ntx, model, spec, stream, iters=3):
-    """Time every decode GEMV of one step on its own (the same weights and shapes as
-    the step, plain store epilogue, same stream) with CUDA events.  Per shape: bytes
-    per launch (packed weights + x + y) and the average launch time, cycling over the
-    layers so no launch finds its weights in L2.  The aggregate over a step's launches
-    is the dominant kernel's achieved HBM bandwidth.  Only HBM-resident layers count;
-    streamed layers are bound by the host link, which is reported on its own."""
+def fmt_name(spec):
+    return {0: "q8_0", 1: "q4_0", 2: "q4_k", 3: "q6_k"}[spec.qtype] + ("_t" if spec.tiled else "")
+
+
+def measure_gemv_roofline(ntx, model, spec, stream, logits, rounds=5):
+    """Time the step's own fused GEMV launches, kind by kind: ntx_model_replay_gemv enqueues
+    them exactly as the decode step does (same kernels, prologues, epilogues, programmatic
+    launch), cycling over the resident layers so no launch finds its weights in L2; n of
+    them are captured in a CUDA graph and replayed on the bench stream between CUDA events.
+    Per kind: average launch time (median over `rounds` replays) and algorithmic bytes per
+    launch.  The launch-weighted aggregate over one step is the dominant kernel's achieved
+    HBM bandwidth.  Only HBM-resident layers count (streamed ones are bound by the host link)."""
     import torch
-    import synth
-    x = torch.randn(max(spec.hidden, spec.ffn, spec.q_dim), device="cuda")
-    y = torch.empty(max(spec.vocab, spec.ffn, spec.qkv_rows), device="cuda")
-    res = model.layers[:model.n_resident]
-    shapes = [("qkv", [t["w_qkv"] for t in res], spec.qkv_rows, spec.hidden),
-              ("o", [t["w_o"] for t in res], spec.hidden, spec.q_dim),
-              ("gate_up", [t[k] for t in res for k in ("w_gate", "w_up")], spec.ffn, spec.hidden),
-              ("down", [t["w_down"] for t in res], spec.hidden, spec.ffn),
-              ("lm_head", [model.output], spec.vocab, spec.hidden)]
-    q = lib_qtype(spec)
-    fmt = {0: "q8_0", 1: "q4_0", 2: "q4_k", 3: "q6_k"}[spec.qtype] + ("_t" if spec.tiled else "")
+    fmt = fmt_name(spec)
     sha = gemv_sources_sha()
+    nres = model.n_resident
     out, tot_bytes, tot_ms, tot_launch, tot_traffic = {}, 0.0, 0.0, 0, 0.0
-    with torch.cuda.stream(stream):
-        for name, mats, r, c in shapes:
-            per = r * synth.row_bytes(spec.qtype, c) + 4 * (c + r)
-            n = max(len(mats) * iters, 4)
-            for W in mats[:4]:
-                ntx.ntx_gemv_q(q, W, r, c, x, y, stream.cuda_stream)
+    for name, kind, r, c, nmat, per_step, per in gemv_kinds(spec):
+        if kind != 4 and nres < 1:
+            continue
+        launches = per_step if kind == 4 else nres     # launches of this kind in one step's resident part
+        n = max(3 * launches, 8) if kind != 4 else 8
+        with torch.cuda.stream(stream):
+            ntx.ntx_model_replay_gemv(model.handle, kind, min(n, 4), logits, stream.cuda_stream)
             torch.cuda.synchronize()
-            # the n launches back to back in a CUDA graph, so the host's launch rate does
-            # not bound the small shapes
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
-                for i in range(n):
-                    ntx.ntx_gemv_q(q, mats[i % len(mats)], r, c, x, y, stream.cuda_stream)
+                ntx.ntx_model_replay_gemv(model.handle, kind, n, logits, stream.cuda_stream)
             g.replay()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
-            e0.record(stream)
-            g.replay()
-            e1.record(stream)
-            torch.cuda.synchronize()
+            times = []
+            for _ in range(rounds):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                g.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1) / n)
             del g
-            ms = e0.elapsed_time(e1) / n
-            launches = len(mats)    # launches of this shape in one decode step
-            tr = GEMV_TRAFFIC.get(f"{fmt}:{r}x{c}") if sha == GEMV_TRAFFIC_SRC_SHA else None
-            out[name] = {"shape": f"{fmt}:{r}x{c}", "bytes_per_launch": per, "avg_launch_us": ms * 1e3,
-                         "achieved_gbs": per / (ms * 1e-3) / 1e9, "launches_per_step": launches,
-                         "traffic_per_launch": tr}
-            tot_bytes += per * launches
-            tot_ms += ms * launches
-            tot_launch += launches
-            tot_traffic = None if (tr is None or tot_traffic is None) else tot_traffic + tr * launches
+        ms = statistics.median(times)
+        shape = f"{fmt}:{'2x' if nmat == 2 else ''}{r}x{c}"
+        tr = GEMV_TRAFFIC.get(f"{fmt}:{name}:{r}x{c}") if sha == GEMV_TRAFFIC_SRC_SHA else None
+        out[name] = {"shape": shape, "fused": ["rmsnorm+rope+kv_append", "residual_add", "rmsnorm+swiglu",
+                                                "residual_add", "rmsnorm"][kind],
+                     "bytes_per_launch": per, "avg_launch_us": ms * 1e3, "best_launch_us": min(times) * 1e3,
+                     "achieved_gbs": per / (ms * 1e-3) / 1e9, "launches_per_step": launches,
+                     "traffic_per_launch": tr}
+        tot_bytes += per * launches
+        tot_ms += ms * launches
+        tot_launch += launches
+        tot_traffic = None if (tr is None or tot_traffic is None) else tot_traffic + tr * launches
     agg = {"achieved": tot_bytes / (tot_ms * 1e-3) / 1e9, "bytes_per_launch": tot_bytes / tot_launch,
-           "avg_launch_us": tot_ms * 1e3 / tot_launch,
+           "avg_launch_us": tot_ms * 1e3 / tot_launch, "launches": tot_launch,
            "traffic": None if tot_traffic is None else tot_traffic / tot_launch}
     return agg, out
 
@@ -257,7 +263,7 @@ def run_decode_bench(args, rank, world, local):
     from synth.device_model import DeviceModel
 
     name = args.workload
-    spec = spec_for(name, args.layout)
+    spec = spec_for(name, args.layout, args.layers)
     streamed = name == "llama70b_q4k_stream"
     n_res = 36 if streamed else None
     t0 = time.time()
@@ -293,22 +299,36 @@ def run_decode_bench(args, rank, world, local):
     ms = max_over_ranks(ms, world)
     dev_err = ntx.ntx_device_error()
 
-    # end to end through the public API: token in from the host, logits back to pinned host memory
+    # end to end through the public API, the same number of steps: token in from the host,
+    # logits back to pinned host memory, the host waiting for each step
     host_logits = torch.empty(spec.vocab, dtype=torch.float32, pin_memory=True)
-    e2e_steps = max(3, min(args.steps, 10))
     torch.cuda.synchronize()
     t_e2e = time.perf_counter()
-    for _ in range(e2e_steps):
+    for _ in range(args.steps):
         step()
         with torch.cuda.stream(stream):
             host_logits.copy_(logits, non_blocking=True)
         stream.synchronize()
-    e2e_ms = (time.perf_counter() - t_e2e) * 1e3 / e2e_steps
+    e2e_ms = (time.perf_counter() - t_e2e) * 1e3 / args.steps
     e2e_ms = max_over_ranks(e2e_ms, world)
 
-    out = {"ms_per_step": ms, "tok_s": world * 1e3 / ms, "e2e_tok_s": world * 1e3 / e2e_ms, "setup_s": setup_s,
-           "clocks": clk.summary(), "launches": launches_per_step * args.steps, "device_error": dev_err,
-           "bytes": step_bytes(spec), "spec": spec, "model": model, "stream": stream}
+    # per-step spread: >= 50 replays, each between its own pair of events
+    replay_ms = []
+    for _ in range(max(50, args.steps)):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        step()
+        b.record(stream)
+        replay_ms.append((a, b))
+    torch.cuda.synchronize()
+    replay_ms = sorted(a.elapsed_time(b) for a, b in replay_ms)
+
+    out = {"ms_per_step": ms, "tok_s": world * 1e3 / ms, "e2e_tok_s": world * 1e3 / e2e_ms, "e2e_ms": e2e_ms,
+           "setup_s": setup_s, "clocks": clk.summary(), "launches": launches_per_step * args.steps,
+           "device_error": dev_err, "bytes": step_bytes(spec), "spec": spec, "model": model, "stream": stream,
+           "logits": logits,
+           "replays": {"n": len(replay_ms), "median_ms": statistics.median(replay_ms), "best_ms": replay_ms[0],
+                       "worst_ms": replay_ms[-1]}}
     if streamed:
         h2d, step_ms = ntx.ntx_stream_stats(model.handle)
         out["h2d_bytes"] = h2d
@@ -335,76 +355,113 @@ def measure_h2d():
     return best
 
 
-def cpu_baseline(spec, budget_s=20.0):
-    """The CPU oracle, as it stands, on a bounded sample of the decode step: whole
-    layers at the workload's shape (weights generated before timing) and a slice of
-    the LM head; extrapolated to one token."""
-    import numpy as np
+CPU_SAMPLE_LAYERS = 4     # whole layers the CPU baseline times per token (both arms alike)
+
+
+def cpu_baseline(spec, n_layers_timed=CPU_SAMPLE_LAYERS):
+    """The CPU oracle, as it stands, on a bounded sample of the decode step: the first
+    `n_layers_timed` whole layers at the workload's shape (weights generated before timing)
+    and 1/32 of the LM-head rows; the per-token time is extrapolated from them (layers x
+    n_layers / n_layers_timed, head x 32)."""
     import oracle
     from oracle import model as om
-    import synth
     oracle.build()
     dims = oracle.dims_of(spec)
-    t = om.layer_tensors(spec, 0)
     h = om.embedding_row(spec, spec.token()).copy()
-    n_layers_timed, t_layers = 0, 0.0
-    while t_layers < budget_s * 0.7 and n_layers_timed < spec.n_layers:
+    n = min(n_layers_timed, spec.n_layers)
+    t_layers = 0.0
+    for layer in range(n):
+        t = om.layer_tensors(spec, layer)
         t0 = time.perf_counter()
         oracle.decode_layer(dims, spec.qtype, h, spec.n_prefill, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"],
                             t["w_gate"], t["w_up"], t["w_down"], t["k_cache"], t["v_cache"])
         t_layers += time.perf_counter() - t0
-        n_layers_timed += 1
     head_rows = max(256, spec.vocab // 32)
     norm, W = om.head_tensors(spec, (0, head_rows))
     t0 = time.perf_counter()
     oracle.lm_head(spec.qtype, norm, W, head_rows, spec.hidden, spec.rms_eps, h)
     t_head = (time.perf_counter() - t0) * spec.vocab / head_rows
-    s_per_tok = t_layers / n_layers_timed * spec.n_layers + t_head
+    s_per_tok = t_layers / n * spec.n_layers + t_head
     return {"value": 1.0 / s_per_tok, "unit": "tok/s", "cores": oracle.threads(), "kind": "oracle",
-            "sample": f"{n_layers_timed} of {spec.n_layers} layers (full shape, ctx {spec.n_prefill + 1}) "
-                      f"+ {head_rows} of {spec.vocab} LM-head rows, extrapolated to one token"}
+            "extrapolated": True,
+            "sample": f"{n} of {spec.n_layers} layers (full shape, ctx {spec.n_prefill + 1}) "
+                      f"+ {head_rows} of {spec.vocab} LM-head rows timed, extrapolated to one token"}
 
 
-def gemv_bench(ntx, iters=50, tiled=True):
-    """Q8_0 4096 x 4096 GEMV rotating over 16 weight copies (> 2 x L2)."""
+SWEEP_SHAPES = [("qkv", 6144, 4096), ("o", 4096, 4096), ("gate_or_up", 14336, 4096), ("down", 4096, 14336),
+                ("lm_head", 128256, 4096)]
+
+
+def gemv_rotation_bench(ntx, qtype, rows, cols, tiled, stream, n_launch=48, rounds=5):
+    """One GEMV shape on its own: enough weight copies that one pass over them exceeds
+    2 x L2 (so every launch streams its weights from HBM), n_launch launches cycling over
+    the copies captured in a CUDA graph (programmatic launch between them, as in the step)
+    and replayed `rounds` times between CUDA events; the median and best per-launch times."""
+    import math
     import torch
     import synth
-    rows = cols = 4096
-    qp = synth.sweep_qparams(synth.Q8_0)
-    rb = synth.row_bytes(synth.Q8_0, cols)
-    copies = [torch.empty(rows * rb, dtype=torch.uint8, device="cuda") for _ in range(16)]
-    tmp = torch.empty(rows * rb, dtype=torch.uint8, device="cuda")
-    for i, c in enumerate(copies):
-        if tiled:
-            synth.blocks_dev(tmp, synth.Q8_0, 0, 1, rows, cols, qp)
-            ntx.ntx_repack_q(synth.Q8_0, tmp, c, rows, cols)
-        else:
-            synth.blocks_dev(c, synth.Q8_0, 0, 1, rows, cols, qp)
-    q = synth.Q8_0 | (16 if tiled else 0)
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    rb = synth.row_bytes(qtype, cols)
+    nbytes = rows * rb
+    n_copies = max(2, math.ceil(2 * l2 / nbytes) + 1)
+    qp = synth.sweep_qparams(qtype)
+    base = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    synth.blocks_dev(base, qtype, 0, 1, rows, cols, qp)
+    if tiled:
+        t = torch.empty_like(base)
+        ntx.ntx_repack_q(qtype, base, t, rows, cols)
+        base = t
+    copies = [base] + [base.clone() for _ in range(n_copies - 1)]
+    q = qtype | (16 if tiled else 0)
     x = torch.empty(cols, device="cuda")
     synth.normal_f32_dev(x, 0, 2)
     y = torch.empty(rows, device="cuda")
-    s = torch.cuda.Stream()
-    for c in copies:
-        ntx.ntx_gemv_q(q, c, rows, cols, x, y, s.cuda_stream)
-    torch.cuda.synchronize()
-    # back to back from a CUDA graph, so the host's launch rate does not bound them
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=s):
-        for i in range(iters):
-            ntx.ntx_gemv_q(q, copies[i % 16], rows, cols, x, y, s.cuda_stream)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(s):   # replay() launches on the current stream
+    with torch.cuda.stream(stream):
+        for c in copies[:4]:
+            ntx.ntx_gemv_q(q, c, rows, cols, x, y, stream.cuda_stream)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n_launch):
+                ntx.ntx_gemv_q(q, copies[i % n_copies], rows, cols, x, y, stream.cuda_stream)
         g.replay()
         torch.cuda.synchronize()
-        e0.record(s)
-        g.replay()
-        e1.record(s)
-    torch.cuda.synchronize()
-    del g
-    us = e0.elapsed_time(e1) * 1e3 / iters
-    nbytes = rows * rb + 4 * (rows + cols)
-    return {"us": us, "gbs": nbytes / (us * 1e-6) / 1e9}
+        times = []
+        for _ in range(rounds):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            g.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3 / n_launch)
+        del g
+    del copies, base
+    torch.cuda.empty_cache()
+    per = nbytes + 4 * (rows + cols)
+    us = statistics.median(times)
+    return {"bytes_per_launch": per, "us": us, "best_us": min(times), "gbs": per / (us * 1e-6) / 1e9,
+            "copies": n_copies}
+
+
+def gemv_sweep(ntx, stream, peak, peak_kind, ceiling):
+    """The quantized GEMV sweep at the Llama-8B layer shapes (4096 -> 6144 fused QKV,
+    4096 -> 4096 O, 4096 -> 14336 gate or up, 14336 -> 4096 down, 4096 -> 128256 LM head)
+    in Q4_0 and Q4_K, in both layouts, plus the single Q8_0 4096 x 4096 GEMV."""
+    import synth
+    rows_out = []
+    for qname, q in (("q4_0", synth.Q4_0), ("q4_k", synth.Q4_K)):
+        for layout in ("tiled", "gguf"):
+            for name, rows, cols in SWEEP_SHAPES:
+                r = gemv_rotation_bench(ntx, q, rows, cols, layout == "tiled", stream)
+                r.update({"format": qname, "layout": layout, "shape": name, "rows": rows, "cols": cols,
+                          "frac_of_%s" % peak_kind: r["gbs"] / peak, "frac_of_read_ceiling": r["gbs"] / ceiling})
+                rows_out.append(r)
+    single = {}
+    for layout in ("tiled", "gguf"):
+        r = gemv_rotation_bench(ntx, synth.Q8_0, 4096, 4096, layout == "tiled", stream)
+        r.update({"frac_of_%s" % peak_kind: r["gbs"] / peak, "frac_of_read_ceiling": r["gbs"] / ceiling})
+        single[layout] = r
+    return rows_out, single
 
 
 def measure_read_ceiling(ntx, stream, nbytes=4 << 30, iters=10):
@@ -502,6 +559,18 @@ def profile_attn(what, launches):
     print(json.dumps({"attn": what, "kv_bytes": kv, "us_median": us, "gbs": kv / (us * 1e-6) / 1e9}))
 
 
+DTYPE = "i8*i24->i32+f32"
+DTYPE_DETAIL = ("weights: packed block codes (4/6/8-bit) unpacked to int8; GEMV: integer dot products (dp4a) "
+                "of the codes with x as 24-bit fixed point (three int8 limbs, one exponent per 32-column step), "
+                "exact int32 block sums, block scales and sums in fp32; attention: fp16 KV cache, fp32 softmax and "
+                "accumulation (fp16 tensor-core products of exact split operands); activations fp32")
+ROOFLINE_FRAC_LIMIT = 1.2   # a GEMV timed above 1.2 x the copy peak is not doing the work: refuse the figure
+
+
+def print_line(line):
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -509,15 +578,20 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ntx", choices=["ntx", "reference"])
     ap.add_argument("--workload", default="llama70b_q6k_decode",
-                    choices=["llama70b_q6k_decode", "llama8b_q8_0_decode", "llama70b_q4k_stream"])
+                    choices=["llama70b_q6k_decode", "llama8b_q8_0_decode", "llama70b_q4k_stream", "gemv_sweep"])
     ap.add_argument("--layout", default="tiled", choices=["tiled", "gguf"],
                     help="weights handed to the library as tiled (repacked once at load) or GGUF-style blocks")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="shorten the model to this many layers (profiler captures only; the line says so)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--profile-gemv", default=None, metavar="FMT:ROWSxCOLS[,...]",
                     help="only run the GEMV kernel on one matrix (for profilers), e.g. q6_k:28672x8192")
     ap.add_argument("--profile-attn", default=None, metavar="QHEADS:KVHEADS:CONTEXT",
                     help="only run the decode attention on one shape (for profilers), e.g. 64:8:8193")
+    ap.add_argument("--profile-step-gemv", action="store_true",
+                    help="build the model, run --warmup steps, then one launch of each of the step's fused GEMV "
+                         "kinds (for profilers; use with --layers)")
     args = ap.parse_args()
     if args.profile_gemv:
         return profile_gemv(args.profile_gemv, args.steps)
@@ -531,12 +605,19 @@ def main():
         rank, world, local = int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), 0
     else:
         rank, world, local = dist_setup(args.gpus)
-    spec = spec_for(args.workload, args.layout)
+    peak, peak_kind = load_peaks()
+
+    if args.workload == "gemv_sweep":
+        return run_sweep(args, rank, world, local, peak, peak_kind)
+
+    spec = spec_for(args.workload, args.layout, args.layers)
     config = {"workload": args.workload, "layers": spec.n_layers, "hidden": spec.hidden, "ffn": spec.ffn,
               "q_heads": spec.n_q_heads, "kv_heads": spec.n_kv_heads, "vocab": spec.vocab, "format": ["q8_0", "q4_0",
               "q4_k", "q6_k"][spec.qtype], "layout": args.layout, "context": spec.n_prefill + 1, "batch": 1,
               "l2": "inputs larger than L2 (weights %.1f GB per step)" % (step_bytes(spec) / 1e9),
               "parallelism": "replicas" if world > 1 else "single"}
+    if args.layers:
+        config["shortened_for_profiling"] = True
 
     if args.impl == "reference":
         if rank != 0:
@@ -544,16 +625,17 @@ def main():
         cb = None
         vals = []
         for i in range(args.warmup + args.steps):
-            cb = cpu_baseline(spec, budget_s=6.0)
+            cb = cpu_baseline(spec)
             if i >= args.warmup:
                 vals.append(cb["value"])
         v = statistics.median(vals)
         cb["value"] = v
-        print(json.dumps({"metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps,
-                          "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
-                          "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-                          "impl": "reference", "config": config, "cpu_baseline": cb,
-                          "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}))
+        print_line({"metric": METRIC, "value": v, "unit": "tok/s", "n_gpus": args.gpus, "steps": args.steps,
+                    "warmup": args.warmup, "ms_per_step": 1e3 / v, "higher_is_better": True,
+                    "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                    "impl": "reference", "config": config, "cpu_baseline": cb,
+                    "note": "each step times a sample of one token (cpu_baseline.sample) and extrapolates",
+                    "e2e": {"value": v, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
         return
 
     import torch
@@ -563,16 +645,20 @@ def main():
     build.build()
     synth.build_dev()
     torch.cuda.set_device(local)
+    if args.profile_step_gemv:
+        return profile_step_gemv(args, spec)
     r = run_decode_bench(args, rank, world, local)
     spec, model, stream = r["spec"], r["model"], r["stream"]
-    peak, peak_kind = load_peaks()
 
     line = {"metric": METRIC, "value": r["tok_s"], "unit": "tok/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded random weights and KV cache)",
+            "vs_baseline": None, "dtype": DTYPE, "dtype_detail": DTYPE_DETAIL,
+            "data": "synthetic (seeded random weights and KV cache)",
             "config": config, "clocks": r["clocks"], "gpu_launches": r["launches"],
             "e2e": {"value": r["e2e_tok_s"], "unit": "tok/s", "h2d_bytes_per_step": 8,
-                    "d2h_bytes_per_step": 4 * spec.vocab}}
+                    "d2h_bytes_per_step": 4 * spec.vocab, "steps": args.steps,
+                    "not_faster_than_device_timed": r["e2e_tok_s"] <= r["tok_s"] * 1.01},
+            "replays": r["replays"]}
     step_gbs = r["bytes"] / (r["ms_per_step"] * 1e-3) / 1e9
     line["step_hbm"] = {"bytes_per_step": r["bytes"], "achieved_gbs": step_gbs, "frac_of_%s" % peak_kind:
                         step_gbs / peak, "frac_of_8000": step_gbs / 8000.0}
@@ -580,27 +666,117 @@ def main():
         line["host_link"] = {"h2d_bytes_per_step": r["h2d_bytes"], "achieved_gbs": r["h2d_gbs"],
                              "measured_pinned_h2d_gbs": r["h2d_peak_gbs"], "frac": r["h2d_gbs"] / r["h2d_peak_gbs"]}
     if rank == 0:
-        agg, per_shape = measure_gemv_roofline(ntx, model, spec, stream)
-        line["roofline"] = {"bound": "hbm", "kernel": "qmma_kernel<%s> (all GEMV launches of one step)" % config["format"],
+        agg, per_kind = measure_gemv_roofline(ntx, model, spec, stream, r["logits"])
+        frac = agg["achieved"] / peak
+        line["roofline"] = {"bound": "hbm",
+                            "kernel": "qmma_kernel<%s> (the step's fused GEMV launches, all kinds, launch-weighted)"
+                                      % fmt_name(spec),
                             "achieved": agg["achieved"], "peak": peak, "peak_kind": peak_kind, "unit": "GB/s",
-                            "frac": agg["achieved"] / peak, "traffic": agg["traffic"],
-                            "bytes_per_launch": agg["bytes_per_launch"], "avg_launch_us": agg["avg_launch_us"]}
-        line["gemv_shapes"] = per_shape
+                            "frac": frac, "traffic": agg["traffic"],
+                            "bytes_per_launch": agg["bytes_per_launch"], "avg_launch_us": agg["avg_launch_us"],
+                            "launches_per_step": agg["launches"]}
+        if frac > ROOFLINE_FRAC_LIMIT:
+            line["roofline"]["rejected"] = "achieved above %.1f x the copy peak: the timed kernel is not doing " \
+                                           "the work" % ROOFLINE_FRAC_LIMIT
+            line["roofline"]["frac"] = None
+        line["gemv_kinds"] = per_kind
         ceil_gbs = measure_read_ceiling(ntx, stream)
         line["read_ceiling"] = {"kernel": "ntx_stream_read_probe (bulk-copy ring, one CTA per SM, no arithmetic)",
                                 "gbs": ceil_gbs, "frac_of_%s" % peak_kind: ceil_gbs / peak}
         line["roofline"]["frac_of_read_ceiling"] = agg["achieved"] / ceil_gbs
         if not args.no_extras:
-            line["gemv_q8_0_4096x4096"] = {"tiled": gemv_bench(ntx, tiled=True), "gguf": gemv_bench(ntx, tiled=False)}
+            line["gemv_q8_0_4096x4096"] = {lay: gemv_rotation_bench(ntx, synth.Q8_0, 4096, 4096, lay == "tiled",
+                                                                    stream) for lay in ("tiled", "gguf")}
         if not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(spec)
         if r["device_error"]:
             line["device_error"] = r["device_error"]
-        print(json.dumps(line))
+        print_line(line)
     model.close()
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_sweep(args, rank, world, local, peak, peak_kind):
+    """--workload gemv_sweep: the GEMV sweep's line (metric: quantized GEMV HBM GB/s)."""
+    config = {"workload": "gemv_sweep", "shapes": [f"{c}->{r}" for _, r, c in SWEEP_SHAPES],
+              "formats": ["q4_0", "q4_k"], "layouts": ["tiled", "gguf"], "batch": 1,
+              "l2": "weights rotated over copies larger than 2 x L2", "parallelism": "single"}
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import numpy as np
+        import oracle
+        import synth
+        oracle.build()
+        vals = []
+        for i in range(args.warmup + args.steps):
+            tot_b, tot_s = 0, 0.0
+            for qname, q in (("q4_0", synth.Q4_0), ("q4_k", synth.Q4_K)):
+                for name, rows, cols in SWEEP_SHAPES:
+                    n = 64
+                    W = synth.blocks_host(q, 0, 1, n, cols, synth.sweep_qparams(q))
+                    x = synth.normal_f32_host(0, 2, cols)
+                    t0 = time.perf_counter()
+                    oracle.gemv(q, W, n, cols, x)
+                    tot_s += time.perf_counter() - t0
+                    tot_b += W.size
+            if i >= args.warmup:
+                vals.append(tot_b / tot_s / 1e9)
+        v = statistics.median(vals)
+        print_line({"metric": "quantized GEMV GB/s", "value": v, "unit": "GB/s", "n_gpus": args.gpus,
+                    "steps": args.steps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                    "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference", "config": config,
+                    "cpu_baseline": {"value": v, "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+                                     "sample": "64 rows of each sweep shape and format"},
+                    "e2e": {"value": v, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}})
+        return
+    import torch
+    import quantized_weight_gemv_block_b200 as ntx
+    from quantized_weight_gemv_block_b200 import build
+    import synth
+    build.build()
+    synth.build_dev()
+    torch.cuda.set_device(local)
+    stream = torch.cuda.Stream()
+    ceil_gbs = measure_read_ceiling(ntx, stream)
+    with ClockSampler(local) as clk:
+        rows_out, single = gemv_sweep(ntx, stream, peak, peak_kind, ceil_gbs)
+    tiled = [r for r in rows_out if r["layout"] == "tiled"]
+    tot_b = sum(r["bytes_per_launch"] for r in tiled)
+    tot_us = sum(r["us"] for r in tiled)
+    v = tot_b / (tot_us * 1e-6) / 1e9
+    top = max(tiled, key=lambda r: r["bytes_per_launch"])
+    line = {"metric": "quantized GEMV HBM GB/s", "value": v, "unit": "GB/s", "n_gpus": world, "steps": 5,
+            "warmup": 1, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE,
+            "data": "synthetic (seeded random blocks, x ~ N(0,1))", "config": config, "clocks": clk.summary(),
+            "gpu_launches": 48 * 5 * (len(rows_out) + 2),
+            "roofline": {"bound": "hbm", "kernel": "qmma_kernel (tiled Q4_0 / Q4_K, all sweep shapes, one launch each)",
+                         "achieved": v, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": v / peak,
+                         "traffic": None, "frac_of_read_ceiling": v / ceil_gbs,
+                         "largest_shape": {"shape": f"{top['format']}:{top['rows']}x{top['cols']}",
+                                           "gbs": top["gbs"]}},
+            "read_ceiling": {"gbs": ceil_gbs}, "sweep": rows_out, "gemv_q8_0_4096x4096": single}
+    print_line(line)
+
+
+def profile_step_gemv(args, spec):
+    """The step's fused GEMV kinds, one launch each, after `warmup` decode steps of a
+    (shortened) model: the case that profiler captures of the fused instances run."""
+    import torch
+    import quantized_weight_gemv_block_b200 as ntx
+    from synth.device_model import DeviceModel
+    model = DeviceModel(spec)
+    logits = torch.empty(spec.vocab, dtype=torch.float32, device="cuda")
+    for _ in range(args.warmup):
+        ntx.ntx_decode_step(model.handle, spec.token(), spec.n_prefill, logits)
+    torch.cuda.synchronize()
+    for name, kind, *_ in gemv_kinds(spec):
+        ntx.ntx_model_replay_gemv(model.handle, kind, 1, logits)
+        torch.cuda.synchronize()
+        print(json.dumps({"profiled": name}), flush=True)
+    model.close()
 
 
 if __name__ == "__main__":

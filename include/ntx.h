@@ -277,6 +277,22 @@ ntx_status ntx_decode_step(ntx_model* model, int32_t token, int32_t pos, float* 
 ntx_status ntx_stream_layers(ntx_model* model, int32_t token, int32_t pos, float* logits, void* compute,
                              void* copy, int64_t timeout_ms);
 
+/* Measurement helper, not part of the decode path: enqueue `n_launches` launches of
+ * one kind of the step's fused GEMVs on `stream`, exactly as ntx_decode_step issues
+ * them (same kernels, prologues, epilogues and launch attributes), cycling over the
+ * resident layers 0, 1, ... so consecutive launches read different weights:
+ *   NTX_GEMV_QKV      RMSNorm prologue, RoPE and fp16 K/V append at the step's position
+ *   NTX_GEMV_O        residual add into the hidden state
+ *   NTX_GEMV_GATE_UP  RMSNorm prologue, gate and up rows streamed together, SwiGLU
+ *   NTX_GEMV_DOWN     residual add into the hidden state
+ *   NTX_GEMV_HEAD     final RMSNorm prologue, logits into `logits` (device fp32 [vocab];
+ *                     unused by the other kinds, may be NULL there)
+ * Inputs are the model's activation buffers as the last step left them; outputs
+ * overwrite them (and the KV rows at the last step's position), so run a decode step
+ * again before relying on its results.  The launches may be captured in a CUDA graph. */
+enum { NTX_GEMV_QKV = 0, NTX_GEMV_O = 1, NTX_GEMV_GATE_UP = 2, NTX_GEMV_DOWN = 3, NTX_GEMV_HEAD = 4 };
+ntx_status ntx_model_replay_gemv(ntx_model* model, int kind, int n_launches, float* logits, void* stream);
+
 /* Per-step counters of the last ntx_stream_layers call: bytes copied host ->
  * device, and device milliseconds of the whole step (between the step's first
  * and last event; valid once the step finished). */

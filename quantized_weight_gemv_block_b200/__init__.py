@@ -17,6 +17,7 @@ NTX_OK, NTX_EINVAL, NTX_EUNSUPPORTED, NTX_ENOMEM, NTX_ECUDA, NTX_ETIMEOUT = rang
 NTX_Q8_0, NTX_Q4_0, NTX_Q4_K, NTX_Q6_K = range(4)
 NTX_TILED = 16
 NTX_Q8_0_T, NTX_Q4_0_T, NTX_Q4_K_T, NTX_Q6_K_T = 16, 17, 18, 19
+NTX_GEMV_QKV, NTX_GEMV_O, NTX_GEMV_GATE_UP, NTX_GEMV_DOWN, NTX_GEMV_HEAD = range(5)
 STATUS_NAMES = {0: "NTX_OK", 1: "NTX_EINVAL", 2: "NTX_EUNSUPPORTED", 3: "NTX_ENOMEM", 4: "NTX_ECUDA",
                 5: "NTX_ETIMEOUT"}
 
@@ -25,7 +26,7 @@ EXPORTS = ("ntx_last_error", "ntx_version", "ntx_row_bytes", "ntx_block_elems", 
            "ntx_stream_read_probe",
            "ntx_dequant_q", "ntx_repack_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_decode_noalloc", "ntx_attn_workspace_bytes", "ntx_swiglu",
            "ntx_softmax", "ntx_argmax", "ntx_embed", "ntx_model_create", "ntx_model_destroy", "ntx_decode_step",
-           "ntx_stream_layers", "ntx_stream_stats")
+           "ntx_stream_layers", "ntx_stream_stats", "ntx_model_replay_gemv")
 
 
 class NtxError(RuntimeError):
@@ -85,6 +86,7 @@ def lib() -> ctypes.CDLL:
             "ntx_decode_step": ([vp, i32, i32, vp, vp], ci),
             "ntx_stream_layers": ([vp, i32, i32, vp, vp, vp, i64], ci),
             "ntx_stream_stats": ([vp, ctypes.POINTER(i64), ctypes.POINTER(cf)], ci),
+            "ntx_model_replay_gemv": ([vp, ci, ci, vp, vp], ci),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -217,3 +219,7 @@ def ntx_stream_stats(model: int):
     ms = ctypes.c_float(0)
     check(lib().ntx_stream_stats(model, ctypes.byref(b), ctypes.byref(ms)))
     return b.value, ms.value
+
+
+def ntx_model_replay_gemv(model: int, kind: int, n_launches: int, logits=None, stream=None) -> None:
+    check(lib().ntx_model_replay_gemv(model, kind, n_launches, _p(logits), _s(stream)))

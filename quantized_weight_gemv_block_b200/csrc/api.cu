@@ -1,5 +1,8 @@
 // api.cu - status handling and small C-ABI helpers of the ntx library.
+#include <mutex>
+#include <set>
 #include <string>
+#include <tuple>
 
 #include "common.cuh"
 
@@ -21,6 +24,22 @@ ntx_status check_launch(const char* what)
 {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(NTX_ECUDA, std::string(what) + ": " + cudaGetErrorString(e));
+    return NTX_OK;
+}
+
+ntx_status ensure_smem_limit(const void* func, int bytes)
+{
+    static std::mutex mu;
+    static std::set<std::tuple<int, const void*, int>> done;
+    int dev = 0;
+    NTX_CUDA_TRY(cudaGetDevice(&dev));
+    const auto key = std::make_tuple(dev, func, bytes);
+    std::lock_guard<std::mutex> lock(mu);
+    if (done.count(key)) return NTX_OK;
+    const cudaError_t e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess)
+        return fail(NTX_ECUDA, std::string("setting a kernel's shared-memory limit: ") + cudaGetErrorString(e));
+    done.insert(key);
     return NTX_OK;
 }
 

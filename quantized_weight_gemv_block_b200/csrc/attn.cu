@@ -480,11 +480,8 @@ __global__ void __launch_bounds__(HD) attn_merge_kernel(const float* part, float
 template <int G>
 ntx_status launch_g(const KArgs& k, int n_q_heads, cudaStream_t s, bool pdl)
 {
-    static bool configured = false;
-    if (!configured) {
-        cudaFuncSetAttribute(attn_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-        configured = true;
-    }
+    const ntx_status st = ensure_smem_limit((const void*)attn_kernel<G>, kSmem);
+    if (st != NTX_OK) return st;
     const int grid = (n_q_heads / G) * k.n_split;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

@@ -59,6 +59,10 @@ cudaError_t take_device_error_probe(uint32_t* out);
 
 int num_sms();
 
+// Raise the dynamic shared-memory limit of kernel `func` to `bytes` on the current
+// device, once per (device, kernel, size); thread-safe.  NTX_ECUDA if the driver refuses.
+ntx_status ensure_smem_limit(const void* func, int bytes);
+
 // ------------------------------------------------------------------ formats
 
 struct QTraits {

@@ -4,17 +4,19 @@
 // principales": host read, PCIe DMA and GPU compute overlapped with double
 // buffering; here pinned host memory -> a two-slot HBM ring on a copy stream).
 //
-// Per layer, five kernels:
+// Per layer, six kernels:
 //   1. fused QKV GEMV: RMSNorm(h) prologue, RoPE + fp16 K/V append epilogue
-//   2. split-KV GQA attention (merge by the last CTA of each kv head)
-//   3. O GEMV, residual add into h
-//   4. fused gate/up GEMV: RMSNorm(h) prologue, SwiGLU epilogue
-//   5. down GEMV, residual add into h
-// plus the embedding before layer 0 and the RMSNorm + LM-head GEMV after the
-// last layer.  Kernels use programmatic dependent launch so each one's weight
-// stream starts while the previous one drains; the resident step is recorded
-// once as a CUDA graph and replayed, with token and position read from device
-// memory.
+//   2. split-context GQA attention, each split's partial (max, sum, accumulator)
+//      to a workspace
+//   3. merge of the splits (log-sum-exp rule, fixed order)
+//   4. O GEMV, residual add into h
+//   5. fused gate/up GEMV: RMSNorm(h) prologue, SwiGLU epilogue
+//   6. down GEMV, residual add into h
+// plus the step word / RoPE table kernel and the embedding before layer 0 and the
+// RMSNorm + LM-head GEMV after the last layer.  Kernels use programmatic dependent
+// launch so each one's weight stream starts while the previous one drains; the
+// resident step is recorded once as a CUDA graph and replayed, with token and
+// position read from device memory.
 #include <chrono>
 #include <cstdlib>
 #include <cstring>
@@ -63,33 +65,84 @@ struct LayerW {
     const void *qkv, *o, *gate, *up, *down;
 };
 
-ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl)
+// The fused GEMV launches of a layer, one function per kind, exactly as the step issues them.
+ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl)
 {
     const ntx_model_desc& d = m->d;
     const ntx_layer_desc& L = m->layers[l];
     const int qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim;
+    Params P{};
+    P.W = (const uint8_t*)w;
+    P.row_bytes = m->rb_h;
+    P.M = qd + 2 * kvd;
+    P.K = d.hidden;
+    P.x = m->h;
+    P.norm_w = L.attn_norm;
+    P.eps = d.rms_eps;
+    P.q_rows = qd;
+    P.kv_rows = kvd;
+    P.head_dim = d.head_dim;
+    P.max_ctx = d.max_ctx;
+    P.pos_dev = m->step + 1;
+    P.rope_cs = m->rope;
+    P.k_cache = (__half*)L.k_cache;
+    P.v_cache = (__half*)L.v_cache;
+    P.q_out = m->q;
+    P.use_pdl = pdl;
+    return gemv_launch(d.qtype, gemv::EPI_QKV, gemv::PRO_RMSNORM, P, s);
+}
+
+ntx_status launch_o(ntx_model* m, const void* w, cudaStream_t s, bool pdl)
+{
+    const ntx_model_desc& d = m->d;
+    Params P{};
+    P.W = (const uint8_t*)w;
+    P.row_bytes = m->rb_q;
+    P.M = d.hidden;
+    P.K = d.n_q_heads * d.head_dim;
+    P.x = m->att;
+    P.y = m->h;
+    P.use_pdl = pdl;
+    return gemv_launch(d.qtype, gemv::EPI_ADD, gemv::PRO_X, P, s);
+}
+
+ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, cudaStream_t s, bool pdl)
+{
+    const ntx_model_desc& d = m->d;
+    Params P{};
+    P.W = (const uint8_t*)wg;
+    P.W2 = (const uint8_t*)wu;
+    P.row_bytes = m->rb_h;
+    P.M = d.ffn;
+    P.K = d.hidden;
+    P.x = m->h;
+    P.norm_w = m->layers[l].ffn_norm;
+    P.eps = d.rms_eps;
+    P.y = m->act;
+    P.use_pdl = pdl;
+    return gemv_launch(d.qtype, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, P, s);
+}
+
+ntx_status launch_down(ntx_model* m, const void* w, cudaStream_t s, bool pdl)
+{
+    const ntx_model_desc& d = m->d;
+    Params P{};
+    P.W = (const uint8_t*)w;
+    P.row_bytes = m->rb_f;
+    P.M = d.hidden;
+    P.K = d.ffn;
+    P.x = m->act;
+    P.y = m->h;
+    P.use_pdl = pdl;
+    return gemv_launch(d.qtype, gemv::EPI_ADD, gemv::PRO_X, P, s);
+}
+
+ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl)
+{
+    const ntx_model_desc& d = m->d;
+    const ntx_layer_desc& L = m->layers[l];
     ntx_status st;
-    {
-        Params P{};
-        P.W = (const uint8_t*)w.qkv;
-        P.row_bytes = m->rb_h;
-        P.M = qd + 2 * kvd;
-        P.K = d.hidden;
-        P.x = m->h;
-        P.norm_w = L.attn_norm;
-        P.eps = d.rms_eps;
-        P.q_rows = qd;
-        P.kv_rows = kvd;
-        P.head_dim = d.head_dim;
-        P.max_ctx = d.max_ctx;
-        P.pos_dev = m->step + 1;
-        P.rope_cs = m->rope;
-        P.k_cache = (__half*)L.k_cache;
-        P.v_cache = (__half*)L.v_cache;
-        P.q_out = m->q;
-        P.use_pdl = pdl;
-        if ((st = gemv_launch(d.qtype, gemv::EPI_QKV, gemv::PRO_RMSNORM, P, s)) != NTX_OK) return st;
-    }
+    if ((st = launch_qkv(m, l, w.qkv, s, pdl)) != NTX_OK) return st;
     {
         AttnArgs a{};
         a.q = m->q;
@@ -106,43 +159,9 @@ ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, b
         a.pdl = pdl;
         if ((st = attn_launch(a, s)) != NTX_OK) return st;
     }
-    {
-        Params P{};
-        P.W = (const uint8_t*)w.o;
-        P.row_bytes = m->rb_q;
-        P.M = d.hidden;
-        P.K = qd;
-        P.x = m->att;
-        P.y = m->h;
-        P.use_pdl = pdl;
-        if ((st = gemv_launch(d.qtype, gemv::EPI_ADD, gemv::PRO_X, P, s)) != NTX_OK) return st;
-    }
-    {
-        Params P{};
-        P.W = (const uint8_t*)w.gate;
-        P.W2 = (const uint8_t*)w.up;
-        P.row_bytes = m->rb_h;
-        P.M = d.ffn;
-        P.K = d.hidden;
-        P.x = m->h;
-        P.norm_w = L.ffn_norm;
-        P.eps = d.rms_eps;
-        P.y = m->act;
-        P.use_pdl = pdl;
-        if ((st = gemv_launch(d.qtype, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, P, s)) != NTX_OK) return st;
-    }
-    {
-        Params P{};
-        P.W = (const uint8_t*)w.down;
-        P.row_bytes = m->rb_f;
-        P.M = d.hidden;
-        P.K = d.ffn;
-        P.x = m->act;
-        P.y = m->h;
-        P.use_pdl = pdl;
-        if ((st = gemv_launch(d.qtype, gemv::EPI_ADD, gemv::PRO_X, P, s)) != NTX_OK) return st;
-    }
-    return NTX_OK;
+    if ((st = launch_o(m, w.o, s, pdl)) != NTX_OK) return st;
+    if ((st = launch_gate_up(m, l, w.gate, w.up, s, pdl)) != NTX_OK) return st;
+    return launch_down(m, w.down, s, pdl);
 }
 
 ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
@@ -434,4 +453,29 @@ NTX_EXPORT ntx_status ntx_stream_stats(ntx_model* m, int64_t* h2d_bytes, float* 
         *step_ms = ms;
     }
     return NTX_OK;
+}
+
+NTX_EXPORT ntx_status ntx_model_replay_gemv(ntx_model* m, int kind, int n_launches, float* logits, void* stream)
+{
+    if (!m) return fail(NTX_EINVAL, "ntx_model_replay_gemv: null model");
+    if (kind < NTX_GEMV_QKV || kind > NTX_GEMV_HEAD) return fail(NTX_EINVAL, "ntx_model_replay_gemv: unknown kind");
+    if (n_launches < 1) return fail(NTX_EINVAL, "ntx_model_replay_gemv: n_launches must be >= 1");
+    if (kind == NTX_GEMV_HEAD && (!logits || !aligned(logits, 4)))
+        return fail(NTX_EINVAL, "ntx_model_replay_gemv: the LM head needs 4-byte aligned logits");
+    const int nres = m->d.n_resident;
+    if (kind != NTX_GEMV_HEAD && nres < 1) return fail(NTX_EINVAL, "ntx_model_replay_gemv: no resident layer");
+    cudaStream_t s = (cudaStream_t)stream;
+    ntx_status st = NTX_OK;
+    for (int i = 0; i < n_launches && st == NTX_OK; ++i) {
+        const int l = i % std::max(1, nres);
+        const ntx_layer_desc& L = m->layers[l];
+        switch (kind) {
+        case NTX_GEMV_QKV: st = launch_qkv(m, l, L.w_qkv, s, m->pdl); break;
+        case NTX_GEMV_O: st = launch_o(m, L.w_o, s, m->pdl); break;
+        case NTX_GEMV_GATE_UP: st = launch_gate_up(m, l, L.w_gate, L.w_up, s, m->pdl); break;
+        case NTX_GEMV_DOWN: st = launch_down(m, L.w_down, s, m->pdl); break;
+        default: st = enqueue_head(m, logits, s, m->pdl); break;
+        }
+    }
+    return st;
 }

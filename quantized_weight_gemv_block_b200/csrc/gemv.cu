@@ -64,10 +64,8 @@ ntx_status launch_t(Params P, cudaStream_t s, int grid_cap)
     if (!shape<QT>(P, 0)) return fail(NTX_EUNSUPPORTED, "gemv: row too long for the shared-memory pipeline");
     auto kern = gemv_kernel<QT, EPI, PRO>;
     const int smem = smem_bytes(P);
-    static std::once_flag once[20][4][2];
-    std::call_once(once[QT][EPI][PRO], [&] {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-    });
+    const ntx_status st = ensure_smem_limit((const void*)kern, kSmemLimit);
+    if (st != NTX_OK) return st;
     P.m24 = 1u << 24;
     const int outs = Outs<QT, EPI>::value;
     int grid = std::min(grid_cap, (P.M + outs - 1) / outs);

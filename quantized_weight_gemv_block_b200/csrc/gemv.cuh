@@ -72,6 +72,9 @@ struct Params {
     int x_bytes;
     int use_pdl;
     int recv_bytes;       // tiled GEMV: bytes of the per-group row sums of a CTA pair
+    int fs_off;           // tiled GEMV: byte offset of the per-step factors from the x words
+    int stall_stage;      // tiled GEMV, tests of the bounded waits: the producer issues no copy
+                          // from this stage on, so the consumers' wait for it runs out (-1: off)
     // multiplier that lets a shift run as an integer multiply on the FMA pipe
     // (v >> 8 == umulhi(v, 2^24)); passed in so it stays a multiply
     uint32_t m24;

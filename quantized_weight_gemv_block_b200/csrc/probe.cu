@@ -99,7 +99,8 @@ NTX_EXPORT ntx_status ntx_stream_read_probe(const void* src, size_t bytes, void*
     if (!src || bytes < 16 || bytes % 16) return fail(NTX_EINVAL, "ntx_stream_read_probe: bytes must be a positive multiple of 16");
     if (!aligned(src, 16)) return fail(NTX_EINVAL, "ntx_stream_read_probe: src must be 16-byte aligned");
     const int smem = 256 + kStages * (int)kStageBytes;
-    NTX_CUDA_TRY(cudaFuncSetAttribute(stream_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    const ntx_status st = ensure_smem_limit((const void*)stream_probe_kernel, smem);
+    if (st != NTX_OK) return st;
     stream_probe_kernel<<<num_sms(), 64, smem, (cudaStream_t)stream>>>((const uint8_t*)src, bytes);
     return check_launch("ntx_stream_read_probe");
 }

@@ -2,6 +2,7 @@
 // of CUDA-core or tensor-core units) and the repack kernel GGUF-style -> tiled.
 #include <algorithm>
 #include <cstdlib>
+#include <map>
 #include <mutex>
 
 #include "qmma.cuh"
@@ -138,7 +139,9 @@ bool shape(Params& P, int n_clusters, int csize, int n_mats)
 {
     using T = gemv::Tiled<QT>;
     const int kh = cta_cols<QT>(P.K, csize);
-    P.x_bytes = kh * 4;   // 32 words per 32-column step of the half
+    // 32 words per 32-column step of the half, then one float per step (16-byte multiple)
+    P.fs_off = kh * 4;
+    P.x_bytes = kh * 4 + (kh / 32 * 4 + 15) / 16 * 16;
     const int max_groups = (P.M / 16 + n_clusters - 1) / n_clusters;
     P.recv_bytes = max_groups * n_mats * 16 * 4;
     const int avail = kSmemLimit - kHeader - P.x_bytes - P.recv_bytes - 128;
@@ -156,32 +159,37 @@ bool shape(Params& P, int n_clusters, int csize, int n_mats)
     return true;
 }
 
-// Clusters of `csize` CTAs (one per SM) that fit on the device at once, per kernel.
+// Clusters of `csize` CTAs (one per SM) that fit on the current device at once, per
+// kernel (queried once per device and cluster size).
 template <int QT, int EPI, int PRO, int CORE>
 int max_clusters(int csize)
 {
-    static std::once_flag once[3];
-    static int n[3] = {0, 0, 0};
-    std::call_once(once[csize], [csize] {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(csize * 256);
-        cfg.blockDim = dim3(kThreads);
-        cfg.dynamicSmemBytes = kSmemLimit;
-        cudaLaunchAttribute attr[1];
-        attr[0].id = cudaLaunchAttributeClusterDimension;
-        attr[0].val.clusterDim.x = csize;
-        attr[0].val.clusterDim.y = 1;
-        attr[0].val.clusterDim.z = 1;
-        cfg.attrs = attr;
-        cfg.numAttrs = 1;
-        int c = 0;
-        if (cudaOccupancyMaxActiveClusters(&c, qmma_kernel<QT, EPI, PRO, CORE>, &cfg) != cudaSuccess || c < 1) {
-            cudaGetLastError();
-            c = std::max(1, num_sms() / csize);
-        }
-        n[csize] = c;
-    });
-    return n[csize];
+    static std::mutex mu;
+    static std::map<std::pair<int, int>, int> cache;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lock(mu);
+    const auto key = std::make_pair(dev, csize);
+    const auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(csize * 256);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = kSmemLimit;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = csize;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int c = 0;
+    if (cudaOccupancyMaxActiveClusters(&c, qmma_kernel<QT, EPI, PRO, CORE>, &cfg) != cudaSuccess || c < 1) {
+        cudaGetLastError();
+        c = std::max(1, num_sms() / csize);
+    }
+    cache[key] = c;
+    return c;
 }
 
 // Whether CTA pairs split the columns: when whole rows would leave the last round of
@@ -202,10 +210,12 @@ template <int QT, int EPI, int PRO, int CORE>
 ntx_status launch_t(Params P, cudaStream_t s)
 {
     auto kern = qmma_kernel<QT, EPI, PRO, CORE>;
-    static std::once_flag once[4][4][2];
-    std::call_once(once[QT & 3][EPI][PRO], [&] {
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemLimit);
-    });
+    const ntx_status st = ensure_smem_limit((const void*)kern, kSmemLimit);
+    if (st != NTX_OK) return st;
+    // NTX_TEST_STALL_STAGE=k (tests of the failure path only): the producer stops before
+    // stage k, so the consumers' bounded wait runs out and the kernel records an error
+    const char* stall = std::getenv("NTX_TEST_STALL_STAGE");
+    P.stall_stage = (stall && stall[0]) ? std::atoi(stall) : -1;
     const int csize = pick_cluster_size(P.M, P.K);
     const int n_clusters = std::max(1, std::min(max_clusters<QT, EPI, PRO, CORE>(csize), P.M / 16));
     if (!shape<QT>(P, n_clusters, csize, EPI == gemv::EPI_SWIGLU ? 2 : 1))

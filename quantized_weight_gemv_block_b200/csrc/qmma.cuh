@@ -5,20 +5,25 @@
 // weight once, so the work per weight must stay far below the SM's issue rate to
 // keep HBM busy.  Dequantizing each weight to fp32 and multiplying costs several
 // instructions per weight; here the packed codes are multiplied as integers:
-//  * the input vector x is turned once per CTA into 24-bit fixed point,
-//    x_int = rint(x 2^S) with |x_int| < 2^22, written as three balanced signed
-//    8-bit limbs, x_int = l0 + 2^8 l1 + 2^16 l2 (S from max |x|, a power of two);
+//  * the input vector x is turned once per CTA into 24-bit fixed point with one
+//    exponent per 32-column step u: x_int = rint(x 2^(S + e_u)) with |x_int| < 2^22,
+//    written as three balanced signed 8-bit limbs, x_int = l0 + 2^8 l1 + 2^16 l2.
+//    S comes from max |x| over the CTA's columns; e_u >= 0 adds the bits a step whose
+//    values are all small can carry (from the step's own max |x|), so every step keeps
+//    23 bits relative to its own largest value and an outlier channel only costs
+//    precision to the 31 columns that share its step;
 //  * the codes (int8 for Q8_0, unsigned 4- or 6-bit codes for the others, unpacked
 //    to bytes with a few logic ops per word) are dotted with each limb, four bytes
 //    at a time, by dp4a on the CUDA cores (CORE 1, the default): every partial sum is
 //    an exact integer;
 //  * the format's per-block scale (fp16 d, int8 or 6-bit sub-block scales, the
 //    Q4_K mins, the code offsets 8 and 32) is applied to those integers, in
-//    integer arithmetic where it is exact, in fp32 once per block otherwise;
+//    integer arithmetic where it is exact, and in fp32 once per step together with
+//    the step's 2^-e_u (exact: a power of two);
 //  * the limbs are recombined (weights 1, 2^8, 2^16) and the row total is scaled
 //    by 2^-S, exactly.
-// The products are exact; x carries 23 bits (relative to max |x|) where fp32
-// carries 24; sums round at fp32 once per block or superblock.
+// The products are exact; x carries 23 bits relative to the largest value of its
+// 32-column step where fp32 carries 24 per value; sums round at fp32 once per step.
 // CORE 0 does the same integer dots with one m16n8k32 integer MMA per 16 x 32 block
 // (codes as A, the limbs as the 8 columns of B); it is kept as a measured
 // alternative (NTX_GEMV_CORE=tc): on B200 the dp4a path streams as fast or faster on
@@ -67,6 +72,9 @@ constexpr int kOffRope = kOffRed + 2 * kWarps * 32 * 4;   // [64][cos, sin]
 constexpr int kHeader = kOffRope + 512 + 256;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr uint32_t kWaitPolls = 1u << 22;
+// Extra bits a step may take beyond the CTA's exponent S: a step whose largest value is
+// 2^40 below the CTA's largest keeps 23 bits; smaller steps keep 23 - (their shortfall).
+constexpr int kMaxStepShift = 40;
 
 // ------------------------------------------------------------------ MMA helpers
 
@@ -176,6 +184,8 @@ __device__ __forceinline__ void red_add_cluster(uint32_t addr, float v)
 // four consecutive steps, and a warp converting x writes four consecutive steps, which
 // then fall in four different bank groups.  The Q8_0 lane units read no sums (words
 // 24..31 hold no data there); only the tensor-core units read the zero words.
+// A separate array of floats holds, per step u, 2^-e_u: the factor that brings the
+// step's integer dots back to the CTA's common scale 2^S (fs below).
 
 // The limb words and column sums of the 4 columns a lane holds (lane w of the 8 lanes
 // of a step); the sums are already reduced over the step's lanes (or each half's).
@@ -327,8 +337,8 @@ struct Unit;
 
 template <>
 struct Unit<NTX_Q8_0_T> {
-    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
-                                               float& acc1)
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, const Lane& L,
+                                               float& acc0, float& acc1)
     {
         const uint4 a4 = *reinterpret_cast<const uint4*>(U + 16 * L.lane);
         const uint32_t a[4] = {a4.x, a4.y, a4.z, a4.w};
@@ -337,15 +347,16 @@ struct Unit<NTX_Q8_0_T> {
         int c[4];
         mma_s8(c, a, b0, b1);
         const float2 d = d_pair(U + 512 + 4 * L.gid);
-        acc0 = fmaf((float)(c[0] + 256 * c[1]), d.x, acc0);
-        acc1 = fmaf((float)(c[2] + 256 * c[3]), d.y, acc1);
+        const float f = fs[0];
+        acc0 = fmaf((float)(c[0] + 256 * c[1]), d.x * f, acc0);
+        acc1 = fmaf((float)(c[2] + 256 * c[3]), d.y * f, acc1);
     }
 };
 
 template <>
 struct Unit<NTX_Q4_0_T> {
-    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
-                                               float& acc1)
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, const Lane& L,
+                                               float& acc0, float& acc1)
     {
         const uint2 pq = *reinterpret_cast<const uint2*>(U + 8 * L.lane);
         const uint32_t M = 0x0F0F0F0Fu;
@@ -358,20 +369,20 @@ struct Unit<NTX_Q4_0_T> {
         const int2 X = *reinterpret_cast<const int2*>(xs + 24 + 2 * L.tig);
         const int off = -8 * (X.x + 256 * X.y);
         const float2 d = d_pair(U + 256 + 4 * L.gid);
-        acc0 = fmaf((float)(c[0] + 256 * c[1] + off), d.x, acc0);
-        acc1 = fmaf((float)(c[2] + 256 * c[3] + off), d.y, acc1);
+        const float f = fs[0];
+        acc0 = fmaf((float)(c[0] + 256 * c[1] + off), d.x * f, acc0);
+        acc1 = fmaf((float)(c[2] + 256 * c[3] + off), d.y * f, acc1);
     }
 };
 
 template <>
 struct Unit<NTX_Q6_K_T> {
-    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
-                                               float& acc1)
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, const Lane& L,
+                                               float& acc0, float& acc1)
     {
         // this lane's scales: sub-blocks 2m + (tig / 2) of rows gid (bytes 0-7) and gid + 8 (8-15)
         const uint4 sv = *reinterpret_cast<const uint4*>(U + 3072 + 16 * (2 * L.gid + (L.tig >> 1)));
-        // per row: s * (limb-0 column), s * (limb-1 column), s * (the columns' limb sums)
-        int p0 = 0, p1 = 0, q0 = 0, q1 = 0, o0 = 0, o1 = 0, r0 = 0, r1 = 0;
+        const float2 d = d_pair(U + 3328 + 4 * L.gid);
         const uint32_t M6 = 0x3F3F3F3Fu;
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
@@ -398,30 +409,26 @@ struct Unit<NTX_Q6_K_T> {
                 s0 = m == 4 ? sbyte<0>(sv.y) : m == 5 ? sbyte<1>(sv.y) : m == 6 ? sbyte<2>(sv.y) : sbyte<3>(sv.y);
                 s1 = m == 4 ? sbyte<0>(sv.w) : m == 5 ? sbyte<1>(sv.w) : m == 6 ? sbyte<2>(sv.w) : sbyte<3>(sv.w);
             }
-            p0 += s0 * c[0];
-            p1 += s0 * c[1];
-            o0 += s0 * X.x;
-            o1 += s0 * X.y;
-            q0 += s1 * c[2];
-            q1 += s1 * c[3];
-            r0 += s1 * X.x;
-            r1 += s1 * X.y;
+            // codes carry +32; the step's column totals are exact integers before the fp32 step
+            const int p0 = s0 * (c[0] - 32 * X.x), p1 = s0 * (c[1] - 32 * X.y);
+            const int q0 = s1 * (c[2] - 32 * X.x), q1 = s1 * (c[3] - 32 * X.y);
+            const float f = fs[m];
+            acc0 = fmaf(d.x * f, fmaf(256.f, (float)p1, (float)p0), acc0);
+            acc1 = fmaf(d.y * f, fmaf(256.f, (float)q1, (float)q0), acc1);
         }
-        // codes carry +32; every column's integer total is exact before the fp32 step
-        const float2 d = d_pair(U + 3328 + 4 * L.gid);
-        acc0 = fmaf(d.x, fmaf(256.f, (float)(p1 - 32 * o1), (float)(p0 - 32 * o0)), acc0);
-        acc1 = fmaf(d.y, fmaf(256.f, (float)(q1 - 32 * r1), (float)(q0 - 32 * r0)), acc1);
     }
 };
 
 template <>
 struct Unit<NTX_Q4_K_T> {
-    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
-                                               float& acc1)
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, const Lane& L,
+                                               float& acc0, float& acc1)
     {
         uint32_t S[8];
         q4k_scale_words(U, L.gid, S);
-        int p0 = 0, p1 = 0, q0 = 0, q1 = 0, o0 = 0, r0 = 0;
+        const uint2 dd = *reinterpret_cast<const uint2*>(U + 2240 + 8 * L.gid);
+        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
         const uint32_t M = 0x0F0F0F0Fu;
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
@@ -435,18 +442,12 @@ struct Unit<NTX_Q4_K_T> {
             const int2 X = *reinterpret_cast<const int2*>(x + 24 + 2 * L.tig);
             const int xp = X.x + 256 * X.y;
             const int sc0 = ubyte<0>(S[m]), sc1 = ubyte<1>(S[m]), mn0 = ubyte<2>(S[m]), mn1 = ubyte<3>(S[m]);
-            p0 += sc0 * c[0];
-            p1 += sc0 * c[1];
-            q0 += sc1 * c[2];
-            q1 += sc1 * c[3];
-            o0 += mn0 * xp;
-            r0 += mn1 * xp;
+            const float f = fs[m];
+            acc0 = fmaf(d.x * f, fmaf(256.f, (float)(sc0 * c[1]), (float)(sc0 * c[0])),
+                        fmaf(-dm.x * f, (float)(mn0 * xp), acc0));
+            acc1 = fmaf(d.y * f, fmaf(256.f, (float)(sc1 * c[3]), (float)(sc1 * c[2])),
+                        fmaf(-dm.y * f, (float)(mn1 * xp), acc1));
         }
-        const uint2 dd = *reinterpret_cast<const uint2*>(U + 2240 + 8 * L.gid);
-        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
-        const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
-        acc0 = fmaf(d.x, fmaf(256.f, (float)p1, (float)p0), fmaf(-dm.x, (float)o0, acc0));
-        acc1 = fmaf(d.y, fmaf(256.f, (float)q1, (float)q0), fmaf(-dm.y, (float)r0, acc1));
     }
 };
 
@@ -487,8 +488,8 @@ struct Dot;
 
 template <>
 struct Dot<NTX_Q8_0_T> {
-    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const Lane& L, float& acc0,
-                                               float& acc1)
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, const Lane& L,
+                                               float& acc0, float& acc1)
     {
         const uint4 a = *reinterpret_cast<const uint4*>(U + 16 * L.lane);
         uint2 X[3];
@@ -500,8 +501,9 @@ struct Dot<NTX_Q8_0_T> {
             c1[l] = dp4(a.w, X[l].y, dp4(a.y, X[l].x, 0));
         }
         const float2 d = d_pair(U + 512 + 4 * L.gid);
-        acc0 = fmaf(d.x, limbs_f(c0[0], c0[1], c0[2]), acc0);
-        acc1 = fmaf(d.y, limbs_f(c1[0], c1[1], c1[2]), acc1);
+        const float f = fs[0];
+        acc0 = fmaf(d.x * f, limbs_f(c0[0], c0[1], c0[2]), acc0);
+        acc1 = fmaf(d.y * f, limbs_f(c1[0], c1[1], c1[2]), acc1);
     }
 };
 
@@ -546,9 +548,9 @@ struct Row;
 
 template <>
 struct Row<NTX_Q4_0_T> {
-    // U: the unit (one step), xs: its x words, sx: the step's x swizzle
-    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, int sx, int g, float& acc0,
-                                               float& acc1)
+    // U: the unit (one step), xs: its x words, sx: the step's x swizzle, f: the step's factor
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, int sx, float f, int g,
+                                               float& acc0, float& acc1)
     {
         const uint4* L = reinterpret_cast<const uint4*>(U + 32 * g);   // (P, Q) of lanes tig 0..3
         const uint4 u0 = L[0], u1 = L[1];
@@ -569,16 +571,17 @@ struct Row<NTX_Q4_0_T> {
             }
         }
         const float2 d = d_pair(U + 256 + 4 * g);
-        acc0 = fmaf(d.x, limbs_f(c0[0], c0[1], c0[2]), acc0);
-        acc1 = fmaf(d.y, limbs_f(c1[0], c1[1], c1[2]), acc1);
+        acc0 = fmaf(d.x * f, limbs_f(c0[0], c0[1], c0[2]), acc0);
+        acc1 = fmaf(d.y * f, limbs_f(c1[0], c1[1], c1[2]), acc1);
     }
 };
 
 template <>
 struct Row<NTX_Q6_K_T> {
-    // U: the superblock unit, xs: its x words; the thread takes steps j and j + 4
-    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, int g, int j, float& acc0,
-                                               float& acc1)
+    // U: the superblock unit, xs: its x words, fs: its steps' factors; the thread takes
+    // steps j and j + 4
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, int g, int j,
+                                               float& acc0, float& acc1)
     {
         // int8 scales: vector (g, parity) holds row g at bytes 0-7 and row g + 8 at bytes
         // 8-15, byte m of each = sub-block 2m + parity (se: parity 0, so: parity 1)
@@ -586,9 +589,10 @@ struct Row<NTX_Q6_K_T> {
         const uint4 so = *reinterpret_cast<const uint4*>(U + 3072 + 32 * g + 16);
         const uint32_t sel = sbyte_sel(j);   // byte m mod 4 = j
         const uint32_t M6 = 0x3F3F3F3Fu;
-        int p0[3] = {0, 0, 0}, p1[3] = {0, 0, 0};   // per limb: rows g, g + 8
+        const float2 d = d_pair(U + 3328 + 4 * g);
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
+            int p0[3] = {0, 0, 0}, p1[3] = {0, 0, 0};   // per limb: rows g, g + 8
             const int m = j + 4 * k;
             // lanes tig 0..3 of gid g: words A, B, C of each
             const uint4* L = reinterpret_cast<const uint4*>(U + 384 * m + 48 * g);
@@ -627,25 +631,29 @@ struct Row<NTX_Q6_K_T> {
                 p0[l] += s_e0 * e0 + s_o0 * o0;
                 p1[l] += s_e1 * e1 + s_o1 * o1;
             }
+            const float f = fs[m];
+            acc0 = fmaf(d.x * f, limbs_f(p0[0], p0[1], p0[2]), acc0);
+            acc1 = fmaf(d.y * f, limbs_f(p1[0], p1[1], p1[2]), acc1);
         }
-        const float2 d = d_pair(U + 3328 + 4 * g);
-        acc0 = fmaf(d.x, limbs_f(p0[0], p0[1], p0[2]), acc0);
-        acc1 = fmaf(d.y, limbs_f(p1[0], p1[1], p1[2]), acc1);
     }
 };
 
 template <>
 struct Row<NTX_Q4_K_T> {
-    // U: the superblock unit, xs: its x words; the thread takes steps (= sub-blocks) j and j + 4
-    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, int g, int j, float& acc0,
-                                               float& acc1)
+    // U: the superblock unit, xs: its x words, fs: its steps' factors; the thread takes
+    // steps (= sub-blocks) j and j + 4
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, int g, int j,
+                                               float& acc0, float& acc1)
     {
         const uint8_t* v = U + 2048 + 24 * g;   // packed 6-bit scales / mins of rows g, g + 8
         const uint32_t M = 0x0F0F0F0Fu;
-        int p0[3] = {0, 0, 0}, p1[3] = {0, 0, 0};   // per limb: rows g, g + 8
-        int n0[3] = {0, 0, 0}, n1[3] = {0, 0, 0};   // mins x limb sums
+        const uint2 dd = *reinterpret_cast<const uint2*>(U + 2240 + 8 * g);
+        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
 #pragma unroll
         for (int k = 0; k < 2; ++k) {
+            int p0[3] = {0, 0, 0}, p1[3] = {0, 0, 0};   // per limb: rows g, g + 8
+            int n0[3] = {0, 0, 0}, n1[3] = {0, 0, 0};   // mins x limb sums
             const int m = j + 4 * k;
             // sub-block m: byte 0 scale row g, 1 scale row g + 8, 2 min row g, 3 min row g + 8
             const uint32_t nw = *reinterpret_cast<const uint32_t*>(v + 4 * (m >> 1));
@@ -673,12 +681,10 @@ struct Row<NTX_Q4_K_T> {
                 n0[l] += mn0 * (int)comp(xsum, l);
                 n1[l] += mn1 * (int)comp(xsum, l);
             }
+            const float f = fs[m];
+            acc0 = fmaf(d.x * f, limbs_f(p0[0], p0[1], p0[2]), fmaf(-dm.x * f, limbs_f(n0[0], n0[1], n0[2]), acc0));
+            acc1 = fmaf(d.y * f, limbs_f(p1[0], p1[1], p1[2]), fmaf(-dm.y * f, limbs_f(n1[0], n1[1], n1[2]), acc1));
         }
-        const uint2 dd = *reinterpret_cast<const uint2*>(U + 2240 + 8 * g);
-        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
-        const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
-        acc0 = fmaf(d.x, limbs_f(p0[0], p0[1], p0[2]), fmaf(-dm.x, limbs_f(n0[0], n0[1], n0[2]), acc0));
-        acc1 = fmaf(d.y, limbs_f(p1[0], p1[1], p1[2]), fmaf(-dm.y, limbs_f(n1[0], n1[1], n1[2]), acc1));
     }
 };
 
@@ -742,6 +748,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
     float* red = reinterpret_cast<float*>(smem + kOffRed);
     float* rope_cs = reinterpret_cast<float*>(smem + kOffRope);
     uint32_t* xq = reinterpret_cast<uint32_t*>(smem + kHeader);
+    float* xsf = reinterpret_cast<float*>(smem + kHeader + P.fs_off);   // per-step factors 2^-e_u
     uint8_t* stages = smem + kHeader + P.x_bytes;
     float* sums = reinterpret_cast<float*>(stages + (size_t)P.n_stages * P.stage_bytes);   // [group][mat][16]
 
@@ -788,6 +795,12 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                 for (int mat = 0; mat < NM && okay; ++mat) {
                     const uint8_t* base = (mat ? P.W2 : P.W) + (int64_t)gi * group_bytes + (int64_t)u0 * T::UB;
                     for (int c = 0; c < NCH; ++c) {
+                        if (issued == P.stall_stage) {
+                            // test of the consumers' bounded wait: stop issuing (every copy issued
+                            // so far lands before the consumers reach this stage)
+                            okay = false;
+                            break;
+                        }
                         if (!mbar_wait(&empty[s], ph ^ 1u, kWaitPolls)) {
                             record_device_error(DEVERR_EMPTY_WAIT);
                             okay = false;
@@ -899,30 +912,42 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
         // the normalised value is fl(fl(x w) inv): its largest magnitude is fl(max |x w| inv)
         const float inv = RMS ? 1.0f / sqrtf(tot / (float)P.K + P.eps) : 1.f;
         if (RMS) mx *= inv;
-        // |x| 2^S < 2^22; a zero half keeps S = 0 (all limbs zero)
+        // |x| 2^S < 2^22 over the CTA's columns; a zero half keeps S = 0 (all limbs zero)
         const int S = (mx > 0.f && mx <= 3.4e38f) ? max(-100, min(127, 21 - ilogbf(mx))) : 0;
-        const float two_s = __uint_as_float((uint32_t)(127 + S) << 23);
+        const int e_cap = min(kMaxStepShift, 127 - S);
         // (3) normalised fp32 -> limbs, in place: 8 lanes per 32-column step, float4
-        // i = tid + j kCons; 4 rounds at a time, all reads of a round before its stores
+        // i = tid + j kCons; 4 rounds at a time, all reads of a round before its stores.
+        // Step u takes 2^(S + e_u) with e_u the extra bits its own largest value leaves room
+        // for (|x| 2^(S + e_u) < 2^22 still holds), and records 2^-e_u.
         {
             const int n_steps = KR / 32, n_rounds = (n_steps + 31) / 32, wl = lane & 7;
             auto convert4 = [&](int j0, const float4 (&w)[4]) {
                 XLimbs r[4];
+                float fk[4];
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int i = tid + (j0 + k) * kCons;
                     float4 v = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
                     if (RMS)
                         v = make_float4(v.x * w[k].x * inv, v.y * w[k].y * inv, v.z * w[k].z * inv, v.w * w[k].w * inv);
-                    r[k] = x_limbs<QT == NTX_Q6_K_T, XSUMS>(v, two_s);
+                    // the step's largest magnitude over its 8 lanes
+                    float m = fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w)));
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 2));
+                    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 4));
+                    const int e = (m > 0.f && m <= 3.4e38f) ? max(0, min(e_cap, 21 - ilogbf(m) - S)) : 0;
+                    r[k] = x_limbs<QT == NTX_Q6_K_T, XSUMS>(v, __uint_as_float((uint32_t)(127 + S + e) << 23));
+                    fk[k] = __uint_as_float((uint32_t)(127 - e) << 23);
                 }
                 __syncwarp();   // every lane of a step has read its floats before any limb word lands
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int u = (tid + (j0 + k) * kCons) >> 3;
-                    if (u < n_steps)
+                    if (u < n_steps) {
                         x_store<QT == NTX_Q6_K_T, CORE == 1 && QT == NTX_Q8_0_T, XSUMS, CORE == 0>(
                             xq + 32 * u, wl, r[k], ROWS ? 8 * (u & 3) : 0);
+                        if (wl == 0) xsf[u] = fk[k];
+                    }
                 }
             };
 #pragma unroll
@@ -969,23 +994,26 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                     const uint8_t* st = stages + (size_t)s * P.stage_bytes;
                     if (!dead) {
                         const uint32_t* xc = xq + 32 * (c * CE / 32);
+                        const float* fc = xsf + c * CE / 32;
                         if (CORE == 0) {
                             for (int un = warp; un < n_units; un += kWarps)
-                                Unit<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, L, acc0, acc1);
+                                Unit<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, fc + SPU * un, L, acc0,
+                                              acc1);
                         } else if constexpr (QT == NTX_Q8_0_T) {
                             for (int un = warp; un < n_units; un += kWarps)
-                                Dot<QT>::run(st + (size_t)un * T::UB, xc + 32 * un, L, acc0, acc1);
+                                Dot<QT>::run(st + (size_t)un * T::UB, xc + 32 * un, fc + un, L, acc0, acc1);
                         } else if constexpr (QT == NTX_Q4_0_T) {
                             // a warp takes 4 units (steps) at a time, one per 8 threads
                             const int sx = 8 * ((c * CE / 32 + rj) & 3);
                             for (int u4 = 4 * warp; u4 < n_units; u4 += 4 * kWarps) {
                                 const int un = u4 + rj;
                                 if (un < n_units)
-                                    Row<QT>::run(st + (size_t)un * T::UB, xc + 32 * un, sx, rgid, acc0, acc1);
+                                    Row<QT>::run(st + (size_t)un * T::UB, xc + 32 * un, sx, fc[un], rgid, acc0, acc1);
                             }
                         } else {
                             for (int un = warp; un < n_units; un += kWarps)
-                                Row<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, rgid, rj, acc0, acc1);
+                                Row<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, fc + SPU * un, rgid, rj,
+                                             acc0, acc1);
                         }
                     }
                     __syncwarp();

@@ -4,7 +4,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import GEMV_TIGHT, TOL, ntx_module, rel_err
+from gpu_util import GEMV_TIGHT, TOL, elem_err, ntx_module, rel_err
 
 pytestmark = pytest.mark.gpu
 
@@ -49,6 +49,7 @@ def test_gemv_fast_path(ntx, orc, syn, qtype, rows, cols):
     o = orc.gemv(qtype, host, rows, cols, x)
     e = rel_err(y, o)
     assert e <= TOL and e <= GEMV_TIGHT, e
+    assert elem_err(y, o) <= TOL
     assert ntx.ntx_device_error() == 0
 
 
@@ -140,27 +141,100 @@ def test_gemv_full_shapes(ntx, orc, syn, qtype, rows, cols):
     host, dev = make(syn, qtype, rows, cols)
     x = syn.normal_f32_host(5, 12, cols)
     y = gpu_gemv(ntx, qtype, dev, rows, cols, x)
-    e = rel_err(y, orc.gemv(qtype, host, rows, cols, x))
+    o = orc.gemv(qtype, host, rows, cols, x)
+    e = rel_err(y, o)
     assert e <= GEMV_TIGHT, e
+    assert elem_err(y, o) <= TOL
 
 
+@pytest.mark.parametrize("tiled", [False, True], ids=["gguf", "tiled"])
 @pytest.mark.parametrize("qtype", [Q4_0, Q4_K, Q8_0, Q6_K], ids=["q4_0", "q4_k", "q8_0", "q6_k"])
-def test_gemv_lm_head_sampled_rows(ntx, orc, syn, qtype):
-    """The 4096 -> 128256 (8192 -> 128256 for Q6_K) LM-head GEMV at full size, checked on
-    sampled rows the oracle computes one by one."""
+def test_gemv_lm_head_sampled_rows(ntx, orc, syn, qtype, tiled):
+    """The 4096 -> 128256 (8192 -> 128256 for Q6_K) LM-head GEMV at full size, in the GGUF-style
+    and the tiled layout, checked on sampled rows the oracle computes one by one."""
     rows, cols = 128256, (8192 if qtype == Q6_K else 4096)
     qp = syn.sweep_qparams(qtype)
     dev = torch.empty(rows * syn.row_bytes(qtype, cols), dtype=torch.uint8, device="cuda")
     syn.blocks_dev(dev, qtype, 9, 21, rows, cols, qp)
+    if tiled:
+        t = torch.empty_like(dev)
+        ntx.ntx_repack_q(qtype, dev, t, rows, cols)
+        dev = t
     x = syn.normal_f32_host(9, 22, cols)
-    y = gpu_gemv(ntx, qtype, dev, rows, cols, x)
+    y = gpu_gemv(ntx, qtype | (T if tiled else 0), dev, rows, cols, x)
     rng = np.random.default_rng(0)
-    sample = np.unique(np.concatenate([[0, 1, rows // 2, rows - 2, rows - 1], rng.integers(0, rows, 300)]))
+    sample = np.unique(np.concatenate([[0, 1, 15, 16, rows // 2, rows - 17, rows - 2, rows - 1],
+                                       rng.integers(0, rows, 300)]))
     o = np.empty(sample.size, dtype=np.float32)
     for i, r in enumerate(sample):
         Wr = syn.blocks_host(qtype, 9, 21, 1, cols, qp, row0=int(r))
         o[i] = orc.gemv(qtype, Wr, 1, cols, x)[0]
     assert rel_err(y[sample], o) <= GEMV_TIGHT
+    assert elem_err(y[sample], o) <= TOL
+
+
+# ------------------------------------------------------------ outlier channels
+
+ZERO_CODE = {Q8_0: 0, Q4_0: 8, Q4_K: 0, Q6_K: 32}
+
+
+def outlier_matrix(qtype, rows, cols, cols_out, seed):
+    """Packed GGUF-style [rows, cols] with random fields, whose first rows // 2 rows hold a
+    zero weight at every column of cols_out (the format's zero code; for Q4_K also a zero
+    min for that sub-block), built with the test-side packer."""
+    import blockpack as bp
+    rng = np.random.default_rng(seed)
+    be = 32 if qtype in (Q8_0, Q4_0) else 256
+    out = bytearray()
+    for r in range(rows):
+        for b in range(cols // be):
+            f = bp.random_fields(qtype, rng)
+            if r < rows // 2:
+                for c in cols_out:
+                    if b * be <= c < (b + 1) * be:
+                        f["q"] = np.array(f["q"])
+                        f["q"][c - b * be] = ZERO_CODE[qtype]
+                        if qtype == Q4_K:
+                            f["m"] = np.array(f["m"])
+                            f["m"][(c - b * be) // 32] = 0
+            out += bp.pack(qtype, f)
+    return np.frombuffer(bytes(out), dtype=np.uint8).reshape(rows, -1).copy()
+
+
+def outlier_input(syn, cols, cols_out):
+    """x ~ N(0, 1) with LLM-style outlier channels: six at 1e3 and two at 1e4 times the rest."""
+    x = syn.normal_f32_host(31, 12, cols)
+    for i, c in enumerate(cols_out):
+        x[c] = np.float32((1e4 if i >= 6 else 1e3) * (1.0 if i % 2 else -1.0) * (1.0 + 0.1 * i))
+    return x
+
+
+@pytest.mark.parametrize("layout", ["gguf", "tiled-dp4a", "tiled-tc"])
+@pytest.mark.parametrize("qtype", [Q8_0, Q4_0, Q4_K, Q6_K], ids=list(NAMES.values()))
+def test_gemv_outlier_channels(ntx, orc, syn, monkeypatch, qtype, layout):
+    """A few input channels 1e3..1e4 times the rest, and half of the rows with zero weight at
+    those channels: those rows' outputs are far below the largest output, and must keep their
+    own precision (per-element error against the oracle, floor 1e-3 max |o|), not only the
+    normwise one."""
+    rows, cols = 64, 4096
+    cols_out = [5, 700, 1031, 2047, 2048, 3333, 3900, 4095]
+    host = outlier_matrix(qtype, rows, cols, cols_out, seed=qtype + 40)
+    dev = torch.from_numpy(host.reshape(-1)).cuda()
+    q = qtype
+    if layout != "gguf":
+        monkeypatch.setenv("NTX_GEMV_CORE", "tc" if layout.endswith("tc") else "dp4a")
+        t = torch.empty_like(dev)
+        ntx.ntx_repack_q(qtype, dev, t, rows, cols)
+        dev, q = t, qtype | T
+    x = outlier_input(syn, cols, cols_out)
+    y = gpu_gemv(ntx, q, dev, rows, cols, x)
+    o = orc.gemv(qtype, host, rows, cols, x)
+    # the rows that ignore the outliers are the small ones
+    assert np.max(np.abs(o[: rows // 2])) < 0.05 * np.max(np.abs(o[rows // 2:]))
+    assert rel_err(y, o) <= GEMV_TIGHT
+    e = elem_err(y, o)
+    print(f"outlier channels {NAMES[qtype]} {layout}: normwise {rel_err(y, o):.2e} per-element {e:.2e}")
+    assert e <= TOL, e
 
 
 # ------------------------------------------------------------------ tiled layouts
@@ -187,8 +261,10 @@ TILED_FAST = [(Q8_0, 48, 4096 + 256), (Q4_0, 48, 4096 + 256), (Q4_K, 48, 8192 + 
 def test_gemv_tiled(ntx, orc, syn, qtype, rows, cols):
     host, W = make_tiled(ntx, syn, qtype, rows, cols)
     x = syn.normal_f32_host(1, 13, cols)
-    e = rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x))
+    y, o = gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)
+    e = rel_err(y, o)
     assert e <= TOL and e <= GEMV_TIGHT, e
+    assert elem_err(y, o) <= TOL
 
 
 @pytest.mark.parametrize("qtype", [Q8_0, Q4_0, Q4_K, Q6_K], ids=list(NAMES.values()))
@@ -220,15 +296,18 @@ def test_tiled_one_hot_bit_exact(ntx, syn, qtype):
         assert np.array_equal(gpu_gemv(ntx, qtype | T, W, rows, cols, x), dq[:, k].cpu().numpy()), k
 
 
-TSWEEP = [(q, n, k) for q in (Q4_0, Q4_K, Q8_0) for (k, n) in ((4096, 6144), (4096, 14336), (14336, 4096))]
-TSWEEP += [(Q6_K, 10240, 8192), (Q6_K, 8192, 28672), (Q6_K, 28672, 8192), (Q8_0, 4096, 4096)]
+TSWEEP = [(q, n, k) for q in (Q4_0, Q4_K, Q8_0) for (k, n) in ((4096, 6144), (4096, 4096), (4096, 14336),
+                                                                 (14336, 4096))]
+TSWEEP += [(Q6_K, 10240, 8192), (Q6_K, 8192, 8192), (Q6_K, 8192, 28672), (Q6_K, 28672, 8192)]
 
 
 @pytest.mark.parametrize("qtype,rows,cols", TSWEEP, ids=[f"{NAMES[q]}_t-{r}x{c}" for q, r, c in TSWEEP])
 def test_gemv_tiled_full_shapes(ntx, orc, syn, qtype, rows, cols):
     host, W = make_tiled(ntx, syn, qtype, rows, cols)
     x = syn.normal_f32_host(6, 12, cols)
-    assert rel_err(gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)) <= GEMV_TIGHT
+    y, o = gpu_gemv(ntx, qtype | T, W, rows, cols, x), orc.gemv(qtype, host, rows, cols, x)
+    assert rel_err(y, o) <= GEMV_TIGHT
+    assert elem_err(y, o) <= TOL
 
 
 @pytest.mark.parametrize("qtype,rows,cols", [(Q8_0, 32, 512), (Q4_0, 16, 256), (Q4_K, 32, 512), (Q6_K, 16, 768)],

@@ -2,10 +2,11 @@
 callers that have no device memory to hand over as a workspace.
 
 Checked through the C ABI against the allocating entry point on the same
-inputs, for two calls in a row (the shared scratch keeps the previous call's
-contents, so the second call shows the counters are cleared), and for the
-size limit of the fixed scratch.  Collected last on purpose: it must pass in a
-fresh process and after every other test."""
+inputs, for two calls in a row with different inputs and context lengths (the
+shared scratch keeps the previous call's partials, and the second call must not
+be affected by them: every split's partial is rewritten before the merge reads
+it), and for the size limit of the fixed scratch.  Collected last on purpose: it
+must pass in a fresh process and after every other test."""
 import numpy as np
 import pytest
 import torch
