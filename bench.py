@@ -164,8 +164,9 @@ def step_bytes(spec):
     """Algorithmic bytes of one decode step: packed weights read + KV cache read
     (positions 0..pos) + the embedding row (vectors are negligible)."""
     import synth
-    w = spec.n_layers * spec.layer_weight_bytes() + spec.vocab * synth.row_bytes(spec.qtype, spec.hidden)
-    return w + kv_read_bytes(spec) + synth.row_bytes(spec.qtype, spec.hidden)
+    w = sum(spec.layer_weight_bytes(l) for l in range(spec.n_layers))
+    w += spec.vocab * synth.row_bytes(spec.qtype_of("output"), spec.hidden)
+    return w + kv_read_bytes(spec) + synth.row_bytes(spec.qtype_of("tok_embd"), spec.hidden)
 
 
 def gemv_kinds(spec):
@@ -273,8 +274,9 @@ def run_decode_bench(args, rank, world, local):
     stream = torch.cuda.Stream()
     copy_stream = torch.cuda.Stream() if streamed else None
     logits = torch.empty(spec.vocab, dtype=torch.float32, device="cuda")
-    # step word + embedding, per layer QKV, attention, split merge, O, gate/up, down, then the LM head
-    launches_per_step = 2 + 6 * spec.n_layers + 1
+    # step word + embedding, per layer QKV, attention (with the split merge), O, gate/up, down,
+    # then the LM head
+    launches_per_step = 2 + 5 * spec.n_layers + 1
 
     def step():
         if streamed:
@@ -373,13 +375,14 @@ def cpu_baseline(spec, n_layers_timed=CPU_SAMPLE_LAYERS):
     for layer in range(n):
         t = om.layer_tensors(spec, layer)
         t0 = time.perf_counter()
-        oracle.decode_layer(dims, spec.qtype, h, spec.n_prefill, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"],
+        qts = [spec.qtype_of(k, layer) for k in ("w_qkv", "w_o", "w_gate", "w_down")]
+        oracle.decode_layer(dims, qts, h, spec.n_prefill, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"],
                             t["w_gate"], t["w_up"], t["w_down"], t["k_cache"], t["v_cache"])
         t_layers += time.perf_counter() - t0
     head_rows = max(256, spec.vocab // 32)
     norm, W = om.head_tensors(spec, (0, head_rows))
     t0 = time.perf_counter()
-    oracle.lm_head(spec.qtype, norm, W, head_rows, spec.hidden, spec.rms_eps, h)
+    oracle.lm_head(spec.qtype_of("output"), norm, W, head_rows, spec.hidden, spec.rms_eps, h)
     t_head = (time.perf_counter() - t0) * spec.vocab / head_rows
     s_per_tok = t_layers / n * spec.n_layers + t_head
     return {"value": 1.0 / s_per_tok, "unit": "tok/s", "cores": oracle.threads(), "kind": "oracle",
@@ -461,7 +464,16 @@ def gemv_sweep(ntx, stream, peak, peak_kind, ceiling):
         r = gemv_rotation_bench(ntx, synth.Q8_0, 4096, 4096, layout == "tiled", stream)
         r.update({"frac_of_%s" % peak_kind: r["gbs"] / peak, "frac_of_read_ceiling": r["gbs"] / ceiling})
         single[layout] = r
-    return rows_out, single
+    # the further formats at the same shapes: Q5_K in its tiled layout, F16 and F32 rows
+    further = []
+    for qname, q, tiled in (("q5_k", synth.Q5_K, True), ("f16", synth.F16, False), ("f32", synth.F32, False)):
+        for name, rows, cols in SWEEP_SHAPES:
+            r = gemv_rotation_bench(ntx, q, rows, cols, tiled, stream)
+            r.update({"format": qname, "layout": "tiled" if tiled else "rows", "shape": name, "rows": rows,
+                      "cols": cols, "frac_of_%s" % peak_kind: r["gbs"] / peak,
+                      "frac_of_read_ceiling": r["gbs"] / ceiling})
+            further.append(r)
+    return rows_out, single, further
 
 
 def measure_read_ceiling(ntx, stream, nbytes=4 << 30, iters=10):
@@ -742,7 +754,7 @@ def run_sweep(args, rank, world, local, peak, peak_kind):
     stream = torch.cuda.Stream()
     ceil_gbs = measure_read_ceiling(ntx, stream)
     with ClockSampler(local) as clk:
-        rows_out, single = gemv_sweep(ntx, stream, peak, peak_kind, ceil_gbs)
+        rows_out, single, further = gemv_sweep(ntx, stream, peak, peak_kind, ceil_gbs)
     tiled = [r for r in rows_out if r["layout"] == "tiled"]
     tot_b = sum(r["bytes_per_launch"] for r in tiled)
     tot_us = sum(r["us"] for r in tiled)
@@ -751,13 +763,14 @@ def run_sweep(args, rank, world, local, peak, peak_kind):
     line = {"metric": "quantized GEMV HBM GB/s", "value": v, "unit": "GB/s", "n_gpus": world, "steps": 5,
             "warmup": 1, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": DTYPE,
             "data": "synthetic (seeded random blocks, x ~ N(0,1))", "config": config, "clocks": clk.summary(),
-            "gpu_launches": 48 * 5 * (len(rows_out) + 2),
+            "gpu_launches": 48 * 5 * (len(rows_out) + 2 + len(further)),
             "roofline": {"bound": "hbm", "kernel": "qmma_kernel (tiled Q4_0 / Q4_K, all sweep shapes, one launch each)",
                          "achieved": v, "peak": peak, "peak_kind": peak_kind, "unit": "GB/s", "frac": v / peak,
                          "traffic": None, "frac_of_read_ceiling": v / ceil_gbs,
                          "largest_shape": {"shape": f"{top['format']}:{top['rows']}x{top['cols']}",
                                            "gbs": top["gbs"]}},
-            "read_ceiling": {"gbs": ceil_gbs}, "sweep": rows_out, "gemv_q8_0_4096x4096": single}
+            "read_ceiling": {"gbs": ceil_gbs}, "sweep": rows_out, "gemv_q8_0_4096x4096": single,
+            "further_formats": further}
     print_line(line)
 
 

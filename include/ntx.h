@@ -69,6 +69,14 @@ typedef enum ntx_qtype {
     NTX_Q4_0 = 1,
     NTX_Q4_K = 2,
     NTX_Q6_K = 3,
+    /* Q5_K 176 B / 256: fp16 d | fp16 dmin | 12 B of 6-bit scales and mins packed as in
+     * Q4_K | 32 B of fifth code bits | 128 B of low 4-bit codes    w = d sc_j q - dmin m_j
+     * (q in 0..31, j = element / 32; element 64c + l and 64c + 32 + l, l < 32, take the
+     * low and high nibble of low-code byte 32c + l and bits 2c and 2c + 1 of fifth-bit
+     * byte l).  F16 / F32: one little-endian IEEE value per weight. */
+    NTX_Q5_K = 4,
+    NTX_F16 = 5,
+    NTX_F32 = 6,
     /* Tiled layouts (flag NTX_TILED): the same information in the same bytes per
      * row, reordered for the streaming GEMV.  Produced from the GGUF-style
      * layout by ntx_repack_q, lossless.  Rows come in groups of 16 (a tiled
@@ -87,12 +95,17 @@ typedef enum ntx_qtype {
      *               bytes) | 256 B int8 sub-block scales | 8 x (d[r], d[r+8])
      *   NTX_Q4_K_T  unit 2304 B: 8 steps x 32 lanes x 8 B | 8 x 24 B of 6-bit scales
      *               and mins | 8 x (d[r], d[r+8], dmin[r], dmin[r+8])
-     * A row of a tiled tensor must hold whole units. */
+     *   NTX_Q5_K_T  unit 2816 B: 8 steps x (32 lanes x 8 B of low 4 bits as Q4_K | 8 gids x
+     *               8 B of fifth bits: word H0 row gid, H1 row gid + 8, the bit of column
+     *               4 tig + j at 8 j + 2 tig, of column 16 + 4 tig + j at 8 j + 2 tig + 1) |
+     *               scales, mins, d and dmin as NTX_Q4_K_T
+     * A row of a tiled tensor must hold whole units.  F16 and F32 have no tiled form. */
     NTX_TILED = 16,
     NTX_Q8_0_T = 16,
     NTX_Q4_0_T = 17,
     NTX_Q4_K_T = 18,
-    NTX_Q6_K_T = 19
+    NTX_Q6_K_T = 19,
+    NTX_Q5_K_T = 20
 } ntx_qtype;
 
 /* Message of the last failing ntx_* call on this thread ("" if none). */
@@ -175,9 +188,13 @@ ntx_status ntx_rope(float* q, float* k, int n_q_heads, int n_kv_heads, int head_
  *   k_cache, v_cache  device fp16 [n_kv_heads, max_ctx, head_dim]
  *   out     device fp32 [n_q_heads, head_dim]
  *   workspace / workspace_bytes: device scratch of at least
- *           ntx_attn_workspace_bytes(...) bytes, 16-byte aligned, for the partial
- *           results of the context splits; it needs no initialisation.
- * Two kernels run on `stream`: the split kernel, then the merge of the splits.
+ *           ntx_attn_workspace_bytes(...) bytes, 16-byte aligned: the first 256
+ *           bytes hold one merge ticket counter per kv head (cleared by the call with
+ *           cudaMemsetAsync on `stream`), the rest the partial results of the context
+ *           splits; it needs no initialisation by the caller.
+ * One kernel runs on `stream`: each CTA takes a context range of one kv head, and
+ * the last of them to finish merges that head's ranges (log-sum-exp rule, in range
+ * order, so the result does not depend on which CTA merges).
  * head_dim == 128, n_q_heads a multiple of n_kv_heads with at most 8 q heads per
  * kv head, 1 <= n_ctx <= max_ctx.  Calls sharing a workspace must not overlap. */
 ntx_status ntx_attn_decode(const float* q, const void* k_cache, const void* v_cache, float* out, int n_q_heads,
@@ -189,8 +206,9 @@ size_t ntx_attn_workspace_bytes(int n_q_heads, int n_kv_heads, int head_dim, int
  * memory: code that runs under a fixed, pre-planned memory budget or inside a
  * host framework whose allocator hands out no scratch, and so has no workspace
  * to pass.  (The pages have no counterpart; this is an addition of this library.)
- * The split partials live in a device array of 512 KiB that the
- * library holds on every GPU that loads it, until the process exits.  Shapes
+ * The merge tickets and split partials live in a device array of 512 KiB that the
+ * library holds on every GPU that loads it, until the process exits (the call clears
+ * the tickets with cudaMemsetAsync, which allocates nothing).  Shapes
  * whose workspace (ntx_attn_workspace_bytes) exceeds 512 KiB are rejected with
  * NTX_EUNSUPPORTED (on a 148-SM B200: 8 q heads per kv head with 8 kv heads, as
  * in Llama-70B, needs about 600 KB; 4 per kv head, as in Llama-8B, about 300 KB).  Nothing is allocated: the first call on a device looks up
@@ -242,7 +260,7 @@ typedef struct ntx_layer_desc {
 typedef struct ntx_model_desc {
     int32_t n_layers, hidden, n_q_heads, n_kv_heads, head_dim, ffn, vocab, max_ctx;
     float rms_eps, rope_theta;
-    int32_t qtype;                 /* format of every packed tensor */
+    int32_t qtype;                 /* format of every packed tensor (unless tensor_qtypes says otherwise) */
     const void* tok_embd;          /* packed [vocab, hidden], device */
     const float* out_norm;         /* device fp32 [hidden] */
     const void* output;            /* packed [vocab, hidden], device */
@@ -253,6 +271,13 @@ typedef struct ntx_model_desc {
      * ntx_stream_layers.  Norm weights and KV caches of every layer stay in HBM.
      * n_resident == n_layers: fully resident model. */
     int32_t n_resident;
+    /* Per-tensor formats, for models that mix formats (the "Q4_K_M" models of
+     * "Rendimiento y estructura de caché", e.g. most matrices Q4_K and some Q6_K):
+     * NULL (every tensor in qtype), or a host array of 2 + 4 n_layers formats, copied
+     * by ntx_model_create: tok_embd, output, then per layer w_qkv, w_o, w_gate and w_up
+     * (one format for both), w_down.  Any format of ntx_qtype; GGUF-style Q5_K rows have
+     * no streaming kernel, so a Q5_K matrix is given in its tiled form NTX_Q5_K_T. */
+    const int32_t* tensor_qtypes;
 } ntx_model_desc;
 
 typedef struct ntx_model ntx_model;

@@ -46,7 +46,7 @@ class Dims(ctypes.Structure):
 
 
 class Layer(ctypes.Structure):
-    _fields_ = [("qtype", ctypes.c_int32), ("attn_norm", ctypes.c_void_p), ("w_qkv", ctypes.c_void_p),
+    _fields_ = [("qtype", ctypes.c_int32 * 4), ("attn_norm", ctypes.c_void_p), ("w_qkv", ctypes.c_void_p),
                 ("w_o", ctypes.c_void_p), ("ffn_norm", ctypes.c_void_p), ("w_gate", ctypes.c_void_p),
                 ("w_up", ctypes.c_void_p), ("w_down", ctypes.c_void_p), ("k_cache", ctypes.c_void_p),
                 ("v_cache", ctypes.c_void_p)]
@@ -195,14 +195,17 @@ def lm_head(qtype: int, out_norm, W_out: np.ndarray, vocab: int, hidden: int, ep
     return logits
 
 
-def decode_layer(dims: Dims, qtype: int, h: np.ndarray, pos: int, attn_norm, w_qkv, w_o, ffn_norm, w_gate, w_up,
+def decode_layer(dims: Dims, qtype, h: np.ndarray, pos: int, attn_norm, w_qkv, w_o, ffn_norm, w_gate, w_up,
                  w_down, k_cache: np.ndarray, v_cache: np.ndarray) -> None:
-    """One layer in place on h (fp32) and on the fp16-bit caches (uint16)."""
+    """One layer in place on h (fp32) and on the fp16-bit caches (uint16).  qtype: the format
+    of every matrix, or four formats (QKV, O, gate and up, down)."""
     keep = [_f32(attn_norm), np.ascontiguousarray(w_qkv), np.ascontiguousarray(w_o), _f32(ffn_norm),
             np.ascontiguousarray(w_gate), np.ascontiguousarray(w_up), np.ascontiguousarray(w_down)]
     assert h.dtype == np.float32 and h.flags["C_CONTIGUOUS"]
     assert k_cache.dtype == np.uint16 and v_cache.dtype == np.uint16
-    L = Layer(qtype, *[_p(a) for a in keep], _p(k_cache), _p(v_cache))
+    qts = [int(qtype)] * 4 if np.isscalar(qtype) else [int(v) for v in qtype]
+    assert len(qts) == 4
+    L = Layer((ctypes.c_int32 * 4)(*qts), *[_p(a) for a in keep], _p(k_cache), _p(v_cache))
     if lib().orc_decode_layer(ctypes.byref(dims), ctypes.byref(L), _p(h), pos) != 0:
         raise ValueError("bad decode layer arguments")
 

@@ -16,10 +16,10 @@ from . import decode_layer, dims_of, embed, lm_head
 
 def layer_tensors(spec: ModelSpec, layer: int) -> dict:
     """Host copies of one layer's tensors, generated from the seed."""
-    q, s, hd = spec.qtype, spec.seed, spec.head_dim
+    s, hd = spec.seed, spec.head_dim
     t = {}
     for kind in ("w_qkv", "w_o", "w_gate", "w_up", "w_down"):
-        rows, cols, qp = spec.packed(kind)
+        rows, cols, qp, q = spec.packed(kind, layer)
         t[kind] = synth.blocks_host(q, s, tensor_id(layer, kind), rows, cols, qp)
     for kind in ("attn_norm", "ffn_norm"):
         t[kind] = synth.uniform_f32_host(s, tensor_id(layer, kind), spec.hidden, *synth.NORM_W)
@@ -30,16 +30,16 @@ def layer_tensors(spec: ModelSpec, layer: int) -> dict:
 
 
 def embedding_row(spec: ModelSpec, token: int) -> np.ndarray:
-    rows, cols, qp = spec.packed("tok_embd")
-    row = synth.blocks_host(spec.qtype, spec.seed, tensor_id(GLOBAL_LAYER, "tok_embd"), 1, cols, qp, row0=token)
-    return embed(spec.qtype, row, spec.hidden, 0)
+    rows, cols, qp, q = spec.packed("tok_embd")
+    row = synth.blocks_host(q, spec.seed, tensor_id(GLOBAL_LAYER, "tok_embd"), 1, cols, qp, row0=token)
+    return embed(q, row, spec.hidden, 0)
 
 
 def head_tensors(spec: ModelSpec, rows=None):
     """(out_norm, packed LM-head rows); rows = (row0, n) for a slice of the vocabulary."""
-    vocab, cols, qp = spec.packed("output")
+    vocab, cols, qp, q = spec.packed("output")
     row0, n = (0, vocab) if rows is None else rows
-    W = synth.blocks_host(spec.qtype, spec.seed, tensor_id(GLOBAL_LAYER, "output"), n, cols, qp, row0=row0)
+    W = synth.blocks_host(q, spec.seed, tensor_id(GLOBAL_LAYER, "output"), n, cols, qp, row0=row0)
     norm = synth.uniform_f32_host(spec.seed, tensor_id(GLOBAL_LAYER, "out_norm"), spec.hidden, *synth.NORM_W)
     return norm, W
 
@@ -60,7 +60,8 @@ def decode(spec: ModelSpec, pos: int | None = None, token: int | None = None, n_
     hidden = []
     for layer in range(n_layers):
         t = layer_tensors(spec, layer)
-        decode_layer(dims, spec.qtype, h, pos, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"], t["w_gate"],
+        qts = [spec.qtype_of(k, layer) for k in ("w_qkv", "w_o", "w_gate", "w_down")]
+        decode_layer(dims, qts, h, pos, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"], t["w_gate"],
                      t["w_up"], t["w_down"], t["k_cache"], t["v_cache"])
         if keep_hidden:
             hidden.append(h.copy())
@@ -68,5 +69,5 @@ def decode(spec: ModelSpec, pos: int | None = None, token: int | None = None, n_
             layer_hook(layer, t)
     norm, W = head_tensors(spec, head_rows)
     n_rows = W.shape[0]
-    logits = lm_head(spec.qtype, norm, W, n_rows, spec.hidden, spec.rms_eps, h)
+    logits = lm_head(spec.qtype_of("output"), norm, W, n_rows, spec.hidden, spec.rms_eps, h)
     return logits, hidden

@@ -369,8 +369,10 @@ ORC_EXPORT int orc_decode_layer(const orc_dims* D, const orc_layer* L, float* h,
 {
     int64_t H = D->hidden, hd = D->head_dim, qd = (int64_t)D->n_q_heads * hd, kvd = (int64_t)D->n_kv_heads * hd;
     int64_t F = D->ffn;
-    int qt = L->qtype;
-    if (!shape_ok(qt, H) || !shape_ok(qt, qd) || !shape_ok(qt, F) || pos < 0 || pos >= D->max_ctx) return -1;
+    const int qt_qkv = L->qtype[0], qt_o = L->qtype[1], qt_ffn = L->qtype[2], qt_down = L->qtype[3];
+    if (!shape_ok(qt_qkv, H) || !shape_ok(qt_o, qd) || !shape_ok(qt_ffn, H) || !shape_ok(qt_down, F) || pos < 0 ||
+        pos >= D->max_ctx)
+        return -1;
     float* xn = (float*)malloc((size_t)H * sizeof(float));
     float* qkv = (float*)malloc((size_t)(qd + 2 * kvd) * sizeof(float));
     float* att = (float*)malloc((size_t)qd * sizeof(float));
@@ -380,7 +382,7 @@ ORC_EXPORT int orc_decode_layer(const orc_dims* D, const orc_layer* L, float* h,
     float* a = (float*)malloc((size_t)F * sizeof(float));
 
     orc_rmsnorm(h, L->attn_norm, xn, H, D->rms_eps);
-    orc_gemv(qt, L->w_qkv, qd + 2 * kvd, H, xn, qkv);
+    orc_gemv(qt_qkv, L->w_qkv, qd + 2 * kvd, H, xn, qkv);
     float *q = qkv, *k = qkv + qd, *v = qkv + qd + kvd;
     orc_rope(q, k, D->n_q_heads, D->n_kv_heads, D->head_dim, pos, D->rope_theta);
     for (int gi = 0; gi < D->n_kv_heads; ++gi)
@@ -390,14 +392,14 @@ ORC_EXPORT int orc_decode_layer(const orc_dims* D, const orc_layer* L, float* h,
             L->v_cache[at] = orc_f32_to_f16(v[gi * hd + d]);
         }
     orc_attn_decode(q, L->k_cache, L->v_cache, att, D->n_q_heads, D->n_kv_heads, D->head_dim, pos + 1, D->max_ctx);
-    orc_gemv(qt, L->w_o, H, qd, att, o);
+    orc_gemv(qt_o, L->w_o, H, qd, att, o);
     for (int64_t i = 0; i < H; ++i) h[i] = h[i] + o[i];
 
     orc_rmsnorm(h, L->ffn_norm, xn, H, D->rms_eps);
-    orc_gemv(qt, L->w_gate, F, H, xn, g);
-    orc_gemv(qt, L->w_up, F, H, xn, u);
+    orc_gemv(qt_ffn, L->w_gate, F, H, xn, g);
+    orc_gemv(qt_ffn, L->w_up, F, H, xn, u);
     orc_swiglu(g, u, a, F);
-    orc_gemv(qt, L->w_down, H, F, a, o);
+    orc_gemv(qt_down, L->w_down, H, F, a, o);
     for (int64_t i = 0; i < H; ++i) h[i] = h[i] + o[i];
 
     free(xn); free(qkv); free(att); free(o); free(g); free(u); free(a);

@@ -58,7 +58,7 @@ typedef struct orc_dims {
 } orc_dims;
 
 typedef struct orc_layer {
-    int32_t qtype;
+    int32_t qtype[4];        /* formats of w_qkv, w_o, w_gate and w_up, w_down */
     const float* attn_norm;
     const uint8_t* w_qkv;    /* [(nq + 2 nkv) * hd, hidden]: q rows, then k rows, then v rows */
     const uint8_t* w_o;      /* [hidden, nq * hd] */

@@ -14,9 +14,9 @@ import os
 from .build import LIB
 
 NTX_OK, NTX_EINVAL, NTX_EUNSUPPORTED, NTX_ENOMEM, NTX_ECUDA, NTX_ETIMEOUT = range(6)
-NTX_Q8_0, NTX_Q4_0, NTX_Q4_K, NTX_Q6_K = range(4)
+NTX_Q8_0, NTX_Q4_0, NTX_Q4_K, NTX_Q6_K, NTX_Q5_K, NTX_F16, NTX_F32 = range(7)
 NTX_TILED = 16
-NTX_Q8_0_T, NTX_Q4_0_T, NTX_Q4_K_T, NTX_Q6_K_T = 16, 17, 18, 19
+NTX_Q8_0_T, NTX_Q4_0_T, NTX_Q4_K_T, NTX_Q6_K_T, NTX_Q5_K_T = 16, 17, 18, 19, 20
 NTX_GEMV_QKV, NTX_GEMV_O, NTX_GEMV_GATE_UP, NTX_GEMV_DOWN, NTX_GEMV_HEAD = range(5)
 STATUS_NAMES = {0: "NTX_OK", 1: "NTX_EINVAL", 2: "NTX_EUNSUPPORTED", 3: "NTX_ENOMEM", 4: "NTX_ECUDA",
                 5: "NTX_ETIMEOUT"}
@@ -47,7 +47,7 @@ class ModelDesc(ctypes.Structure):
                 ("vocab", ctypes.c_int32), ("max_ctx", ctypes.c_int32), ("rms_eps", ctypes.c_float),
                 ("rope_theta", ctypes.c_float), ("qtype", ctypes.c_int32), ("tok_embd", ctypes.c_void_p),
                 ("out_norm", ctypes.c_void_p), ("output", ctypes.c_void_p), ("layers", ctypes.POINTER(LayerDesc)),
-                ("n_resident", ctypes.c_int32)]
+                ("n_resident", ctypes.c_int32), ("tensor_qtypes", ctypes.POINTER(ctypes.c_int32))]
 
 
 _lib = None

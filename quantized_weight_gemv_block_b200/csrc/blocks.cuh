@@ -23,12 +23,29 @@ __device__ __forceinline__ void q4k_sm(const uint8_t* s, int j, int& sc, int& m)
     }
 }
 
-// Weight e (0 <= e < cols) of one packed row in a GGUF-style layout QT (0..3).
+// Weight e (0 <= e < cols) of one packed row in a GGUF-style layout QT (or F16 / F32).
 template <int QT>
 __device__ __forceinline__ float weight_in_row(const uint8_t* row, int64_t e)
 {
-    static_assert(QT >= NTX_Q8_0 && QT <= NTX_Q6_K, "GGUF-style layouts only");
-    if constexpr (QT == NTX_Q8_0) {
+    static_assert(QT >= NTX_Q8_0 && QT <= NTX_F32, "GGUF-style layouts only");
+    if constexpr (QT == NTX_F16) {
+        return ldh(row + 2 * e);
+    } else if constexpr (QT == NTX_F32) {
+        float v;
+        memcpy(&v, row + 4 * e, 4);
+        return v;
+    } else if constexpr (QT == NTX_Q5_K) {
+        // fp16 d | fp16 dmin | 12 B scales and mins | 32 B fifth bits | 128 B low nibbles
+        const uint8_t* b = row + (e >> 8) * 176;
+        const int r256 = (int)(e & 255);
+        const float d = ldh(b), dmin = ldh(b + 2);
+        const int c = r256 >> 6, r = r256 & 63, l = r & 31, up = r >> 5;
+        const int byte = b[48 + 32 * c + l];
+        const int q = (up ? (byte >> 4) : (byte & 15)) | (((b[16 + l] >> (2 * c + up)) & 1) << 4);
+        int sc, m;
+        q4k_sm(b + 4, r256 >> 5, sc, m);
+        return __fsub_rn(__fmul_rn(__fmul_rn(d, (float)sc), (float)q), __fmul_rn(dmin, (float)m));
+    } else if constexpr (QT == NTX_Q8_0) {
         const uint8_t* blk = row + (e >> 5) * 34;
         return ldh(blk) * (float)(int8_t)blk[2 + (e & 31)];
     } else if constexpr (QT == NTX_Q4_0) {
@@ -88,6 +105,13 @@ __device__ __forceinline__ float weight_in_row(const uint8_t* row, int64_t e)
 //                        even m) then 2 words of their top 2 bits (word m/4, byte b,
 //                        bits 2 (m mod 4)); [2240, 2304) 8 bytes per gid: d[gid],
 //                        d[gid+8], dmin[gid], dmin[gid+8] fp16.
+//  Q5_K (UK 256, 2816 B): 8 steps (one 32-column sub-block each), step m at 320 m:
+//                        [0, 256) lane L at 8 L: the low 4 bits of the codes as Q4_K's
+//                        words P, Q; [256, 320) 8 bytes per gid at 256 + 8 gid: words
+//                        H0 (row gid), H1 (row gid + 8) of fifth bits, the bit of column
+//                        4 t + j at bit 8 j + 2 t and that of column 16 + 4 t + j at bit
+//                        8 j + 2 t + 1 (t = tig); then [2560, 2752) scales and mins and
+//                        [2752, 2816) d, dmin exactly as Q4_K's [2048, 2304).
 template <int QT>
 struct Tiled;
 template <>
@@ -105,6 +129,10 @@ struct Tiled<NTX_Q4_K_T> {
 template <>
 struct Tiled<NTX_Q6_K_T> {
     static constexpr int UK = 256, UB = 3360;
+};
+template <>
+struct Tiled<NTX_Q5_K_T> {
+    static constexpr int UK = 256, UB = 2816;
 };
 
 // Weight (r, e) of a tiled matrix W whose rows hold rb bytes each.
@@ -134,6 +162,21 @@ __device__ __forceinline__ float weight_tiled(const uint8_t* W, int64_t r, int64
         const int sb = c >> 4;
         const int sc = (int8_t)U[3072 + 16 * (2 * gid + (sb & 1)) + 8 * hi + (sb >> 1)];
         return __fmul_rn(__fmul_rn(ldh(U + 3328 + 4 * gid + 2 * hi), (float)sc), (float)(q - 32));
+    } else if constexpr (QT == NTX_Q5_K_T) {
+        const int m = c >> 5;
+        const int lo = (U[320 * m + 8 * lane + 4 * hi + j] >> (4 * kh)) & 15;
+        const int b5 = (U[320 * m + 256 + 8 * gid + 4 * hi + j] >> (2 * tig + kh)) & 1;
+        const int q = lo | (b5 << 4);
+        const uint8_t* v = U + 2560 + 24 * gid;
+        auto val = [&](int b) {
+            const int lo4 = (v[4 * (m >> 1) + b] >> (4 * (m & 1))) & 15;
+            const int hi2 = (v[16 + 4 * (m >> 2) + b] >> (2 * (m & 3))) & 3;
+            return lo4 | (hi2 << 4);
+        };
+        const int sc = val(hi), mn = val(2 + hi);
+        const uint8_t* dd = U + 2752 + 8 * gid;
+        const float d = ldh(dd + 2 * hi), dmin = ldh(dd + 4 + 2 * hi);
+        return __fsub_rn(__fmul_rn(__fmul_rn(d, (float)sc), (float)q), __fmul_rn(dmin, (float)mn));
     } else {
         const int m = c >> 5;
         const int q = (U[256 * m + 8 * lane + 4 * hi + j] >> (4 * kh)) & 15;

@@ -78,16 +78,19 @@ inline int tile_elems(int qtype)
 {
     switch (base_qtype(qtype)) {
     case NTX_Q8_0: case NTX_Q4_0: return 32;
-    case NTX_Q4_K: case NTX_Q6_K: return 256;
+    case NTX_Q4_K: case NTX_Q6_K: case NTX_Q5_K: return 256;
     default: return 0;
     }
 }
+
+// F16 / F32: unquantized weights (no blocks, no tiled form).
+inline bool is_float_format(int qtype) { return qtype == NTX_F16 || qtype == NTX_F32; }
 
 inline QTraits qtraits(int qtype)
 {
     if (is_tiled(qtype)) {
         const int b = base_qtype(qtype);
-        if (b < NTX_Q8_0 || b > NTX_Q6_K) return {0, 0};
+        if (b < NTX_Q8_0 || b > NTX_Q5_K) return {0, 0};
         qtype = b;
     }
     switch (qtype) {
@@ -95,6 +98,9 @@ inline QTraits qtraits(int qtype)
     case NTX_Q4_0: return {32, 18};
     case NTX_Q4_K: return {256, 144};
     case NTX_Q6_K: return {256, 210};
+    case NTX_Q5_K: return {256, 176};
+    case NTX_F16: return {1, 2};
+    case NTX_F32: return {1, 4};
     default: return {0, 0};
     }
 }

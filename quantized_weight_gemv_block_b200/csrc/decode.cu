@@ -4,14 +4,13 @@
 // principales": host read, PCIe DMA and GPU compute overlapped with double
 // buffering; here pinned host memory -> a two-slot HBM ring on a copy stream).
 //
-// Per layer, six kernels:
+// Per layer, five kernels:
 //   1. fused QKV GEMV: RMSNorm(h) prologue, RoPE + fp16 K/V append epilogue
-//   2. split-context GQA attention, each split's partial (max, sum, accumulator)
-//      to a workspace
-//   3. merge of the splits (log-sum-exp rule, fixed order)
-//   4. O GEMV, residual add into h
-//   5. fused gate/up GEMV: RMSNorm(h) prologue, SwiGLU epilogue
-//   6. down GEMV, residual add into h
+//   2. split-context GQA attention; the last split of each kv head to finish merges
+//      the splits' partials (log-sum-exp rule, fixed order)
+//   3. O GEMV, residual add into h
+//   4. fused gate/up GEMV: RMSNorm(h) prologue, SwiGLU epilogue
+//   5. down GEMV, residual add into h
 // plus the step word / RoPE table kernel and the embedding before layer 0 and the
 // RMSNorm + LM-head GEMV after the last layer.  Kernels use programmatic dependent
 // launch so each one's weight stream starts while the previous one drains; the
@@ -25,11 +24,17 @@
 
 #include "ops.h"
 
+// Formats of one layer's matrices: QKV, O, gate and up, down.
+struct ntx_layer_qt {
+    int32_t qkv, o, ffn, down;
+};
+
 struct ntx_model {
     ntx_model_desc d;
     std::vector<ntx_layer_desc> layers;
+    std::vector<ntx_layer_qt> lqt;
+    int32_t qt_embd = 0, qt_out = 0;
     int device = 0;
-    int64_t rb_h = 0, rb_q = 0, rb_f = 0;
     float* h = nullptr;
     float* q = nullptr;
     float* att = nullptr;
@@ -71,9 +76,10 @@ ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool p
     const ntx_model_desc& d = m->d;
     const ntx_layer_desc& L = m->layers[l];
     const int qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim;
+    const int qt = m->lqt[l].qkv;
     Params P{};
     P.W = (const uint8_t*)w;
-    P.row_bytes = m->rb_h;
+    P.row_bytes = row_bytes(qt, d.hidden);
     P.M = qd + 2 * kvd;
     P.K = d.hidden;
     P.x = m->h;
@@ -89,30 +95,32 @@ ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool p
     P.v_cache = (__half*)L.v_cache;
     P.q_out = m->q;
     P.use_pdl = pdl;
-    return gemv_launch(d.qtype, gemv::EPI_QKV, gemv::PRO_RMSNORM, P, s);
+    return gemv_launch(qt, gemv::EPI_QKV, gemv::PRO_RMSNORM, P, s);
 }
 
-ntx_status launch_o(ntx_model* m, const void* w, cudaStream_t s, bool pdl)
+ntx_status launch_o(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl)
 {
     const ntx_model_desc& d = m->d;
+    const int qt = m->lqt[l].o;
     Params P{};
     P.W = (const uint8_t*)w;
-    P.row_bytes = m->rb_q;
-    P.M = d.hidden;
     P.K = d.n_q_heads * d.head_dim;
+    P.row_bytes = row_bytes(qt, P.K);
+    P.M = d.hidden;
     P.x = m->att;
     P.y = m->h;
     P.use_pdl = pdl;
-    return gemv_launch(d.qtype, gemv::EPI_ADD, gemv::PRO_X, P, s);
+    return gemv_launch(qt, gemv::EPI_ADD, gemv::PRO_X, P, s);
 }
 
 ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, cudaStream_t s, bool pdl)
 {
     const ntx_model_desc& d = m->d;
+    const int qt = m->lqt[l].ffn;
     Params P{};
     P.W = (const uint8_t*)wg;
     P.W2 = (const uint8_t*)wu;
-    P.row_bytes = m->rb_h;
+    P.row_bytes = row_bytes(qt, d.hidden);
     P.M = d.ffn;
     P.K = d.hidden;
     P.x = m->h;
@@ -120,21 +128,22 @@ ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, c
     P.eps = d.rms_eps;
     P.y = m->act;
     P.use_pdl = pdl;
-    return gemv_launch(d.qtype, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, P, s);
+    return gemv_launch(qt, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, P, s);
 }
 
-ntx_status launch_down(ntx_model* m, const void* w, cudaStream_t s, bool pdl)
+ntx_status launch_down(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl)
 {
     const ntx_model_desc& d = m->d;
+    const int qt = m->lqt[l].down;
     Params P{};
     P.W = (const uint8_t*)w;
-    P.row_bytes = m->rb_f;
+    P.row_bytes = row_bytes(qt, d.ffn);
     P.M = d.hidden;
     P.K = d.ffn;
     P.x = m->act;
     P.y = m->h;
     P.use_pdl = pdl;
-    return gemv_launch(d.qtype, gemv::EPI_ADD, gemv::PRO_X, P, s);
+    return gemv_launch(qt, gemv::EPI_ADD, gemv::PRO_X, P, s);
 }
 
 ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl)
@@ -159,9 +168,9 @@ ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, b
         a.pdl = pdl;
         if ((st = attn_launch(a, s)) != NTX_OK) return st;
     }
-    if ((st = launch_o(m, w.o, s, pdl)) != NTX_OK) return st;
+    if ((st = launch_o(m, l, w.o, s, pdl)) != NTX_OK) return st;
     if ((st = launch_gate_up(m, l, w.gate, w.up, s, pdl)) != NTX_OK) return st;
-    return launch_down(m, w.down, s, pdl);
+    return launch_down(m, l, w.down, s, pdl);
 }
 
 ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
@@ -169,7 +178,7 @@ ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
     const ntx_model_desc& d = m->d;
     Params P{};
     P.W = (const uint8_t*)d.output;
-    P.row_bytes = m->rb_h;
+    P.row_bytes = row_bytes(m->qt_out, d.hidden);
     P.M = d.vocab;
     P.K = d.hidden;
     P.x = m->h;
@@ -177,7 +186,7 @@ ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
     P.eps = d.rms_eps;
     P.y = logits;
     P.use_pdl = pdl;
-    return gemv_launch(d.qtype, gemv::EPI_STORE, gemv::PRO_RMSNORM, P, s);
+    return gemv_launch(m->qt_out, gemv::EPI_STORE, gemv::PRO_RMSNORM, P, s);
 }
 
 LayerW resident_w(const ntx_layer_desc& L) { return {L.w_qkv, L.w_o, L.w_gate, L.w_up, L.w_down}; }
@@ -185,7 +194,7 @@ LayerW resident_w(const ntx_layer_desc& L) { return {L.w_qkv, L.w_o, L.w_gate, L
 // Embedding + resident layers [0, n) (+ head if with_head), token/pos from m->step.
 ntx_status enqueue_resident(ntx_model* m, int n, float* logits, cudaStream_t s, bool with_head)
 {
-    ntx_status st = embed_launch(m->d.qtype, m->d.tok_embd, m->d.hidden, m->step, m->h, s, m->pdl);
+    ntx_status st = embed_launch(m->qt_embd, m->d.tok_embd, m->d.hidden, m->step, m->h, s, m->pdl);
     if (st != NTX_OK) return st;
     for (int l = 0; l < n; ++l)
         if ((st = enqueue_layer(m, l, resident_w(m->layers[l]), s, m->pdl)) != NTX_OK) return st;
@@ -197,6 +206,20 @@ bool env_flag(const char* name)
 {
     const char* v = std::getenv(name);
     return v && v[0] && v[0] != '0';
+}
+
+// Format of tensor i of the descriptor: 0 tok_embd, 1 output, then 4 per layer.
+int32_t tensor_qtype(const ntx_model_desc* d, int i) { return d->tensor_qtypes ? d->tensor_qtypes[i] : d->qtype; }
+
+// A packed matrix of `cols` columns in format qt that a decode-step GEMV can stream.
+ntx_status check_matrix_format(int32_t qt, int64_t cols, const char* what)
+{
+    const std::string w(what);
+    if (qtraits(qt).block_elems == 0) return fail(NTX_EINVAL, "model: unknown format for " + w);
+    if (qt == NTX_Q5_K) return fail(NTX_EUNSUPPORTED, "model: " + w + ": Q5_K matrices need the tiled layout NTX_Q5_K_T");
+    if (row_bytes(qt, cols) == 0) return fail(NTX_EINVAL, "model: " + w + ": row length not a multiple of the block size");
+    if (row_bytes(qt, cols) % 16) return fail(NTX_EUNSUPPORTED, "model: " + w + ": packed rows must be multiples of 16 bytes");
+    return NTX_OK;
 }
 
 ntx_status check_desc(const ntx_model_desc* d)
@@ -215,10 +238,20 @@ ntx_status check_desc(const ntx_model_desc* d)
     if (d->n_resident < 0 || d->n_resident > d->n_layers) return fail(NTX_EINVAL, "model: n_resident out of range");
     if (!d->tok_embd || !d->out_norm || !d->output || !d->layers) return fail(NTX_EINVAL, "model: null pointer");
     const int qd = d->n_q_heads * d->head_dim;
-    for (int64_t k : {(int64_t)d->hidden, (int64_t)qd, (int64_t)d->ffn}) {
-        if (row_bytes(d->qtype, k) == 0) return fail(NTX_EINVAL, "model: a row length is not a multiple of the block size");
-        if (row_bytes(d->qtype, k) % 16) return fail(NTX_EUNSUPPORTED, "model: packed rows must be multiples of 16 bytes");
+    for (int64_t k : {(int64_t)d->hidden, (int64_t)qd, (int64_t)d->ffn})
         if (k > 32768) return fail(NTX_EUNSUPPORTED, "model: row length above 32768");
+    ntx_status st;
+    // the embedding is read one row at a time (any layout); every other matrix is streamed
+    if (qtraits(tensor_qtype(d, 0)).block_elems == 0 || row_bytes(tensor_qtype(d, 0), d->hidden) == 0)
+        return fail(NTX_EINVAL, "model: bad format for tok_embd");
+    if ((st = check_matrix_format(tensor_qtype(d, 1), d->hidden, "output")) != NTX_OK) return st;
+    for (int l = 0; l < d->n_layers; ++l) {
+        const int b = 2 + 4 * l;
+        if ((st = check_matrix_format(tensor_qtype(d, b), d->hidden, "w_qkv")) != NTX_OK ||
+            (st = check_matrix_format(tensor_qtype(d, b + 1), qd, "w_o")) != NTX_OK ||
+            (st = check_matrix_format(tensor_qtype(d, b + 2), d->hidden, "w_gate / w_up")) != NTX_OK ||
+            (st = check_matrix_format(tensor_qtype(d, b + 3), d->ffn, "w_down")) != NTX_OK)
+            return st;
     }
     if (!aligned(d->tok_embd, 16) || !aligned(d->output, 16) || !aligned(d->out_norm, 16))
         return fail(NTX_EINVAL, "model: tensors must be 16-byte aligned");
@@ -273,12 +306,17 @@ NTX_EXPORT ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** m
     m->d = *desc;
     m->layers.assign(desc->layers, desc->layers + desc->n_layers);
     m->d.layers = nullptr;
+    m->d.tensor_qtypes = nullptr;
+    m->qt_embd = tensor_qtype(desc, 0);
+    m->qt_out = tensor_qtype(desc, 1);
+    for (int l = 0; l < desc->n_layers; ++l) {
+        const int b = 2 + 4 * l;
+        m->lqt.push_back({tensor_qtype(desc, b), tensor_qtype(desc, b + 1), tensor_qtype(desc, b + 2),
+                          tensor_qtype(desc, b + 3)});
+    }
     cudaGetDevice(&m->device);
     const ntx_model_desc& d = m->d;
     const int qd = d.n_q_heads * d.head_dim;
-    m->rb_h = row_bytes(d.qtype, d.hidden);
-    m->rb_q = row_bytes(d.qtype, qd);
-    m->rb_f = row_bytes(d.qtype, d.ffn);
     m->pdl = !env_flag("NTX_NO_PDL");
     m->use_graph = !env_flag("NTX_NO_GRAPH");
     m->n_split = attn_split_for(d.n_q_heads, d.n_kv_heads, d.max_ctx);
@@ -298,10 +336,14 @@ NTX_EXPORT ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** m
     if (e == cudaSuccess) e = cudaMemset(m->step, 0, 16);
     if (e == cudaSuccess && d.n_resident < d.n_layers) {
         const int kvd = d.n_kv_heads * d.head_dim;
-        m->sz_qkv = (size_t)(qd + 2 * kvd) * m->rb_h;
-        m->sz_o = (size_t)d.hidden * m->rb_q;
-        m->sz_ffn = (size_t)d.ffn * m->rb_h;
-        m->sz_down = (size_t)d.hidden * m->rb_f;
+        // ring slots sized for the largest of each matrix over the streamed layers
+        for (int l = d.n_resident; l < d.n_layers; ++l) {
+            const ntx_layer_qt& q = m->lqt[l];
+            m->sz_qkv = std::max(m->sz_qkv, (size_t)(qd + 2 * kvd) * row_bytes(q.qkv, d.hidden));
+            m->sz_o = std::max(m->sz_o, (size_t)d.hidden * row_bytes(q.o, qd));
+            m->sz_ffn = std::max(m->sz_ffn, (size_t)d.ffn * row_bytes(q.ffn, d.hidden));
+            m->sz_down = std::max(m->sz_down, (size_t)d.hidden * row_bytes(q.down, d.ffn));
+        }
         m->off_qkv = 0;
         m->off_o = align256(m->sz_qkv);
         m->off_gate = m->off_o + align256(m->sz_o);
@@ -342,7 +384,8 @@ NTX_EXPORT ntx_status ntx_decode_step(ntx_model* m, int32_t token, int32_t pos, 
     if (pos < 0 || pos >= m->d.max_ctx) return fail(NTX_EINVAL, "ntx_decode_step: pos out of range");
     if (!aligned(logits, 4)) return fail(NTX_EINVAL, "ntx_decode_step: logits must be 4-byte aligned");
     cudaStream_t s = (cudaStream_t)stream;
-    ntx_status st = set_step_launch(m->step, token, pos, m->rope, m->d.rope_theta, m->d.head_dim, s);
+    ntx_status st = set_step_launch(m->step, token, pos, m->rope, m->d.rope_theta, m->d.head_dim,
+                                    (unsigned*)m->attn_ws, m->d.n_kv_heads, s);
     if (st != NTX_OK) return st;
     if (!m->use_graph) return enqueue_resident(m, m->d.n_layers, logits, s, true);
     if (!m->graph || m->graph_logits != logits) {
@@ -391,7 +434,8 @@ NTX_EXPORT ntx_status ntx_stream_layers(ntx_model* m, int32_t token, int32_t pos
     const ntx_model_desc& d = m->d;
     const int nres = d.n_resident;
     NTX_CUDA_TRY(cudaEventRecord(m->ev_start, cs));
-    ntx_status st = set_step_launch(m->step, token, pos, m->rope, d.rope_theta, d.head_dim, cs);
+    ntx_status st = set_step_launch(m->step, token, pos, m->rope, d.rope_theta, d.head_dim, (unsigned*)m->attn_ws,
+                                    d.n_kv_heads, cs);
     if (st != NTX_OK) return st;
     int64_t h2d = 0;
     // copies of streamed layer j into slot (j - nres) % 2; the slot is free once
@@ -401,13 +445,20 @@ NTX_EXPORT ntx_status ntx_stream_layers(ntx_model* m, int32_t token, int32_t pos
         const ntx_layer_desc& L = m->layers[j];
         uint8_t* base = m->ring + (size_t)slot * m->slot_bytes;
         NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->slot_free[slot], 0));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_qkv, L.w_qkv, m->sz_qkv, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_o, L.w_o, m->sz_o, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_gate, L.w_gate, m->sz_ffn, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_up, L.w_up, m->sz_ffn, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_down, L.w_down, m->sz_down, cudaMemcpyHostToDevice, ks));
+        // this layer's own matrix sizes (its formats may differ from the largest the slot holds)
+        const ntx_layer_qt& q = m->lqt[j];
+        const int kvd = d.n_kv_heads * d.head_dim, qd = d.n_q_heads * d.head_dim;
+        const size_t b_qkv = (size_t)(qd + 2 * kvd) * row_bytes(q.qkv, d.hidden);
+        const size_t b_o = (size_t)d.hidden * row_bytes(q.o, qd);
+        const size_t b_ffn = (size_t)d.ffn * row_bytes(q.ffn, d.hidden);
+        const size_t b_down = (size_t)d.hidden * row_bytes(q.down, d.ffn);
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_qkv, L.w_qkv, b_qkv, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_o, L.w_o, b_o, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_gate, L.w_gate, b_ffn, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_up, L.w_up, b_ffn, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_down, L.w_down, b_down, cudaMemcpyHostToDevice, ks));
         NTX_CUDA_TRY(cudaEventRecord(m->copy_done[slot], ks));
-        h2d += (int64_t)(m->sz_qkv + m->sz_o + 2 * m->sz_ffn + m->sz_down);
+        h2d += (int64_t)(b_qkv + b_o + 2 * b_ffn + b_down);
         return NTX_OK;
     };
     if (nres < d.n_layers) {
@@ -471,9 +522,9 @@ NTX_EXPORT ntx_status ntx_model_replay_gemv(ntx_model* m, int kind, int n_launch
         const ntx_layer_desc& L = m->layers[l];
         switch (kind) {
         case NTX_GEMV_QKV: st = launch_qkv(m, l, L.w_qkv, s, m->pdl); break;
-        case NTX_GEMV_O: st = launch_o(m, L.w_o, s, m->pdl); break;
+        case NTX_GEMV_O: st = launch_o(m, l, L.w_o, s, m->pdl); break;
         case NTX_GEMV_GATE_UP: st = launch_gate_up(m, l, L.w_gate, L.w_up, s, m->pdl); break;
-        case NTX_GEMV_DOWN: st = launch_down(m, L.w_down, s, m->pdl); break;
+        case NTX_GEMV_DOWN: st = launch_down(m, l, L.w_down, s, m->pdl); break;
         default: st = enqueue_head(m, logits, s, m->pdl); break;
         }
     }

@@ -93,6 +93,9 @@ ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaS
     if (epi == EPI_QKV && (!P.rope_cs || P.head_dim > 128))
         return fail(NTX_EINVAL, "gemv: the fused QKV epilogue needs the step's RoPE table (head_dim <= 128)");
     if (is_tiled(qtype)) return qmma_launch(qtype, epi, pro, P, s);
+    if (is_float_format(qtype)) return fgemv_launch(qtype, epi, pro, P, s);
+    if (qtype == NTX_Q5_K)
+        return fail(NTX_EUNSUPPORTED, "gemv: Q5_K streams in its tiled layout only (ntx_repack_q to NTX_Q5_K_T)");
     const int cap = num_sms();
     if (epi == EPI_STORE && pro == PRO_X) return launch_q<EPI_STORE, PRO_X>(qtype, P, s, cap);
     if (epi == EPI_ADD && pro == PRO_X) return launch_q<EPI_ADD, PRO_X>(qtype, P, s, cap);
@@ -106,7 +109,9 @@ cudaError_t take_device_error_gemv(uint32_t* out) { return take_tu_device_error(
 
 bool gemv_fast_path_ok(int qtype, const void* W, int64_t cols)
 {
-    // the tiled layouts need only a 16-byte aligned base (their 16-row groups are 16-byte multiples)
+    // the tiled layouts need only a 16-byte aligned base (their 16-row groups are 16-byte multiples);
+    // GGUF-style Q5_K has no streaming kernel (its tiled form has), F16 / F32 have their own
+    if (qtype == NTX_Q5_K || is_float_format(qtype)) return false;
     return aligned(W, 16) && (is_tiled(qtype) || row_bytes(qtype, cols) % 16 == 0);
 }
 
@@ -127,7 +132,7 @@ NTX_EXPORT ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t
     if (!aligned(W, 2)) return fail(NTX_EINVAL, "ntx_gemv_q: W must be at least 2-byte aligned");
     cudaStream_t s = (cudaStream_t)stream;
     const int64_t rb = row_bytes(qtype, cols);
-    if (gemv_fast_path_ok(qtype, W, cols) && cols <= 32768 && aligned(x, 16)) {
+    if ((gemv_fast_path_ok(qtype, W, cols) && cols <= 32768 && aligned(x, 16)) || fgemv_shape_ok(qtype, W, x, cols)) {
         gemv::Params P{};
         P.W = (const uint8_t*)W;
         P.row_bytes = rb;
@@ -148,10 +153,14 @@ NTX_EXPORT ntx_status ntx_gemv_q(int qtype, const void* W, int64_t rows, int64_t
     case NTX_Q4_0: NTX_SIMPLE(NTX_Q4_0); break;
     case NTX_Q4_K: NTX_SIMPLE(NTX_Q4_K); break;
     case NTX_Q6_K: NTX_SIMPLE(NTX_Q6_K); break;
+    case NTX_Q5_K: NTX_SIMPLE(NTX_Q5_K); break;
+    case NTX_F16: NTX_SIMPLE(NTX_F16); break;
+    case NTX_F32: NTX_SIMPLE(NTX_F32); break;
     case NTX_Q8_0_T: NTX_SIMPLE(NTX_Q8_0_T); break;
     case NTX_Q4_0_T: NTX_SIMPLE(NTX_Q4_0_T); break;
     case NTX_Q4_K_T: NTX_SIMPLE(NTX_Q4_K_T); break;
     case NTX_Q6_K_T: NTX_SIMPLE(NTX_Q6_K_T); break;
+    case NTX_Q5_K_T: NTX_SIMPLE(NTX_Q5_K_T); break;
     }
 #undef NTX_SIMPLE
     return check_launch("ntx_gemv_q (simple kernel)");
@@ -175,10 +184,14 @@ NTX_EXPORT ntx_status ntx_dequant_q(int qtype, const void* W, int64_t rows, int6
     case NTX_Q4_0: NTX_DQ(NTX_Q4_0); break;
     case NTX_Q4_K: NTX_DQ(NTX_Q4_K); break;
     case NTX_Q6_K: NTX_DQ(NTX_Q6_K); break;
+    case NTX_Q5_K: NTX_DQ(NTX_Q5_K); break;
+    case NTX_F16: NTX_DQ(NTX_F16); break;
+    case NTX_F32: NTX_DQ(NTX_F32); break;
     case NTX_Q8_0_T: NTX_DQ(NTX_Q8_0_T); break;
     case NTX_Q4_0_T: NTX_DQ(NTX_Q4_0_T); break;
     case NTX_Q4_K_T: NTX_DQ(NTX_Q4_K_T); break;
     case NTX_Q6_K_T: NTX_DQ(NTX_Q6_K_T); break;
+    case NTX_Q5_K_T: NTX_DQ(NTX_Q5_K_T); break;
     }
 #undef NTX_DQ
     return check_launch("ntx_dequant_q");

@@ -140,14 +140,18 @@ __global__ void embed_kernel(const uint8_t* E, int64_t rb, int64_t hidden, const
 // The step word (token, position) and the RoPE table of the position: rope[2i] and
 // rope[2i + 1] = cos and sin of pos theta^(-2i/head_dim), computed in double, for
 // i < head_dim / 2 (the rotation of "RoPE" in the ntransformer news summary's kernel
-// list).  Later kernels of the step read both.
-__global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim)
+// list).  Later kernels of the step read both.  Also zeroes the attention's merge
+// tickets (each attention launch leaves them at zero; this covers a step that did not
+// finish).
+__global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
+                                unsigned* counters, int n_counters)
 {
     const int i = threadIdx.x;
     if (i == 0) {
         step[0] = token;
         step[1] = pos;
     }
+    for (int c = i; c < n_counters; c += blockDim.x) counters[c] = 0u;
     if (rope && i < head_dim / 2) {
         const double ang = (double)pos * pow((double)theta, -(2.0 * i) / (double)head_dim);
         double sn, cs;
@@ -182,19 +186,24 @@ ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t*
     case NTX_Q4_0: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q4_0>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q4_K: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q4_K>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q6_K: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q6_K>, e, rb, hidden, token_dev, h, p); break;
+    case NTX_Q5_K: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q5_K>, e, rb, hidden, token_dev, h, p); break;
+    case NTX_F16: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_F16>, e, rb, hidden, token_dev, h, p); break;
+    case NTX_F32: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_F32>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q8_0_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q8_0_T>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q4_0_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q4_0_T>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q4_K_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q4_K_T>, e, rb, hidden, token_dev, h, p); break;
     case NTX_Q6_K_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q6_K_T>, e, rb, hidden, token_dev, h, p); break;
+    case NTX_Q5_K_T: err = cudaLaunchKernelEx(&cfg, embed_kernel<NTX_Q5_K_T>, e, rb, hidden, token_dev, h, p); break;
     }
     if (err != cudaSuccess) return fail(NTX_ECUDA, std::string("embedding launch: ") + cudaGetErrorString(err));
     return NTX_OK;
 }
 
 ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
-                           cudaStream_t s)
+                           unsigned* counters, int n_counters, cudaStream_t s)
 {
-    set_step_kernel<<<1, std::max(32, head_dim / 2), 0, s>>>(step, token, pos, rope, theta, head_dim);
+    set_step_kernel<<<1, std::max(32, head_dim / 2), 0, s>>>(step, token, pos, rope, theta, head_dim, counters,
+                                                               counters ? n_counters : 0);
     return check_launch("step counter");
 }
 

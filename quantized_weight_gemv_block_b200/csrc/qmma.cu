@@ -37,13 +37,47 @@ __device__ __forceinline__ int src_q4_k(const uint8_t* row, int64_t e)
     return r < 32 ? (byte & 15) : (byte >> 4);
 }
 
-// Q4_K 6-bit value V(m, b) of the tiled layout for rows (gid, gid + 8) of group W16.
-__device__ __forceinline__ int src_q4_k_v(const uint8_t* W16, int64_t rb, int64_t sb, int gid, int m, int b)
+// Q5_K: the low 4 bits and the fifth bit of element e of a GGUF-style row.
+__device__ __forceinline__ int src_q5_k_lo(const uint8_t* row, int64_t e)
 {
-    const uint8_t* blk = W16 + (int64_t)(gid + 8 * (b & 1)) * rb + sb * 144;
+    const uint8_t* b = row + (e >> 8) * 176;
+    const int r256 = (int)(e & 255), c = r256 >> 6, r = r256 & 63;
+    const int byte = b[48 + 32 * c + (r & 31)];
+    return r < 32 ? (byte & 15) : (byte >> 4);
+}
+
+__device__ __forceinline__ int src_q5_k_b5(const uint8_t* row, int64_t e)
+{
+    const uint8_t* b = row + (e >> 8) * 176;
+    const int r256 = (int)(e & 255), c = r256 >> 6, r = r256 & 63;
+    return (b[16 + (r & 31)] >> (2 * c + (r >> 5))) & 1;
+}
+
+// Q4_K / Q5_K 6-bit value V(m, b) of the tiled layout for rows (gid, gid + 8) of group W16
+// (BB: bytes of one GGUF-style superblock; the scales sit at byte 4 of it in both).
+template <int BB>
+__device__ __forceinline__ int src_k_v(const uint8_t* W16, int64_t rb, int64_t sb, int gid, int m, int b)
+{
+    const uint8_t* blk = W16 + (int64_t)(gid + 8 * (b & 1)) * rb + sb * BB;
     int sc, mn;
     gemv::q4k_sm(blk + 4, m, sc, mn);
     return (b & 2) ? mn : sc;
+}
+
+// Byte p (< 192) of the scale section of a Q4_K / Q5_K tiled unit.
+template <int BB>
+__device__ __forceinline__ uint8_t k_scale_byte(const uint8_t* W16, int64_t rb, int64_t u, int p)
+{
+    const int gid = p / 24, r = p % 24;
+    if (r < 16) {
+        const int wn = r >> 2, b = r & 3;
+        return (uint8_t)((src_k_v<BB>(W16, rb, u, gid, 2 * wn, b) & 15) |
+                         ((src_k_v<BB>(W16, rb, u, gid, 2 * wn + 1, b) & 15) << 4));
+    }
+    const int wh = (r - 16) >> 2, b = r & 3;
+    int v = 0;
+    for (int t = 0; t < 4; ++t) v |= ((src_k_v<BB>(W16, rb, u, gid, 4 * wh + t, b) >> 4) & 3) << (2 * t);
+    return (uint8_t)v;
 }
 
 // Byte `o` of unit u of the 16-row group that starts at GGUF row pointer W16.
@@ -93,23 +127,40 @@ __device__ __forceinline__ uint8_t tiled_byte(const uint8_t* W16, int64_t rb, in
             const int64_t e = 256 * u + 32 * m + 4 * (lane & 3) + j;
             return (uint8_t)(src_q4_k(row, e) | (src_q4_k(row, e + 16) << 4));
         }
-        if (o < 2240) {
-            const int p = o - 2048, gid = p / 24, r = p % 24;
-            if (r < 16) {
-                const int wn = r >> 2, b = r & 3;
-                return (uint8_t)((src_q4_k_v(W16, rb, u, gid, 2 * wn, b) & 15) |
-                                 ((src_q4_k_v(W16, rb, u, gid, 2 * wn + 1, b) & 15) << 4));
-            }
-            const int wh = (r - 16) >> 2, b = r & 3;
-            int v = 0;
-            for (int t = 0; t < 4; ++t) v |= ((src_q4_k_v(W16, rb, u, gid, 4 * wh + t, b) >> 4) & 3) << (2 * t);
-            return (uint8_t)v;
-        }
+        if (o < 2240) return k_scale_byte<144>(W16, rb, u, o - 2048);
         const int p = o - 2240, gid = p >> 3, k = (p >> 1) & 3;
         // k: 0 d(gid), 1 d(gid+8), 2 dmin(gid), 3 dmin(gid+8)
         const int row = gid + 8 * (k & 1);
         return W16[(int64_t)row * rb + u * 144 + 2 * (k >> 1) + (p & 1)];
     }
+}
+
+// Byte `o` of Q5_K unit u of the 16-row group that starts at GGUF row pointer W16.
+__device__ __forceinline__ uint8_t tiled_byte_q5_k(const uint8_t* W16, int64_t rb, int64_t u, int o)
+{
+    if (o < 2560) {
+        const int m = o / 320, r = o % 320;
+        const int64_t e0 = 256 * u + 32 * m;
+        if (r < 256) {
+            // low 4 bits as Q4_K: lane, word P / Q, byte j
+            const int lane = r >> 3, hi = (r >> 2) & 1, j = r & 3;
+            const uint8_t* row = W16 + (int64_t)((lane >> 2) + 8 * hi) * rb;
+            const int64_t e = e0 + 4 * (lane & 3) + j;
+            return (uint8_t)(src_q5_k_lo(row, e) | (src_q5_k_lo(row, e + 16) << 4));
+        }
+        // fifth bits: gid, word H0 / H1 (row gid / gid + 8), byte j holds bit 2t (column
+        // 4t + j) and bit 2t + 1 (column 16 + 4t + j) for t = 0..3
+        const int p = r - 256, gid = p >> 3, hi = (p >> 2) & 1, j = p & 3;
+        const uint8_t* row = W16 + (int64_t)(gid + 8 * hi) * rb;
+        int v = 0;
+        for (int t = 0; t < 4; ++t)
+            v |= (src_q5_k_b5(row, e0 + 4 * t + j) << (2 * t)) | (src_q5_k_b5(row, e0 + 16 + 4 * t + j) << (2 * t + 1));
+        return (uint8_t)v;
+    }
+    if (o < 2752) return k_scale_byte<176>(W16, rb, u, o - 2560);
+    const int p = o - 2752, gid = p >> 3, k = (p >> 1) & 3;
+    const int row = gid + 8 * (k & 1);
+    return W16[(int64_t)row * rb + u * 176 + 2 * (k >> 1) + (p & 1)];
 }
 
 template <int QT>
@@ -120,7 +171,10 @@ __global__ void repack_kernel(const uint8_t* in, uint8_t* out, int64_t n_bytes, 
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n_bytes; i += (int64_t)gridDim.x * blockDim.x) {
         const int64_t grp = i / gb, o = i - grp * gb;
         const int64_t u = o / T::UB;
-        out[i] = tiled_byte<QT>(in + grp * gb, rb, u, (int)(o - u * T::UB));
+        if constexpr (QT == NTX_Q5_K_T)
+            out[i] = tiled_byte_q5_k(in + grp * gb, rb, u, (int)(o - u * T::UB));
+        else
+            out[i] = tiled_byte<QT>(in + grp * gb, rb, u, (int)(o - u * T::UB));
     }
 }
 
@@ -267,6 +321,7 @@ ntx_status launch_q(int qtype, const Params& P, cudaStream_t s)
     case NTX_Q4_0_T: return launch_c<NTX_Q4_0_T, EPI, PRO>(P, s);
     case NTX_Q4_K_T: return launch_c<NTX_Q4_K_T, EPI, PRO>(P, s);
     case NTX_Q6_K_T: return launch_c<NTX_Q6_K_T, EPI, PRO>(P, s);
+    case NTX_Q5_K_T: return launch_c<NTX_Q5_K_T, EPI, PRO>(P, s);
     default: return fail(NTX_EINVAL, "unknown tiled qtype");
     }
 }
@@ -298,6 +353,7 @@ ntx_status repack_launch(int qtype, const void* W, void* W_tiled, int64_t rows, 
     case NTX_Q4_0: qmma::repack_kernel<NTX_Q4_0_T><<<grid, threads, 0, s>>>(in, out, n, rb); break;
     case NTX_Q4_K: qmma::repack_kernel<NTX_Q4_K_T><<<grid, threads, 0, s>>>(in, out, n, rb); break;
     case NTX_Q6_K: qmma::repack_kernel<NTX_Q6_K_T><<<grid, threads, 0, s>>>(in, out, n, rb); break;
+    case NTX_Q5_K: qmma::repack_kernel<NTX_Q5_K_T><<<grid, threads, 0, s>>>(in, out, n, rb); break;
     default: return fail(NTX_EINVAL, "ntx_repack_q: qtype must be a GGUF-style format");
     }
     return check_launch("ntx_repack_q");

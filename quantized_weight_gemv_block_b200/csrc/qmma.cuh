@@ -173,8 +173,10 @@ __device__ __forceinline__ void red_add_cluster(uint32_t addr, float v)
 // ------------------------------------------------------------------ x staging
 // Step u (columns 32u .. 32u + 31) of x occupies 32 words at xq + 32u:
 //  words 8l + w (l = 0..2, w = 0..7): limb l of columns 32u + 4w .. + 3, one byte each
-//    (PAIRED, the CUDA-core lane units: word 8l + 2(w mod 4) + w / 4 instead, so the two
-//    words a lane needs, columns 4 tig.. and 16 + 4 tig.., are adjacent);
+//    (PAIRED, the CUDA-core lane units: word 8 (w mod 4) + 2l + w / 4 instead, and the
+//    step's factor 2^-e_u as a float at word 8 tig + 6 for tig = 0..3, so the seven words
+//    lane tig needs, limbs 0..2 of columns 4 tig.. and 16 + 4 tig.. and the factor, are
+//    contiguous: two 16-byte loads);
 //  words 24..31: per-column sums of the limbs over what one C column covers
 //    (Q6_K: words 24 + 4h + l = sum of limb l over the 16 columns of half h, words
 //    27 and 31 zero; other formats: word 24 + l = sum of limb l over the 32 columns,
@@ -229,12 +231,19 @@ __device__ __forceinline__ XLimbs x_limbs(float4 v, float two_s)
 // (SUMS) and the zero words (ZEROS: words 27..31, or 27 and 31 with HALVES, which the
 // tensor-core units read; the CUDA-core units leave them unread).
 template <bool HALVES, bool PAIRED, bool SUMS, bool ZEROS>
-__device__ __forceinline__ void x_store(uint32_t* xs, int w, const XLimbs& r, int sx)
+__device__ __forceinline__ void x_store(uint32_t* xs, int w, const XLimbs& r, int sx, float f)
 {
-    const int wp = PAIRED ? 2 * (w & 3) + (w >> 2) : w;
-    xs[wp ^ sx] = r.w0;
-    xs[(8 + wp) ^ sx] = r.w1;
-    xs[(16 + wp) ^ sx] = r.w2;
+    if (PAIRED) {
+        const int b = 8 * (w & 3) + (w >> 2);
+        xs[b] = r.w0;
+        xs[b + 2] = r.w1;
+        xs[b + 4] = r.w2;
+        if (w < 4) xs[8 * w + 6] = __float_as_uint(f);
+    } else {
+        xs[w ^ sx] = r.w0;
+        xs[(8 + w) ^ sx] = r.w1;
+        xs[(16 + w) ^ sx] = r.w2;
+    }
     if (!SUMS) return;
     if (HALVES) {
         if ((w & 3) == 0) {
@@ -309,11 +318,13 @@ __device__ __forceinline__ float2 d_pair(const uint8_t* p)
     return __half22float2(*reinterpret_cast<const __half2*>(p));
 }
 
-// Q4_K: the 32 six-bit scales / mins of rows gid and gid + 8 of a unit, one word per
-// step m: byte 0 scale row gid, 1 scale row gid + 8, 2 min row gid, 3 min row gid + 8.
+// Q4_K / Q5_K: the 32 six-bit scales / mins of rows gid and gid + 8 of a unit, one word
+// per step m: byte 0 scale row gid, 1 scale row gid + 8, 2 min row gid, 3 min row gid + 8
+// (SOFF: byte offset of the unit's scale section).
+template <int SOFF = 2048>
 __device__ __forceinline__ void q4k_scale_words(const uint8_t* U, int gid, uint32_t (&S)[8])
 {
-    const uint8_t* v = U + 2048 + 24 * gid;    // 8-byte aligned
+    const uint8_t* v = U + SOFF + 24 * gid;    // 8-byte aligned
     const uint2 na = *reinterpret_cast<const uint2*>(v);
     const uint2 nb = *reinterpret_cast<const uint2*>(v + 8);
     const uint2 hw = *reinterpret_cast<const uint2*>(v + 16);
@@ -451,6 +462,50 @@ struct Unit<NTX_Q4_K_T> {
     }
 };
 
+// Q5_K: the fifth bits of the 4 codes of group gi (columns 4 t .. + 3 for gi = 2 t, 16 + 4 t
+// .. + 3 for gi = 2 t + 1) of one row, from its fifth-bit word h, at bit 4 of each byte.
+template <int gi>
+__device__ __forceinline__ uint32_t q5_bits(uint32_t h)
+{
+    return (gi <= 4 ? (h << (4 - gi)) : (h >> (gi - 4))) & 0x10101010u;
+}
+__device__ __forceinline__ uint32_t q5_bits_r(uint32_t h, int gi) { return ((h >> gi) & 0x01010101u) << 4; }
+
+template <>
+struct Unit<NTX_Q5_K_T> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, const Lane& L,
+                                               float& acc0, float& acc1)
+    {
+        uint32_t S[8];
+        q4k_scale_words<2560>(U, L.gid, S);
+        const uint2 dd = *reinterpret_cast<const uint2*>(U + 2752 + 8 * L.gid);
+        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+        const uint32_t M = 0x0F0F0F0Fu;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const uint2 pq = *reinterpret_cast<const uint2*>(U + 320 * m + 8 * L.lane);
+            const uint2 H = *reinterpret_cast<const uint2*>(U + 320 * m + 256 + 8 * L.gid);
+            const uint32_t a[4] = {(pq.x & M) | q5_bits_r(H.x, 2 * L.tig), (pq.y & M) | q5_bits_r(H.y, 2 * L.tig),
+                                   ((pq.x >> 4) & M) | q5_bits_r(H.x, 2 * L.tig + 1),
+                                   ((pq.y >> 4) & M) | q5_bits_r(H.y, 2 * L.tig + 1)};
+            const uint32_t* x = xs + 32 * m;
+            uint32_t b0, b1;
+            b_frag<NTX_Q5_K_T>(x, L, b0, b1);
+            int c[4];
+            mma_u8(c, a, b0, b1);
+            const int2 X = *reinterpret_cast<const int2*>(x + 24 + 2 * L.tig);
+            const int xp = X.x + 256 * X.y;
+            const int sc0 = ubyte<0>(S[m]), sc1 = ubyte<1>(S[m]), mn0 = ubyte<2>(S[m]), mn1 = ubyte<3>(S[m]);
+            const float f = fs[m];
+            acc0 = fmaf(d.x * f, fmaf(256.f, (float)(sc0 * c[1]), (float)(sc0 * c[0])),
+                        fmaf(-dm.x * f, (float)(mn0 * xp), acc0));
+            acc1 = fmaf(d.y * f, fmaf(256.f, (float)(sc1 * c[3]), (float)(sc1 * c[2])),
+                        fmaf(-dm.y * f, (float)(mn1 * xp), acc1));
+        }
+    }
+};
+
 // ------------------------------------------------------------------ CUDA-core units
 // The same tiled bytes, reduced on the CUDA cores with dp4a (four 8-bit products and
 // an int32 add per instruction).  Integer partial sums (exact) are weighted by the
@@ -476,11 +531,16 @@ __device__ __forceinline__ float limbs_f(int c0, int c1, int c2)
     return fmaf((float)c2, 65536.f, fmaf((float)c1, 256.f, (float)c0));
 }
 
-// limb words of a step for lane tig: X[l].x = columns 4 tig.., X[l].y = 16 + 4 tig..
-__device__ __forceinline__ void x_words(const uint32_t* xs, int tig, uint2 (&X)[3])
+// limb words of a step for lane tig (the PAIRED layout): X[l].x = columns 4 tig..,
+// X[l].y = 16 + 4 tig..; f = the step's factor 2^-e_u
+__device__ __forceinline__ void x_words(const uint32_t* xs, int tig, uint2 (&X)[3], float& f)
 {
-#pragma unroll
-    for (int l = 0; l < 3; ++l) X[l] = *reinterpret_cast<const uint2*>(xs + 8 * l + 2 * tig);
+    const uint4 a = *reinterpret_cast<const uint4*>(xs + 8 * tig);
+    const uint4 b = *reinterpret_cast<const uint4*>(xs + 8 * tig + 4);
+    X[0] = make_uint2(a.x, a.y);
+    X[1] = make_uint2(a.z, a.w);
+    X[2] = make_uint2(b.x, b.y);
+    f = __uint_as_float(b.z);
 }
 
 template <int QT>
@@ -493,7 +553,9 @@ struct Dot<NTX_Q8_0_T> {
     {
         const uint4 a = *reinterpret_cast<const uint4*>(U + 16 * L.lane);
         uint2 X[3];
-        x_words(xs, L.tig, X);
+        float f;
+        x_words(xs, L.tig, X, f);
+        (void)fs;
         int c0[3], c1[3];
 #pragma unroll
         for (int l = 0; l < 3; ++l) {
@@ -501,7 +563,6 @@ struct Dot<NTX_Q8_0_T> {
             c1[l] = dp4(a.w, X[l].y, dp4(a.y, X[l].x, 0));
         }
         const float2 d = d_pair(U + 512 + 4 * L.gid);
-        const float f = fs[0];
         acc0 = fmaf(d.x * f, limbs_f(c0[0], c0[1], c0[2]), acc0);
         acc1 = fmaf(d.y * f, limbs_f(c1[0], c1[1], c1[2]), acc1);
     }
@@ -675,6 +736,73 @@ struct Row<NTX_Q4_K_T> {
                 for (int t = 0; t < 4; ++t) {
                     c0 = dp4((Pw[t] >> 4) & M, comp(X[l][1], t), dp4(Pw[t] & M, comp(X[l][0], t), c0));
                     c1 = dp4((Qw[t] >> 4) & M, comp(X[l][1], t), dp4(Qw[t] & M, comp(X[l][0], t), c1));
+                }
+                p0[l] += sc0 * c0;
+                p1[l] += sc1 * c1;
+                n0[l] += mn0 * (int)comp(xsum, l);
+                n1[l] += mn1 * (int)comp(xsum, l);
+            }
+            const float f = fs[m];
+            acc0 = fmaf(d.x * f, limbs_f(p0[0], p0[1], p0[2]), fmaf(-dm.x * f, limbs_f(n0[0], n0[1], n0[2]), acc0));
+            acc1 = fmaf(d.y * f, limbs_f(p1[0], p1[1], p1[2]), fmaf(-dm.y * f, limbs_f(n1[0], n1[1], n1[2]), acc1));
+        }
+    }
+};
+
+template <>
+struct Row<NTX_Q5_K_T> {
+    // As Row<NTX_Q4_K_T>, with each code's fifth bit ORed in from the step's fifth-bit words
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, int g, int j,
+                                               float& acc0, float& acc1)
+    {
+        const uint8_t* v = U + 2560 + 24 * g;   // packed 6-bit scales / mins of rows g, g + 8
+        const uint32_t M = 0x0F0F0F0Fu;
+        const uint2 dd = *reinterpret_cast<const uint2*>(U + 2752 + 8 * g);
+        const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+        const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            int p0[3] = {0, 0, 0}, p1[3] = {0, 0, 0};   // per limb: rows g, g + 8
+            int n0[3] = {0, 0, 0}, n1[3] = {0, 0, 0};   // mins x limb sums
+            const int m = j + 4 * k;
+            const uint32_t nw = *reinterpret_cast<const uint32_t*>(v + 4 * (m >> 1));
+            const uint32_t hw = *reinterpret_cast<const uint32_t*>(v + 16 + 4 * k);
+            const uint32_t S = ((nw >> (4 * (m & 1))) & 0x0F0F0F0Fu) | (((hw >> (2 * j)) & 0x03030303u) << 4);
+            const uint4* L = reinterpret_cast<const uint4*>(U + 320 * m + 32 * g);
+            const uint4 u0 = L[0], u1 = L[1];
+            const uint2 H = *reinterpret_cast<const uint2*>(U + 320 * m + 256 + 8 * g);
+            const uint32_t Pw[4] = {u0.x, u0.z, u1.x, u1.z}, Qw[4] = {u0.y, u0.w, u1.y, u1.w};
+            // 5-bit codes of rows g (P) and g + 8 (Q): columns 4 t .. (lo) and 16 + 4 t .. (hi) of lane t
+            uint32_t Plo[4], Phi[4], Qlo[4], Qhi[4];
+            Plo[0] = (Pw[0] & M) | q5_bits<0>(H.x);
+            Phi[0] = ((Pw[0] >> 4) & M) | q5_bits<1>(H.x);
+            Plo[1] = (Pw[1] & M) | q5_bits<2>(H.x);
+            Phi[1] = ((Pw[1] >> 4) & M) | q5_bits<3>(H.x);
+            Plo[2] = (Pw[2] & M) | q5_bits<4>(H.x);
+            Phi[2] = ((Pw[2] >> 4) & M) | q5_bits<5>(H.x);
+            Plo[3] = (Pw[3] & M) | q5_bits<6>(H.x);
+            Phi[3] = ((Pw[3] >> 4) & M) | q5_bits<7>(H.x);
+            Qlo[0] = (Qw[0] & M) | q5_bits<0>(H.y);
+            Qhi[0] = ((Qw[0] >> 4) & M) | q5_bits<1>(H.y);
+            Qlo[1] = (Qw[1] & M) | q5_bits<2>(H.y);
+            Qhi[1] = ((Qw[1] >> 4) & M) | q5_bits<3>(H.y);
+            Qlo[2] = (Qw[2] & M) | q5_bits<4>(H.y);
+            Qhi[2] = ((Qw[2] >> 4) & M) | q5_bits<5>(H.y);
+            Qlo[3] = (Qw[3] & M) | q5_bits<6>(H.y);
+            Qhi[3] = ((Qw[3] >> 4) & M) | q5_bits<7>(H.y);
+            const uint32_t* x = xs + 32 * m;
+            const int sx = 8 * j;   // step m mod 4 = j (a unit starts on a multiple of 8 steps)
+            uint4 X[3][2];
+            x_step(x, sx, X);
+            const uint4 xsum = *reinterpret_cast<const uint4*>(x + (24 ^ sx));
+            const int sc0 = ubyte<0>(S), sc1 = ubyte<1>(S), mn0 = ubyte<2>(S), mn1 = ubyte<3>(S);
+#pragma unroll
+            for (int l = 0; l < 3; ++l) {
+                int c0 = 0, c1 = 0;
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    c0 = dp4(Phi[t], comp(X[l][1], t), dp4(Plo[t], comp(X[l][0], t), c0));
+                    c1 = dp4(Qhi[t], comp(X[l][1], t), dp4(Qlo[t], comp(X[l][0], t), c1));
                 }
                 p0[l] += sc0 * c0;
                 p1[l] += sc1 * c1;
@@ -945,7 +1073,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                     const int u = (tid + (j0 + k) * kCons) >> 3;
                     if (u < n_steps) {
                         x_store<QT == NTX_Q6_K_T, CORE == 1 && QT == NTX_Q8_0_T, XSUMS, CORE == 0>(
-                            xq + 32 * u, wl, r[k], ROWS ? 8 * (u & 3) : 0);
+                            xq + 32 * u, wl, r[k], ROWS ? 8 * (u & 3) : 0, fk[k]);
                         if (wl == 0) xsf[u] = fk[k];
                     }
                 }
@@ -1000,11 +1128,13 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                                 Unit<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, fc + SPU * un, L, acc0,
                                               acc1);
                         } else if constexpr (QT == NTX_Q8_0_T) {
+#pragma unroll 4
                             for (int un = warp; un < n_units; un += kWarps)
                                 Dot<QT>::run(st + (size_t)un * T::UB, xc + 32 * un, fc + un, L, acc0, acc1);
                         } else if constexpr (QT == NTX_Q4_0_T) {
                             // a warp takes 4 units (steps) at a time, one per 8 threads
                             const int sx = 8 * ((c * CE / 32 + rj) & 3);
+#pragma unroll 2
                             for (int u4 = 4 * warp; u4 < n_units; u4 += 4 * kWarps) {
                                 const int un = u4 + rj;
                                 if (un < n_units)

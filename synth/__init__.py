@@ -18,6 +18,8 @@ estructura de caché" sections):
     [0.5 s, 1.5 s], s = 1 / sqrt(K * E[c^2] * 13/12) where c is the integer
     factor of d in one weight (Q4_K: scales 1..8, mins round(7.5 scale),
     dmin = d; Q6_K: sub-scales 1..16);
+  * F16 / F32 weights: an Irwin-Hall(12) value times a power of two (1/4 for the
+    sweep, the power of two nearest 1 / sqrt(K) for decode tensors);
   * vectors and the fp16 KV cache: Irwin-Hall(12) stand-in for N(0,1)
     (mean 0, variance 1, support [-6, 6], resolution 2^-16);
   * RMSNorm weights uniform in [0.9, 1.1].
@@ -36,10 +38,11 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 HOST_LIB = os.path.join(_HERE, "libsynth_host.so")
 DEV_LIB = os.path.join(_HERE, "libsynth_dev.so")
 
-Q8_0, Q4_0, Q4_K, Q6_K, Q5_K = 0, 1, 2, 3, 4
-QTYPE_NAMES = {"q8_0": Q8_0, "q4_0": Q4_0, "q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K}
+Q8_0, Q4_0, Q4_K, Q6_K, Q5_K, F16, F32 = 0, 1, 2, 3, 4, 5, 6
+QTYPE_NAMES = {"q8_0": Q8_0, "q4_0": Q4_0, "q4_k": Q4_K, "q6_k": Q6_K, "q5_k": Q5_K, "f16": F16, "f32": F32}
 # (elements per block, bytes per block)
-BLOCK = {Q8_0: (32, 34), Q4_0: (32, 18), Q4_K: (256, 144), Q6_K: (256, 210), Q5_K: (256, 176)}
+BLOCK = {Q8_0: (32, 34), Q4_0: (32, 18), Q4_K: (256, 144), Q6_K: (256, 210), Q5_K: (256, 176), F16: (1, 2),
+         F32: (1, 4)}
 
 
 def qtype_of(name) -> int:
@@ -68,7 +71,10 @@ def _scale_range(lo: float, hi: float, mode: int) -> QParams:
 
 
 def sweep_qparams(qtype: int) -> QParams:
-    """Scales of the GEMV sweep tensors: d (and dmin) uniform in [1e-3, 1e-2]."""
+    """Scales of the GEMV sweep tensors: d (and dmin) uniform in [1e-3, 1e-2]; F16 / F32
+    weights N(0, 1) / 4."""
+    if qtype in (F16, F32):
+        return QParams(0, 0, -2, 0)
     return _scale_range(1e-3, 1e-2, 0)
 
 
@@ -97,7 +103,10 @@ def _code_mean_square(qtype: int) -> float:
 
 
 def decode_qparams(qtype: int, k: int) -> QParams:
-    """Scales of a decode tensor whose rows have k columns (unit-RMS conditioning)."""
+    """Scales of a decode tensor whose rows have k columns (unit-RMS conditioning; F16 / F32
+    weights N(0, 1) times the power of two nearest 1 / sqrt(k))."""
+    if qtype in (F16, F32):
+        return QParams(0, 0, -int(round(math.log2(math.sqrt(k)))), 1)
     s = 1.0 / math.sqrt(k * _code_mean_square(qtype) * 13.0 / 12.0)
     return _scale_range(0.5 * s, 1.5 * s, 1)
 
@@ -267,7 +276,31 @@ class ModelSpec:
     rope_theta: float = 500000.0
     seed: int = 0
     tiled: bool = False       # weights handed to the library in the tiled layout (same bytes, regrouped)
+    mix: str | None = None    # per-tensor formats: None (every tensor in qtype) or "q4_k_m" (below)
     extra: dict = field(default_factory=dict)
+
+    def qtype_of(self, kind: str, layer: int = GLOBAL_LAYER) -> int:
+        """Format of one tensor.  mix "q4_k_m" (a reading of the pages' "Q4_K_M" models, which
+        mix formats per tensor without saying how): Q4_K everywhere except the LM head and the
+        down projection of every even-numbered layer, which are Q6_K."""
+        if self.mix == "q4_k_m":
+            return Q6_K if kind == "output" or (kind == "w_down" and layer % 2 == 0) else Q4_K
+        return self.qtype
+
+    def lib_code(self, qtype: int) -> int:
+        """The library's code of a tensor in `qtype` as this model hands it over (the tiled form
+        when the model is tiled; F16 / F32 have none)."""
+        return qtype | 16 if self.tiled and qtype not in (F16, F32) else qtype
+
+    def tensor_qtypes(self):
+        """Library codes of every tensor (tok_embd, output, then per layer w_qkv, w_o, w_gate and
+        w_up, w_down), or None when every tensor has the model's format."""
+        if self.mix is None:
+            return None
+        out = [self.lib_code(self.qtype_of("tok_embd")), self.lib_code(self.qtype_of("output"))]
+        for l in range(self.n_layers):
+            out += [self.lib_code(self.qtype_of(k, l)) for k in ("w_qkv", "w_o", "w_gate", "w_down")]
+        return out
 
     @property
     def qkv_rows(self) -> int:
@@ -277,10 +310,10 @@ class ModelSpec:
     def q_dim(self) -> int:
         return self.n_q_heads * self.head_dim
 
-    def layer_weight_bytes(self) -> int:
-        h, f, q = self.hidden, self.ffn, self.qtype
-        return (self.qkv_rows * row_bytes(q, h) + h * row_bytes(q, self.q_dim) + 2 * f * row_bytes(q, h)
-                + h * row_bytes(q, f))
+    def layer_weight_bytes(self, layer: int = 0) -> int:
+        h, f, q = self.hidden, self.ffn, lambda k: self.qtype_of(k, layer)
+        return (self.qkv_rows * row_bytes(q("w_qkv"), h) + h * row_bytes(q("w_o"), self.q_dim)
+                + 2 * f * row_bytes(q("w_gate"), h) + h * row_bytes(q("w_down"), f))
 
     def kv_bytes_per_layer(self) -> int:
         return 2 * self.n_kv_heads * self.max_ctx * self.head_dim * 2
@@ -288,17 +321,18 @@ class ModelSpec:
     def token(self) -> int:
         return uniform_index(self.seed, tensor_id(GLOBAL_LAYER, "token"), self.vocab)
 
-    # (rows, cols, scale params) of each packed tensor
-    def packed(self, kind: str):
-        h, f, q = self.hidden, self.ffn, self.qtype
-        shapes = {"tok_embd": (self.vocab, h, decode_qparams(q, 1)),
-                  "output": (self.vocab, h, decode_qparams(q, h)),
-                  "w_qkv": (self.qkv_rows, h, decode_qparams(q, h)),
-                  "w_o": (h, self.q_dim, decode_qparams(q, self.q_dim)),
-                  "w_gate": (f, h, decode_qparams(q, h)),
-                  "w_up": (f, h, decode_qparams(q, h)),
-                  "w_down": (h, f, decode_qparams(q, f))}
-        return shapes[kind]
+    # (rows, cols, scale params, format) of each packed tensor
+    def packed(self, kind: str, layer: int = GLOBAL_LAYER):
+        h, f, q = self.hidden, self.ffn, self.qtype_of(kind, layer)
+        shapes = {"tok_embd": (self.vocab, h, 1),
+                  "output": (self.vocab, h, h),
+                  "w_qkv": (self.qkv_rows, h, h),
+                  "w_o": (h, self.q_dim, self.q_dim),
+                  "w_gate": (f, h, h),
+                  "w_up": (f, h, h),
+                  "w_down": (h, f, f)}
+        rows, cols, k = shapes[kind]
+        return rows, cols, decode_qparams(q, k), q
 
 
 LLAMA_8B_Q8_0 = dict(n_layers=32, hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, ffn=14336,
@@ -306,3 +340,4 @@ LLAMA_8B_Q8_0 = dict(n_layers=32, hidden=4096, n_q_heads=32, n_kv_heads=8, head_
 LLAMA_70B_Q6_K = dict(n_layers=80, hidden=8192, n_q_heads=64, n_kv_heads=8, head_dim=128, ffn=28672,
                       vocab=128256, max_ctx=8193, n_prefill=8192, qtype=Q6_K, rope_theta=500000.0)
 LLAMA_70B_Q4_K = dict(LLAMA_70B_Q6_K, qtype=Q4_K)
+LLAMA_70B_Q4_K_M = dict(LLAMA_70B_Q6_K, qtype=Q4_K, mix="q4_k_m")

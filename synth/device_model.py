@@ -12,14 +12,14 @@ from . import (GLOBAL_LAYER, NORM_W, BLOCK, ModelSpec, blocks_dev, normal_f16_de
 
 
 def _alloc_packed(spec: ModelSpec, kind: str, layer: int, device, host: bool = False) -> torch.Tensor:
-    rows, cols, qp = spec.packed(kind)
-    nbytes = rows * row_bytes(spec.qtype, cols)
+    rows, cols, qp, q = spec.packed(kind, layer)
+    nbytes = rows * row_bytes(q, cols)
     t = torch.empty(nbytes, dtype=torch.uint8, device=device)
-    blocks_dev(t, spec.qtype, spec.seed, tensor_id(layer, kind), rows, cols, qp)
-    if spec.tiled:
+    blocks_dev(t, q, spec.seed, tensor_id(layer, kind), rows, cols, qp)
+    if spec.lib_code(q) != q:
         import quantized_weight_gemv_block_b200 as ntx
         tt = torch.empty_like(t)
-        ntx.ntx_repack_q(spec.qtype, t, tt, rows, cols)
+        ntx.ntx_repack_q(q, t, tt, rows, cols)
         t = tt
     if host:
         h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
@@ -63,11 +63,19 @@ class DeviceModel:
             self._layer_descs[l] = ntx.LayerDesc(*[t[k].data_ptr() for k in ("attn_norm", "w_qkv", "w_o", "ffn_norm",
                                                                             "w_gate", "w_up", "w_down", "k_cache",
                                                                             "v_cache")])
+        qts = s.tensor_qtypes()
+        if qts is not None:
+            qts = qts[:2 + 4 * self.n_layers]
+            self._qts = (ctypes.c_int32 * len(qts))(*qts)
+            qts_p = ctypes.cast(self._qts, ctypes.POINTER(ctypes.c_int32))
+        else:
+            qts_p = None
         self.desc = ntx.ModelDesc(self.n_layers, s.hidden, s.n_q_heads, s.n_kv_heads, s.head_dim, s.ffn, s.vocab,
-                                  s.max_ctx, s.rms_eps, s.rope_theta, s.qtype | (16 if s.tiled else 0),
+                                  s.max_ctx, s.rms_eps, s.rope_theta, s.lib_code(s.qtype),
                                   self.tok_embd.data_ptr(),
                                   self.out_norm.data_ptr(), self.output.data_ptr(),
-                                  ctypes.cast(self._layer_descs, ctypes.POINTER(ntx.LayerDesc)), self.n_resident)
+                                  ctypes.cast(self._layer_descs, ctypes.POINTER(ntx.LayerDesc)), self.n_resident,
+                                  qts_p)
         self.handle = ntx.ntx_model_create(self.desc)
 
     def reset_caches(self):

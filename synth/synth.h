@@ -27,6 +27,7 @@
 #define SYNTH_H
 
 #include <stdint.h>
+#include <string.h>
 
 #ifdef __CUDACC__
 #define SYN_HD __host__ __device__ __forceinline__
@@ -40,6 +41,8 @@
 #define SYN_Q4_K 2
 #define SYN_Q6_K 3
 #define SYN_Q5_K 4
+#define SYN_F16 5
+#define SYN_F32 6
 
 /* Scale-field distribution of one tensor.
  *   d = fp16(k * 2^d_exp) with k uniform in [d_lo, d_hi]
@@ -141,19 +144,21 @@ SYN_HD uint16_t syn_scale_bits(uint32_t r, const syn_qparams* P)
 SYN_HD int syn_block_bytes(int qtype)
 {
     return qtype == SYN_Q8_0 ? 34 : qtype == SYN_Q4_0 ? 18 : qtype == SYN_Q4_K ? 144 : qtype == SYN_Q6_K ? 210
-         : qtype == SYN_Q5_K ? 176 : 0;
+         : qtype == SYN_Q5_K ? 176 : qtype == SYN_F16 ? 2 : qtype == SYN_F32 ? 4 : 0;
 }
 
 SYN_HD int syn_block_elems(int qtype)
 {
     return (qtype == SYN_Q8_0 || qtype == SYN_Q4_0) ? 32
-         : (qtype == SYN_Q4_K || qtype == SYN_Q6_K || qtype == SYN_Q5_K) ? 256 : 0;
+         : (qtype == SYN_Q4_K || qtype == SYN_Q6_K || qtype == SYN_Q5_K) ? 256
+         : (qtype == SYN_F16 || qtype == SYN_F32) ? 1 : 0;
 }
 
 /* Draws consumed per block (block b uses draws [b*D, b*D + D)). */
 SYN_HD uint64_t syn_block_draws(int qtype)
 {
-    return qtype == SYN_Q8_0 ? 17 : qtype == SYN_Q4_0 ? 3 : qtype == SYN_Q4_K ? 19 : qtype == SYN_Q5_K ? 23 : 33;
+    return qtype == SYN_Q8_0 ? 17 : qtype == SYN_Q4_0 ? 3 : qtype == SYN_Q4_K ? 19 : qtype == SYN_Q5_K ? 23
+         : (qtype == SYN_F16 || qtype == SYN_F32) ? 3 : 33;
 }
 
 /* 6-bit scale / min packing of the K-quants: sub-blocks 0..3 whole in bytes 0..3 (scale)
@@ -169,10 +174,40 @@ SYN_HD void syn_pack_k_scales(const uint8_t* s6, const uint8_t* m6, uint8_t* sc)
     }
 }
 
-/* Write block number `b` of the tensor with stream key `key` to out[0 .. block_bytes). */
+/* Irwin-Hall(12) stand-in for N(0,1): sum of twelve 16-bit uniforms
+ * U = (u + 1/2) / 65536, minus 6.  Returns the numerator n of n * 2^-16. */
+SYN_HD int32_t syn_ih12(uint64_t key, uint64_t i)
+{
+    int32_t s = 0;
+    for (int j = 0; j < 3; ++j) {
+        uint64_t r = syn_draw(key, 3 * i + j);
+        s += (int32_t)(r & 0xFFFF) + (int32_t)((r >> 16) & 0xFFFF) + (int32_t)((r >> 32) & 0xFFFF) + (int32_t)(r >> 48);
+    }
+    return s - 393210;
+}
+
+/* Write block number `b` of the tensor with stream key `key` to out[0 .. block_bytes).
+ * F16 / F32 "blocks" are one weight: an Irwin-Hall(12) value times 2^d_exp (a power of
+ * two, no other rounding than fp16's). */
 SYN_HD void syn_fill_block(int qtype, uint64_t key, uint64_t b, const syn_qparams* P, uint8_t* out)
 {
     uint64_t n0 = b * syn_block_draws(qtype);
+    if (qtype == SYN_F16 || qtype == SYN_F32) {
+        const int32_t n = syn_ih12(key, b);
+        if (qtype == SYN_F16) {
+            const uint64_t a = (uint64_t)(n < 0 ? -n : n);
+            syn_put_u16(out, (uint16_t)((n < 0 ? 0x8000 : 0) | syn_f16_from_scaled(a, P->d_exp - 16)));
+        } else {
+            float v = (float)n;
+            int e = P->d_exp - 16;
+            while (e < 0) { v *= 0.5f; ++e; }
+            while (e > 0) { v *= 2.0f; --e; }
+            uint32_t u;
+            memcpy(&u, &v, 4);
+            for (int i = 0; i < 4; ++i) out[i] = (uint8_t)(u >> (8 * i));
+        }
+        return;
+    }
     if (qtype == SYN_Q8_0) {
         syn_put_u16(out, syn_scale_bits((uint32_t)syn_draw(key, n0), P));
         for (int i = 0; i < 16; ++i) {
@@ -242,18 +277,6 @@ SYN_HD void syn_fill_block(int qtype, uint64_t key, uint64_t b, const syn_qparam
         }
         syn_put_u16(out + 208, syn_scale_bits((uint32_t)syn_draw(key, n0), P));
     }
-}
-
-/* Irwin-Hall(12) stand-in for N(0,1): sum of twelve 16-bit uniforms
- * U = (u + 1/2) / 65536, minus 6.  Returns the numerator n of n * 2^-16. */
-SYN_HD int32_t syn_ih12(uint64_t key, uint64_t i)
-{
-    int32_t s = 0;
-    for (int j = 0; j < 3; ++j) {
-        uint64_t r = syn_draw(key, 3 * i + j);
-        s += (int32_t)(r & 0xFFFF) + (int32_t)((r >> 16) & 0xFFFF) + (int32_t)((r >> 32) & 0xFFFF) + (int32_t)(r >> 48);
-    }
-    return s - 393210;
 }
 
 SYN_HD float syn_normal_f32(uint64_t key, uint64_t i)

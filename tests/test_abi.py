@@ -41,7 +41,7 @@ def test_row_bytes_and_block_sizes(ntx):
     assert ntx.ntx_row_bytes(ntx.NTX_Q6_K, 28672) == 23520
     assert ntx.ntx_row_bytes(ntx.NTX_Q4_K, 128) == 0          # not a multiple of 256
     assert ntx.ntx_row_bytes(9, 256) == 0
-    assert [ntx.ntx_block_elems(q) for q in range(4)] == [32, 32, 256, 256]
+    assert [ntx.ntx_block_elems(q) for q in range(7)] == [32, 32, 256, 256, 256, 1, 1]
 
 
 def _status(ntx, fn, *args):
@@ -59,10 +59,15 @@ def test_gemv_rejects_bad_arguments(ntx):
     assert _status(ntx, "ntx_dequant_q", 3, p, 1, 100, p, None) == ntx.NTX_EINVAL
     # tiled layouts take whole 16-row groups
     assert _status(ntx, "ntx_gemv_q", 16, p, 40, 256, p, p, None) == ntx.NTX_EINVAL
-    # formats without GPU kernels yet (Q5_K, F16, F32 codes) are rejected, not misread
-    for q in (4, 5, 6, 20):
+    # unknown codes, and tiled forms that do not exist (F16, F32), are rejected, not misread
+    for q in (7, 8, 15, 21, 22, 23):
         assert _status(ntx, "ntx_gemv_q", q, p, 16, 256, p, p, None) == ntx.NTX_EINVAL
-    assert ntx.lib().ntx_row_bytes(4, 256) == 0
+        assert ntx.lib().ntx_row_bytes(q, 256) == 0
+    assert ntx.lib().ntx_row_bytes(ntx.NTX_Q5_K, 256) == 176
+    assert ntx.lib().ntx_row_bytes(ntx.NTX_Q5_K_T, 512) == 352
+    assert ntx.lib().ntx_row_bytes(ntx.NTX_Q5_K, 128) == 0
+    assert ntx.lib().ntx_row_bytes(ntx.NTX_F16, 3) == 6
+    assert ntx.lib().ntx_row_bytes(ntx.NTX_F32, 7) == 28
 
 
 def test_ops_reject_bad_arguments(ntx):
@@ -74,7 +79,7 @@ def test_ops_reject_bad_arguments(ntx):
     assert _status(ntx, "ntx_softmax", p, p, 0, None) == ntx.NTX_EINVAL
     assert _status(ntx, "ntx_swiglu", p, None, p, 4, None) == ntx.NTX_EINVAL
     assert _status(ntx, "ntx_argmax", p, 0, p, None) == ntx.NTX_EINVAL
-    assert _status(ntx, "ntx_embed", 5, p, 10, 256, p, p, None) == ntx.NTX_EINVAL
+    assert _status(ntx, "ntx_embed", 9, p, 10, 256, p, p, None) == ntx.NTX_EINVAL
 
 
 def test_attention_rejects_bad_arguments(ntx):

@@ -47,12 +47,16 @@ def kv_rows_at(model, layer, pos):
 
 
 def assert_kv_rows_match(got_bits, want_bits):
-    """The K / V rows stored at pos equal the oracle's fp16 rounding of k and v, up to the
-    occasional 1-ulp flip where fp32 summation order moves a value across a rounding
-    boundary (same sign, adjacent patterns)."""
-    diff = np.abs(got_bits - want_bits)
-    assert np.all(diff <= 1), int(diff.max())
-    assert np.mean(diff == 0) > 0.99
+    """The K / V rows stored at pos are the oracle's fp16 rounding of k and v: most are the
+    same bit pattern, and the rest differ only where fp32 summation order moved a value
+    across an fp16 rounding boundary, i.e. by no more than the 2e-3 tolerance relative to
+    the largest value of the head's row (a value near zero has fp16 steps far finer than
+    its absolute error, so it may be several patterns away)."""
+    got = np.asarray(got_bits, dtype=np.int16).view(np.float16).astype(np.float64)
+    want = np.asarray(want_bits, dtype=np.int16).view(np.float16).astype(np.float64)
+    scale = np.max(np.abs(want), axis=-1, keepdims=True)
+    assert np.all(np.abs(got - want) <= TOL * scale)
+    assert np.mean(got_bits == want_bits) > 0.95
 
 
 @pytest.mark.parametrize("qtype", [0, 1, 2, 3], ids=["q8_0", "q4_0", "q4_k", "q6_k"])
@@ -90,6 +94,22 @@ def test_decode_step_tiled(ntx, syn, qtype):
     from synth.device_model import DeviceModel
     kw = dict(hidden=8192, ffn=8192 * 2, n_q_heads=64) if qtype == 3 else {}
     spec = small_spec(syn, qtype, n_layers=2, tiled=True, **kw)
+    m = DeviceModel(spec)
+    got = run_decode(ntx, m, spec.token(), spec.n_prefill)
+    m.close()
+    want, _ = om.decode(spec)
+    assert rel_err(got, want) <= TOL
+    assert elem_err(got, want) <= TOL
+
+
+@pytest.mark.parametrize("qtype,mix", [(4, None), (5, None), (6, None), (2, "q4_k_m")],
+                         ids=["q5_k_t", "f16", "f32", "q4_k_m_t"])
+def test_decode_step_further_formats(ntx, syn, qtype, mix):
+    """Whole decode steps of models in the further formats (Q5_K tiled, F16, F32) and of a
+    model that mixes Q4_K and Q6_K tensors, against the oracle."""
+    from oracle import model as om
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, qtype, n_layers=2, tiled=True, mix=mix)
     m = DeviceModel(spec)
     got = run_decode(ntx, m, spec.token(), spec.n_prefill)
     m.close()
@@ -196,3 +216,11 @@ def test_streamed_llama70b_q4_k_against_oracle(ntx, syn):
     ring, against the oracle's decode of the same four layers."""
     spec = syn.ModelSpec(**dict(syn.LLAMA_70B_Q4_K, n_layers=4), tiled=True)
     compare_full(ntx, spec, "llama70b q4_k tiled, 2 of 4 layers streamed", n_resident=2)
+
+
+def test_streamed_mixed_formats_against_oracle(ntx, syn):
+    """A model mixing Q4_K and Q6_K matrices (the "q4_k_m" recipe) at 70B width, two layers
+    resident and two streamed: the ring's slots hold each streamed layer's own sizes."""
+    spec = syn.ModelSpec(**dict(syn.LLAMA_70B_Q4_K_M, n_layers=4, vocab=4000, max_ctx=600, n_prefill=512),
+                         tiled=True)
+    compare_full(ntx, spec, "llama70b q4_k_m tiled, 2 of 4 layers streamed", n_resident=2)

@@ -4,7 +4,7 @@ separately from the library's repack kernel, so the kernel's output can be
 checked byte for byte against the documented layout."""
 import numpy as np
 
-Q8_0, Q4_0, Q4_K, Q6_K = 0, 1, 2, 3
+Q8_0, Q4_0, Q4_K, Q6_K, Q5_K = 0, 1, 2, 3, 4
 
 
 def _fields(qtype, host, rows, cols):
@@ -30,12 +30,19 @@ def _fields(qtype, host, rows, cols):
         sc = b.reshape(rows, cols // 256, 210)[:, :, 192:208]
         d = b.reshape(rows, cols // 256, 210)[:, :, 208:210].copy().view(np.uint16)[:, :, 0]
         return dict(code=code.reshape(rows, cols), sc=sc.copy(), d=d)
-    blk = b.reshape(rows, cols // 256, 144).astype(np.int32)
+    bb = 176 if qtype == Q5_K else 144
+    blk = b.reshape(rows, cols // 256, bb).astype(np.int32)
     code = np.zeros((rows, cols // 256, 256), np.int32)
     for e in range(256):
         c, r = e >> 6, e & 63
-        byte = blk[:, :, 16 + 32 * c + (r & 31)]
-        code[:, :, e] = (byte & 15) if r < 32 else (byte >> 4)
+        if qtype == Q5_K:
+            # fp16 d | fp16 dmin | 12 B scales | 32 B fifth bits | 128 B low nibbles
+            byte = blk[:, :, 48 + 32 * c + (r & 31)]
+            b5 = (blk[:, :, 16 + (r & 31)] >> (2 * c + (r >> 5))) & 1
+            code[:, :, e] = ((byte & 15) if r < 32 else (byte >> 4)) | (b5 << 4)
+        else:
+            byte = blk[:, :, 16 + 32 * c + (r & 31)]
+            code[:, :, e] = (byte & 15) if r < 32 else (byte >> 4)
     s = blk[:, :, 4:16]
     sc = np.zeros((rows, cols // 256, 8), np.int32)
     mn = np.zeros((rows, cols // 256, 8), np.int32)
@@ -46,7 +53,7 @@ def _fields(qtype, host, rows, cols):
         else:
             sc[:, :, j] = (s[:, :, j + 4] & 15) | ((s[:, :, j - 4] >> 6) << 4)
             mn[:, :, j] = (s[:, :, j + 4] >> 4) | ((s[:, :, j] >> 6) << 4)
-    raw = b.reshape(rows, cols // 256, 144)
+    raw = b.reshape(rows, cols // 256, bb)
     return dict(code=code.reshape(rows, cols), sc=sc, mn=mn, d=raw[:, :, 0:2].copy().view(np.uint16)[:, :, 0],
                 dmin=raw[:, :, 2:4].copy().view(np.uint16)[:, :, 0])
 
@@ -111,7 +118,20 @@ def tile(qtype, host, rows, cols):
                             row = r0 + gid + 8 * hi
                             for j in range(4):
                                 c = c0 + 32 * m + 4 * tig + j
-                                unit.append(code[row, c] | (code[row, c + 16] << 4))
+                                unit.append((code[row, c] & 15) | ((code[row, c + 16] & 15) << 4))
+                    if qtype == Q5_K:
+                        # fifth bits: per gid words H0 (row gid), H1 (row gid + 8); the bit of
+                        # column 4 t + j at 8 j + 2 t, of column 16 + 4 t + j at 8 j + 2 t + 1
+                        for gid in range(8):
+                            for hi in range(2):
+                                row = r0 + gid + 8 * hi
+                                for j in range(4):
+                                    v = 0
+                                    for t in range(4):
+                                        c = c0 + 32 * m + 4 * t + j
+                                        v |= ((code[row, c] >> 4) & 1) << (2 * t)
+                                        v |= ((code[row, c + 16] >> 4) & 1) << (2 * t + 1)
+                                    unit.append(v)
                 for gid in range(8):
                     V = lambda m, b: int((f["mn"] if b & 2 else f["sc"])[r0 + gid + 8 * (b & 1), u, m])
                     for wn in range(4):
