@@ -274,9 +274,8 @@ def run_decode_bench(args, rank, world, local):
     stream = torch.cuda.Stream()
     copy_stream = torch.cuda.Stream() if streamed else None
     logits = torch.empty(spec.vocab, dtype=torch.float32, device="cuda")
-    # step word + embedding, per layer QKV, attention (with the split merge), O, gate/up, down,
-    # then the LM head
-    launches_per_step = 2 + 5 * spec.n_layers + 1
+    # step word + embedding, per layer QKV, attention, split merge, O, gate/up, down, then the LM head
+    launches_per_step = 2 + 6 * spec.n_layers + 1
 
     def step():
         if streamed:

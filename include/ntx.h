@@ -188,13 +188,9 @@ ntx_status ntx_rope(float* q, float* k, int n_q_heads, int n_kv_heads, int head_
  *   k_cache, v_cache  device fp16 [n_kv_heads, max_ctx, head_dim]
  *   out     device fp32 [n_q_heads, head_dim]
  *   workspace / workspace_bytes: device scratch of at least
- *           ntx_attn_workspace_bytes(...) bytes, 16-byte aligned: the first 256
- *           bytes hold one merge ticket counter per kv head (cleared by the call with
- *           cudaMemsetAsync on `stream`), the rest the partial results of the context
- *           splits; it needs no initialisation by the caller.
- * One kernel runs on `stream`: each CTA takes a context range of one kv head, and
- * the last of them to finish merges that head's ranges (log-sum-exp rule, in range
- * order, so the result does not depend on which CTA merges).
+ *           ntx_attn_workspace_bytes(...) bytes, 16-byte aligned, for the partial
+ *           results of the context splits; it needs no initialisation.
+ * Two kernels run on `stream`: the split kernel, then the merge of the splits.
  * head_dim == 128, n_q_heads a multiple of n_kv_heads with at most 8 q heads per
  * kv head, 1 <= n_ctx <= max_ctx.  Calls sharing a workspace must not overlap. */
 ntx_status ntx_attn_decode(const float* q, const void* k_cache, const void* v_cache, float* out, int n_q_heads,
@@ -206,9 +202,8 @@ size_t ntx_attn_workspace_bytes(int n_q_heads, int n_kv_heads, int head_dim, int
  * memory: code that runs under a fixed, pre-planned memory budget or inside a
  * host framework whose allocator hands out no scratch, and so has no workspace
  * to pass.  (The pages have no counterpart; this is an addition of this library.)
- * The merge tickets and split partials live in a device array of 512 KiB that the
- * library holds on every GPU that loads it, until the process exits (the call clears
- * the tickets with cudaMemsetAsync, which allocates nothing).  Shapes
+ * The split partials live in a device array of 512 KiB that the
+ * library holds on every GPU that loads it, until the process exits.  Shapes
  * whose workspace (ntx_attn_workspace_bytes) exceeds 512 KiB are rejected with
  * NTX_EUNSUPPORTED (on a 148-SM B200: 8 q heads per kv head with 8 kv heads, as
  * in Llama-70B, needs about 600 KB; 4 per kv head, as in Llama-8B, about 300 KB).  Nothing is allocated: the first call on a device looks up
@@ -317,6 +312,25 @@ ntx_status ntx_stream_layers(ntx_model* model, int32_t token, int32_t pos, float
  * again before relying on its results.  The launches may be captured in a CUDA graph. */
 enum { NTX_GEMV_QKV = 0, NTX_GEMV_O = 1, NTX_GEMV_GATE_UP = 2, NTX_GEMV_DOWN = 3, NTX_GEMV_HEAD = 4 };
 ntx_status ntx_model_replay_gemv(ntx_model* model, int kind, int n_launches, float* logits, void* stream);
+
+/* Layer skip ("Rendimiento y estructura de caché": layers whose hidden states barely
+ * change, judged by cosine similarity, are left out; 20 of 80 on the pages' 70B run).
+ *
+ * ntx_model_layer_similarity runs one decode step of token at pos with every layer (the
+ * skip mask ignored; the LM head is not run) and writes, for each layer l, the cosine
+ * similarity of the hidden state before and after it, cos_out[l] = h_in . h_out /
+ * (|h_in| |h_out|), to the host array cos_out [n_layers]; it returns once they are there.
+ * Like a step, it writes the K / V rows at pos.  Streamed models need distinct compute and
+ * copy streams (copy is unused otherwise).
+ *
+ * ntx_model_set_layer_skip sets the layers the decode step leaves out: skip is a host
+ * array [n_layers], nonzero = skip (NULL clears the mask).  A skipped layer is neither
+ * computed nor, if streamed, copied, and writes no K / V rows (its cache is never read
+ * while it stays skipped).  The next ntx_decode_step records its CUDA graph again.  Which
+ * layers to skip is the caller's choice, e.g. the k layers of highest similarity. */
+ntx_status ntx_model_layer_similarity(ntx_model* model, int32_t token, int32_t pos, float* cos_out, void* compute,
+                                      void* copy);
+ntx_status ntx_model_set_layer_skip(ntx_model* model, const uint8_t* skip);
 
 /* Per-step counters of the last ntx_stream_layers call: bytes copied host ->
  * device, and device milliseconds of the whole step (between the step's first

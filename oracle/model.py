@@ -45,12 +45,13 @@ def head_tensors(spec: ModelSpec, rows=None):
 
 
 def decode(spec: ModelSpec, pos: int | None = None, token: int | None = None, n_layers: int | None = None,
-           head_rows=None, keep_hidden: bool = False, layer_hook=None):
+           head_rows=None, keep_hidden: bool = False, layer_hook=None, skip=()):
     """Logits of one decode step (token at position pos, default n_prefill).
 
     Returns (logits, hidden_states) where hidden_states[l] is h after layer l
     when keep_hidden is set.  layer_hook(l, tensors) may inspect the layer's
-    tensors after the step (e.g. the KV rows written at pos).
+    tensors after the step (e.g. the KV rows written at pos).  Layers in `skip` are
+    left out (h passes through them unchanged).
     """
     pos = spec.n_prefill if pos is None else pos
     token = spec.token() if token is None else token
@@ -59,6 +60,10 @@ def decode(spec: ModelSpec, pos: int | None = None, token: int | None = None, n_
     h = embedding_row(spec, token).copy()
     hidden = []
     for layer in range(n_layers):
+        if layer in skip:        # a skipped layer leaves h as it is
+            if keep_hidden:
+                hidden.append(h.copy())
+            continue
         t = layer_tensors(spec, layer)
         qts = [spec.qtype_of(k, layer) for k in ("w_qkv", "w_o", "w_gate", "w_down")]
         decode_layer(dims, qts, h, pos, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"], t["w_gate"],
@@ -71,3 +76,18 @@ def decode(spec: ModelSpec, pos: int | None = None, token: int | None = None, n_
     n_rows = W.shape[0]
     logits = lm_head(spec.qtype_of("output"), norm, W, n_rows, spec.hidden, spec.rms_eps, h)
     return logits, hidden
+
+
+def layer_similarity(spec: ModelSpec, pos: int | None = None, token: int | None = None):
+    """Cosine similarity of each layer's input and output hidden states, in double, from the
+    oracle's hidden states (every layer run)."""
+    import numpy as np
+    token = spec.token() if token is None else token
+    h0 = embedding_row(spec, token).astype(np.float64)
+    _, hidden = decode(spec, pos=pos, token=token, keep_hidden=True, head_rows=(0, 16))
+    out, prev = [], h0
+    for h in hidden:
+        cur = h.astype(np.float64)
+        out.append(float(prev @ cur / np.sqrt((prev @ prev) * (cur @ cur))))
+        prev = cur
+    return out

@@ -26,7 +26,8 @@ EXPORTS = ("ntx_last_error", "ntx_version", "ntx_row_bytes", "ntx_block_elems", 
            "ntx_stream_read_probe",
            "ntx_dequant_q", "ntx_repack_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_decode_noalloc", "ntx_attn_workspace_bytes", "ntx_swiglu",
            "ntx_softmax", "ntx_argmax", "ntx_embed", "ntx_model_create", "ntx_model_destroy", "ntx_decode_step",
-           "ntx_stream_layers", "ntx_stream_stats", "ntx_model_replay_gemv")
+           "ntx_stream_layers", "ntx_stream_stats", "ntx_model_replay_gemv", "ntx_model_layer_similarity",
+           "ntx_model_set_layer_skip")
 
 
 class NtxError(RuntimeError):
@@ -87,6 +88,8 @@ def lib() -> ctypes.CDLL:
             "ntx_stream_layers": ([vp, i32, i32, vp, vp, vp, i64], ci),
             "ntx_stream_stats": ([vp, ctypes.POINTER(i64), ctypes.POINTER(cf)], ci),
             "ntx_model_replay_gemv": ([vp, ci, ci, vp, vp], ci),
+            "ntx_model_layer_similarity": ([vp, i32, i32, ctypes.POINTER(cf), vp, vp], ci),
+            "ntx_model_set_layer_skip": ([vp, ctypes.POINTER(ctypes.c_uint8)], ci),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -223,3 +226,19 @@ def ntx_stream_stats(model: int):
 
 def ntx_model_replay_gemv(model: int, kind: int, n_launches: int, logits=None, stream=None) -> None:
     check(lib().ntx_model_replay_gemv(model, kind, n_launches, _p(logits), _s(stream)))
+
+
+def ntx_model_layer_similarity(model: int, token: int, pos: int, n_layers: int, compute=None, copy=None):
+    """Cosine similarity of each layer's input and output hidden states (list of floats)."""
+    out = (ctypes.c_float * n_layers)()
+    check(lib().ntx_model_layer_similarity(model, token, pos, out, _s(compute), _s(copy) if copy is not None else None))
+    return list(out)
+
+
+def ntx_model_set_layer_skip(model: int, skip) -> None:
+    """skip: sequence of n_layers flags (nonzero = leave the layer out), or None to clear."""
+    if skip is None:
+        check(lib().ntx_model_set_layer_skip(model, None))
+        return
+    arr = (ctypes.c_uint8 * len(skip))(*[1 if v else 0 for v in skip])
+    check(lib().ntx_model_set_layer_skip(model, arr))

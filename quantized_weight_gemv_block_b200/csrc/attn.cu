@@ -18,11 +18,10 @@
 //    warps, which form O^T = V^T P^T (P split the same way) while the score warps
 //    move on to stage i + 1.  K and V are fp16 already, so every product is exact
 //    and only the fp32 accumulation rounds;
-//  * the partial (m, l, acc[128]) of each query head goes to the workspace; the
-//    CTA that finishes last among the splits of a kv head (a ticket from one atomic
-//    counter per kv head) merges that head's splits with the log-sum-exp rule, in a
-//    fixed split order whichever CTA it is, so the result is deterministic and no
-//    second kernel is launched.
+//  * the partial (m, l, acc[128]) of each query head goes to the workspace, and a
+//    second kernel (one CTA per query head, launched as a programmatic dependent)
+//    merges the splits with the log-sum-exp rule in a fixed order, so the result
+//    is deterministic.
 // Every wait is bounded; a wait that runs out records an error and the CTA still
 // finishes.
 #include <cuda.h>
@@ -48,14 +47,12 @@ constexpr int kStages = 4;
 constexpr int kPartFloats = 4 + HD;               // m, l, 2 pad, acc[128]: 528-byte records
 constexpr int kMaxSplit = 128;
 constexpr uint32_t kPolls = 1u << 22;
-constexpr size_t kCounterBytes = 256;             // one merge ticket counter per kv head (<= 64)
 
 struct KArgs {
     CUtensorMap tk, tv;         // K and V caches as [n_kv][max_ctx][128] fp16, 64 x 64 boxes
     const float* q;
     float* out;
     float* part;
-    unsigned* counters;         // [n_kv] arrivals of the splits of each kv head; 0 between launches
     int max_ctx, n_split;
     int32_t n_ctx;
     const int32_t* pos_dev;
@@ -118,59 +115,6 @@ __device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int x
         "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
-}
-
-// Merge of the splits of kv head g into out, by one CTA: with M = max_s m_s over the
-// splits that saw a position, w_s = e^(m_s - M) / L and L = sum_s l_s e^(m_s - M),
-// out[h][d] = sum_s w_s acc_s[h][d], the splits taken in order s = 0, 1, ... (so the
-// result does not depend on which CTA merges).  ws: shared memory for the weights.
-template <int G>
-__device__ __forceinline__ void merge_splits(const KArgs& a, int g, float* ws)
-{
-    const int tid = threadIdx.x, ns = a.n_split;
-    const float* base = a.part + (size_t)g * ns * G * kPartFloats;
-    // (m, l) of every split and head
-    for (int i = tid; i < ns * G; i += kThreads) {
-        const float2 ml = __ldcg(reinterpret_cast<const float2*>(base + (size_t)i * kPartFloats));
-        ws[2 * i] = ml.x;
-        ws[2 * i + 1] = ml.y;
-    }
-    __syncthreads();
-    // per head: the normalised weight of each split, in place of its m
-    if (tid < G) {
-        const int h = tid;
-        float M = -INFINITY;
-        for (int s = 0; s < ns; ++s)
-            if (ws[2 * (s * G + h) + 1] > 0.f) M = fmaxf(M, ws[2 * (s * G + h)]);
-        float L = 0.f;
-        for (int s = 0; s < ns; ++s) {
-            const float l = ws[2 * (s * G + h) + 1];
-            if (l > 0.f) L = fmaf(l, expf(ws[2 * (s * G + h)] - M), L);
-        }
-        for (int s = 0; s < ns; ++s) {
-            const float l = ws[2 * (s * G + h) + 1];
-            ws[2 * (s * G + h)] = l > 0.f ? expf(ws[2 * (s * G + h)] - M) / L : 0.f;
-        }
-    }
-    __syncthreads();
-    // outputs: thread t takes dim t % 128 of heads t / 128, t / 128 + R, ... (R = 3 rounds
-    // of 128 threads); the accumulator loads of a batch of splits are issued together
-    constexpr int R = 3;
-    if (tid >= R * HD) return;
-    const int d = tid % HD;
-    for (int h = tid / HD; h < G; h += R) {
-        float o = 0.f;
-        for (int s0 = 0; s0 < ns; s0 += 16) {
-            float v[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                v[k] = s0 + k < ns ? __ldcg(base + (size_t)((s0 + k) * G + h) * kPartFloats + 4 + d) : 0.f;
-#pragma unroll
-            for (int k = 0; k < 16; ++k)
-                if (s0 + k < ns) o = fmaf(ws[2 * ((s0 + k) * G + h)], v[k], o);
-        }
-        a.out[(size_t)(g * G + h) * HD + d] = o;
-    }
 }
 
 template <int G>
@@ -484,23 +428,53 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
         }
     }
 
-    // ---------------------------------------------------------------- merge
-    // Every split's partial is in the workspace once its CTA has arrived; the CTA that
-    // takes the last ticket of its kv head merges all of them (its own ring is free now:
-    // every copy it issued has been consumed).
-    __threadfence();
-    __syncthreads();
-    int* flag = reinterpret_cast<int*>(sm + kOffWSum);
-    if (tid == 0) {
-        const unsigned ticket = atomicAdd(&a.counters[g], 1u);
-        const int last = ticket == (unsigned)(a.n_split - 1);
-        if (last) a.counters[g] = 0u;   // every split of this head has arrived: ready for the next launch
-        __threadfence();
-        *flag = last;
+}
+
+// Merge of the splits, one CTA per query head and one thread per dim: with
+// M = max_s m_s over splits that saw a position, w_s = e^(m_s - M) and
+// L = sum_s l_s w_s, out[d] = (sum_s w_s acc_s[d]) / L.  Each thread reads every
+// split's (m, l) (the same addresses across the CTA) and its dim of every split's
+// accumulator, 32 splits per round of loads, and merges the rounds online (the
+// running sums rescaled when the maximum grows), so one round trip to L2 serves up
+// to 32 splits and no barrier is needed.
+template <int G>
+__global__ void __launch_bounds__(HD) attn_merge_kernel(const float* part, float* out, int n_split, int use_pdl)
+{
+    constexpr int B = 32;   // splits whose records are loaded together
+    if (use_pdl) {
+        pdl_launch_dependents();
+        pdl_wait();
     }
-    __syncthreads();
-    if (!*flag) return;
-    merge_splits<G>(a, g, reinterpret_cast<float*>(ring));
+    const int qh = blockIdx.x, g = qh / G, h = qh % G, d = threadIdx.x;
+    const size_t rec = (size_t)G * kPartFloats;   // floats from one split's record of this head to the next
+    const float* base = part + ((size_t)g * n_split * G + h) * kPartFloats;
+    float M = -INFINITY, L = 0.f, o = 0.f;
+    for (int s0 = 0; s0 < n_split; s0 += B) {
+        float2 ml[B];
+        float v[B];
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+            const bool ok = s0 + k < n_split;
+            ml[k] = ok ? __ldcg(reinterpret_cast<const float2*>(base + (s0 + k) * rec)) : make_float2(0.f, 0.f);
+            v[k] = ok ? __ldcg(base + (s0 + k) * rec + 4 + d) : 0.f;
+        }
+        float Mb = M;
+#pragma unroll
+        for (int k = 0; k < B; ++k)
+            if (ml[k].y > 0.f) Mb = fmaxf(Mb, ml[k].x);
+        if (Mb == -INFINITY) continue;   // no split of this round saw a position
+        const float r = M == -INFINITY ? 0.f : expf(M - Mb);
+        L *= r;
+        o *= r;
+#pragma unroll
+        for (int k = 0; k < B; ++k) {
+            const float w = ml[k].y > 0.f ? expf(ml[k].x - Mb) : 0.f;
+            L = fmaf(ml[k].y, w, L);
+            o = fmaf(w, v[k], o);
+        }
+        M = Mb;
+    }
+    out[(size_t)qh * HD + d] = o / L;
 }
 
 template <int G>
@@ -519,8 +493,17 @@ ntx_status launch_g(const KArgs& k, int n_q_heads, cudaStream_t s, bool pdl)
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G>, k);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, attn_kernel<G>, k);
     if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("attention launch: ") + cudaGetErrorString(e));
+    // the merge always waits for the split kernel through the programmatic dependency
+    cudaLaunchConfig_t mc = {};
+    mc.gridDim = dim3(n_q_heads);
+    mc.blockDim = dim3(HD);
+    mc.stream = s;
+    mc.attrs = attr;
+    mc.numAttrs = 1;
+    e = cudaLaunchKernelEx(&mc, attn_merge_kernel<G>, (const float*)k.part, k.out, k.n_split, 1);
+    if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("attention merge launch: ") + cudaGetErrorString(e));
     return NTX_OK;
 }
 
@@ -572,10 +555,8 @@ size_t attn_workspace_bytes_for(int n_q_heads, int n_kv_heads, int head_dim, int
 {
     (void)head_dim;
     const int G = n_q_heads / n_kv_heads;
-    return kCounterBytes + (size_t)n_kv_heads * n_split * G * kPartFloats * sizeof(float);
+    return (size_t)n_kv_heads * n_split * G * kPartFloats * sizeof(float);
 }
-
-size_t attn_counter_bytes() { return kCounterBytes; }
 
 ntx_status attn_launch(const AttnArgs& a, cudaStream_t s)
 {
@@ -588,8 +569,7 @@ ntx_status attn_launch(const AttnArgs& a, cudaStream_t s)
     if ((st = encode_kv_map(&k.tv, a.v_cache, a.n_kv_heads, a.max_ctx)) != NTX_OK) return st;
     k.q = a.q;
     k.out = a.out;
-    k.counters = reinterpret_cast<unsigned*>(a.workspace);
-    k.part = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a.workspace) + kCounterBytes);
+    k.part = reinterpret_cast<float*>(a.workspace);
     k.max_ctx = a.max_ctx;
     k.n_split = a.n_split;
     k.n_ctx = a.n_ctx;
@@ -662,8 +642,5 @@ NTX_EXPORT ntx_status ntx_attn_decode(const float* q, const void* k_cache, const
     a.workspace = workspace;
     a.n_split = n_split;
     a.pdl = false;
-    // the merge tickets start from zero (each launch leaves them at zero; clearing them here
-    // also covers a workspace that was never used or a launch that did not finish)
-    NTX_CUDA_TRY(cudaMemsetAsync(workspace, 0, kCounterBytes, (cudaStream_t)stream));
     return attn_launch(a, (cudaStream_t)stream);
 }

@@ -60,9 +60,8 @@ NTX_EXPORT ntx_status ntx_attn_decode_noalloc(const float* q, const void* k_cach
     void* ws = nullptr;
     if ((st = static_scratch(&ws)) != NTX_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
-    // the merge tickets at the start of the scratch must start from zero (every launch
-    // leaves them at zero; clearing them also covers a launch that did not finish); the
-    // split partials after them are all written before the merge reads them
+    // nothing in the scratch carries over between calls: every split's partial is
+    // written before the merge reads it, so it needs no clearing
     AttnArgs a{};
     a.q = q;
     a.k_cache = (const __half*)k_cache;
@@ -77,6 +76,5 @@ NTX_EXPORT ntx_status ntx_attn_decode_noalloc(const float* q, const void* k_cach
     a.workspace = ws;
     a.n_split = n_split;
     a.pdl = false;
-    NTX_CUDA_TRY(cudaMemsetAsync(ws, 0, attn_counter_bytes(), s));
     return attn_launch(a, s);
 }

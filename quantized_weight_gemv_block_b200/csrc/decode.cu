@@ -4,13 +4,14 @@
 // principales": host read, PCIe DMA and GPU compute overlapped with double
 // buffering; here pinned host memory -> a two-slot HBM ring on a copy stream).
 //
-// Per layer, five kernels:
+// Per layer, six kernels:
 //   1. fused QKV GEMV: RMSNorm(h) prologue, RoPE + fp16 K/V append epilogue
-//   2. split-context GQA attention; the last split of each kv head to finish merges
-//      the splits' partials (log-sum-exp rule, fixed order)
-//   3. O GEMV, residual add into h
-//   4. fused gate/up GEMV: RMSNorm(h) prologue, SwiGLU epilogue
-//   5. down GEMV, residual add into h
+//   2. split-context GQA attention, each split's partial (max, sum, accumulator)
+//      to a workspace
+//   3. merge of the splits (log-sum-exp rule, fixed order)
+//   4. O GEMV, residual add into h
+//   5. fused gate/up GEMV: RMSNorm(h) prologue, SwiGLU epilogue
+//   6. down GEMV, residual add into h
 // plus the step word / RoPE table kernel and the embedding before layer 0 and the
 // RMSNorm + LM-head GEMV after the last layer.  Kernels use programmatic dependent
 // launch so each one's weight stream starts while the previous one drains; the
@@ -23,6 +24,7 @@
 #include <vector>
 
 #include "ops.h"
+#include "ring.h"
 
 // Formats of one layer's matrices: QKV, O, gate and up, down.
 struct ntx_layer_qt {
@@ -33,7 +35,11 @@ struct ntx_model {
     ntx_model_desc d;
     std::vector<ntx_layer_desc> layers;
     std::vector<ntx_layer_qt> lqt;
+    std::vector<uint8_t> skip;   // layers the step leaves out (1), set by ntx_model_set_layer_skip
     int32_t qt_embd = 0, qt_out = 0;
+    float* h_prev = nullptr;     // calibration: h before the current layer
+    float* cos_dev = nullptr;    // calibration: cosine similarity per layer
+    bool calibrating = false;
     int device = 0;
     float* h = nullptr;
     float* q = nullptr;
@@ -151,6 +157,11 @@ ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, b
     const ntx_model_desc& d = m->d;
     const ntx_layer_desc& L = m->layers[l];
     ntx_status st;
+    if (m->calibrating) {
+        // h before the layer, for the similarity of its input and output
+        NTX_CUDA_TRY(cudaMemcpyAsync(m->h_prev, m->h, (size_t)d.hidden * 4, cudaMemcpyDeviceToDevice, s));
+        pdl = false;
+    }
     if ((st = launch_qkv(m, l, w.qkv, s, pdl)) != NTX_OK) return st;
     {
         AttnArgs a{};
@@ -170,7 +181,9 @@ ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, b
     }
     if ((st = launch_o(m, l, w.o, s, pdl)) != NTX_OK) return st;
     if ((st = launch_gate_up(m, l, w.gate, w.up, s, pdl)) != NTX_OK) return st;
-    return launch_down(m, l, w.down, s, pdl);
+    if ((st = launch_down(m, l, w.down, s, pdl)) != NTX_OK) return st;
+    if (m->calibrating) return cosine_launch(m->h_prev, m->h, d.hidden, m->cos_dev + l, s);
+    return NTX_OK;
 }
 
 ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
@@ -196,8 +209,10 @@ ntx_status enqueue_resident(ntx_model* m, int n, float* logits, cudaStream_t s, 
 {
     ntx_status st = embed_launch(m->qt_embd, m->d.tok_embd, m->d.hidden, m->step, m->h, s, m->pdl);
     if (st != NTX_OK) return st;
-    for (int l = 0; l < n; ++l)
+    for (int l = 0; l < n; ++l) {
+        if (m->skip[l] && !m->calibrating) continue;
         if ((st = enqueue_layer(m, l, resident_w(m->layers[l]), s, m->pdl)) != NTX_OK) return st;
+    }
     if (with_head) return enqueue_head(m, logits, s, m->pdl);
     return NTX_OK;
 }
@@ -283,6 +298,8 @@ void free_model(ntx_model* m)
     cudaFree(m->act);
     cudaFree(m->step);
     cudaFree(m->rope);
+    cudaFree(m->h_prev);
+    cudaFree(m->cos_dev);
     cudaFree(m->attn_ws);
     cudaFree(m->ring);
     delete m;
@@ -307,6 +324,7 @@ NTX_EXPORT ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** m
     m->layers.assign(desc->layers, desc->layers + desc->n_layers);
     m->d.layers = nullptr;
     m->d.tensor_qtypes = nullptr;
+    m->skip.assign(desc->n_layers, 0);
     m->qt_embd = tensor_qtype(desc, 0);
     m->qt_out = tensor_qtype(desc, 1);
     for (int l = 0; l < desc->n_layers; ++l) {
@@ -331,6 +349,8 @@ NTX_EXPORT ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** m
     alloc((void**)&m->act, (size_t)d.ffn * 4);
     alloc((void**)&m->step, 16);
     alloc((void**)&m->rope, (size_t)d.head_dim * 4);
+    alloc((void**)&m->h_prev, (size_t)d.hidden * 4);
+    alloc((void**)&m->cos_dev, (size_t)d.n_layers * 4);
     alloc(&m->attn_ws, ws);
     if (e == cudaSuccess) e = cudaMemset(m->attn_ws, 0, ws);
     if (e == cudaSuccess) e = cudaMemset(m->step, 0, 16);
@@ -384,8 +404,7 @@ NTX_EXPORT ntx_status ntx_decode_step(ntx_model* m, int32_t token, int32_t pos, 
     if (pos < 0 || pos >= m->d.max_ctx) return fail(NTX_EINVAL, "ntx_decode_step: pos out of range");
     if (!aligned(logits, 4)) return fail(NTX_EINVAL, "ntx_decode_step: logits must be 4-byte aligned");
     cudaStream_t s = (cudaStream_t)stream;
-    ntx_status st = set_step_launch(m->step, token, pos, m->rope, m->d.rope_theta, m->d.head_dim,
-                                    (unsigned*)m->attn_ws, m->d.n_kv_heads, s);
+    ntx_status st = set_step_launch(m->step, token, pos, m->rope, m->d.rope_theta, m->d.head_dim, s);
     if (st != NTX_OK) return st;
     if (!m->use_graph) return enqueue_resident(m, m->d.n_layers, logits, s, true);
     if (!m->graph || m->graph_logits != logits) {
@@ -421,6 +440,99 @@ NTX_EXPORT ntx_status ntx_decode_step(ntx_model* m, int32_t token, int32_t pos, 
     return NTX_OK;
 }
 
+namespace ntx {
+namespace {
+
+// The ring's operations on two CUDA streams: copies (cudaMemcpyAsync from the host
+// pointers of the layer descriptors) on `ks`, compute on `cs`, events between them.
+struct CudaRing final : ring::Ops {
+    ntx_model* m;
+    cudaStream_t cs, ks;
+    int64_t h2d = 0;
+    CudaRing(ntx_model* m_, cudaStream_t cs_, cudaStream_t ks_) : m(m_), cs(cs_), ks(ks_) {}
+
+    uint8_t* slot_base(int slot) const { return m->ring + (size_t)slot * m->slot_bytes; }
+
+    ntx_status copy_wait_slot(int slot) override
+    {
+        NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->slot_free[slot], 0));
+        return NTX_OK;
+    }
+    ntx_status copy_layer(int j, int slot) override
+    {
+        // this layer's own matrix sizes (its formats may differ from the largest the slot holds)
+        const ntx_model_desc& d = m->d;
+        const ntx_layer_desc& L = m->layers[j];
+        const ntx_layer_qt& q = m->lqt[j];
+        const int kvd = d.n_kv_heads * d.head_dim, qd = d.n_q_heads * d.head_dim;
+        const size_t b_qkv = (size_t)(qd + 2 * kvd) * row_bytes(q.qkv, d.hidden);
+        const size_t b_o = (size_t)d.hidden * row_bytes(q.o, qd);
+        const size_t b_ffn = (size_t)d.ffn * row_bytes(q.ffn, d.hidden);
+        const size_t b_down = (size_t)d.hidden * row_bytes(q.down, d.ffn);
+        uint8_t* base = slot_base(slot);
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_qkv, L.w_qkv, b_qkv, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_o, L.w_o, b_o, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_gate, L.w_gate, b_ffn, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_up, L.w_up, b_ffn, cudaMemcpyHostToDevice, ks));
+        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_down, L.w_down, b_down, cudaMemcpyHostToDevice, ks));
+        h2d += (int64_t)(b_qkv + b_o + 2 * b_ffn + b_down);
+        return NTX_OK;
+    }
+    ntx_status copy_done(int slot) override
+    {
+        NTX_CUDA_TRY(cudaEventRecord(m->copy_done[slot], ks));
+        return NTX_OK;
+    }
+    ntx_status compute_wait_copy(int slot) override
+    {
+        NTX_CUDA_TRY(cudaStreamWaitEvent(cs, m->copy_done[slot], 0));
+        return NTX_OK;
+    }
+    ntx_status compute_layer(int j, int slot) override
+    {
+        uint8_t* base = slot_base(slot);
+        const LayerW w{base + m->off_qkv, base + m->off_o, base + m->off_gate, base + m->off_up, base + m->off_down};
+        return enqueue_layer(m, j, w, cs, false);
+    }
+    ntx_status compute_done(int slot) override
+    {
+        NTX_CUDA_TRY(cudaEventRecord(m->slot_free[slot], cs));
+        return NTX_OK;
+    }
+    ntx_status before_streamed() override { return enqueue_resident(m, m->d.n_resident, nullptr, cs, false); }
+};
+
+}  // namespace
+}  // namespace ntx
+
+namespace ntx {
+namespace {
+
+// Queue one step of a partly resident model: resident layers and the streamed layers
+// through the ring; the head when logits is not null.
+ntx_status enqueue_streamed_step(ntx_model* m, int32_t token, int32_t pos, float* logits, cudaStream_t cs,
+                                 cudaStream_t ks)
+{
+    const ntx_model_desc& d = m->d;
+    NTX_CUDA_TRY(cudaEventRecord(m->ev_start, cs));
+    ntx_status st = set_step_launch(m->step, token, pos, m->rope, d.rope_theta, d.head_dim, cs);
+    if (st != NTX_OK) return st;
+    // the streamed layers that run (skipped layers are neither copied nor computed)
+    std::vector<int> streamed;
+    for (int j = d.n_resident; j < d.n_layers; ++j)
+        if (!m->skip[j] || m->calibrating) streamed.push_back(j);
+    if (!streamed.empty()) NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->ev_start, 0));
+    CudaRing ops(m, cs, ks);
+    if ((st = ring::schedule(ops, streamed.data(), (int)streamed.size(), 2)) != NTX_OK) return st;
+    if (logits && (st = enqueue_head(m, logits, cs, false)) != NTX_OK) return st;
+    NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
+    m->last_h2d = ops.h2d;
+    return NTX_OK;
+}
+
+}  // namespace
+}  // namespace ntx
+
 NTX_EXPORT ntx_status ntx_stream_layers(ntx_model* m, int32_t token, int32_t pos, float* logits, void* compute,
                                         void* copy, int64_t timeout_ms)
 {
@@ -428,68 +540,25 @@ NTX_EXPORT ntx_status ntx_stream_layers(ntx_model* m, int32_t token, int32_t pos
     if (token < 0 || token >= m->d.vocab) return fail(NTX_EINVAL, "ntx_stream_layers: token out of range");
     if (pos < 0 || pos >= m->d.max_ctx) return fail(NTX_EINVAL, "ntx_stream_layers: pos out of range");
     if (timeout_ms < 0) return fail(NTX_EINVAL, "ntx_stream_layers: timeout_ms must be >= 0");
+    if (!aligned(logits, 4)) return fail(NTX_EINVAL, "ntx_stream_layers: logits must be 4-byte aligned");
     if (compute == copy && m->d.n_resident < m->d.n_layers)
         return fail(NTX_EINVAL, "ntx_stream_layers: compute and copy streams must differ");
-    cudaStream_t cs = (cudaStream_t)compute, ks = (cudaStream_t)copy;
-    const ntx_model_desc& d = m->d;
-    const int nres = d.n_resident;
-    NTX_CUDA_TRY(cudaEventRecord(m->ev_start, cs));
-    ntx_status st = set_step_launch(m->step, token, pos, m->rope, d.rope_theta, d.head_dim, (unsigned*)m->attn_ws,
-                                    d.n_kv_heads, cs);
+    ntx_status st = enqueue_streamed_step(m, token, pos, logits, (cudaStream_t)compute, (cudaStream_t)copy);
     if (st != NTX_OK) return st;
-    int64_t h2d = 0;
-    // copies of streamed layer j into slot (j - nres) % 2; the slot is free once
-    // the compute of the layer that used it before has finished
-    auto enqueue_copy = [&](int j) -> ntx_status {
-        const int slot = (j - nres) & 1;
-        const ntx_layer_desc& L = m->layers[j];
-        uint8_t* base = m->ring + (size_t)slot * m->slot_bytes;
-        NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->slot_free[slot], 0));
-        // this layer's own matrix sizes (its formats may differ from the largest the slot holds)
-        const ntx_layer_qt& q = m->lqt[j];
-        const int kvd = d.n_kv_heads * d.head_dim, qd = d.n_q_heads * d.head_dim;
-        const size_t b_qkv = (size_t)(qd + 2 * kvd) * row_bytes(q.qkv, d.hidden);
-        const size_t b_o = (size_t)d.hidden * row_bytes(q.o, qd);
-        const size_t b_ffn = (size_t)d.ffn * row_bytes(q.ffn, d.hidden);
-        const size_t b_down = (size_t)d.hidden * row_bytes(q.down, d.ffn);
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_qkv, L.w_qkv, b_qkv, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_o, L.w_o, b_o, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_gate, L.w_gate, b_ffn, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_up, L.w_up, b_ffn, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaMemcpyAsync(base + m->off_down, L.w_down, b_down, cudaMemcpyHostToDevice, ks));
-        NTX_CUDA_TRY(cudaEventRecord(m->copy_done[slot], ks));
-        h2d += (int64_t)(b_qkv + b_o + 2 * b_ffn + b_down);
-        return NTX_OK;
-    };
-    if (nres < d.n_layers) {
-        NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->ev_start, 0));
-        for (int j = nres; j < std::min(d.n_layers, nres + 2); ++j)
-            if ((st = enqueue_copy(j)) != NTX_OK) return st;
-    }
-    if ((st = enqueue_resident(m, nres, logits, cs, false)) != NTX_OK) return st;
-    for (int j = nres; j < d.n_layers; ++j) {
-        const int slot = (j - nres) & 1;
-        uint8_t* base = m->ring + (size_t)slot * m->slot_bytes;
-        NTX_CUDA_TRY(cudaStreamWaitEvent(cs, m->copy_done[slot], 0));
-        const LayerW w{base + m->off_qkv, base + m->off_o, base + m->off_gate, base + m->off_up, base + m->off_down};
-        if ((st = enqueue_layer(m, j, w, cs, false)) != NTX_OK) return st;
-        NTX_CUDA_TRY(cudaEventRecord(m->slot_free[slot], cs));
-        if (j + 2 < d.n_layers)
-            if ((st = enqueue_copy(j + 2)) != NTX_OK) return st;
-    }
-    if ((st = enqueue_head(m, logits, cs, false)) != NTX_OK) return st;
-    NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
-    m->last_h2d = h2d;
     if (timeout_ms > 0) {
-        const auto deadline = std::chrono::steady_clock::now() + std::chrono::milliseconds(timeout_ms);
-        for (;;) {
-            cudaError_t q = cudaEventQuery(m->ev_end);
-            if (q == cudaSuccess) break;
-            if (q != cudaErrorNotReady) return fail(NTX_ECUDA, std::string("ntx_stream_layers: ") + cudaGetErrorString(q));
-            if (std::chrono::steady_clock::now() > deadline)
-                return fail(NTX_ETIMEOUT, "ntx_stream_layers: step not finished within timeout_ms (work stays queued)");
-            std::this_thread::sleep_for(std::chrono::microseconds(200));
-        }
+        cudaError_t qerr = cudaSuccess;
+        st = ring::wait_bounded(
+            [&]() -> ntx_status {
+                const cudaError_t q = cudaEventQuery(m->ev_end);
+                if (q == cudaSuccess) return NTX_OK;
+                if (q == cudaErrorNotReady) return NTX_ETIMEOUT;
+                qerr = q;
+                return NTX_ECUDA;
+            },
+            timeout_ms);
+        if (st == NTX_ETIMEOUT)
+            return fail(NTX_ETIMEOUT, "ntx_stream_layers: step not finished within timeout_ms (work stays queued)");
+        if (st != NTX_OK) return fail(st, std::string("ntx_stream_layers: ") + cudaGetErrorString(qerr));
     }
     return NTX_OK;
 }
@@ -529,4 +598,45 @@ NTX_EXPORT ntx_status ntx_model_replay_gemv(ntx_model* m, int kind, int n_launch
         }
     }
     return st;
+}
+
+NTX_EXPORT ntx_status ntx_model_set_layer_skip(ntx_model* m, const uint8_t* skip)
+{
+    if (!m) return fail(NTX_EINVAL, "ntx_model_set_layer_skip: null model");
+    for (int l = 0; l < m->d.n_layers; ++l) m->skip[l] = skip && skip[l] ? 1 : 0;
+    // the recorded step holds the old set of layers: record it again on the next call
+    if (m->graph) {
+        cudaGraphExecDestroy(m->graph);
+        m->graph = nullptr;
+    }
+    return NTX_OK;
+}
+
+NTX_EXPORT ntx_status ntx_model_layer_similarity(ntx_model* m, int32_t token, int32_t pos, float* cos_out,
+                                                 void* compute, void* copy)
+{
+    if (!m || !cos_out) return fail(NTX_EINVAL, "ntx_model_layer_similarity: null pointer");
+    if (token < 0 || token >= m->d.vocab) return fail(NTX_EINVAL, "ntx_model_layer_similarity: token out of range");
+    if (pos < 0 || pos >= m->d.max_ctx) return fail(NTX_EINVAL, "ntx_model_layer_similarity: pos out of range");
+    const bool streamed = m->d.n_resident < m->d.n_layers;
+    if (streamed && compute == copy)
+        return fail(NTX_EINVAL, "ntx_model_layer_similarity: compute and copy streams must differ");
+    cudaStream_t cs = (cudaStream_t)compute;
+    NTX_CUDA_TRY(cudaMemsetAsync(m->cos_dev, 0, (size_t)m->d.n_layers * 4, cs));
+    m->calibrating = true;
+    const bool pdl = m->pdl;
+    m->pdl = false;
+    ntx_status st;
+    if (streamed) {
+        st = enqueue_streamed_step(m, token, pos, nullptr, cs, (cudaStream_t)copy);
+    } else {
+        st = set_step_launch(m->step, token, pos, m->rope, m->d.rope_theta, m->d.head_dim, cs);
+        if (st == NTX_OK) st = enqueue_resident(m, m->d.n_layers, nullptr, cs, false);
+    }
+    m->calibrating = false;
+    m->pdl = pdl;
+    if (st != NTX_OK) return st;
+    NTX_CUDA_TRY(cudaMemcpyAsync(cos_out, m->cos_dev, (size_t)m->d.n_layers * 4, cudaMemcpyDeviceToHost, cs));
+    NTX_CUDA_TRY(cudaStreamSynchronize(cs));
+    return NTX_OK;
 }

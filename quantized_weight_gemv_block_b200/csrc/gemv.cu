@@ -199,7 +199,8 @@ NTX_EXPORT ntx_status ntx_dequant_q(int qtype, const void* W, int64_t rows, int6
 
 NTX_EXPORT ntx_status ntx_repack_q(int qtype, const void* W, void* W_tiled, int64_t rows, int64_t cols, void* stream)
 {
-    if (qtype < NTX_Q8_0 || qtype > NTX_Q6_K) return fail(NTX_EINVAL, "ntx_repack_q: qtype must be a GGUF-style format");
+    if (qtype < NTX_Q8_0 || qtype > NTX_Q5_K)
+        return fail(NTX_EINVAL, "ntx_repack_q: qtype must be a GGUF-style block format (F16 / F32 have no tiled form)");
     if (!W || !W_tiled) return fail(NTX_EINVAL, "ntx_repack_q: null pointer");
     if (rows < 1 || row_bytes(qtype | NTX_TILED, cols) == 0)
         return fail(NTX_EINVAL, "ntx_repack_q: cols must be a positive multiple of the tile size");

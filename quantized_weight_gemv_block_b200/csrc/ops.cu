@@ -140,18 +140,14 @@ __global__ void embed_kernel(const uint8_t* E, int64_t rb, int64_t hidden, const
 // The step word (token, position) and the RoPE table of the position: rope[2i] and
 // rope[2i + 1] = cos and sin of pos theta^(-2i/head_dim), computed in double, for
 // i < head_dim / 2 (the rotation of "RoPE" in the ntransformer news summary's kernel
-// list).  Later kernels of the step read both.  Also zeroes the attention's merge
-// tickets (each attention launch leaves them at zero; this covers a step that did not
-// finish).
-__global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
-                                unsigned* counters, int n_counters)
+// list).  Later kernels of the step read both.
+__global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim)
 {
     const int i = threadIdx.x;
     if (i == 0) {
         step[0] = token;
         step[1] = pos;
     }
-    for (int c = i; c < n_counters; c += blockDim.x) counters[c] = 0u;
     if (rope && i < head_dim / 2) {
         const double ang = (double)pos * pow((double)theta, -(2.0 * i) / (double)head_dim);
         double sn, cs;
@@ -161,7 +157,49 @@ __global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos, float
     }
 }
 
+// Cosine similarity of two vectors, by one CTA (the similarity of a layer's input and
+// output hidden states, the measure the layer skip of "Rendimiento y estructura de
+// caché" in the ntransformer news summary ranks layers by); sums in double.
+__global__ void cosine_kernel(const float* a, const float* b, int64_t n, float* out)
+{
+    __shared__ double red[3][32];
+    double ab = 0.0, aa = 0.0, bb = 0.0;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const double x = a[i], y = b[i];
+        ab += x * y;
+        aa += x * x;
+        bb += y * y;
+    }
+    for (int o = 16; o > 0; o >>= 1) {
+        ab += __shfl_xor_sync(0xffffffffu, ab, o);
+        aa += __shfl_xor_sync(0xffffffffu, aa, o);
+        bb += __shfl_xor_sync(0xffffffffu, bb, o);
+    }
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        red[0][w] = ab;
+        red[1][w] = aa;
+        red[2][w] = bb;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0;
+        for (int k = 0; k < (int)(blockDim.x >> 5); ++k) {
+            s0 += red[0][k];
+            s1 += red[1][k];
+            s2 += red[2][k];
+        }
+        *out = (s1 > 0.0 && s2 > 0.0) ? (float)(s0 / sqrt(s1 * s2)) : 0.f;
+    }
+}
+
 }  // namespace
+
+ntx_status cosine_launch(const float* a, const float* b, int64_t n, float* out, cudaStream_t s)
+{
+    cosine_kernel<<<1, 1024, 0, s>>>(a, b, n, out);
+    return check_launch("cosine similarity");
+}
 
 ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t* token_dev, float* h, cudaStream_t s,
                         bool pdl)
@@ -200,10 +238,9 @@ ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t*
 }
 
 ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
-                           unsigned* counters, int n_counters, cudaStream_t s)
+                           cudaStream_t s)
 {
-    set_step_kernel<<<1, std::max(32, head_dim / 2), 0, s>>>(step, token, pos, rope, theta, head_dim, counters,
-                                                               counters ? n_counters : 0);
+    set_step_kernel<<<1, std::max(32, head_dim / 2), 0, s>>>(step, token, pos, rope, theta, head_dim);
     return check_launch("step counter");
 }
 

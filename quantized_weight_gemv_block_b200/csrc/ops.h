@@ -9,11 +9,12 @@ namespace ntx {
 ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t* token_dev, float* h, cudaStream_t s,
                         bool pdl);
 // Writes the step word (token, pos) and, if rope is not null, the RoPE table of pos
-// ([head_dim / 2][cos, sin] floats) for the kernels of the step, and zeroes the
-// attention's merge tickets (`counters`, n_counters words; may be null).
+// ([head_dim / 2][cos, sin] floats) for the kernels of the step.
 ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
-                           unsigned* counters, int n_counters, cudaStream_t s);
+                           cudaStream_t s);
 ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
+// *out = a . b / (|a| |b|) for device fp32 vectors of n <= 2^26 elements (0 if either is zero).
+ntx_status cosine_launch(const float* a, const float* b, int64_t n, float* out, cudaStream_t s);
 ntx_status qmma_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
 // F16 / F32 weights (fgemv.cu): the streaming kernel needs W and x 16-byte aligned,
 // rows that are 16-byte multiples and at most 32768 columns.
@@ -31,8 +32,7 @@ struct AttnArgs {
     int n_q_heads, n_kv_heads, head_dim, max_ctx;
     int32_t n_ctx;              // used when n_ctx_from_pos is null
     const int32_t* pos_dev;     // if set: n_ctx = *pos_dev + 1 (read on the device)
-    void* workspace;            // merge tickets (attn_counter_bytes(), zero before the launch), then the
-                                // split partials
+    void* workspace;            // split partials (no initialisation needed)
     int n_split;                // CTAs per kv head
     bool pdl;
 };
@@ -40,7 +40,6 @@ ntx_status attn_check(const void* q, const void* k_cache, const void* v_cache, c
                       int n_kv_heads, int head_dim, int32_t n_ctx, int32_t max_ctx, const char* who);
 int attn_split_for(int n_q_heads, int n_kv_heads, int32_t max_ctx);
 size_t attn_workspace_bytes_for(int n_q_heads, int n_kv_heads, int head_dim, int n_split);
-size_t attn_counter_bytes();
 ntx_status attn_launch(const AttnArgs& a, cudaStream_t s);
 
 }  // namespace ntx

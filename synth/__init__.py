@@ -277,6 +277,8 @@ class ModelSpec:
     seed: int = 0
     tiled: bool = False       # weights handed to the library in the tiled layout (same bytes, regrouped)
     mix: str | None = None    # per-tensor formats: None (every tensor in qtype) or "q4_k_m" (below)
+    # extra["quiet_layers"]: layers whose O and down projections are scaled by 2^-10 (their
+    # output barely changes the hidden state: a planted candidate for the layer skip)
     extra: dict = field(default_factory=dict)
 
     def qtype_of(self, kind: str, layer: int = GLOBAL_LAYER) -> int:
@@ -332,7 +334,11 @@ class ModelSpec:
                   "w_up": (f, h, h),
                   "w_down": (h, f, f)}
         rows, cols, k = shapes[kind]
-        return rows, cols, decode_qparams(q, k), q
+        qp = decode_qparams(q, k)
+        if kind in ("w_o", "w_down") and layer in self.extra.get("quiet_layers", ()):
+            # a near-identity layer: its two residual contributions scaled by 2^-10
+            qp = QParams(qp.d_lo, qp.d_hi, qp.d_exp - 10, qp.mode)
+        return rows, cols, qp, q
 
 
 LLAMA_8B_Q8_0 = dict(n_layers=32, hidden=4096, n_q_heads=32, n_kv_heads=8, head_dim=128, ffn=14336,

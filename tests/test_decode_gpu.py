@@ -224,3 +224,53 @@ def test_streamed_mixed_formats_against_oracle(ntx, syn):
     spec = syn.ModelSpec(**dict(syn.LLAMA_70B_Q4_K_M, n_layers=4, vocab=4000, max_ctx=600, n_prefill=512),
                          tiled=True)
     compare_full(ntx, spec, "llama70b q4_k_m tiled, 2 of 4 layers streamed", n_resident=2)
+
+
+def test_layer_skip_by_similarity(ntx, syn):
+    """The layer skip: per-layer cosine similarity of the hidden state before and after
+    each layer matches the oracle's; a planted near-identity layer has the highest
+    similarity; skipping it gives the oracle's logits with that layer left out, and
+    clearing the mask gives the full model's again."""
+    from oracle import model as om
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, 0, n_layers=4, tiled=True, extra={"quiet_layers": [2]})
+    m = DeviceModel(spec)
+    token, pos = spec.token(), spec.n_prefill
+    cos = ntx.ntx_model_layer_similarity(m.handle, token, pos, spec.n_layers)
+    want = om.layer_similarity(spec)
+    print("layer similarity gpu", [round(c, 6) for c in cos], "oracle", [round(c, 6) for c in want])
+    assert np.max(np.abs(np.array(cos) - np.array(want))) <= 1e-4
+    assert int(np.argmax(cos)) == 2 and cos[2] > 0.999
+    m.reset_caches()
+    ntx.ntx_model_set_layer_skip(m.handle, [0, 0, 1, 0])
+    got = run_decode(ntx, m, token, pos)
+    ref, _ = om.decode(spec, skip={2})
+    assert rel_err(got, ref) <= TOL and elem_err(got, ref) <= TOL
+    m.reset_caches()
+    ntx.ntx_model_set_layer_skip(m.handle, None)
+    full = run_decode(ntx, m, token, pos)
+    m.close()
+    want_full, _ = om.decode(spec)
+    assert rel_err(full, want_full) <= TOL
+
+
+def test_layer_skip_streamed_layers_are_not_copied(ntx, syn):
+    """A skipped streamed layer is neither copied nor computed: the step copies one layer
+    fewer and still matches the oracle with that layer left out."""
+    from oracle import model as om
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, 2, n_layers=4, tiled=True, extra={"quiet_layers": [3]})
+    m = DeviceModel(spec, n_resident=2)
+    token, pos = spec.token(), spec.n_prefill
+    cs, ks = torch.cuda.Stream(), torch.cuda.Stream()
+    cos = ntx.ntx_model_layer_similarity(m.handle, token, pos, spec.n_layers, cs.cuda_stream, ks.cuda_stream)
+    assert int(np.argmax(cos)) == 3
+    m.reset_caches()
+    torch.cuda.synchronize()
+    ntx.ntx_model_set_layer_skip(m.handle, [0, 0, 0, 1])
+    got = run_decode(ntx, m, token, pos, stream_layers=True)
+    h2d, _ = ntx.ntx_stream_stats(m.handle)
+    m.close()
+    assert h2d == spec.layer_weight_bytes(2)
+    ref, _ = om.decode(spec, skip={3})
+    assert rel_err(got, ref) <= TOL and elem_err(got, ref) <= TOL
