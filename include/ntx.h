@@ -277,6 +277,30 @@ typedef struct ntx_model_desc {
 
 typedef struct ntx_model ntx_model;
 
+/* Automatic tier split ("Rendimiento y estructura de caché": as many layers as fit stay
+ * in VRAM, the rest are streamed from host memory each token).  From the descriptor's
+ * shapes and formats alone (no pointer is read; it may be a planning copy with null
+ * pointers), the largest n_resident such that everything the model keeps in HBM fits
+ * in hbm_budget bytes: the embedding and LM-head matrices, the norm weights, the KV
+ * caches of every layer, the matrices of layers [0, n_resident), the two-slot ring for
+ * the others (when n_resident < n_layers: each slot holds the largest of each matrix
+ * over the streamed layers), and the model's own scratch.  *hbm_used receives that
+ * total (may be NULL).  NTX_ENOMEM if even n_resident = 0 does not fit.  Host only: it
+ * launches nothing.  Place layers [0, *n_resident) in device memory and the others in
+ * host memory, and set desc.n_resident to it. */
+ntx_status ntx_plan_resident(const ntx_model_desc* desc, size_t hbm_budget, int32_t* n_resident, size_t* hbm_used);
+
+/* How the streamed layers' matrices are copied (decided by ntx_model_create, the data-path
+ * selection of "Funciones principales"): page-locked host memory is copied by DMA as it
+ * is; other host memory is page-locked in place (cudaHostRegister, undone by
+ * ntx_model_destroy) unless the environment variable NTX_NO_HOST_REGISTER is set or the
+ * system refuses, and is otherwise copied from pageable memory (the driver stages each
+ * copy and the host waits for it, so copy and compute overlap less).  The model's path is
+ * the slowest any streamed matrix takes.  Streamed matrices in device memory are
+ * rejected by ntx_model_create. */
+enum { NTX_HOST_PATH_NONE = 0, NTX_HOST_PATH_PINNED = 1, NTX_HOST_PATH_REGISTERED = 2, NTX_HOST_PATH_PAGEABLE = 3 };
+ntx_status ntx_model_host_path(ntx_model* model, int32_t* path);
+
 /* Validate the descriptor and allocate the model's scratch (activations,
  * attention partials, and the HBM ring when n_resident < n_layers).  The model
  * must be used on the device that was current at creation. */

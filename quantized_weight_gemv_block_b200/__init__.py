@@ -18,6 +18,7 @@ NTX_Q8_0, NTX_Q4_0, NTX_Q4_K, NTX_Q6_K, NTX_Q5_K, NTX_F16, NTX_F32 = range(7)
 NTX_TILED = 16
 NTX_Q8_0_T, NTX_Q4_0_T, NTX_Q4_K_T, NTX_Q6_K_T, NTX_Q5_K_T = 16, 17, 18, 19, 20
 NTX_GEMV_QKV, NTX_GEMV_O, NTX_GEMV_GATE_UP, NTX_GEMV_DOWN, NTX_GEMV_HEAD = range(5)
+NTX_HOST_PATH_NONE, NTX_HOST_PATH_PINNED, NTX_HOST_PATH_REGISTERED, NTX_HOST_PATH_PAGEABLE = range(4)
 STATUS_NAMES = {0: "NTX_OK", 1: "NTX_EINVAL", 2: "NTX_EUNSUPPORTED", 3: "NTX_ENOMEM", 4: "NTX_ECUDA",
                 5: "NTX_ETIMEOUT"}
 
@@ -27,7 +28,7 @@ EXPORTS = ("ntx_last_error", "ntx_version", "ntx_row_bytes", "ntx_block_elems", 
            "ntx_dequant_q", "ntx_repack_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_decode_noalloc", "ntx_attn_workspace_bytes", "ntx_swiglu",
            "ntx_softmax", "ntx_argmax", "ntx_embed", "ntx_model_create", "ntx_model_destroy", "ntx_decode_step",
            "ntx_stream_layers", "ntx_stream_stats", "ntx_model_replay_gemv", "ntx_model_layer_similarity",
-           "ntx_model_set_layer_skip")
+           "ntx_model_set_layer_skip", "ntx_plan_resident", "ntx_model_host_path")
 
 
 class NtxError(RuntimeError):
@@ -90,6 +91,8 @@ def lib() -> ctypes.CDLL:
             "ntx_model_replay_gemv": ([vp, ci, ci, vp, vp], ci),
             "ntx_model_layer_similarity": ([vp, i32, i32, ctypes.POINTER(cf), vp, vp], ci),
             "ntx_model_set_layer_skip": ([vp, ctypes.POINTER(ctypes.c_uint8)], ci),
+            "ntx_plan_resident": ([ctypes.POINTER(ModelDesc), sz, ctypes.POINTER(i32), ctypes.POINTER(sz)], ci),
+            "ntx_model_host_path": ([vp, ctypes.POINTER(i32)], ci),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -242,3 +245,17 @@ def ntx_model_set_layer_skip(model: int, skip) -> None:
         return
     arr = (ctypes.c_uint8 * len(skip))(*[1 if v else 0 for v in skip])
     check(lib().ntx_model_set_layer_skip(model, arr))
+
+
+def ntx_plan_resident(desc: ModelDesc, hbm_budget: int):
+    """(n_resident, hbm_bytes): the most leading layers that fit in hbm_budget bytes of HBM."""
+    n = ctypes.c_int32(0)
+    used = ctypes.c_size_t(0)
+    check(lib().ntx_plan_resident(ctypes.byref(desc), hbm_budget, ctypes.byref(n), ctypes.byref(used)))
+    return n.value, used.value
+
+
+def ntx_model_host_path(model: int) -> int:
+    p = ctypes.c_int32(0)
+    check(lib().ntx_model_host_path(model, ctypes.byref(p)))
+    return p.value

@@ -40,6 +40,8 @@ struct ntx_model {
     float* h_prev = nullptr;     // calibration: h before the current layer
     float* cos_dev = nullptr;    // calibration: cosine similarity per layer
     bool calibrating = false;
+    int32_t host_path = NTX_HOST_PATH_NONE;   // how streamed layers leave host memory
+    std::vector<void*> registered;            // host ranges this library registered (unregistered at destroy)
     int device = 0;
     float* h = nullptr;
     float* q = nullptr;
@@ -237,7 +239,61 @@ ntx_status check_matrix_format(int32_t qt, int64_t cols, const char* what)
     return NTX_OK;
 }
 
-ntx_status check_desc(const ntx_model_desc* d)
+// How the streamed layers' matrices leave host memory ("Funciones principales" of the
+// ntransformer news summary picks the data path by what the system offers): page-locked
+// memory is copied by DMA directly (NTX_HOST_PATH_PINNED); other host memory is
+// page-locked in place with cudaHostRegister (NTX_HOST_PATH_REGISTERED; undone at
+// destroy); if that is refused, or NTX_NO_HOST_REGISTER is set, the copies go from
+// pageable memory (NTX_HOST_PATH_PAGEABLE: the driver stages them, the host waits for
+// each).  The model's path is the slowest one any streamed matrix takes.
+ntx_status choose_host_path(ntx_model* m)
+{
+    const ntx_model_desc& d = m->d;
+    const char* no_reg = std::getenv("NTX_NO_HOST_REGISTER");
+    const bool may_register = !(no_reg && no_reg[0] && no_reg[0] != '0');
+    int path = NTX_HOST_PATH_PINNED;
+    for (int l = d.n_resident; l < d.n_layers; ++l) {
+        size_t b[5];
+        const ntx_layer_qt& q = m->lqt[l];
+        const int qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim;
+        b[0] = (size_t)(qd + 2 * kvd) * row_bytes(q.qkv, d.hidden);
+        b[1] = (size_t)d.hidden * row_bytes(q.o, qd);
+        b[2] = b[3] = (size_t)d.ffn * row_bytes(q.ffn, d.hidden);
+        b[4] = (size_t)d.hidden * row_bytes(q.down, d.ffn);
+        const ntx_layer_desc& L = m->layers[l];
+        const void* ptrs[5] = {L.w_qkv, L.w_o, L.w_gate, L.w_up, L.w_down};
+        for (int k = 0; k < 5; ++k) {
+            cudaPointerAttributes a{};
+            const cudaError_t e = cudaPointerGetAttributes(&a, ptrs[k]);
+            if (e != cudaSuccess) cudaGetLastError();
+            const cudaMemoryType t = e == cudaSuccess ? a.type : cudaMemoryTypeUnregistered;
+            if (t == cudaMemoryTypeDevice || t == cudaMemoryTypeManaged)
+                return fail(NTX_EINVAL, "ntx_model_create: streamed layer " + std::to_string(l) +
+                                            " has a matrix in device memory (streamed matrices live in host memory)");
+            if (t == cudaMemoryTypeHost) continue;
+            bool ok = false;
+            if (may_register) {
+                ok = cudaHostRegister(const_cast<void*>(ptrs[k]), b[k], cudaHostRegisterReadOnly) == cudaSuccess;
+                if (!ok) {
+                    cudaGetLastError();
+                    ok = cudaHostRegister(const_cast<void*>(ptrs[k]), b[k], cudaHostRegisterDefault) == cudaSuccess;
+                    if (!ok) cudaGetLastError();
+                }
+            }
+            if (ok) {
+                m->registered.push_back(const_cast<void*>(ptrs[k]));
+                path = std::max(path, (int)NTX_HOST_PATH_REGISTERED);
+            } else {
+                path = NTX_HOST_PATH_PAGEABLE;
+            }
+        }
+    }
+    m->host_path = path;
+    return NTX_OK;
+}
+
+// Shapes and formats of the descriptor (no pointer is looked at).
+ntx_status check_shapes(const ntx_model_desc* d)
 {
     if (!d) return fail(NTX_EINVAL, "model: null descriptor");
     if (qtraits(d->qtype).block_elems == 0) return fail(NTX_EINVAL, "model: unknown qtype");
@@ -251,7 +307,6 @@ ntx_status check_desc(const ntx_model_desc* d)
     if (d->max_ctx < 1) return fail(NTX_EINVAL, "model: max_ctx must be >= 1");
     if (!(d->rms_eps >= 0.f) || !(d->rope_theta > 0.f)) return fail(NTX_EINVAL, "model: bad eps / theta");
     if (d->n_resident < 0 || d->n_resident > d->n_layers) return fail(NTX_EINVAL, "model: n_resident out of range");
-    if (!d->tok_embd || !d->out_norm || !d->output || !d->layers) return fail(NTX_EINVAL, "model: null pointer");
     const int qd = d->n_q_heads * d->head_dim;
     for (int64_t k : {(int64_t)d->hidden, (int64_t)qd, (int64_t)d->ffn})
         if (k > 32768) return fail(NTX_EUNSUPPORTED, "model: row length above 32768");
@@ -268,6 +323,14 @@ ntx_status check_desc(const ntx_model_desc* d)
             (st = check_matrix_format(tensor_qtype(d, b + 3), d->ffn, "w_down")) != NTX_OK)
             return st;
     }
+    return NTX_OK;
+}
+
+ntx_status check_desc(const ntx_model_desc* d)
+{
+    ntx_status st = check_shapes(d);
+    if (st != NTX_OK) return st;
+    if (!d->tok_embd || !d->out_norm || !d->output || !d->layers) return fail(NTX_EINVAL, "model: null pointer");
     if (!aligned(d->tok_embd, 16) || !aligned(d->output, 16) || !aligned(d->out_norm, 16))
         return fail(NTX_EINVAL, "model: tensors must be 16-byte aligned");
     for (int l = 0; l < d->n_layers; ++l) {
@@ -282,9 +345,61 @@ ntx_status check_desc(const ntx_model_desc* d)
     return NTX_OK;
 }
 
+// Bytes of the five packed matrices of layer l, matrix by matrix (QKV, O, gate, up, down).
+void layer_matrix_bytes(const ntx_model_desc* d, int l, size_t (&b)[5])
+{
+    const int qd = d->n_q_heads * d->head_dim, kvd = d->n_kv_heads * d->head_dim, t = 2 + 4 * l;
+    b[0] = (size_t)(qd + 2 * kvd) * row_bytes(tensor_qtype(d, t), d->hidden);
+    b[1] = (size_t)d->hidden * row_bytes(tensor_qtype(d, t + 1), qd);
+    b[2] = b[3] = (size_t)d->ffn * row_bytes(tensor_qtype(d, t + 2), d->hidden);
+    b[4] = (size_t)d->hidden * row_bytes(tensor_qtype(d, t + 3), d->ffn);
+}
+
+// Bytes of the HBM ring for layers [n_resident, n_layers): two slots, each holding the
+// largest of every matrix over those layers (256-byte aligned).
+size_t ring_bytes(const ntx_model_desc* d, int n_resident)
+{
+    if (n_resident >= d->n_layers) return 0;
+    size_t mx[5] = {0, 0, 0, 0, 0};
+    for (int l = n_resident; l < d->n_layers; ++l) {
+        size_t b[5];
+        layer_matrix_bytes(d, l, b);
+        for (int k = 0; k < 5; ++k) mx[k] = std::max(mx[k], b[k]);
+    }
+    size_t slot = 0;
+    for (int k = 0; k < 5; ++k) slot += align256(mx[k]);
+    return 2 * slot;
+}
+
+// Device memory the model itself allocates, besides the ring.
+size_t scratch_bytes(const ntx_model_desc* d)
+{
+    const int qd = d->n_q_heads * d->head_dim;
+    const size_t ws = attn_workspace_bytes_for(d->n_q_heads, d->n_kv_heads, d->head_dim,
+                                               attn_split_for(d->n_q_heads, d->n_kv_heads, d->max_ctx));
+    return (size_t)4 * (2 * d->hidden + 2 * qd + d->ffn + d->head_dim + d->n_layers) + 16 + ws;
+}
+
+// Everything in HBM with the first n layers resident: embedding and LM-head matrices, norm
+// weights, every layer's KV cache, the resident layers' matrices, the ring, the scratch.
+size_t hbm_bytes_for(const ntx_model_desc* d, int n)
+{
+    size_t total = (size_t)d->vocab * row_bytes(tensor_qtype(d, 0), d->hidden) +
+                   (size_t)d->vocab * row_bytes(tensor_qtype(d, 1), d->hidden);
+    total += (size_t)(2 * d->n_layers + 1) * d->hidden * 4;
+    total += (size_t)d->n_layers * 2 * d->n_kv_heads * d->max_ctx * d->head_dim * 2;
+    for (int l = 0; l < n; ++l) {
+        size_t b[5];
+        layer_matrix_bytes(d, l, b);
+        total += b[0] + b[1] + b[2] + b[3] + b[4];
+    }
+    return total + ring_bytes(d, n) + scratch_bytes(d);
+}
+
 void free_model(ntx_model* m)
 {
     if (!m) return;
+    for (void* p : m->registered) cudaHostUnregister(p);
     if (m->graph) cudaGraphExecDestroy(m->graph);
     for (int i = 0; i < 2; ++i) {
         if (m->copy_done[i]) cudaEventDestroy(m->copy_done[i]);
@@ -355,6 +470,11 @@ NTX_EXPORT ntx_status ntx_model_create(const ntx_model_desc* desc, ntx_model** m
     if (e == cudaSuccess) e = cudaMemset(m->attn_ws, 0, ws);
     if (e == cudaSuccess) e = cudaMemset(m->step, 0, 16);
     if (e == cudaSuccess && d.n_resident < d.n_layers) {
+        st = choose_host_path(m);
+        if (st != NTX_OK) {
+            free_model(m);
+            return st;
+        }
         const int kvd = d.n_kv_heads * d.head_dim;
         // ring slots sized for the largest of each matrix over the streamed layers
         for (int l = d.n_resident; l < d.n_layers; ++l) {
@@ -638,5 +758,39 @@ NTX_EXPORT ntx_status ntx_model_layer_similarity(ntx_model* m, int32_t token, in
     if (st != NTX_OK) return st;
     NTX_CUDA_TRY(cudaMemcpyAsync(cos_out, m->cos_dev, (size_t)m->d.n_layers * 4, cudaMemcpyDeviceToHost, cs));
     NTX_CUDA_TRY(cudaStreamSynchronize(cs));
+    return NTX_OK;
+}
+
+NTX_EXPORT ntx_status ntx_plan_resident(const ntx_model_desc* desc, size_t hbm_budget, int32_t* n_resident,
+                                        size_t* hbm_used)
+{
+    if (!n_resident) return fail(NTX_EINVAL, "ntx_plan_resident: null output pointer");
+    *n_resident = 0;
+    if (hbm_used) *hbm_used = 0;
+    const ntx_status st = check_shapes(desc);
+    if (st != NTX_OK) return st;
+    // the HBM need grows with n (each resident layer adds its matrices, the ring shrinks by
+    // at most one layer's worth): take the largest n that fits
+    int best = -1;
+    size_t used = 0;
+    for (int n = 0; n <= desc->n_layers; ++n) {
+        const size_t b = hbm_bytes_for(desc, n);
+        if (b <= hbm_budget) {
+            best = n;
+            used = b;
+        }
+    }
+    if (best < 0)
+        return fail(NTX_ENOMEM, "ntx_plan_resident: even with every layer streamed the model needs " +
+                                    std::to_string(hbm_bytes_for(desc, 0)) + " bytes of HBM");
+    *n_resident = best;
+    if (hbm_used) *hbm_used = used;
+    return NTX_OK;
+}
+
+NTX_EXPORT ntx_status ntx_model_host_path(ntx_model* m, int32_t* path)
+{
+    if (!m || !path) return fail(NTX_EINVAL, "ntx_model_host_path: null pointer");
+    *path = m->host_path;
     return NTX_OK;
 }

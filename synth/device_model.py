@@ -11,7 +11,8 @@ from . import (GLOBAL_LAYER, NORM_W, BLOCK, ModelSpec, blocks_dev, normal_f16_de
                uniform_f32_dev)
 
 
-def _alloc_packed(spec: ModelSpec, kind: str, layer: int, device, host: bool = False) -> torch.Tensor:
+def _alloc_packed(spec: ModelSpec, kind: str, layer: int, device, host: bool = False,
+                  pinned: bool = True) -> torch.Tensor:
     rows, cols, qp, q = spec.packed(kind, layer)
     nbytes = rows * row_bytes(q, cols)
     t = torch.empty(nbytes, dtype=torch.uint8, device=device)
@@ -22,7 +23,7 @@ def _alloc_packed(spec: ModelSpec, kind: str, layer: int, device, host: bool = F
         ntx.ntx_repack_q(q, t, tt, rows, cols)
         t = tt
     if host:
-        h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=True)
+        h = torch.empty(nbytes, dtype=torch.uint8, pin_memory=pinned)
         h.copy_(t)
         return h
     return t
@@ -31,11 +32,13 @@ def _alloc_packed(spec: ModelSpec, kind: str, layer: int, device, host: bool = F
 class DeviceModel:
     """Tensors of a synthetic model and the ntx descriptor pointing at them.
 
-    Layers >= n_resident keep their five packed matrices in pinned host memory
-    (streamed through the ring); everything else lives in HBM.
+    Layers >= n_resident keep their five packed matrices in host memory (page-locked
+    unless host_pinned is False) and are streamed through the ring; everything else
+    lives in HBM.
     """
 
-    def __init__(self, spec: ModelSpec, n_resident: int | None = None, device="cuda", n_layers: int | None = None):
+    def __init__(self, spec: ModelSpec, n_resident: int | None = None, device="cuda", n_layers: int | None = None,
+                 host_pinned: bool = True):
         import quantized_weight_gemv_block_b200 as ntx
 
         self.spec = spec
@@ -49,7 +52,8 @@ class DeviceModel:
         self.layers = []
         for l in range(self.n_layers):
             host = l >= self.n_resident
-            t = {k: _alloc_packed(s, k, l, device, host=host) for k in ("w_qkv", "w_o", "w_gate", "w_up", "w_down")}
+            t = {k: _alloc_packed(s, k, l, device, host=host, pinned=host_pinned)
+                 for k in ("w_qkv", "w_o", "w_gate", "w_up", "w_down")}
             for k in ("attn_norm", "ffn_norm"):
                 t[k] = torch.empty(s.hidden, dtype=torch.float32, device=device)
                 uniform_f32_dev(t[k], s.seed, tensor_id(l, k), *NORM_W)

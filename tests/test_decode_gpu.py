@@ -274,3 +274,50 @@ def test_layer_skip_streamed_layers_are_not_copied(ntx, syn):
     assert h2d == spec.layer_weight_bytes(2)
     ref, _ = om.decode(spec, skip={3})
     assert rel_err(got, ref) <= TOL and elem_err(got, ref) <= TOL
+
+
+@pytest.mark.parametrize("register", [True, False], ids=["registered", "pageable"])
+def test_streamed_from_pageable_host_memory(ntx, syn, monkeypatch, register):
+    """Streamed layers in ordinary (pageable) host memory: the library page-locks them in
+    place (or, with NTX_NO_HOST_REGISTER, copies from pageable memory); either way the
+    logits equal those of the same model streamed from page-locked memory."""
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, 2, n_layers=4, tiled=True)
+    pinned = DeviceModel(spec, n_resident=2)
+    assert ntx.ntx_model_host_path(pinned.handle) == ntx.NTX_HOST_PATH_PINNED
+    want = run_decode(ntx, pinned, spec.token(), spec.n_prefill, stream_layers=True)
+    pinned.close()
+    if not register:
+        monkeypatch.setenv("NTX_NO_HOST_REGISTER", "1")
+    m = DeviceModel(spec, n_resident=2, host_pinned=False)
+    path = ntx.ntx_model_host_path(m.handle)
+    assert path == (ntx.NTX_HOST_PATH_REGISTERED if register else ntx.NTX_HOST_PATH_PAGEABLE), path
+    got = run_decode(ntx, m, spec.token(), spec.n_prefill, stream_layers=True)
+    m.close()
+    assert np.array_equal(got, want)
+
+
+def test_planned_split_runs(ntx, syn):
+    """A split chosen by ntx_plan_resident for a given HBM budget builds and decodes: the
+    budget that fits exactly two of four layers gives two resident layers, and the step
+    matches the oracle."""
+    from oracle import model as om
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, 2, n_layers=4, tiled=True)
+    probe = DeviceModel(spec, n_resident=4)
+    d = probe.desc
+    _, full = ntx.ntx_plan_resident(d, 1 << 62)
+    budget = None
+    for b in range(full, 0, -(1 << 20)):
+        n, used = ntx.ntx_plan_resident(d, b)
+        if n == 2:
+            budget = b
+            break
+    probe.close()
+    assert budget is not None
+    m = DeviceModel(spec, n_resident=ntx.ntx_plan_resident(d, budget)[0])
+    assert m.n_resident == 2
+    got = run_decode(ntx, m, spec.token(), spec.n_prefill, stream_layers=True)
+    m.close()
+    want, _ = om.decode(spec)
+    assert rel_err(got, want) <= TOL
