@@ -335,7 +335,37 @@ def run_decode_bench(args, rank, world, local):
         out["h2d_bytes"] = h2d
         out["h2d_gbs"] = h2d / (ms * 1e-3) / 1e9
         out["h2d_peak_gbs"] = measure_h2d()
+    if args.speculative:
+        out["speculative"] = run_speculative(ntx, model, spec, token, pos, args.speculative, stream, copy_stream,
+                                             max(3, args.steps // 2))
     return out
+
+
+def run_speculative(ntx, model, spec, token, pos, k, stream, copy_stream, n_calls):
+    """Self-speculative decoding: n_calls steps of (draft k - 1 tokens with the resident
+    layers, verify k tokens in one pass), each timed with CUDA events on the compute stream.
+    With random weights the draft's picks agree with the full model's by chance only, so the
+    measured tokens per pass say nothing about trained models; the verify pass's positions
+    per second (k per pass) is what full acceptance would give."""
+    import torch
+    cs = stream.cuda_stream
+    ks = copy_stream.cuda_stream if copy_stream is not None else None
+    times, counts, t, p = [], [], token, pos
+    for i in range(n_calls + 1):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        out = ntx.ntx_speculative_step(model.handle, t, p, k, None, cs, ks)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i:     # the first call allocates the pass buffers
+            times.append(a.elapsed_time(b))
+            counts.append(len(out))
+        t = out[-1]
+        p = spec.n_prefill + ((p - spec.n_prefill + len(out)) % max(1, spec.max_ctx - spec.n_prefill - k))
+    ms = statistics.median(times)
+    return {"k": k, "calls": n_calls, "median_ms_per_call": ms, "tokens_per_call": statistics.mean(counts),
+            "tok_s": sum(counts) / (sum(times) * 1e-3), "verify_positions_per_s_at_full_acceptance": k / (ms * 1e-3),
+            "note": "random weights: acceptance is by chance; see verify_positions_per_s_at_full_acceptance"}
 
 
 def measure_h2d():
@@ -594,6 +624,8 @@ def main():
                     help="weights handed to the library as tiled (repacked once at load) or GGUF-style blocks")
     ap.add_argument("--layers", type=int, default=None,
                     help="shorten the model to this many layers (profiler captures only; the line says so)")
+    ap.add_argument("--speculative", type=int, default=0, metavar="K",
+                    help="also time self-speculative decoding steps verifying K tokens per pass")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--profile-gemv", default=None, metavar="FMT:ROWSxCOLS[,...]",
@@ -676,6 +708,8 @@ def main():
     if args.workload == "llama70b_q4k_stream":
         line["host_link"] = {"h2d_bytes_per_step": r["h2d_bytes"], "achieved_gbs": r["h2d_gbs"],
                              "measured_pinned_h2d_gbs": r["h2d_peak_gbs"], "frac": r["h2d_gbs"] / r["h2d_peak_gbs"]}
+    if "speculative" in r:
+        line["speculative"] = r["speculative"]
     if rank == 0:
         agg, per_kind = measure_gemv_roofline(ntx, model, spec, stream, r["logits"])
         frac = agg["achieved"] / peak

@@ -356,6 +356,34 @@ ntx_status ntx_model_layer_similarity(ntx_model* model, int32_t token, int32_t p
                                       void* copy);
 ntx_status ntx_model_set_layer_skip(ntx_model* model, const uint8_t* skip);
 
+/* Self-speculative decoding ("Funciones principales": the layers resident in VRAM act as
+ * the draft model and the full model verifies several drafted tokens in one pass, so each
+ * streamed layer crosses the host link once for all of them; "Hoja de ruta de
+ * desarrollo").
+ *
+ * ntx_verify_tokens: one pass of the model as ntx_decode_step / ntx_stream_layers run it
+ * (skip mask included) over n tokens (host array, 1 <= n <= 8) at positions pos0 ..
+ * pos0 + n - 1.  Token i attends to positions 0 .. pos0 + i, including the K / V rows the
+ * earlier tokens of the pass write; its logits go to logits + i vocab (device fp32
+ * [n, vocab]).  Every layer runs for all n tokens before the next, so a streamed layer is
+ * copied once per pass.  Queued on `compute` (and `copy` for a partly resident model, which
+ * must differ); returns after queueing.
+ *
+ * ntx_speculative_step: from `token` at `pos`, drafts k - 1 tokens (2 <= k <= 8) greedily
+ * with the draft model (the resident layers, minus the layers draft_skip marks: host array
+ * [n_layers] or NULL), verifies token and drafts with one ntx_verify_tokens pass, and
+ * accepts the drafted tokens up to the first one the full model's greedy pick disagrees
+ * with, followed by the full model's own pick there.  out_tokens (host [k]) receives those
+ * tokens, *n_out their number (1 .. k): exactly the tokens greedy decoding of the full model
+ * gives from (token, pos).  The K / V rows at pos .. pos + *n_out - 1 hold the accepted
+ * tokens' values; continue from out_tokens[*n_out - 1] at pos + *n_out.  Synchronises with
+ * the work it queued (bounded by timeout_ms when > 0: NTX_ETIMEOUT leaves the work queued).
+ * Drafting uses greedy picks (argmax, lowest index among ties). */
+ntx_status ntx_verify_tokens(ntx_model* model, const int32_t* tokens, int32_t n, int32_t pos0, float* logits,
+                             void* compute, void* copy);
+ntx_status ntx_speculative_step(ntx_model* model, int32_t token, int32_t pos, int32_t k, const uint8_t* draft_skip,
+                                int32_t* out_tokens, int32_t* n_out, void* compute, void* copy, int64_t timeout_ms);
+
 /* Per-step counters of the last ntx_stream_layers call: bytes copied host ->
  * device, and device milliseconds of the whole step (between the step's first
  * and last event; valid once the step finished). */

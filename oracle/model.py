@@ -91,3 +91,22 @@ def layer_similarity(spec: ModelSpec, pos: int | None = None, token: int | None 
         out.append(float(prev @ cur / np.sqrt((prev @ prev) * (cur @ cur))))
         prev = cur
     return out
+
+
+def decode_sequence(spec: ModelSpec, tokens, pos0: int):
+    """Logits of each of `tokens` decoded one after another at positions pos0, pos0 + 1, ...
+    (token i attends to the K / V rows tokens 0..i-1 wrote).  Keeps every layer's tensors in
+    host memory: small models only."""
+    import numpy as np
+    dims = dims_of(spec)
+    layers = [layer_tensors(spec, l) for l in range(spec.n_layers)]
+    norm, W = head_tensors(spec)
+    out = []
+    for i, token in enumerate(tokens):
+        h = embedding_row(spec, int(token)).copy()
+        for layer, t in enumerate(layers):
+            qts = [spec.qtype_of(k, layer) for k in ("w_qkv", "w_o", "w_gate", "w_down")]
+            decode_layer(dims, qts, h, pos0 + i, t["attn_norm"], t["w_qkv"], t["w_o"], t["ffn_norm"], t["w_gate"],
+                         t["w_up"], t["w_down"], t["k_cache"], t["v_cache"])
+        out.append(lm_head(spec.qtype_of("output"), norm, W, W.shape[0], spec.hidden, spec.rms_eps, h))
+    return np.stack(out)

@@ -28,7 +28,8 @@ EXPORTS = ("ntx_last_error", "ntx_version", "ntx_row_bytes", "ntx_block_elems", 
            "ntx_dequant_q", "ntx_repack_q", "ntx_rmsnorm", "ntx_rope", "ntx_attn_decode", "ntx_attn_decode_noalloc", "ntx_attn_workspace_bytes", "ntx_swiglu",
            "ntx_softmax", "ntx_argmax", "ntx_embed", "ntx_model_create", "ntx_model_destroy", "ntx_decode_step",
            "ntx_stream_layers", "ntx_stream_stats", "ntx_model_replay_gemv", "ntx_model_layer_similarity",
-           "ntx_model_set_layer_skip", "ntx_plan_resident", "ntx_model_host_path")
+           "ntx_model_set_layer_skip", "ntx_plan_resident", "ntx_model_host_path", "ntx_verify_tokens",
+           "ntx_speculative_step")
 
 
 class NtxError(RuntimeError):
@@ -93,6 +94,9 @@ def lib() -> ctypes.CDLL:
             "ntx_model_set_layer_skip": ([vp, ctypes.POINTER(ctypes.c_uint8)], ci),
             "ntx_plan_resident": ([ctypes.POINTER(ModelDesc), sz, ctypes.POINTER(i32), ctypes.POINTER(sz)], ci),
             "ntx_model_host_path": ([vp, ctypes.POINTER(i32)], ci),
+            "ntx_verify_tokens": ([vp, ctypes.POINTER(i32), i32, i32, vp, vp, vp], ci),
+            "ntx_speculative_step": ([vp, i32, i32, i32, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(i32),
+                                      ctypes.POINTER(i32), vp, vp, i64], ci),
         }
         for name, (args, res) in sigs.items():
             f = getattr(L, name)
@@ -259,3 +263,21 @@ def ntx_model_host_path(model: int) -> int:
     p = ctypes.c_int32(0)
     check(lib().ntx_model_host_path(model, ctypes.byref(p)))
     return p.value
+
+
+def ntx_verify_tokens(model: int, tokens, pos0: int, logits, compute=None, copy=None) -> None:
+    """One pass of the full model over len(tokens) tokens at positions pos0..; logits [n, vocab]."""
+    arr = (ctypes.c_int32 * len(tokens))(*[int(t) for t in tokens])
+    check(lib().ntx_verify_tokens(model, arr, len(tokens), pos0, _p(logits), _s(compute),
+                                  _s(copy) if copy is not None else None))
+
+
+def ntx_speculative_step(model: int, token: int, pos: int, k: int, draft_skip=None, compute=None, copy=None,
+                         timeout_ms: int = 0):
+    """Draft k - 1 tokens, verify them in one pass; returns the accepted tokens (1..k of them)."""
+    out = (ctypes.c_int32 * k)()
+    n = ctypes.c_int32(0)
+    skip = None if draft_skip is None else (ctypes.c_uint8 * len(draft_skip))(*[1 if v else 0 for v in draft_skip])
+    check(lib().ntx_speculative_step(model, token, pos, k, skip, out, ctypes.byref(n), _s(compute),
+                                     _s(copy) if copy is not None else None, timeout_ms))
+    return list(out[:n.value])

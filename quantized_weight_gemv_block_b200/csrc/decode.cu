@@ -41,6 +41,13 @@ struct ntx_model {
     float* cos_dev = nullptr;    // calibration: cosine similarity per layer
     bool calibrating = false;
     int32_t host_path = NTX_HOST_PATH_NONE;   // how streamed layers leave host memory
+    // multi-token passes (verification of drafted tokens): per-token hidden states, step
+    // words and RoPE tables, drafted and predicted tokens, logits of every token
+    float* lane_h = nullptr;
+    int32_t* lane_step = nullptr;
+    float* lane_rope = nullptr;
+    int32_t* spec_tokens = nullptr;   // [2 kMaxLanes]: drafted tokens, then the full model's predictions
+    float* spec_logits = nullptr;     // [kMaxLanes, vocab]
     std::vector<void*> registered;            // host ranges this library registered (unregistered at destroy)
     int device = 0;
     float* h = nullptr;
@@ -78,8 +85,18 @@ struct LayerW {
     const void *qkv, *o, *gate, *up, *down;
 };
 
+// The per-token state of a step: hidden state h, the step word (token, pos) and the RoPE
+// table of pos.  A plain step has one; a verification pass has one per token.
+struct Lane {
+    float* h;
+    int32_t* step;
+    float* rope;
+};
+
+Lane lane0(ntx_model* m) { return {m->h, m->step, m->rope}; }
+
 // The fused GEMV launches of a layer, one function per kind, exactly as the step issues them.
-ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl)
+ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
     const ntx_layer_desc& L = m->layers[l];
@@ -90,15 +107,15 @@ ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool p
     P.row_bytes = row_bytes(qt, d.hidden);
     P.M = qd + 2 * kvd;
     P.K = d.hidden;
-    P.x = m->h;
+    P.x = ln.h;
     P.norm_w = L.attn_norm;
     P.eps = d.rms_eps;
     P.q_rows = qd;
     P.kv_rows = kvd;
     P.head_dim = d.head_dim;
     P.max_ctx = d.max_ctx;
-    P.pos_dev = m->step + 1;
-    P.rope_cs = m->rope;
+    P.pos_dev = ln.step + 1;
+    P.rope_cs = ln.rope;
     P.k_cache = (__half*)L.k_cache;
     P.v_cache = (__half*)L.v_cache;
     P.q_out = m->q;
@@ -106,7 +123,7 @@ ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool p
     return gemv_launch(qt, gemv::EPI_QKV, gemv::PRO_RMSNORM, P, s);
 }
 
-ntx_status launch_o(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl)
+ntx_status launch_o(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
     const int qt = m->lqt[l].o;
@@ -116,12 +133,13 @@ ntx_status launch_o(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl
     P.row_bytes = row_bytes(qt, P.K);
     P.M = d.hidden;
     P.x = m->att;
-    P.y = m->h;
+    P.y = ln.h;
     P.use_pdl = pdl;
     return gemv_launch(qt, gemv::EPI_ADD, gemv::PRO_X, P, s);
 }
 
-ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, cudaStream_t s, bool pdl)
+ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, cudaStream_t s, bool pdl,
+                          const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
     const int qt = m->lqt[l].ffn;
@@ -131,7 +149,7 @@ ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, c
     P.row_bytes = row_bytes(qt, d.hidden);
     P.M = d.ffn;
     P.K = d.hidden;
-    P.x = m->h;
+    P.x = ln.h;
     P.norm_w = m->layers[l].ffn_norm;
     P.eps = d.rms_eps;
     P.y = m->act;
@@ -139,7 +157,7 @@ ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, c
     return gemv_launch(qt, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, P, s);
 }
 
-ntx_status launch_down(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl)
+ntx_status launch_down(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
     const int qt = m->lqt[l].down;
@@ -149,22 +167,22 @@ ntx_status launch_down(ntx_model* m, int l, const void* w, cudaStream_t s, bool 
     P.M = d.hidden;
     P.K = d.ffn;
     P.x = m->act;
-    P.y = m->h;
+    P.y = ln.h;
     P.use_pdl = pdl;
     return gemv_launch(qt, gemv::EPI_ADD, gemv::PRO_X, P, s);
 }
 
-ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl)
+ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
     const ntx_layer_desc& L = m->layers[l];
     ntx_status st;
     if (m->calibrating) {
         // h before the layer, for the similarity of its input and output
-        NTX_CUDA_TRY(cudaMemcpyAsync(m->h_prev, m->h, (size_t)d.hidden * 4, cudaMemcpyDeviceToDevice, s));
+        NTX_CUDA_TRY(cudaMemcpyAsync(m->h_prev, ln.h, (size_t)d.hidden * 4, cudaMemcpyDeviceToDevice, s));
         pdl = false;
     }
-    if ((st = launch_qkv(m, l, w.qkv, s, pdl)) != NTX_OK) return st;
+    if ((st = launch_qkv(m, l, w.qkv, s, pdl, ln)) != NTX_OK) return st;
     {
         AttnArgs a{};
         a.q = m->q;
@@ -175,20 +193,20 @@ ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, b
         a.n_kv_heads = d.n_kv_heads;
         a.head_dim = d.head_dim;
         a.max_ctx = d.max_ctx;
-        a.pos_dev = m->step + 1;
+        a.pos_dev = ln.step + 1;
         a.workspace = m->attn_ws;
         a.n_split = m->n_split;
         a.pdl = pdl;
         if ((st = attn_launch(a, s)) != NTX_OK) return st;
     }
-    if ((st = launch_o(m, l, w.o, s, pdl)) != NTX_OK) return st;
-    if ((st = launch_gate_up(m, l, w.gate, w.up, s, pdl)) != NTX_OK) return st;
-    if ((st = launch_down(m, l, w.down, s, pdl)) != NTX_OK) return st;
-    if (m->calibrating) return cosine_launch(m->h_prev, m->h, d.hidden, m->cos_dev + l, s);
+    if ((st = launch_o(m, l, w.o, s, pdl, ln)) != NTX_OK) return st;
+    if ((st = launch_gate_up(m, l, w.gate, w.up, s, pdl, ln)) != NTX_OK) return st;
+    if ((st = launch_down(m, l, w.down, s, pdl, ln)) != NTX_OK) return st;
+    if (m->calibrating) return cosine_launch(m->h_prev, ln.h, d.hidden, m->cos_dev + l, s);
     return NTX_OK;
 }
 
-ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
+ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
     Params P{};
@@ -196,7 +214,7 @@ ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
     P.row_bytes = row_bytes(m->qt_out, d.hidden);
     P.M = d.vocab;
     P.K = d.hidden;
-    P.x = m->h;
+    P.x = ln.h;
     P.norm_w = d.out_norm;
     P.eps = d.rms_eps;
     P.y = logits;
@@ -206,17 +224,41 @@ ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl)
 
 LayerW resident_w(const ntx_layer_desc& L) { return {L.w_qkv, L.w_o, L.w_gate, L.w_up, L.w_down}; }
 
-// Embedding + resident layers [0, n) (+ head if with_head), token/pos from m->step.
+// Whether layer l runs: not in the skip mask (the calibration runs every layer), and not
+// in the extra mask `also_skip` (the draft model of a speculative step; may be null).
+bool layer_runs(const ntx_model* m, int l, const uint8_t* also_skip)
+{
+    if (m->calibrating) return true;
+    return !m->skip[l] && !(also_skip && also_skip[l]);
+}
+
+// Embedding + resident layers [0, n) for every lane (token / pos from each lane's step
+// word), then, if logits is not null, the head of each lane into logits + i vocab.  The
+// lanes go through a layer one after another, so lane i's attention sees the K / V rows
+// lanes 0..i-1 wrote at their positions.
+ntx_status enqueue_resident(ntx_model* m, int n, float* logits, cudaStream_t s, const Lane* lanes, int n_lanes,
+                            const uint8_t* also_skip = nullptr)
+{
+    const bool pdl = m->pdl && n_lanes == 1;
+    ntx_status st;
+    for (int i = 0; i < n_lanes; ++i)
+        if ((st = embed_launch(m->qt_embd, m->d.tok_embd, m->d.hidden, lanes[i].step, lanes[i].h, s, pdl)) != NTX_OK)
+            return st;
+    for (int l = 0; l < n; ++l) {
+        if (!layer_runs(m, l, also_skip)) continue;
+        for (int i = 0; i < n_lanes; ++i)
+            if ((st = enqueue_layer(m, l, resident_w(m->layers[l]), s, pdl, lanes[i])) != NTX_OK) return st;
+    }
+    if (logits)
+        for (int i = 0; i < n_lanes; ++i)
+            if ((st = enqueue_head(m, logits + (size_t)i * m->d.vocab, s, pdl, lanes[i])) != NTX_OK) return st;
+    return NTX_OK;
+}
+
 ntx_status enqueue_resident(ntx_model* m, int n, float* logits, cudaStream_t s, bool with_head)
 {
-    ntx_status st = embed_launch(m->qt_embd, m->d.tok_embd, m->d.hidden, m->step, m->h, s, m->pdl);
-    if (st != NTX_OK) return st;
-    for (int l = 0; l < n; ++l) {
-        if (m->skip[l] && !m->calibrating) continue;
-        if ((st = enqueue_layer(m, l, resident_w(m->layers[l]), s, m->pdl)) != NTX_OK) return st;
-    }
-    if (with_head) return enqueue_head(m, logits, s, m->pdl);
-    return NTX_OK;
+    const Lane ln = lane0(m);
+    return enqueue_resident(m, n, with_head ? logits : nullptr, s, &ln, 1);
 }
 
 bool env_flag(const char* name)
@@ -396,9 +438,16 @@ size_t hbm_bytes_for(const ntx_model_desc* d, int n)
     return total + ring_bytes(d, n) + scratch_bytes(d);
 }
 
+constexpr int kMaxLanes = 8;   // tokens of one verification pass
+
 void free_model(ntx_model* m)
 {
     if (!m) return;
+    cudaFree(m->lane_h);
+    cudaFree(m->lane_step);
+    cudaFree(m->lane_rope);
+    cudaFree(m->spec_tokens);
+    cudaFree(m->spec_logits);
     for (void* p : m->registered) cudaHostUnregister(p);
     if (m->graph) cudaGraphExecDestroy(m->graph);
     for (int i = 0; i < 2; ++i) {
@@ -568,8 +617,11 @@ namespace {
 struct CudaRing final : ring::Ops {
     ntx_model* m;
     cudaStream_t cs, ks;
+    const Lane* lanes;
+    int n_lanes;
     int64_t h2d = 0;
-    CudaRing(ntx_model* m_, cudaStream_t cs_, cudaStream_t ks_) : m(m_), cs(cs_), ks(ks_) {}
+    CudaRing(ntx_model* m_, cudaStream_t cs_, cudaStream_t ks_, const Lane* lanes_, int n_lanes_)
+        : m(m_), cs(cs_), ks(ks_), lanes(lanes_), n_lanes(n_lanes_) {}
 
     uint8_t* slot_base(int slot) const { return m->ring + (size_t)slot * m->slot_bytes; }
 
@@ -612,14 +664,23 @@ struct CudaRing final : ring::Ops {
     {
         uint8_t* base = slot_base(slot);
         const LayerW w{base + m->off_qkv, base + m->off_o, base + m->off_gate, base + m->off_up, base + m->off_down};
-        return enqueue_layer(m, j, w, cs, false);
+        // every lane goes through the layer while its matrices are in the slot: one copy
+        // over the host link serves all of them
+        for (int i = 0; i < n_lanes; ++i) {
+            const ntx_status st = enqueue_layer(m, j, w, cs, false, lanes[i]);
+            if (st != NTX_OK) return st;
+        }
+        return NTX_OK;
     }
     ntx_status compute_done(int slot) override
     {
         NTX_CUDA_TRY(cudaEventRecord(m->slot_free[slot], cs));
         return NTX_OK;
     }
-    ntx_status before_streamed() override { return enqueue_resident(m, m->d.n_resident, nullptr, cs, false); }
+    ntx_status before_streamed() override
+    {
+        return enqueue_resident(m, m->d.n_resident, nullptr, cs, lanes, n_lanes);
+    }
 };
 
 }  // namespace
@@ -628,26 +689,40 @@ struct CudaRing final : ring::Ops {
 namespace ntx {
 namespace {
 
-// Queue one step of a partly resident model: resident layers and the streamed layers
-// through the ring; the head when logits is not null.
+// Queue one pass of a partly resident model over the given lanes (their step words
+// already written): resident layers, then the streamed layers through the ring, each
+// streamed layer copied once for all lanes; the heads when logits is not null.
+ntx_status enqueue_streamed_pass(ntx_model* m, float* logits, cudaStream_t cs, cudaStream_t ks, const Lane* lanes,
+                                 int n_lanes)
+{
+    const ntx_model_desc& d = m->d;
+    ntx_status st;
+    // the streamed layers that run (skipped layers are neither copied nor computed)
+    std::vector<int> streamed;
+    for (int j = d.n_resident; j < d.n_layers; ++j)
+        if (layer_runs(m, j, nullptr)) streamed.push_back(j);
+    if (!streamed.empty()) NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->ev_start, 0));
+    CudaRing ops(m, cs, ks, lanes, n_lanes);
+    if ((st = ring::schedule(ops, streamed.data(), (int)streamed.size(), 2)) != NTX_OK) return st;
+    if (logits)
+        for (int i = 0; i < n_lanes; ++i)
+            if ((st = enqueue_head(m, logits + (size_t)i * d.vocab, cs, false, lanes[i])) != NTX_OK) return st;
+    NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
+    m->last_h2d = ops.h2d;
+    return NTX_OK;
+}
+
+// One step of a partly resident model (the model's own lane); the head when logits is
+// not null.
 ntx_status enqueue_streamed_step(ntx_model* m, int32_t token, int32_t pos, float* logits, cudaStream_t cs,
                                  cudaStream_t ks)
 {
     const ntx_model_desc& d = m->d;
     NTX_CUDA_TRY(cudaEventRecord(m->ev_start, cs));
-    ntx_status st = set_step_launch(m->step, token, pos, m->rope, d.rope_theta, d.head_dim, cs);
+    const ntx_status st = set_step_launch(m->step, token, pos, m->rope, d.rope_theta, d.head_dim, cs);
     if (st != NTX_OK) return st;
-    // the streamed layers that run (skipped layers are neither copied nor computed)
-    std::vector<int> streamed;
-    for (int j = d.n_resident; j < d.n_layers; ++j)
-        if (!m->skip[j] || m->calibrating) streamed.push_back(j);
-    if (!streamed.empty()) NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->ev_start, 0));
-    CudaRing ops(m, cs, ks);
-    if ((st = ring::schedule(ops, streamed.data(), (int)streamed.size(), 2)) != NTX_OK) return st;
-    if (logits && (st = enqueue_head(m, logits, cs, false)) != NTX_OK) return st;
-    NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
-    m->last_h2d = ops.h2d;
-    return NTX_OK;
+    const Lane ln = lane0(m);
+    return enqueue_streamed_pass(m, logits, cs, ks, &ln, 1);
 }
 
 }  // namespace
@@ -710,11 +785,11 @@ NTX_EXPORT ntx_status ntx_model_replay_gemv(ntx_model* m, int kind, int n_launch
         const int l = i % std::max(1, nres);
         const ntx_layer_desc& L = m->layers[l];
         switch (kind) {
-        case NTX_GEMV_QKV: st = launch_qkv(m, l, L.w_qkv, s, m->pdl); break;
-        case NTX_GEMV_O: st = launch_o(m, l, L.w_o, s, m->pdl); break;
-        case NTX_GEMV_GATE_UP: st = launch_gate_up(m, l, L.w_gate, L.w_up, s, m->pdl); break;
-        case NTX_GEMV_DOWN: st = launch_down(m, l, L.w_down, s, m->pdl); break;
-        default: st = enqueue_head(m, logits, s, m->pdl); break;
+        case NTX_GEMV_QKV: st = launch_qkv(m, l, L.w_qkv, s, m->pdl, lane0(m)); break;
+        case NTX_GEMV_O: st = launch_o(m, l, L.w_o, s, m->pdl, lane0(m)); break;
+        case NTX_GEMV_GATE_UP: st = launch_gate_up(m, l, L.w_gate, L.w_up, s, m->pdl, lane0(m)); break;
+        case NTX_GEMV_DOWN: st = launch_down(m, l, L.w_down, s, m->pdl, lane0(m)); break;
+        default: st = enqueue_head(m, logits, s, m->pdl, lane0(m)); break;
         }
     }
     return st;
@@ -792,5 +867,146 @@ NTX_EXPORT ntx_status ntx_model_host_path(ntx_model* m, int32_t* path)
 {
     if (!m || !path) return fail(NTX_EINVAL, "ntx_model_host_path: null pointer");
     *path = m->host_path;
+    return NTX_OK;
+}
+
+namespace ntx {
+namespace {
+
+// The buffers of multi-token passes, allocated on first use.
+ntx_status ensure_lanes(ntx_model* m)
+{
+    if (m->lane_h) return NTX_OK;
+    const ntx_model_desc& d = m->d;
+    cudaError_t e = cudaMalloc((void**)&m->lane_h, (size_t)kMaxLanes * d.hidden * 4);
+    if (e == cudaSuccess) e = cudaMalloc((void**)&m->lane_step, (size_t)kMaxLanes * 16);
+    if (e == cudaSuccess) e = cudaMalloc((void**)&m->lane_rope, (size_t)kMaxLanes * d.head_dim * 4);
+    if (e == cudaSuccess) e = cudaMalloc((void**)&m->spec_tokens, (size_t)2 * kMaxLanes * 4);
+    if (e == cudaSuccess) e = cudaMalloc((void**)&m->spec_logits, (size_t)kMaxLanes * d.vocab * 4);
+    if (e != cudaSuccess) {
+        cudaFree(m->lane_h);
+        cudaFree(m->lane_step);
+        cudaFree(m->lane_rope);
+        cudaFree(m->spec_tokens);
+        cudaFree(m->spec_logits);
+        m->lane_h = nullptr;
+        m->lane_step = nullptr;
+        m->lane_rope = nullptr;
+        m->spec_tokens = nullptr;
+        m->spec_logits = nullptr;
+        return fail(e == cudaErrorMemoryAllocation ? NTX_ENOMEM : NTX_ECUDA,
+                    std::string("multi-token pass buffers: ") + cudaGetErrorString(e));
+    }
+    return NTX_OK;
+}
+
+Lane lane_at(ntx_model* m, int i)
+{
+    return {m->lane_h + (size_t)i * m->d.hidden, m->lane_step + 4 * i, m->lane_rope + (size_t)i * m->d.head_dim};
+}
+
+// One pass of the full model over n tokens at positions pos0 .. pos0 + n - 1 (token i
+// from host tokens[i], or from device tokens_dev[i] when that is not null), logits of
+// token i into logits + i vocab.  Resident models run on `cs` alone.
+ntx_status enqueue_multi(ntx_model* m, const int32_t* tokens, const int32_t* tokens_dev, int n, int32_t pos0,
+                         float* logits, cudaStream_t cs, cudaStream_t ks)
+{
+    const ntx_model_desc& d = m->d;
+    Lane lanes[kMaxLanes];
+    NTX_CUDA_TRY(cudaEventRecord(m->ev_start, cs));
+    for (int i = 0; i < n; ++i) {
+        lanes[i] = lane_at(m, i);
+        const ntx_status st = set_step_launch(lanes[i].step, tokens ? tokens[i] : 0, pos0 + i, lanes[i].rope,
+                                              d.rope_theta, d.head_dim, cs, tokens_dev ? tokens_dev + i : nullptr);
+        if (st != NTX_OK) return st;
+    }
+    if (d.n_resident == d.n_layers) {
+        const ntx_status st = enqueue_resident(m, d.n_layers, logits, cs, lanes, n);
+        if (st != NTX_OK) return st;
+        NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
+        return NTX_OK;
+    }
+    return enqueue_streamed_pass(m, logits, cs, ks, lanes, n);
+}
+
+ntx_status check_multi(ntx_model* m, int n, int32_t pos0, void* compute, void* copy, const char* who)
+{
+    const std::string w(who);
+    if (!m) return fail(NTX_EINVAL, w + ": null model");
+    if (n < 1 || n > kMaxLanes) return fail(NTX_EINVAL, w + ": between 1 and 8 tokens");
+    if (pos0 < 0 || pos0 + n > m->d.max_ctx) return fail(NTX_EINVAL, w + ": positions out of range");
+    if (m->d.n_resident < m->d.n_layers && compute == copy)
+        return fail(NTX_EINVAL, w + ": compute and copy streams must differ");
+    return ensure_lanes(m);
+}
+
+}  // namespace
+}  // namespace ntx
+
+NTX_EXPORT ntx_status ntx_verify_tokens(ntx_model* m, const int32_t* tokens, int32_t n, int32_t pos0, float* logits,
+                                        void* compute, void* copy)
+{
+    ntx_status st = check_multi(m, n, pos0, compute, copy, "ntx_verify_tokens");
+    if (st != NTX_OK) return st;
+    if (!tokens || !logits || !aligned(logits, 4)) return fail(NTX_EINVAL, "ntx_verify_tokens: bad tokens / logits");
+    for (int i = 0; i < n; ++i)
+        if (tokens[i] < 0 || tokens[i] >= m->d.vocab) return fail(NTX_EINVAL, "ntx_verify_tokens: token out of range");
+    return enqueue_multi(m, tokens, nullptr, n, pos0, logits, (cudaStream_t)compute, (cudaStream_t)copy);
+}
+
+NTX_EXPORT ntx_status ntx_speculative_step(ntx_model* m, int32_t token, int32_t pos, int32_t k,
+                                           const uint8_t* draft_skip, int32_t* out_tokens, int32_t* n_out,
+                                           void* compute, void* copy, int64_t timeout_ms)
+{
+    ntx_status st = check_multi(m, k, pos, compute, copy, "ntx_speculative_step");
+    if (st != NTX_OK) return st;
+    if (k < 2) return fail(NTX_EINVAL, "ntx_speculative_step: k must be at least 2");
+    if (!out_tokens || !n_out) return fail(NTX_EINVAL, "ntx_speculative_step: null output pointer");
+    if (token < 0 || token >= m->d.vocab) return fail(NTX_EINVAL, "ntx_speculative_step: token out of range");
+    if (timeout_ms < 0) return fail(NTX_EINVAL, "ntx_speculative_step: timeout_ms must be >= 0");
+    const ntx_model_desc& d = m->d;
+    cudaStream_t cs = (cudaStream_t)compute, ks = (cudaStream_t)copy;
+    int32_t* drafted = m->spec_tokens;              // [k]: token, then the k - 1 drafted tokens
+    int32_t* predicted = m->spec_tokens + kMaxLanes;
+    // the draft model: the resident layers (streamed layers left out) minus draft_skip
+    std::vector<uint8_t> also(d.n_layers, 0);
+    for (int l = 0; l < d.n_layers; ++l) also[l] = (l >= d.n_resident || (draft_skip && draft_skip[l])) ? 1 : 0;
+    NTX_CUDA_TRY(cudaMemcpyAsync(drafted, &token, 4, cudaMemcpyHostToDevice, cs));
+    const Lane ln = lane0(m);
+    const bool pdl = m->pdl;
+    m->pdl = false;
+    for (int i = 0; i + 1 < k && st == NTX_OK; ++i) {
+        // draft step i: the token drafted last, at pos + i; greedy pick of the next one
+        st = set_step_launch(ln.step, 0, pos + i, ln.rope, d.rope_theta, d.head_dim, cs, drafted + i);
+        if (st == NTX_OK) st = enqueue_resident(m, d.n_layers, m->spec_logits, cs, &ln, 1, also.data());
+        if (st == NTX_OK) st = argmax_launch(m->spec_logits, d.vocab, drafted + i + 1, cs);
+    }
+    m->pdl = pdl;
+    if (st != NTX_OK) return st;
+    // one pass of the full model over the token and the drafted tokens
+    if ((st = enqueue_multi(m, nullptr, drafted, k, pos, m->spec_logits, cs, ks)) != NTX_OK) return st;
+    for (int i = 0; i < k; ++i)
+        if ((st = argmax_launch(m->spec_logits + (size_t)i * d.vocab, d.vocab, predicted + i, cs)) != NTX_OK)
+            return st;
+    int32_t host[2 * kMaxLanes];
+    NTX_CUDA_TRY(cudaMemcpyAsync(host, m->spec_tokens, sizeof(host), cudaMemcpyDeviceToHost, cs));
+    NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
+    st = ring::wait_bounded(
+        [&]() -> ntx_status {
+            const cudaError_t q = cudaEventQuery(m->ev_end);
+            return q == cudaSuccess ? NTX_OK : q == cudaErrorNotReady ? NTX_ETIMEOUT : NTX_ECUDA;
+        },
+        timeout_ms > 0 ? timeout_ms : (int64_t)1 << 40);
+    if (st == NTX_ETIMEOUT)
+        return fail(NTX_ETIMEOUT, "ntx_speculative_step: not finished within timeout_ms (work stays queued)");
+    if (st != NTX_OK) return fail(st, "ntx_speculative_step: a kernel failed");
+    // accept the drafted tokens the full model predicts too, then its own next token
+    int n = 0;
+    while (n + 1 < k && host[kMaxLanes + n] == host[n + 1]) {
+        out_tokens[n] = host[n + 1];
+        ++n;
+    }
+    out_tokens[n] = host[kMaxLanes + n];
+    *n_out = n + 1;
     return NTX_OK;
 }

@@ -141,11 +141,12 @@ __global__ void embed_kernel(const uint8_t* E, int64_t rb, int64_t hidden, const
 // rope[2i + 1] = cos and sin of pos theta^(-2i/head_dim), computed in double, for
 // i < head_dim / 2 (the rotation of "RoPE" in the ntransformer news summary's kernel
 // list).  Later kernels of the step read both.
-__global__ void set_step_kernel(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim)
+__global__ void set_step_kernel(int32_t* step, int32_t token, const int32_t* token_dev, int32_t pos, float* rope,
+                                float theta, int head_dim)
 {
     const int i = threadIdx.x;
     if (i == 0) {
-        step[0] = token;
+        step[0] = token_dev ? *token_dev : token;
         step[1] = pos;
     }
     if (rope && i < head_dim / 2) {
@@ -238,9 +239,9 @@ ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t*
 }
 
 ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
-                           cudaStream_t s)
+                           cudaStream_t s, const int32_t* token_dev)
 {
-    set_step_kernel<<<1, std::max(32, head_dim / 2), 0, s>>>(step, token, pos, rope, theta, head_dim);
+    set_step_kernel<<<1, std::max(32, head_dim / 2), 0, s>>>(step, token, token_dev, pos, rope, theta, head_dim);
     return check_launch("step counter");
 }
 
@@ -290,12 +291,19 @@ NTX_EXPORT ntx_status ntx_softmax(const float* x, float* y, int64_t n, void* str
     return check_launch("ntx_softmax");
 }
 
+namespace ntx {
+ntx_status argmax_launch(const float* x, int64_t n, int32_t* out_index, cudaStream_t s)
+{
+    argmax_kernel<<<1, kBlock, 0, s>>>(x, n, out_index);
+    return check_launch("argmax");
+}
+}  // namespace ntx
+
 NTX_EXPORT ntx_status ntx_argmax(const float* x, int64_t n, int32_t* out_index, void* stream)
 {
     if (!x || !out_index) return fail(NTX_EINVAL, "ntx_argmax: null pointer");
     if (n < 1 || n > (1ll << 26)) return fail(NTX_EINVAL, "ntx_argmax: n out of range");
-    argmax_kernel<<<1, kBlock, 0, (cudaStream_t)stream>>>(x, n, out_index);
-    return check_launch("ntx_argmax");
+    return argmax_launch(x, n, out_index, (cudaStream_t)stream);
 }
 
 NTX_EXPORT ntx_status ntx_embed(int qtype, const void* E, int64_t vocab, int64_t hidden, const int32_t* token_dev,

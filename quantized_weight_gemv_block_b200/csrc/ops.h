@@ -9,10 +9,13 @@ namespace ntx {
 ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t* token_dev, float* h, cudaStream_t s,
                         bool pdl);
 // Writes the step word (token, pos) and, if rope is not null, the RoPE table of pos
-// ([head_dim / 2][cos, sin] floats) for the kernels of the step.
+// ([head_dim / 2][cos, sin] floats) for the kernels of the step; the token is read from
+// device memory (token_dev) when that is not null.
 ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
-                           cudaStream_t s);
+                           cudaStream_t s, const int32_t* token_dev = nullptr);
 ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
+// *out_index = the lowest index of the largest x (n <= 2^26), one CTA.
+ntx_status argmax_launch(const float* x, int64_t n, int32_t* out_index, cudaStream_t s);
 // *out = a . b / (|a| |b|) for device fp32 vectors of n <= 2^26 elements (0 if either is zero).
 ntx_status cosine_launch(const float* a, const float* b, int64_t n, float* out, cudaStream_t s);
 ntx_status qmma_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);

@@ -298,26 +298,86 @@ def test_streamed_from_pageable_host_memory(ntx, syn, monkeypatch, register):
 
 
 def test_planned_split_runs(ntx, syn):
-    """A split chosen by ntx_plan_resident for a given HBM budget builds and decodes: the
-    budget that fits exactly two of four layers gives two resident layers, and the step
-    matches the oracle."""
+    """A split chosen by ntx_plan_resident builds and decodes: one byte below the HBM that
+    all four layers need, the planner streams some of them (a streamed layer also needs its
+    share of the two-slot ring), and the step matches the oracle."""
     from oracle import model as om
     from synth.device_model import DeviceModel
     spec = small_spec(syn, 2, n_layers=4, tiled=True)
     probe = DeviceModel(spec, n_resident=4)
-    d = probe.desc
-    _, full = ntx.ntx_plan_resident(d, 1 << 62)
-    budget = None
-    for b in range(full, 0, -(1 << 20)):
-        n, used = ntx.ntx_plan_resident(d, b)
-        if n == 2:
-            budget = b
-            break
+    n_all, full = ntx.ntx_plan_resident(probe.desc, 1 << 62)
+    n, used = ntx.ntx_plan_resident(probe.desc, full - 1)
     probe.close()
-    assert budget is not None
-    m = DeviceModel(spec, n_resident=ntx.ntx_plan_resident(d, budget)[0])
-    assert m.n_resident == 2
+    assert n_all == 4 and 0 <= n < 4 and used <= full - 1
+    m = DeviceModel(spec, n_resident=n)
     got = run_decode(ntx, m, spec.token(), spec.n_prefill, stream_layers=True)
     m.close()
     want, _ = om.decode(spec)
     assert rel_err(got, want) <= TOL
+
+
+@pytest.mark.parametrize("n_resident", [3, 1], ids=["resident", "streamed"])
+def test_verify_tokens_against_oracle(ntx, syn, n_resident):
+    """One multi-token pass over four tokens (each attending to the rows the earlier ones
+    wrote) against the oracle decoding them one after another; a streamed model copies each
+    streamed layer once for the whole pass."""
+    from oracle import model as om
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, 2, n_layers=3, tiled=True, vocab=1008)
+    m = DeviceModel(spec, n_resident=n_resident)
+    tokens, pos0 = [17, 5, 1007, 0], spec.n_prefill
+    logits = torch.full((len(tokens), spec.vocab), float("nan"), dtype=torch.float32, device="cuda")
+    cs, ks = torch.cuda.Stream(), torch.cuda.Stream()
+    ntx.ntx_verify_tokens(m.handle, tokens, pos0, logits, cs.cuda_stream, ks.cuda_stream)
+    torch.cuda.synchronize()
+    assert ntx.ntx_device_error() == 0
+    if n_resident < spec.n_layers:
+        h2d, _ = ntx.ntx_stream_stats(m.handle)
+        assert h2d == sum(spec.layer_weight_bytes(l) for l in range(n_resident, spec.n_layers))
+    m.close()
+    want = om.decode_sequence(spec, tokens, pos0)
+    got = logits.cpu().numpy()
+    for i in range(len(tokens)):
+        assert rel_err(got[i], want[i]) <= TOL, i
+        assert elem_err(got[i], want[i]) <= TOL, i
+
+
+def greedy(ntx, m, token, pos, n, streamed):
+    """n tokens of plain greedy decoding from (token, pos), one step each."""
+    out = []
+    for i in range(n):
+        logits = run_decode(ntx, m, token, pos + i, stream_layers=streamed)
+        token = int(np.argmax(logits))
+        out.append(token)
+    return out
+
+
+@pytest.mark.parametrize("case", ["same-model", "quiet-layer-skipped", "streamed"])
+def test_speculative_decoding_equals_greedy(ntx, syn, case):
+    """Self-speculative decoding gives exactly the tokens of greedy decoding of the full
+    model: with a draft identical to the model every drafted token is accepted; with a draft
+    that leaves out a near-identity layer, or the streamed layers, some may be rejected, and
+    the output is still the greedy sequence."""
+    from synth.device_model import DeviceModel
+    extra = {"quiet_layers": [1]} if case == "quiet-layer-skipped" else {}
+    spec = small_spec(syn, 2, n_layers=3, tiled=True, vocab=1008, max_ctx=320, extra=extra)
+    streamed = case == "streamed"
+    m = DeviceModel(spec, n_resident=1 if streamed else None)
+    token, pos, n_want, k = spec.token(), spec.n_prefill, 9, 4
+    want = greedy(ntx, m, token, pos, n_want, streamed)
+    m.reset_caches()
+    torch.cuda.synchronize()
+    cs, ks = torch.cuda.Stream(), torch.cuda.Stream()
+    draft_skip = [0, 1, 0] if case == "quiet-layer-skipped" else None
+    got, counts, t, p = [], [], token, pos
+    while len(got) < n_want:
+        out = ntx.ntx_speculative_step(m.handle, t, p, k, draft_skip, cs.cuda_stream, ks.cuda_stream)
+        assert 1 <= len(out) <= k
+        counts.append(len(out))
+        got += out
+        t, p = out[-1], p + len(out)
+    m.close()
+    print(f"speculative {case}: tokens per pass {counts}")
+    assert got[:n_want] == want
+    if case == "same-model":
+        assert all(c == k for c in counts)

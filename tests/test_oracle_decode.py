@@ -123,3 +123,43 @@ def test_synthetic_model_stays_conditioned(orc, syn, qtype):
     rms = [float(np.sqrt(np.mean(h.astype(np.float64) ** 2))) for h in hidden]
     assert all(0.05 < r < 20 for r in rms), rms
     assert 0.2 < float(np.sqrt(np.mean(logits.astype(np.float64) ** 2))) < 5
+
+
+def _tiny_spec(syn, **kw):
+    base = dict(n_layers=3, hidden=256, n_q_heads=4, n_kv_heads=2, head_dim=128, ffn=512, vocab=64, max_ctx=24,
+                n_prefill=16, qtype=syn.Q8_0, seed=5)
+    base.update(kw)
+    return syn.ModelSpec(**base)
+
+
+def test_sequence_decode_structure(orc, syn):
+    """The oracle's multi-token decode: one token equals the plain decode; earlier tokens'
+    logits do not depend on later tokens (causality); a later token's logits depend on the
+    earlier token (it attends to the K / V rows that token wrote)."""
+    from oracle import model as om
+    spec = _tiny_spec(syn)
+    pos0 = spec.n_prefill
+    one = om.decode_sequence(spec, [7], pos0)
+    plain, _ = om.decode(spec, pos=pos0, token=7)
+    assert np.array_equal(one[0], plain)
+    ab = om.decode_sequence(spec, [7, 9, 3], pos0)
+    assert np.array_equal(ab[0], plain)
+    cb = om.decode_sequence(spec, [8, 9, 3], pos0)
+    assert not np.array_equal(ab[1], cb[1]) and not np.array_equal(ab[2], cb[2])
+    # the second token at pos0 + 1 with the prefilled row at pos0 (no first token) differs too
+    alone, _ = om.decode(spec, pos=pos0 + 1, token=9)
+    assert not np.array_equal(ab[1], alone)
+
+
+def test_layer_skip_and_similarity(orc, syn):
+    """Skipping a layer leaves h unchanged through it (the skipped model equals the model
+    whose layer has zero residual contributions); a layer whose residual contributions are
+    scaled by 2^-10 has a similarity within 1e-5 of 1 while ordinary layers are far below."""
+    from oracle import model as om
+    spec = _tiny_spec(syn, extra={"quiet_layers": [1]})
+    cos = om.layer_similarity(spec)
+    assert cos[1] > 1 - 1e-5 and max(cos[0], cos[2]) < 0.99
+    _, hid = om.decode(spec, keep_hidden=True, skip={1})
+    assert np.array_equal(hid[1], hid[0])
+    full, hid_full = om.decode(spec, keep_hidden=True)
+    assert np.array_equal(hid[0], hid_full[0]) and not np.array_equal(hid[2], hid_full[2])
