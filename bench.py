@@ -140,8 +140,9 @@ def max_over_ranks(v, world):
 
 # --------------------------------------------------------------------------- workloads
 
-def spec_for(name, layout="tiled", layers=None):
-    """The workload's model; `layers` shortens it (profiler captures only)."""
+def spec_for(name, layout="tiled", layers=None, extra_ctx=0):
+    """The workload's model; `layers` shortens it (profiler captures only); `extra_ctx` adds
+    KV-cache positions past the decode position (room for multi-token verify passes)."""
     import synth
     tiled = layout == "tiled"
     base = {"llama70b_q6k_decode": synth.LLAMA_70B_Q6_K, "llama8b_q8_0_decode": synth.LLAMA_8B_Q8_0,
@@ -149,6 +150,7 @@ def spec_for(name, layout="tiled", layers=None):
     kw = dict(base)
     if layers:
         kw["n_layers"] = layers
+    kw["max_ctx"] += extra_ctx
     return synth.ModelSpec(**kw, tiled=tiled)
 
 
@@ -264,7 +266,8 @@ def run_decode_bench(args, rank, world, local):
     from synth.device_model import DeviceModel
 
     name = args.workload
-    spec = spec_for(name, args.layout, args.layers)
+    # speculative passes verify k positions from the decode position on: room for 4 passes
+    spec = spec_for(name, args.layout, args.layers, extra_ctx=4 * args.speculative)
     streamed = name == "llama70b_q4k_stream"
     n_res = 36 if streamed else None
     t0 = time.time()
@@ -274,8 +277,8 @@ def run_decode_bench(args, rank, world, local):
     stream = torch.cuda.Stream()
     copy_stream = torch.cuda.Stream() if streamed else None
     logits = torch.empty(spec.vocab, dtype=torch.float32, device="cuda")
-    # step word + embedding, per layer QKV, attention, split merge, O, gate/up, down, then the LM head
-    launches_per_step = 2 + 6 * spec.n_layers + 1
+    # step word + embedding, per layer QKV, attention (+ split merge), O, gate/up, down, LM head
+    launches_per_step = ntx.ntx_model_step_launches(model.handle)
 
     def step():
         if streamed:

@@ -384,6 +384,10 @@ ntx_status ntx_verify_tokens(ntx_model* model, const int32_t* tokens, int32_t n,
 ntx_status ntx_speculative_step(ntx_model* model, int32_t token, int32_t pos, int32_t k, const uint8_t* draft_skip,
                                 int32_t* out_tokens, int32_t* n_out, void* compute, void* copy, int64_t timeout_ms);
 
+/* Number of kernel launches one ntx_decode_step of this model queues (the step word,
+ * the embedding, the layers' kernels, the LM head), for accounting. */
+ntx_status ntx_model_step_launches(ntx_model* model, int32_t* launches);
+
 /* Per-step counters of the last ntx_stream_layers call: bytes copied host ->
  * device, and device milliseconds of the whole step (between the step's first
  * and last event; valid once the step finished). */

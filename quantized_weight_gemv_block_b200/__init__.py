@@ -29,7 +29,7 @@ EXPORTS = ("ntx_last_error", "ntx_version", "ntx_row_bytes", "ntx_block_elems", 
            "ntx_softmax", "ntx_argmax", "ntx_embed", "ntx_model_create", "ntx_model_destroy", "ntx_decode_step",
            "ntx_stream_layers", "ntx_stream_stats", "ntx_model_replay_gemv", "ntx_model_layer_similarity",
            "ntx_model_set_layer_skip", "ntx_plan_resident", "ntx_model_host_path", "ntx_verify_tokens",
-           "ntx_speculative_step")
+           "ntx_speculative_step", "ntx_model_step_launches")
 
 
 class NtxError(RuntimeError):
@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
             "ntx_plan_resident": ([ctypes.POINTER(ModelDesc), sz, ctypes.POINTER(i32), ctypes.POINTER(sz)], ci),
             "ntx_model_host_path": ([vp, ctypes.POINTER(i32)], ci),
             "ntx_verify_tokens": ([vp, ctypes.POINTER(i32), i32, i32, vp, vp, vp], ci),
+            "ntx_model_step_launches": ([vp, ctypes.POINTER(i32)], ci),
             "ntx_speculative_step": ([vp, i32, i32, i32, ctypes.POINTER(ctypes.c_uint8), ctypes.POINTER(i32),
                                       ctypes.POINTER(i32), vp, vp, i64], ci),
         }
@@ -281,3 +282,9 @@ def ntx_speculative_step(model: int, token: int, pos: int, k: int, draft_skip=No
     check(lib().ntx_speculative_step(model, token, pos, k, skip, out, ctypes.byref(n), _s(compute),
                                      _s(copy) if copy is not None else None, timeout_ms))
     return list(out[:n.value])
+
+
+def ntx_model_step_launches(model: int) -> int:
+    n = ctypes.c_int32(0)
+    check(lib().ntx_model_step_launches(model, ctypes.byref(n)))
+    return n.value

@@ -1010,3 +1010,15 @@ NTX_EXPORT ntx_status ntx_speculative_step(ntx_model* m, int32_t token, int32_t 
     *n_out = n + 1;
     return NTX_OK;
 }
+
+NTX_EXPORT ntx_status ntx_model_step_launches(ntx_model* m, int32_t* launches)
+{
+    if (!m || !launches) return fail(NTX_EINVAL, "ntx_model_step_launches: null pointer");
+    int n = 0;
+    for (int l = 0; l < m->d.n_layers; ++l)
+        if (layer_runs(m, l, nullptr)) ++n;
+    // per layer: QKV, attention, the merge of its splits, O, gate/up, down; plus the step
+    // word, the embedding and the LM head
+    *launches = 3 + 6 * n;
+    return NTX_OK;
+}
