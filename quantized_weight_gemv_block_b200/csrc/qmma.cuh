@@ -531,6 +531,15 @@ __device__ __forceinline__ float limbs_f(int c0, int c1, int c2)
     return fmaf((float)c2, 65536.f, fmaf((float)c1, 256.f, (float)c0));
 }
 
+// The same value with the two low limbs combined in int32 first (one conversion fewer):
+// c0 + 256 c1 is exact there when |c0|, |c1| < 2^22, and its single rounding to fp32
+// equals that of fmaf(c1, 256, c0) on the exact operands.  Used by the 4-bit row units
+// (Q4_0 sweep +1 %); on the Q8_0 lane units it measured 0.5 % slower and is not used.
+__device__ __forceinline__ float limbs_f2(int c0, int c1, int c2)
+{
+    return fmaf((float)c2, 65536.f, (float)(c0 + 256 * c1));
+}
+
 // limb words of a step for lane tig (the PAIRED layout): X[l].x = columns 4 tig..,
 // X[l].y = 16 + 4 tig..; f = the step's factor 2^-e_u
 __device__ __forceinline__ void x_words(const uint32_t* xs, int tig, uint2 (&X)[3], float& f)
@@ -632,8 +641,9 @@ struct Row<NTX_Q4_0_T> {
             }
         }
         const float2 d = d_pair(U + 256 + 4 * g);
-        acc0 = fmaf(d.x * f, limbs_f(c0[0], c0[1], c0[2]), acc0);
-        acc1 = fmaf(d.y * f, limbs_f(c1[0], c1[1], c1[2]), acc1);
+        // |c| <= 8 * 32 * 128 + 32 * 15 * 128 per limb
+        acc0 = fmaf(d.x * f, limbs_f2(c0[0], c0[1], c0[2]), acc0);
+        acc1 = fmaf(d.y * f, limbs_f2(c1[0], c1[1], c1[2]), acc1);
     }
 };
 
@@ -743,8 +753,9 @@ struct Row<NTX_Q4_K_T> {
                 n1[l] += mn1 * (int)comp(xsum, l);
             }
             const float f = fs[m];
-            acc0 = fmaf(d.x * f, limbs_f(p0[0], p0[1], p0[2]), fmaf(-dm.x * f, limbs_f(n0[0], n0[1], n0[2]), acc0));
-            acc1 = fmaf(d.y * f, limbs_f(p1[0], p1[1], p1[2]), fmaf(-dm.y * f, limbs_f(n1[0], n1[1], n1[2]), acc1));
+            // |p| <= 63 * 32 * 15 * 128 < 2^22, |n| <= 63 * 32 * 128 per limb
+            acc0 = fmaf(d.x * f, limbs_f2(p0[0], p0[1], p0[2]), fmaf(-dm.x * f, limbs_f2(n0[0], n0[1], n0[2]), acc0));
+            acc1 = fmaf(d.y * f, limbs_f2(p1[0], p1[1], p1[2]), fmaf(-dm.y * f, limbs_f2(n1[0], n1[1], n1[2]), acc1));
         }
     }
 };
@@ -810,8 +821,9 @@ struct Row<NTX_Q5_K_T> {
                 n1[l] += mn1 * (int)comp(xsum, l);
             }
             const float f = fs[m];
-            acc0 = fmaf(d.x * f, limbs_f(p0[0], p0[1], p0[2]), fmaf(-dm.x * f, limbs_f(n0[0], n0[1], n0[2]), acc0));
-            acc1 = fmaf(d.y * f, limbs_f(p1[0], p1[1], p1[2]), fmaf(-dm.y * f, limbs_f(n1[0], n1[1], n1[2]), acc1));
+            // |p| may reach 63 * 32 * 31 * 128 > 2^22: three conversions; |n| <= 63 * 32 * 128
+            acc0 = fmaf(d.x * f, limbs_f(p0[0], p0[1], p0[2]), fmaf(-dm.x * f, limbs_f2(n0[0], n0[1], n0[2]), acc0));
+            acc1 = fmaf(d.y * f, limbs_f(p1[0], p1[1], p1[2]), fmaf(-dm.y * f, limbs_f2(n1[0], n1[1], n1[2]), acc1));
         }
     }
 };
