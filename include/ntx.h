@@ -366,8 +366,12 @@ ntx_status ntx_model_set_layer_skip(ntx_model* model, const uint8_t* skip);
  * pos0 + n - 1.  Token i attends to positions 0 .. pos0 + i, including the K / V rows the
  * earlier tokens of the pass write; its logits go to logits + i vocab (device fp32
  * [n, vocab]).  Every layer runs for all n tokens before the next, so a streamed layer is
- * copied once per pass.  Queued on `compute` (and `copy` for a partly resident model, which
- * must differ); returns after queueing.
+ * copied once per pass, and each fused GEMV of the layer (and the LM head) runs once for up
+ * to 4 tokens, streaming its weights once for all of them (tiled formats whose x vectors
+ * fit in shared memory; otherwise, and with NTX_VERIFY_PER_TOKEN=1 in the environment, one
+ * launch per token).  Per token the arithmetic is that of a one-token step.  Queued on
+ * `compute` (and `copy` for a partly resident model, which must differ); returns after
+ * queueing.
  *
  * ntx_speculative_step: from `token` at `pos`, drafts k - 1 tokens (2 <= k <= 8) greedily
  * with the draft model (the resident layers, minus the layers draft_skip marks: host array

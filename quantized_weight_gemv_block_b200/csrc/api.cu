@@ -72,12 +72,14 @@ NTX_EXPORT ntx_status ntx_device_error(uint32_t* code)
 {
     if (!code) return fail(NTX_EINVAL, "ntx_device_error: null pointer");
     NTX_CUDA_TRY(cudaDeviceSynchronize());
-    uint32_t a = 0, b = 0, c = 0, d = 0, e = 0;
+    uint32_t a = 0, b = 0, c = 0, d = 0, e = 0, f = 0, g = 0;
     NTX_CUDA_TRY(take_device_error_gemv(&a));
     NTX_CUDA_TRY(take_device_error_attn(&b));
     NTX_CUDA_TRY(take_device_error_decode(&c));
     NTX_CUDA_TRY(take_device_error_qmma(&d));
     NTX_CUDA_TRY(take_device_error_probe(&e));
-    *code = a | b | c | d | e;
+    NTX_CUDA_TRY(take_device_error_fgemv(&f));
+    NTX_CUDA_TRY(take_device_error_qmma_multi(&g));
+    *code = a | b | c | d | e | f | g;
     return NTX_OK;
 }

@@ -56,6 +56,8 @@ cudaError_t take_device_error_attn(uint32_t* out);
 cudaError_t take_device_error_decode(uint32_t* out);
 cudaError_t take_device_error_qmma(uint32_t* out);
 cudaError_t take_device_error_probe(uint32_t* out);
+cudaError_t take_device_error_fgemv(uint32_t* out);
+cudaError_t take_device_error_qmma_multi(uint32_t* out);
 
 int num_sms();
 

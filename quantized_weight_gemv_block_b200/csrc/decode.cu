@@ -16,7 +16,9 @@
 // RMSNorm + LM-head GEMV after the last layer.  Kernels use programmatic dependent
 // launch so each one's weight stream starts while the previous one drains; the
 // resident step is recorded once as a CUDA graph and replayed, with token and
-// position read from device memory.
+// position read from device memory.  A verification pass (several tokens, "lanes")
+// runs each layer's fused GEMVs once for up to 4 lanes (qmma_multi.cuh: the weights
+// streamed once), the attention lane by lane.
 #include <chrono>
 #include <cstdlib>
 #include <cstring>
@@ -46,6 +48,7 @@ struct ntx_model {
     float* lane_h = nullptr;
     int32_t* lane_step = nullptr;
     float* lane_rope = nullptr;
+    float* lane_act = nullptr;        // [kMaxLanes]: q [n_q head_dim], attention out [same], SwiGLU out [ffn]
     int32_t* spec_tokens = nullptr;   // [2 kMaxLanes]: drafted tokens, then the full model's predictions
     float* spec_logits = nullptr;     // [kMaxLanes, vocab]
     std::vector<void*> registered;            // host ranges this library registered (unregistered at destroy)
@@ -85,26 +88,30 @@ struct LayerW {
     const void *qkv, *o, *gate, *up, *down;
 };
 
-// The per-token state of a step: hidden state h, the step word (token, pos) and the RoPE
-// table of pos.  A plain step has one; a verification pass has one per token.
+// The per-token state of a step: hidden state h, the step word (token, pos), the RoPE
+// table of pos, and the token's activations (q, attention output, SwiGLU output).  A plain
+// step has one; a verification pass has one per token.
 struct Lane {
     float* h;
     int32_t* step;
     float* rope;
+    float* q;
+    float* att;
+    float* act;
 };
 
-Lane lane0(ntx_model* m) { return {m->h, m->step, m->rope}; }
+Lane lane0(ntx_model* m) { return {m->h, m->step, m->rope, m->q, m->att, m->act}; }
 
-// The fused GEMV launches of a layer, one function per kind, exactly as the step issues them.
-ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
+// The fused GEMV launches of a layer, one function per kind, exactly as the step issues
+// them: the parameters of a kind for one lane, then its launch.
+Params qkv_params(ntx_model* m, int l, const void* w, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
     const ntx_layer_desc& L = m->layers[l];
     const int qd = d.n_q_heads * d.head_dim, kvd = d.n_kv_heads * d.head_dim;
-    const int qt = m->lqt[l].qkv;
     Params P{};
     P.W = (const uint8_t*)w;
-    P.row_bytes = row_bytes(qt, d.hidden);
+    P.row_bytes = row_bytes(m->lqt[l].qkv, d.hidden);
     P.M = qd + 2 * kvd;
     P.K = d.hidden;
     P.x = ln.h;
@@ -118,95 +125,57 @@ ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool p
     P.rope_cs = ln.rope;
     P.k_cache = (__half*)L.k_cache;
     P.v_cache = (__half*)L.v_cache;
-    P.q_out = m->q;
+    P.q_out = ln.q;
     P.use_pdl = pdl;
-    return gemv_launch(qt, gemv::EPI_QKV, gemv::PRO_RMSNORM, P, s);
+    return P;
 }
 
-ntx_status launch_o(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
+Params o_params(ntx_model* m, int l, const void* w, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
-    const int qt = m->lqt[l].o;
     Params P{};
     P.W = (const uint8_t*)w;
     P.K = d.n_q_heads * d.head_dim;
-    P.row_bytes = row_bytes(qt, P.K);
+    P.row_bytes = row_bytes(m->lqt[l].o, P.K);
     P.M = d.hidden;
-    P.x = m->att;
+    P.x = ln.att;
     P.y = ln.h;
     P.use_pdl = pdl;
-    return gemv_launch(qt, gemv::EPI_ADD, gemv::PRO_X, P, s);
+    return P;
 }
 
-ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, cudaStream_t s, bool pdl,
-                          const Lane& ln)
+Params gate_up_params(ntx_model* m, int l, const void* wg, const void* wu, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
-    const int qt = m->lqt[l].ffn;
     Params P{};
     P.W = (const uint8_t*)wg;
     P.W2 = (const uint8_t*)wu;
-    P.row_bytes = row_bytes(qt, d.hidden);
+    P.row_bytes = row_bytes(m->lqt[l].ffn, d.hidden);
     P.M = d.ffn;
     P.K = d.hidden;
     P.x = ln.h;
     P.norm_w = m->layers[l].ffn_norm;
     P.eps = d.rms_eps;
-    P.y = m->act;
+    P.y = ln.act;
     P.use_pdl = pdl;
-    return gemv_launch(qt, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, P, s);
+    return P;
 }
 
-ntx_status launch_down(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
+Params down_params(ntx_model* m, int l, const void* w, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
-    const int qt = m->lqt[l].down;
     Params P{};
     P.W = (const uint8_t*)w;
-    P.row_bytes = row_bytes(qt, d.ffn);
+    P.row_bytes = row_bytes(m->lqt[l].down, d.ffn);
     P.M = d.hidden;
     P.K = d.ffn;
-    P.x = m->act;
+    P.x = ln.act;
     P.y = ln.h;
     P.use_pdl = pdl;
-    return gemv_launch(qt, gemv::EPI_ADD, gemv::PRO_X, P, s);
+    return P;
 }
 
-ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl, const Lane& ln)
-{
-    const ntx_model_desc& d = m->d;
-    const ntx_layer_desc& L = m->layers[l];
-    ntx_status st;
-    if (m->calibrating) {
-        // h before the layer, for the similarity of its input and output
-        NTX_CUDA_TRY(cudaMemcpyAsync(m->h_prev, ln.h, (size_t)d.hidden * 4, cudaMemcpyDeviceToDevice, s));
-        pdl = false;
-    }
-    if ((st = launch_qkv(m, l, w.qkv, s, pdl, ln)) != NTX_OK) return st;
-    {
-        AttnArgs a{};
-        a.q = m->q;
-        a.k_cache = (const __half*)L.k_cache;
-        a.v_cache = (const __half*)L.v_cache;
-        a.out = m->att;
-        a.n_q_heads = d.n_q_heads;
-        a.n_kv_heads = d.n_kv_heads;
-        a.head_dim = d.head_dim;
-        a.max_ctx = d.max_ctx;
-        a.pos_dev = ln.step + 1;
-        a.workspace = m->attn_ws;
-        a.n_split = m->n_split;
-        a.pdl = pdl;
-        if ((st = attn_launch(a, s)) != NTX_OK) return st;
-    }
-    if ((st = launch_o(m, l, w.o, s, pdl, ln)) != NTX_OK) return st;
-    if ((st = launch_gate_up(m, l, w.gate, w.up, s, pdl, ln)) != NTX_OK) return st;
-    if ((st = launch_down(m, l, w.down, s, pdl, ln)) != NTX_OK) return st;
-    if (m->calibrating) return cosine_launch(m->h_prev, ln.h, d.hidden, m->cos_dev + l, s);
-    return NTX_OK;
-}
-
-ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl, const Lane& ln)
+Params head_params(ntx_model* m, float* logits, bool pdl, const Lane& ln)
 {
     const ntx_model_desc& d = m->d;
     Params P{};
@@ -219,7 +188,141 @@ ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl, c
     P.eps = d.rms_eps;
     P.y = logits;
     P.use_pdl = pdl;
-    return gemv_launch(m->qt_out, gemv::EPI_STORE, gemv::PRO_RMSNORM, P, s);
+    return P;
+}
+
+ntx_status launch_qkv(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
+{
+    return gemv_launch(m->lqt[l].qkv, gemv::EPI_QKV, gemv::PRO_RMSNORM, qkv_params(m, l, w, pdl, ln), s);
+}
+
+ntx_status launch_o(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
+{
+    return gemv_launch(m->lqt[l].o, gemv::EPI_ADD, gemv::PRO_X, o_params(m, l, w, pdl, ln), s);
+}
+
+ntx_status launch_gate_up(ntx_model* m, int l, const void* wg, const void* wu, cudaStream_t s, bool pdl,
+                          const Lane& ln)
+{
+    return gemv_launch(m->lqt[l].ffn, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, gate_up_params(m, l, wg, wu, pdl, ln),
+                       s);
+}
+
+ntx_status launch_down(ntx_model* m, int l, const void* w, cudaStream_t s, bool pdl, const Lane& ln)
+{
+    return gemv_launch(m->lqt[l].down, gemv::EPI_ADD, gemv::PRO_X, down_params(m, l, w, pdl, ln), s);
+}
+
+ntx_status launch_attention(ntx_model* m, int l, cudaStream_t s, bool pdl, const Lane& ln)
+{
+    const ntx_model_desc& d = m->d;
+    const ntx_layer_desc& L = m->layers[l];
+    AttnArgs a{};
+    a.q = ln.q;
+    a.k_cache = (const __half*)L.k_cache;
+    a.v_cache = (const __half*)L.v_cache;
+    a.out = ln.att;
+    a.n_q_heads = d.n_q_heads;
+    a.n_kv_heads = d.n_kv_heads;
+    a.head_dim = d.head_dim;
+    a.max_ctx = d.max_ctx;
+    a.pos_dev = ln.step + 1;
+    a.workspace = m->attn_ws;
+    a.n_split = m->n_split;
+    a.pdl = pdl;
+    return attn_launch(a, s);
+}
+
+ntx_status enqueue_layer(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl, const Lane& ln)
+{
+    const ntx_model_desc& d = m->d;
+    ntx_status st;
+    if (m->calibrating) {
+        // h before the layer, for the similarity of its input and output
+        NTX_CUDA_TRY(cudaMemcpyAsync(m->h_prev, ln.h, (size_t)d.hidden * 4, cudaMemcpyDeviceToDevice, s));
+        pdl = false;
+    }
+    if ((st = launch_qkv(m, l, w.qkv, s, pdl, ln)) != NTX_OK) return st;
+    if ((st = launch_attention(m, l, s, pdl, ln)) != NTX_OK) return st;
+    if ((st = launch_o(m, l, w.o, s, pdl, ln)) != NTX_OK) return st;
+    if ((st = launch_gate_up(m, l, w.gate, w.up, s, pdl, ln)) != NTX_OK) return st;
+    if ((st = launch_down(m, l, w.down, s, pdl, ln)) != NTX_OK) return st;
+    if (m->calibrating) return cosine_launch(m->h_prev, ln.h, d.hidden, m->cos_dev + l, s);
+    return NTX_OK;
+}
+
+ntx_status enqueue_head(ntx_model* m, float* logits, cudaStream_t s, bool pdl, const Lane& ln)
+{
+    return gemv_launch(m->qt_out, gemv::EPI_STORE, gemv::PRO_RMSNORM, head_params(m, logits, pdl, ln), s);
+}
+
+// One fused GEMV kind over n lanes (params(i): the kind's parameters for lane i): launches
+// of up to 4 lanes each that stream the weights once (tiled formats, when the lanes' x fit
+// in shared memory), else one launch per lane.  NTX_VERIFY_PER_TOKEN=1 in the environment
+// keeps one launch per lane (a test and tuning override).
+template <typename ParamsOf>
+ntx_status launch_lanes(int qt, int epi, int pro, int n, ParamsOf params, cudaStream_t s)
+{
+    const char* env = std::getenv("NTX_VERIFY_PER_TOKEN");
+    const bool per_token = env && env[0] && env[0] != '0';
+    int i = 0;
+    while (i < n) {
+        int done = 0;
+        for (int c = std::min(gemv::kMaxVecs, n - i); c >= 2 && !per_token && !done; --c) {
+            const Params P = params(i);
+            gemv::Vecs V{};
+            for (int v = 0; v < c; ++v) {
+                const Params Pv = params(i + v);
+                V.x[v] = Pv.x;
+                V.y[v] = Pv.y;
+                V.q_out[v] = Pv.q_out;
+                V.pos_dev[v] = Pv.pos_dev;
+                V.rope_cs[v] = Pv.rope_cs;
+            }
+            const ntx_status st = gemv_multi_launch(qt, epi, pro, P, V, c, s);
+            if (st == NTX_OK) done = c;
+            else if (st != NTX_EUNSUPPORTED) return st;
+        }
+        if (!done) {
+            const ntx_status st = gemv_launch(qt, epi, pro, params(i), s);
+            if (st != NTX_OK) return st;
+            done = 1;
+        }
+        i += done;
+    }
+    return NTX_OK;
+}
+
+// Layer l for n lanes (a verification pass): each fused GEMV kind once for all lanes (the
+// weights streamed once per launch of up to 4 lanes), the attention lane by lane.  All
+// lanes' K / V rows are written before any lane's attention runs, and lane i reads rows
+// 0 .. pos_i only, so lane i sees the rows of lanes 0 .. i as in one-token steps.
+ntx_status enqueue_layer_lanes(ntx_model* m, int l, const LayerW& w, cudaStream_t s, const Lane* lanes, int n)
+{
+    if (n == 1) return enqueue_layer(m, l, w, s, false, lanes[0]);
+    const ntx_layer_qt& q = m->lqt[l];
+    ntx_status st;
+    if ((st = launch_lanes(q.qkv, gemv::EPI_QKV, gemv::PRO_RMSNORM, n,
+                           [&](int i) { return qkv_params(m, l, w.qkv, false, lanes[i]); }, s)) != NTX_OK)
+        return st;
+    for (int i = 0; i < n; ++i)
+        if ((st = launch_attention(m, l, s, false, lanes[i])) != NTX_OK) return st;
+    if ((st = launch_lanes(q.o, gemv::EPI_ADD, gemv::PRO_X, n,
+                           [&](int i) { return o_params(m, l, w.o, false, lanes[i]); }, s)) != NTX_OK)
+        return st;
+    if ((st = launch_lanes(q.ffn, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, n,
+                           [&](int i) { return gate_up_params(m, l, w.gate, w.up, false, lanes[i]); }, s)) != NTX_OK)
+        return st;
+    return launch_lanes(q.down, gemv::EPI_ADD, gemv::PRO_X, n,
+                        [&](int i) { return down_params(m, l, w.down, false, lanes[i]); }, s);
+}
+
+// The heads of n lanes, lane i's logits at logits + i vocab.
+ntx_status enqueue_heads(ntx_model* m, float* logits, cudaStream_t s, bool pdl, const Lane* lanes, int n)
+{
+    if (n == 1) return enqueue_head(m, logits, s, pdl, lanes[0]);
+    return launch_lanes(m->qt_out, gemv::EPI_STORE, gemv::PRO_RMSNORM, n,
+                        [&](int i) { return head_params(m, logits + (size_t)i * m->d.vocab, false, lanes[i]); }, s);
 }
 
 LayerW resident_w(const ntx_layer_desc& L) { return {L.w_qkv, L.w_o, L.w_gate, L.w_up, L.w_down}; }
@@ -246,12 +349,11 @@ ntx_status enqueue_resident(ntx_model* m, int n, float* logits, cudaStream_t s, 
             return st;
     for (int l = 0; l < n; ++l) {
         if (!layer_runs(m, l, also_skip)) continue;
-        for (int i = 0; i < n_lanes; ++i)
-            if ((st = enqueue_layer(m, l, resident_w(m->layers[l]), s, pdl, lanes[i])) != NTX_OK) return st;
+        st = n_lanes == 1 ? enqueue_layer(m, l, resident_w(m->layers[l]), s, pdl, lanes[0])
+                          : enqueue_layer_lanes(m, l, resident_w(m->layers[l]), s, lanes, n_lanes);
+        if (st != NTX_OK) return st;
     }
-    if (logits)
-        for (int i = 0; i < n_lanes; ++i)
-            if ((st = enqueue_head(m, logits + (size_t)i * m->d.vocab, s, pdl, lanes[i])) != NTX_OK) return st;
+    if (logits) return enqueue_heads(m, logits, s, pdl, lanes, n_lanes);
     return NTX_OK;
 }
 
@@ -446,6 +548,7 @@ void free_model(ntx_model* m)
     cudaFree(m->lane_h);
     cudaFree(m->lane_step);
     cudaFree(m->lane_rope);
+    cudaFree(m->lane_act);
     cudaFree(m->spec_tokens);
     cudaFree(m->spec_logits);
     for (void* p : m->registered) cudaHostUnregister(p);
@@ -666,11 +769,7 @@ struct CudaRing final : ring::Ops {
         const LayerW w{base + m->off_qkv, base + m->off_o, base + m->off_gate, base + m->off_up, base + m->off_down};
         // every lane goes through the layer while its matrices are in the slot: one copy
         // over the host link serves all of them
-        for (int i = 0; i < n_lanes; ++i) {
-            const ntx_status st = enqueue_layer(m, j, w, cs, false, lanes[i]);
-            if (st != NTX_OK) return st;
-        }
-        return NTX_OK;
+        return enqueue_layer_lanes(m, j, w, cs, lanes, n_lanes);
     }
     ntx_status compute_done(int slot) override
     {
@@ -704,9 +803,7 @@ ntx_status enqueue_streamed_pass(ntx_model* m, float* logits, cudaStream_t cs, c
     if (!streamed.empty()) NTX_CUDA_TRY(cudaStreamWaitEvent(ks, m->ev_start, 0));
     CudaRing ops(m, cs, ks, lanes, n_lanes);
     if ((st = ring::schedule(ops, streamed.data(), (int)streamed.size(), 2)) != NTX_OK) return st;
-    if (logits)
-        for (int i = 0; i < n_lanes; ++i)
-            if ((st = enqueue_head(m, logits + (size_t)i * d.vocab, cs, false, lanes[i])) != NTX_OK) return st;
+    if (logits && (st = enqueue_heads(m, logits, cs, false, lanes, n_lanes)) != NTX_OK) return st;
     NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
     m->last_h2d = ops.h2d;
     return NTX_OK;
@@ -881,17 +978,21 @@ ntx_status ensure_lanes(ntx_model* m)
     cudaError_t e = cudaMalloc((void**)&m->lane_h, (size_t)kMaxLanes * d.hidden * 4);
     if (e == cudaSuccess) e = cudaMalloc((void**)&m->lane_step, (size_t)kMaxLanes * 16);
     if (e == cudaSuccess) e = cudaMalloc((void**)&m->lane_rope, (size_t)kMaxLanes * d.head_dim * 4);
+    if (e == cudaSuccess)
+        e = cudaMalloc((void**)&m->lane_act, (size_t)kMaxLanes * (2 * d.n_q_heads * d.head_dim + d.ffn) * 4);
     if (e == cudaSuccess) e = cudaMalloc((void**)&m->spec_tokens, (size_t)2 * kMaxLanes * 4);
     if (e == cudaSuccess) e = cudaMalloc((void**)&m->spec_logits, (size_t)kMaxLanes * d.vocab * 4);
     if (e != cudaSuccess) {
         cudaFree(m->lane_h);
         cudaFree(m->lane_step);
         cudaFree(m->lane_rope);
+        cudaFree(m->lane_act);
         cudaFree(m->spec_tokens);
         cudaFree(m->spec_logits);
         m->lane_h = nullptr;
         m->lane_step = nullptr;
         m->lane_rope = nullptr;
+        m->lane_act = nullptr;
         m->spec_tokens = nullptr;
         m->spec_logits = nullptr;
         return fail(e == cudaErrorMemoryAllocation ? NTX_ENOMEM : NTX_ECUDA,
@@ -902,7 +1003,11 @@ ntx_status ensure_lanes(ntx_model* m)
 
 Lane lane_at(ntx_model* m, int i)
 {
-    return {m->lane_h + (size_t)i * m->d.hidden, m->lane_step + 4 * i, m->lane_rope + (size_t)i * m->d.head_dim};
+    const ntx_model_desc& d = m->d;
+    const size_t qd = (size_t)d.n_q_heads * d.head_dim;
+    float* a = m->lane_act + (size_t)i * (2 * qd + d.ffn);
+    return {m->lane_h + (size_t)i * d.hidden, m->lane_step + 4 * i, m->lane_rope + (size_t)i * d.head_dim, a, a + qd,
+            a + 2 * qd};
 }
 
 // One pass of the full model over n tokens at positions pos0 .. pos0 + n - 1 (token i

@@ -281,4 +281,6 @@ ntx_status fgemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cuda
     return fail(NTX_EUNSUPPORTED, "gemv: unsupported prologue / epilogue combination");
 }
 
+cudaError_t take_device_error_fgemv(uint32_t* out) { return take_tu_device_error(out); }
+
 }  // namespace ntx

@@ -80,6 +80,17 @@ struct Params {
     uint32_t m24;
 };
 
+// The vectors of one multi-vector tiled GEMV launch (entries v < the launch's count are
+// used): y_v = W x_v with the same fused prologue and epilogue for every v.
+constexpr int kMaxVecs = 4;
+struct Vecs {
+    const float* x[kMaxVecs];          // input, or the vector to normalise (PRO_RMSNORM)
+    float* y[kMaxVecs];                // output (EPI_STORE / EPI_ADD / EPI_SWIGLU)
+    float* q_out[kMaxVecs];            // EPI_QKV: q
+    const int32_t* pos_dev[kMaxVecs];  // EPI_QKV: the vector's position
+    const float* rope_cs[kMaxVecs];    // EPI_QKV: [head_dim / 2][cos, sin] of that position
+};
+
 template <int QT>
 struct Fmt;
 

@@ -14,6 +14,10 @@ ntx_status embed_launch(int qtype, const void* E, int64_t hidden, const int32_t*
 ntx_status set_step_launch(int32_t* step, int32_t token, int32_t pos, float* rope, float theta, int head_dim,
                            cudaStream_t s, const int32_t* token_dev = nullptr);
 ntx_status gemv_launch(int qtype, int epi, int pro, const gemv::Params& P, cudaStream_t s);
+// y_v = W x_v for nx = 2..4 vectors (tiled formats; qmma_multi.cu), each weight streamed once;
+// NTX_EUNSUPPORTED, with nothing launched, when the format or the shape does not allow it.
+ntx_status gemv_multi_launch(int qtype, int epi, int pro, const gemv::Params& P, const gemv::Vecs& V, int nx,
+                             cudaStream_t s);
 // *out_index = the lowest index of the largest x (n <= 2^26), one CTA.
 ntx_status argmax_launch(const float* x, int64_t n, int32_t* out_index, cudaStream_t s);
 // *out = a . b / (|a| |b|) for device fp32 vectors of n <= 2^26 elements (0 if either is zero).

@@ -14,6 +14,9 @@ def ntx():
     return ntx_module()
 
 
+NAMES_T = {0: "q8_0_t", 1: "q4_0_t", 2: "q4_k_t", 3: "q6_k_t", 4: "q5_k_t"}
+
+
 def run_decode(ntx, model, token, pos, stream_layers=False):
     s = model.spec
     logits = torch.full((s.vocab,), float("nan"), dtype=torch.float32, device="cuda")
@@ -340,6 +343,43 @@ def test_verify_tokens_against_oracle(ntx, syn, n_resident):
     for i in range(len(tokens)):
         assert rel_err(got[i], want[i]) <= TOL, i
         assert elem_err(got[i], want[i]) <= TOL, i
+
+
+VERIFY_BATCH = [(0, 4), (1, 4), (2, 4), (3, 4), (4, 4), (0, 6), (3, 3), (0, 2)]
+
+
+@pytest.mark.parametrize("qtype,k", VERIFY_BATCH, ids=[f"{NAMES_T[q]}-{k}tokens" for q, k in VERIFY_BATCH])
+def test_verify_pass_batches_tokens(ntx, syn, monkeypatch, qtype, k):
+    """The verification pass runs each fused GEMV kind once for up to four tokens (every
+    weight streamed once for all of them: 4 + 2 launches for six tokens; three for the
+    14336-column down projection, whose four x vectors do not fit in shared memory, then
+    one).  Per vector the arithmetic is the one-token kernel's, so with whole rows per CTA
+    (every shape here is below 16384 columns) the logits equal those of one launch per
+    token bit for bit, and they match the oracle."""
+    from oracle import model as om
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, qtype, n_layers=2, tiled=True, vocab=1008)
+    tokens = [17, 5, 1007, 0, 333, 64][:k]
+    pos0 = spec.n_prefill
+    m = DeviceModel(spec)
+    cs, ks = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def verify():
+        out = torch.full((k, spec.vocab), float("nan"), dtype=torch.float32, device="cuda")
+        ntx.ntx_verify_tokens(m.handle, tokens, pos0, out, cs.cuda_stream, ks.cuda_stream)
+        torch.cuda.synchronize()
+        assert ntx.ntx_device_error() == 0
+        return out.cpu().numpy()
+
+    batched = verify()
+    monkeypatch.setenv("NTX_VERIFY_PER_TOKEN", "1")
+    per_token = verify()
+    m.close()
+    assert np.array_equal(batched, per_token)
+    want = om.decode_sequence(spec, tokens, pos0)
+    for i in range(k):
+        assert rel_err(batched[i], want[i]) <= TOL, i
+        assert elem_err(batched[i], want[i]) <= TOL, i
 
 
 def greedy(ntx, m, token, pos, n, streamed):
