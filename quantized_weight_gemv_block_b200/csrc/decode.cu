@@ -297,24 +297,29 @@ ntx_status launch_lanes(int qt, int epi, int pro, int n, ParamsOf params, cudaSt
 // weights streamed once per launch of up to 4 lanes), the attention lane by lane.  All
 // lanes' K / V rows are written before any lane's attention runs, and lane i reads rows
 // 0 .. pos_i only, so lane i sees the rows of lanes 0 .. i as in one-token steps.
-ntx_status enqueue_layer_lanes(ntx_model* m, int l, const LayerW& w, cudaStream_t s, const Lane* lanes, int n)
+// The GEMVs may launch as programmatic dependents (pdl): what they read before their wait
+// (weights, norm weights, the lanes' RoPE tables) was written before the pass.  The
+// attention never does here: its producer prefetches every row but the newest before its
+// wait, and in a pass the rows of the earlier lanes are written by this layer's QKV launch.
+ntx_status enqueue_layer_lanes(ntx_model* m, int l, const LayerW& w, cudaStream_t s, bool pdl, const Lane* lanes,
+                               int n)
 {
-    if (n == 1) return enqueue_layer(m, l, w, s, false, lanes[0]);
+    if (n == 1) return enqueue_layer(m, l, w, s, pdl, lanes[0]);
     const ntx_layer_qt& q = m->lqt[l];
     ntx_status st;
     if ((st = launch_lanes(q.qkv, gemv::EPI_QKV, gemv::PRO_RMSNORM, n,
-                           [&](int i) { return qkv_params(m, l, w.qkv, false, lanes[i]); }, s)) != NTX_OK)
+                           [&](int i) { return qkv_params(m, l, w.qkv, pdl, lanes[i]); }, s)) != NTX_OK)
         return st;
     for (int i = 0; i < n; ++i)
         if ((st = launch_attention(m, l, s, false, lanes[i])) != NTX_OK) return st;
     if ((st = launch_lanes(q.o, gemv::EPI_ADD, gemv::PRO_X, n,
-                           [&](int i) { return o_params(m, l, w.o, false, lanes[i]); }, s)) != NTX_OK)
+                           [&](int i) { return o_params(m, l, w.o, pdl, lanes[i]); }, s)) != NTX_OK)
         return st;
     if ((st = launch_lanes(q.ffn, gemv::EPI_SWIGLU, gemv::PRO_RMSNORM, n,
-                           [&](int i) { return gate_up_params(m, l, w.gate, w.up, false, lanes[i]); }, s)) != NTX_OK)
+                           [&](int i) { return gate_up_params(m, l, w.gate, w.up, pdl, lanes[i]); }, s)) != NTX_OK)
         return st;
     return launch_lanes(q.down, gemv::EPI_ADD, gemv::PRO_X, n,
-                        [&](int i) { return down_params(m, l, w.down, false, lanes[i]); }, s);
+                        [&](int i) { return down_params(m, l, w.down, pdl, lanes[i]); }, s);
 }
 
 // The heads of n lanes, lane i's logits at logits + i vocab.
@@ -322,7 +327,7 @@ ntx_status enqueue_heads(ntx_model* m, float* logits, cudaStream_t s, bool pdl, 
 {
     if (n == 1) return enqueue_head(m, logits, s, pdl, lanes[0]);
     return launch_lanes(m->qt_out, gemv::EPI_STORE, gemv::PRO_RMSNORM, n,
-                        [&](int i) { return head_params(m, logits + (size_t)i * m->d.vocab, false, lanes[i]); }, s);
+                        [&](int i) { return head_params(m, logits + (size_t)i * m->d.vocab, pdl, lanes[i]); }, s);
 }
 
 LayerW resident_w(const ntx_layer_desc& L) { return {L.w_qkv, L.w_o, L.w_gate, L.w_up, L.w_down}; }
@@ -342,16 +347,15 @@ bool layer_runs(const ntx_model* m, int l, const uint8_t* also_skip)
 ntx_status enqueue_resident(ntx_model* m, int n, float* logits, cudaStream_t s, const Lane* lanes, int n_lanes,
                             const uint8_t* also_skip = nullptr)
 {
-    const bool pdl = m->pdl && n_lanes == 1;
+    const bool pdl = m->pdl;
     ntx_status st;
     for (int i = 0; i < n_lanes; ++i)
-        if ((st = embed_launch(m->qt_embd, m->d.tok_embd, m->d.hidden, lanes[i].step, lanes[i].h, s, pdl)) != NTX_OK)
+        if ((st = embed_launch(m->qt_embd, m->d.tok_embd, m->d.hidden, lanes[i].step, lanes[i].h, s,
+                               pdl && n_lanes == 1)) != NTX_OK)
             return st;
     for (int l = 0; l < n; ++l) {
         if (!layer_runs(m, l, also_skip)) continue;
-        st = n_lanes == 1 ? enqueue_layer(m, l, resident_w(m->layers[l]), s, pdl, lanes[0])
-                          : enqueue_layer_lanes(m, l, resident_w(m->layers[l]), s, lanes, n_lanes);
-        if (st != NTX_OK) return st;
+        if ((st = enqueue_layer_lanes(m, l, resident_w(m->layers[l]), s, pdl, lanes, n_lanes)) != NTX_OK) return st;
     }
     if (logits) return enqueue_heads(m, logits, s, pdl, lanes, n_lanes);
     return NTX_OK;
@@ -769,7 +773,7 @@ struct CudaRing final : ring::Ops {
         const LayerW w{base + m->off_qkv, base + m->off_o, base + m->off_gate, base + m->off_up, base + m->off_down};
         // every lane goes through the layer while its matrices are in the slot: one copy
         // over the host link serves all of them
-        return enqueue_layer_lanes(m, j, w, cs, lanes, n_lanes);
+        return enqueue_layer_lanes(m, j, w, cs, false, lanes, n_lanes);
     }
     ntx_status compute_done(int slot) override
     {
@@ -1078,15 +1082,14 @@ NTX_EXPORT ntx_status ntx_speculative_step(ntx_model* m, int32_t token, int32_t 
     for (int l = 0; l < d.n_layers; ++l) also[l] = (l >= d.n_resident || (draft_skip && draft_skip[l])) ? 1 : 0;
     NTX_CUDA_TRY(cudaMemcpyAsync(drafted, &token, 4, cudaMemcpyHostToDevice, cs));
     const Lane ln = lane0(m);
-    const bool pdl = m->pdl;
-    m->pdl = false;
     for (int i = 0; i + 1 < k && st == NTX_OK; ++i) {
-        // draft step i: the token drafted last, at pos + i; greedy pick of the next one
+        // draft step i: the token drafted last, at pos + i; greedy pick of the next one (the
+        // step word, written by a plain launch that reads the drafted token, precedes every
+        // programmatic dependent of the step, as in ntx_decode_step)
         st = set_step_launch(ln.step, 0, pos + i, ln.rope, d.rope_theta, d.head_dim, cs, drafted + i);
         if (st == NTX_OK) st = enqueue_resident(m, d.n_layers, m->spec_logits, cs, &ln, 1, also.data());
         if (st == NTX_OK) st = argmax_launch(m->spec_logits, d.vocab, drafted + i + 1, cs);
     }
-    m->pdl = pdl;
     if (st != NTX_OK) return st;
     // one pass of the full model over the token and the drafted tokens
     if ((st = enqueue_multi(m, nullptr, drafted, k, pos, m->spec_logits, cs, ks)) != NTX_OK) return st;
