@@ -188,9 +188,29 @@ def gemv_kinds(spec):
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum, one ncu capture of the step's
 # fused launch of each kind, bytes per launch) of the tiled GEMV, and a hash of the kernel
-# sources it was taken with: a changed kernel reports traffic as unknown (null).
-GEMV_TRAFFIC_SRC_SHA = None
-GEMV_TRAFFIC = {}
+# sources it was taken with: a changed kernel reports traffic as unknown (null).  Captured with
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum \
+#       --clock-control none -k regex:qmma_kernel -c 40 --csv --log-file traffic.csv \
+#       python bench.py --workload <workload> --layers 2 --profile-step-gemv --warmup 3
+# (the last five launches: QKV, O, gate/up, down, LM head).
+GEMV_TRAFFIC_SRC_SHA = "1ae6ded15cbea745"
+GEMV_TRAFFIC = {
+    "q6_k_t:qkv:10240x8192": 69152000,
+    "q6_k_t:o:8192x8192": 55166976,
+    "q6_k_t:gate_up:28672x8192": 385610240,
+    "q6_k_t:down:8192x28672": 193017344,
+    "q6_k_t:lm_head:128256x8192": 862616064,
+    "q8_0_t:qkv:6144x4096": 26838016,
+    "q8_0_t:o:4096x4096": 17903104,
+    "q8_0_t:gate_up:14336x4096": 125287680,
+    "q8_0_t:down:4096x14336": 62522880,
+    "q8_0_t:lm_head:128256x4096": 558666496,
+    "q4_k_t:qkv:10240x8192": 47319552,
+    "q4_k_t:o:8192x8192": 37863424,
+    "q4_k_t:gate_up:28672x8192": 264517120,
+    "q4_k_t:down:8192x28672": 132749056,
+    "q4_k_t:lm_head:128256x8192": 591269632,
+}
 
 
 def gemv_sources_sha():
