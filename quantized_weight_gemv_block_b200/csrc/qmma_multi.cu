@@ -1,6 +1,7 @@
 // qmma_multi.cu - host side of the multi-vector tiled GEMV (qmma_multi.cuh): launch
 // shaping and the format / epilogue dispatch.
 #include <algorithm>
+#include <cstdlib>
 
 #include "launch.h"
 #include "qmma_multi.cuh"
@@ -46,6 +47,10 @@ ntx_status launch_m(Params P, const Vecs& V, cudaStream_t s)
     const ntx_status st = ensure_smem_limit((const void*)kern, kSmemLimit);
     if (st != NTX_OK) return st;
     const int n_ctas = std::max(1, std::min(num_sms(), P.M / 16));
+    // NTX_TEST_STALL_STAGE=k (tests of the failure path only): the producer stops before
+    // stage k, so the consumers' bounded wait runs out and the kernel records an error
+    const char* stall = std::getenv("NTX_TEST_STALL_STAGE");
+    P.stall_stage = (stall && stall[0]) ? std::atoi(stall) : -1;
     if (!shape_multi<QT>(P, NX, n_ctas, EPI == gemv::EPI_SWIGLU ? 2 : 1))
         return fail(NTX_EUNSUPPORTED, "gemv (several vectors): the vectors do not fit in shared memory");
     const int smem = kMHeader + NX * P.x_bytes + P.n_stages * P.stage_bytes + P.recv_bytes + 128;

@@ -359,6 +359,11 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_multi_kernel(const Params P,
                 for (int mat = 0; mat < NM && okay; ++mat) {
                     const uint8_t* base = (mat ? P.W2 : P.W) + (int64_t)gi * group_bytes;
                     for (int c = 0; c < NCH; ++c) {
+                        if (issued == P.stall_stage) {
+                            // test of the consumers' bounded wait: stop issuing
+                            okay = false;
+                            break;
+                        }
                         if (!mbar_wait(&empty[s], ph ^ 1u, kWaitPolls)) {
                             record_device_error(DEVERR_EMPTY_WAIT);
                             okay = false;

@@ -57,6 +57,39 @@ def test_gemv_bounded_wait_runs_out_and_the_context_stays_usable(ntx, orc, syn, 
     assert rel_err(y.cpu().numpy(), orc.gemv(syn.Q8_0, host, rows, cols, x.cpu().numpy())) <= GEMV_TIGHT
 
 
+def test_batched_gemv_bounded_wait_runs_out_and_the_pass_recovers(ntx, syn, monkeypatch):
+    """The same for the batched GEMV of a verification pass (two tokens, every fused GEMV
+    batched): with its producer stopped, the pass still completes and records the consumer
+    wait bit; the next pass on the same context matches one launch per token bit for bit."""
+    from synth.device_model import DeviceModel
+    spec = syn.ModelSpec(n_layers=2, hidden=1024, n_q_heads=16, n_kv_heads=4, head_dim=128, ffn=2816, vocab=512,
+                         max_ctx=80, n_prefill=64, qtype=syn.Q8_0, seed=2, tiled=True)
+    m = DeviceModel(spec)
+    tokens = [3, 400]
+    s = torch.cuda.current_stream().cuda_stream
+
+    def verify():
+        out = torch.full((2, spec.vocab), float("nan"), dtype=torch.float32, device="cuda")
+        ntx.ntx_verify_tokens(m.handle, tokens, spec.n_prefill, out, s, s)
+        torch.cuda.synchronize()
+        return out.cpu().numpy()
+
+    assert ntx.ntx_device_error() == 0
+    monkeypatch.setenv("NTX_TEST_STALL_STAGE", "1")
+    t0 = time.time()
+    verify()
+    assert time.time() - t0 < 120
+    code = ntx.ntx_device_error()
+    assert code & DEVERR_FULL_WAIT, code
+    monkeypatch.delenv("NTX_TEST_STALL_STAGE")
+    batched = verify()
+    assert ntx.ntx_device_error() == 0
+    monkeypatch.setenv("NTX_VERIFY_PER_TOKEN", "1")
+    per_token = verify()
+    m.close()
+    assert np.array_equal(batched, per_token)
+
+
 def test_stream_layers_host_wait_times_out_and_work_stays_queued(ntx, syn):
     """A 1 ms limit on a step that streams two ~480 MB layers over the host link runs out:
     NTX_ETIMEOUT, nothing lost; once the stream is synchronised the logits equal those of
