@@ -1008,49 +1008,21 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
             bulk_g2s(xf, P.x + k0, (uint32_t)KR * 4u, xbar, policy_evict_last());
         }
         if (KR > 0 && !mbar_wait(xbar, 0, kWaitPolls) && tid == 0) record_device_error(DEVERR_FULL_WAIT);
-        // (2) one pass: the sum of squares (RMSNorm; it runs over the whole vector), max |x w|
-        // (w = 1 without RMSNorm) over the CTA's columns, and each 32-column step's largest
-        // |x w| (the 8 lanes of a step reduce it; kept at xsf[u] for the conversion).  Float4
-        // i = tid + j kCons, four rounds j at a time, so the shuffle chains of the four overlap.
+        // (2) one pass: the sum of squares (RMSNorm; it runs over the whole vector) and max |x w|
+        // (w = 1 without RMSNorm) over the CTA's columns; float4 i = tid + j kCons
         float ss = 0.f, mw = 0.f;
         const int n_steps = KR / 32, n_rounds = (n_steps + 31) / 32, wl = lane & 7;
-        auto pass4 = [&](int j0, const float4 (&w)[4]) {
-            float m[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = tid + (j0 + k) * kCons;
-                const float4 v = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                if (RMS) ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
-                m[k] = fmaxf(fmaxf(fabsf(v.x * w[k].x), fabsf(v.y * w[k].y)),
-                             fmaxf(fabsf(v.z * w[k].z), fabsf(v.w * w[k].w)));
-                mw = fmaxf(mw, m[k]);
-            }
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], __shfl_xor_sync(0xffffffffu, m[k], o));
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int u = (tid + (j0 + k) * kCons) >> 3;
-                if (wl == 0 && u < n_steps) xsf[u] = m[k];
-            }
+        auto pass1 = [&](const float4& v, const float4& w) {
+            if (RMS) ss = fmaf(v.x, v.x, fmaf(v.y, v.y, fmaf(v.z, v.z, fmaf(v.w, v.w, ss))));
+            mw = fmaxf(mw, fmaxf(fmaxf(fabsf(v.x * w.x), fabsf(v.y * w.y)), fmaxf(fabsf(v.z * w.z), fabsf(v.w * w.w))));
         };
 #pragma unroll
-        for (int j0 = 0; j0 < NW; j0 += 4) {
-            if (j0 < n_rounds) {
-                const float4 w[4] = {wr[j0], wr[j0 + 1], wr[j0 + 2], wr[j0 + 3]};
-                pass4(j0, w);
-            }
+        for (int j = 0; j < NW; ++j) {
+            const int i = tid + j * kCons;
+            if (i < nh) pass1(xf[i], wr[j]);
         }
-        for (int j0 = NW; j0 < n_rounds; j0 += 4) {
-            float4 w[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = tid + (j0 + k) * kCons;
-                w[k] = (RMS && i < nh) ? w4[i] : make_float4(1.f, 1.f, 1.f, 1.f);
-            }
-            pass4(j0, w);
-        }
+        for (int i = tid + NW * kCons; i < nh; i += kCons)
+            pass1(xf[i], RMS ? w4[i] : make_float4(1.f, 1.f, 1.f, 1.f));
         if (RMS) {
             // the other CTA's columns, from global memory, 8 loads in flight per thread
             for (int j0 = tid; j0 < K4 - nh; j0 += 8 * kCons) {
@@ -1087,26 +1059,35 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
         // (3) normalised fp32 -> limbs, in place: 8 lanes per 32-column step, float4
         // i = tid + j kCons; 4 rounds at a time, all reads of a round before its stores.
         // Step u takes 2^(S + e_u) with e_u the extra bits its own largest value leaves room
-        // for (|x| 2^(S + e_u) < 2^22 still holds), and records 2^-e_u.  The step's largest
-        // normalised magnitude is fl(m_u inv) for m_u = max |fl(x w)| of the first pass
-        // (rounding is monotonic); its binary exponent is read from the bits (a subnormal
-        // reads as 2^-127, above its true exponent, which only leaves e_u smaller).
+        // for (|x| 2^(S + e_u) < 2^22 still holds), and records 2^-e_u.  The step's binary
+        // exponent is the largest of its 8 lanes' (each lane's from the float bits of its own
+        // largest normalised magnitude; a subnormal reads as 2^-127, above its true exponent,
+        // which only leaves e_u smaller): the four rounds' exponent bytes travel packed in one
+        // word, so one 3-shuffle chain serves them all.
         {
             auto convert4 = [&](int j0, const float4 (&w)[4]) {
                 XLimbs r[4];
                 float fk[4];
+                float4 v[4];
+                uint32_t packed = 0;
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
-                    const int i = tid + (j0 + k) * kCons, u = i >> 3;
-                    float4 v = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    float m = u < n_steps ? xsf[u] : 0.f;
-                    if (RMS) {
-                        v = make_float4(v.x * w[k].x * inv, v.y * w[k].y * inv, v.z * w[k].z * inv, v.w * w[k].w * inv);
-                        m *= inv;
-                    }
-                    const int lg = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;
-                    const int e = (m > 0.f && m <= 3.4e38f) ? max(0, min(e_cap, 21 - lg - S)) : 0;
-                    r[k] = x_limbs<QT == NTX_Q6_K_T, XSUMS>(v, __uint_as_float((uint32_t)(127 + S + e) << 23));
+                    const int i = tid + (j0 + k) * kCons;
+                    v[k] = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (RMS)
+                        v[k] = make_float4(v[k].x * w[k].x * inv, v[k].y * w[k].y * inv, v[k].z * w[k].z * inv,
+                                           v[k].w * w[k].w * inv);
+                    const float m = fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)), fmaxf(fabsf(v[k].z), fabsf(v[k].w)));
+                    packed |= ((__float_as_uint(m) >> 23) & 0xFFu) << (8 * k);
+                }
+#pragma unroll
+                for (int o = 1; o < 8; o <<= 1) packed = __vmaxu4(packed, __shfl_xor_sync(0xffffffffu, packed, o));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int be = (int)((packed >> (8 * k)) & 0xFFu);   // biased exponent of the step's max
+                    // a zero step (be = 0) keeps e = e_cap: its limbs are zero either way
+                    const int e = be < 255 ? max(0, min(e_cap, 21 - (be - 127) - S)) : 0;
+                    r[k] = x_limbs<QT == NTX_Q6_K_T, XSUMS>(v[k], __uint_as_float((uint32_t)(127 + S + e) << 23));
                     fk[k] = __uint_as_float((uint32_t)(127 - e) << 23);
                 }
                 __syncwarp();   // every lane of a step has read its floats before any limb word lands

@@ -412,34 +412,19 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_multi_kernel(const Params P,
     }
     if (!mbar_wait(xbar, 0, kWaitPolls) && tid == 0) record_device_error(DEVERR_FULL_WAIT);
 
-    // (2) + (3) per vector, as the single-vector prologue: sum of squares, max |x w| and
-    // the steps' maxima in one pass, then normalised fp32 -> limbs in place
+    // (2) + (3) per vector, as the single-vector prologue: sum of squares and max |x w| in
+    // one pass, then normalised fp32 -> limbs in place with each step's exponent
 #pragma unroll 1
     for (int v = 0; v < NX; ++v) {
         uint32_t* xv = xq + (size_t)v * XW;
         float4* xf = reinterpret_cast<float4*>(xv);
         float* xsf = reinterpret_cast<float*>(xv) + P.fs_off / 4;
         float ss = 0.f, mw = 0.f;
-        for (int j0 = 0; j0 < n_rounds; j0 += 4) {
-            float m[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = tid + (j0 + k) * kCons;
-                const float4 x = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                const float4 w = (RMS && i < nh) ? w4[i] : make_float4(1.f, 1.f, 1.f, 1.f);
-                if (RMS) ss = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, ss))));
-                m[k] = fmaxf(fmaxf(fabsf(x.x * w.x), fabsf(x.y * w.y)), fmaxf(fabsf(x.z * w.z), fabsf(x.w * w.w)));
-                mw = fmaxf(mw, m[k]);
-            }
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1)
-#pragma unroll
-                for (int k = 0; k < 4; ++k) m[k] = fmaxf(m[k], __shfl_xor_sync(0xffffffffu, m[k], o));
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int u = (tid + (j0 + k) * kCons) >> 3;
-                if (wl == 0 && u < n_steps) xsf[u] = m[k];
-            }
+        for (int i = tid; i < nh; i += kCons) {
+            const float4 x = xf[i];
+            const float4 w = RMS ? w4[i] : make_float4(1.f, 1.f, 1.f, 1.f);
+            if (RMS) ss = fmaf(x.x, x.x, fmaf(x.y, x.y, fmaf(x.z, x.z, fmaf(x.w, x.w, ss))));
+            mw = fmaxf(mw, fmaxf(fmaxf(fabsf(x.x * w.x), fabsf(x.y * w.y)), fmaxf(fabsf(x.z * w.z), fabsf(x.w * w.w))));
         }
         if (RMS) ss = gemv::warp_sum(ss);
         mw = gemv::warp_max(mw);
@@ -462,19 +447,26 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_multi_kernel(const Params P,
         for (int j0 = 0; j0 < n_rounds; j0 += 4) {
             XLimbs r[4];
             float fk[4];
+            float4 x[4];
+            uint32_t packed = 0;   // the four rounds' exponent bytes of each lane's largest value
 #pragma unroll
             for (int k = 0; k < 4; ++k) {
-                const int i = tid + (j0 + k) * kCons, u = i >> 3;
-                float4 x = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
-                float m = u < n_steps ? xsf[u] : 0.f;
+                const int i = tid + (j0 + k) * kCons;
+                x[k] = i < nh ? xf[i] : make_float4(0.f, 0.f, 0.f, 0.f);
                 if (RMS) {
                     const float4 w = i < nh ? w4[i] : make_float4(1.f, 1.f, 1.f, 1.f);
-                    x = make_float4(x.x * w.x * inv, x.y * w.y * inv, x.z * w.z * inv, x.w * w.w * inv);
-                    m *= inv;
+                    x[k] = make_float4(x[k].x * w.x * inv, x[k].y * w.y * inv, x[k].z * w.z * inv, x[k].w * w.w * inv);
                 }
-                const int lg = (int)((__float_as_uint(m) >> 23) & 0xFFu) - 127;
-                const int e = (m > 0.f && m <= 3.4e38f) ? max(0, min(e_cap, 21 - lg - S)) : 0;
-                r[k] = x_limbs<QT == NTX_Q6_K_T, XSUMS>(x, __uint_as_float((uint32_t)(127 + S + e) << 23));
+                const float m = fmaxf(fmaxf(fabsf(x[k].x), fabsf(x[k].y)), fmaxf(fabsf(x[k].z), fabsf(x[k].w)));
+                packed |= ((__float_as_uint(m) >> 23) & 0xFFu) << (8 * k);
+            }
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) packed = __vmaxu4(packed, __shfl_xor_sync(0xffffffffu, packed, o));
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int be = (int)((packed >> (8 * k)) & 0xFFu);
+                const int e = be < 255 ? max(0, min(e_cap, 21 - (be - 127) - S)) : 0;
+                r[k] = x_limbs<QT == NTX_Q6_K_T, XSUMS>(x[k], __uint_as_float((uint32_t)(127 + S + e) << 23));
                 fk[k] = __uint_as_float((uint32_t)(127 - e) << 23);
             }
             __syncwarp();   // every lane of a step has read its floats before any limb word lands
