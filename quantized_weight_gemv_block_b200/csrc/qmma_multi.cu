@@ -40,10 +40,10 @@ bool shape_multi(Params& P, int nx, int n_ctas, int n_mats)
     return true;
 }
 
-template <int QT, int EPI, int PRO, int NX>
+template <int QT, int EPI, int PRO, int NX, int CORE>
 ntx_status launch_m(Params P, const Vecs& V, cudaStream_t s)
 {
-    auto kern = qmma_multi_kernel<QT, EPI, PRO, NX>;
+    auto kern = qmma_multi_kernel<QT, EPI, PRO, NX, CORE>;
     const ntx_status st = ensure_smem_limit((const void*)kern, kSmemLimit);
     if (st != NTX_OK) return st;
     const int n_ctas = std::max(1, std::min(num_sms(), P.M / 16));
@@ -70,17 +70,33 @@ ntx_status launch_m(Params P, const Vecs& V, cudaStream_t s)
     return NTX_OK;
 }
 
+template <int EPI, int PRO, int NX, int CORE>
+ntx_status launch_c(int qtype, const Params& P, const Vecs& V, cudaStream_t s)
+{
+    switch (qtype) {
+    case NTX_Q8_0_T: return launch_m<NTX_Q8_0_T, EPI, PRO, NX, CORE>(P, V, s);
+    case NTX_Q4_0_T: return launch_m<NTX_Q4_0_T, EPI, PRO, NX, CORE>(P, V, s);
+    case NTX_Q4_K_T: return launch_m<NTX_Q4_K_T, EPI, PRO, NX, CORE>(P, V, s);
+    case NTX_Q6_K_T: return launch_m<NTX_Q6_K_T, EPI, PRO, NX, CORE>(P, V, s);
+    case NTX_Q5_K_T: return launch_m<NTX_Q5_K_T, EPI, PRO, NX, CORE>(P, V, s);
+    default: return fail(NTX_EUNSUPPORTED, "gemv (several vectors): tiled formats only");
+    }
+}
+
+// Which units reduce the codes of a batch: the integer tensor cores (0) or dp4a on the CUDA
+// cores (1).  NTX_VERIFY_CORE=tc / dp4a overrides the choice (a tuning override).
+inline int pick_multi_core()
+{
+    const char* env = std::getenv("NTX_VERIFY_CORE");
+    if (env && env[0] == 't') return 0;
+    if (env && env[0] == 'd') return 1;
+    return 1;
+}
+
 template <int EPI, int PRO, int NX>
 ntx_status launch_q(int qtype, const Params& P, const Vecs& V, cudaStream_t s)
 {
-    switch (qtype) {
-    case NTX_Q8_0_T: return launch_m<NTX_Q8_0_T, EPI, PRO, NX>(P, V, s);
-    case NTX_Q4_0_T: return launch_m<NTX_Q4_0_T, EPI, PRO, NX>(P, V, s);
-    case NTX_Q4_K_T: return launch_m<NTX_Q4_K_T, EPI, PRO, NX>(P, V, s);
-    case NTX_Q6_K_T: return launch_m<NTX_Q6_K_T, EPI, PRO, NX>(P, V, s);
-    case NTX_Q5_K_T: return launch_m<NTX_Q5_K_T, EPI, PRO, NX>(P, V, s);
-    default: return fail(NTX_EUNSUPPORTED, "gemv (several vectors): tiled formats only");
-    }
+    return pick_multi_core() == 0 ? launch_c<EPI, PRO, NX, 0>(qtype, P, V, s) : launch_c<EPI, PRO, NX, 1>(qtype, P, V, s);
 }
 
 template <int NX>

@@ -268,6 +268,169 @@ struct RowsN<NTX_Q5_K_T, NX> {
     }
 };
 
+// Tensor-core units (CORE 0): per step the A fragment (the codes) is built once and
+// multiplied with each vector's B fragment (its limbs, columns gid < 3) by one m16n8k32
+// integer MMA each; per vector the products, offsets, scales and the accumulation are
+// those of the single-vector tensor-core unit (Unit<QT> in qmma.cuh), so acc0[v] / acc1[v]
+// end in units of the lane's C columns' limb (the quad reduction applies the weights).
+
+template <int QT, int NX>
+struct UnitsN;
+
+template <int NX>
+struct UnitsN<NTX_Q8_0_T, NX> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, int XW,
+                                               const Lane& L, float (&acc0)[NX], float (&acc1)[NX])
+    {
+        const uint4 a4 = *reinterpret_cast<const uint4*>(U + 16 * L.lane);
+        const uint32_t a[4] = {a4.x, a4.y, a4.z, a4.w};
+        const float2 d = d_pair(U + 512 + 4 * L.gid);
+#pragma unroll
+        for (int v = 0; v < NX; ++v) {
+            uint32_t b0, b1;
+            b_frag<NTX_Q8_0_T>(xs + v * XW, L, b0, b1);
+            int c[4];
+            mma_s8(c, a, b0, b1);
+            const float f = fs[v * XW];
+            acc0[v] = fmaf((float)(c[0] + 256 * c[1]), d.x * f, acc0[v]);
+            acc1[v] = fmaf((float)(c[2] + 256 * c[3]), d.y * f, acc1[v]);
+        }
+    }
+};
+
+template <int NX>
+struct UnitsN<NTX_Q4_0_T, NX> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, int XW,
+                                               const Lane& L, float (&acc0)[NX], float (&acc1)[NX])
+    {
+        const uint2 pq = *reinterpret_cast<const uint2*>(U + 8 * L.lane);
+        const uint32_t M = 0x0F0F0F0Fu;
+        const uint32_t a[4] = {pq.x & M, pq.y & M, (pq.x >> 4) & M, (pq.y >> 4) & M};
+        const float2 d = d_pair(U + 256 + 4 * L.gid);
+#pragma unroll
+        for (int v = 0; v < NX; ++v) {
+            const uint32_t* x = xs + v * XW;
+            uint32_t b0, b1;
+            b_frag<NTX_Q4_0_T>(x, L, b0, b1);
+            int c[4];
+            mma_u8(c, a, b0, b1);
+            // codes carry +8: subtract 8 x (this lane's two columns' limb sums)
+            const int2 X = *reinterpret_cast<const int2*>(x + 24 + 2 * L.tig);
+            const int off = -8 * (X.x + 256 * X.y);
+            const float f = fs[v * XW];
+            acc0[v] = fmaf((float)(c[0] + 256 * c[1] + off), d.x * f, acc0[v]);
+            acc1[v] = fmaf((float)(c[2] + 256 * c[3] + off), d.y * f, acc1[v]);
+        }
+    }
+};
+
+template <int NX>
+struct UnitsN<NTX_Q6_K_T, NX> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, int XW,
+                                               const Lane& L, float (&acc0)[NX], float (&acc1)[NX])
+    {
+        // this lane's scales: sub-blocks 2m + (tig / 2) of rows gid (bytes 0-7) and gid + 8 (8-15)
+        const uint4 sv = *reinterpret_cast<const uint4*>(U + 3072 + 16 * (2 * L.gid + (L.tig >> 1)));
+        const float2 d = d_pair(U + 3328 + 4 * L.gid);
+        const uint32_t M6 = 0x3F3F3F3Fu;
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const uint8_t* w = U + 384 * m + 12 * L.lane;
+            const uint32_t A = *reinterpret_cast<const uint32_t*>(w);
+            const uint32_t B = *reinterpret_cast<const uint32_t*>(w + 4);
+            const uint32_t C = *reinterpret_cast<const uint32_t*>(w + 8);
+            uint32_t a[4];
+            a[0] = A & M6;
+            a[1] = B & M6;
+            a[2] = C & M6;
+            a[3] = ((A >> 6) & 0x03030303u) | ((B >> 4) & 0x0C0C0C0Cu) | ((C >> 2) & 0x30303030u);
+            int s0, s1;
+            if (m < 4) {
+                s0 = m == 0 ? sbyte<0>(sv.x) : m == 1 ? sbyte<1>(sv.x) : m == 2 ? sbyte<2>(sv.x) : sbyte<3>(sv.x);
+                s1 = m == 0 ? sbyte<0>(sv.z) : m == 1 ? sbyte<1>(sv.z) : m == 2 ? sbyte<2>(sv.z) : sbyte<3>(sv.z);
+            } else {
+                s0 = m == 4 ? sbyte<0>(sv.y) : m == 5 ? sbyte<1>(sv.y) : m == 6 ? sbyte<2>(sv.y) : sbyte<3>(sv.y);
+                s1 = m == 4 ? sbyte<0>(sv.w) : m == 5 ? sbyte<1>(sv.w) : m == 6 ? sbyte<2>(sv.w) : sbyte<3>(sv.w);
+            }
+#pragma unroll
+            for (int v = 0; v < NX; ++v) {
+                const uint32_t* x = xs + v * XW + 32 * m;
+                uint32_t b0, b1;
+                b_frag<NTX_Q6_K_T>(x, L, b0, b1);
+                int c[4];
+                mma_u8(c, a, b0, b1);
+                const int2 X = *reinterpret_cast<const int2*>(x + 24 + 2 * L.tig);
+                // codes carry +32; the step's column totals are exact integers before the fp32 step
+                const int p0 = s0 * (c[0] - 32 * X.x), p1 = s0 * (c[1] - 32 * X.y);
+                const int q0 = s1 * (c[2] - 32 * X.x), q1 = s1 * (c[3] - 32 * X.y);
+                const float f = fs[v * XW + m];
+                acc0[v] = fmaf(d.x * f, fmaf(256.f, (float)p1, (float)p0), acc0[v]);
+                acc1[v] = fmaf(d.y * f, fmaf(256.f, (float)q1, (float)q0), acc1[v]);
+            }
+        }
+    }
+};
+
+// Q4_K (FIVE = false) and Q5_K (FIVE = true) on the tensor cores
+template <bool FIVE, int NX>
+__device__ __forceinline__ void units_k4(const uint8_t* U, const uint32_t* xs, const float* fs, int XW, const Lane& L,
+                                         float (&acc0)[NX], float (&acc1)[NX])
+{
+    constexpr int SOFF = FIVE ? 2560 : 2048, DOFF = FIVE ? 2752 : 2240, STEP = FIVE ? 320 : 256;
+    uint32_t S[8];
+    q4k_scale_words<SOFF>(U, L.gid, S);
+    const uint2 dd = *reinterpret_cast<const uint2*>(U + DOFF + 8 * L.gid);
+    const float2 d = __half22float2(*reinterpret_cast<const __half2*>(&dd.x));
+    const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dd.y));
+    const uint32_t M = 0x0F0F0F0Fu;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+        const uint2 pq = *reinterpret_cast<const uint2*>(U + STEP * m + 8 * L.lane);
+        uint32_t a[4] = {pq.x & M, pq.y & M, (pq.x >> 4) & M, (pq.y >> 4) & M};
+        if constexpr (FIVE) {
+            const uint2 H = *reinterpret_cast<const uint2*>(U + STEP * m + 256 + 8 * L.gid);
+            a[0] |= q5_bits_r(H.x, 2 * L.tig);
+            a[1] |= q5_bits_r(H.y, 2 * L.tig);
+            a[2] |= q5_bits_r(H.x, 2 * L.tig + 1);
+            a[3] |= q5_bits_r(H.y, 2 * L.tig + 1);
+        }
+        const int sc0 = ubyte<0>(S[m]), sc1 = ubyte<1>(S[m]), mn0 = ubyte<2>(S[m]), mn1 = ubyte<3>(S[m]);
+#pragma unroll
+        for (int v = 0; v < NX; ++v) {
+            const uint32_t* x = xs + v * XW + 32 * m;
+            uint32_t b0, b1;
+            b_frag<FIVE ? NTX_Q5_K_T : NTX_Q4_K_T>(x, L, b0, b1);
+            int c[4];
+            mma_u8(c, a, b0, b1);
+            const int2 X = *reinterpret_cast<const int2*>(x + 24 + 2 * L.tig);
+            const int xp = X.x + 256 * X.y;
+            const float f = fs[v * XW + m];
+            acc0[v] = fmaf(d.x * f, fmaf(256.f, (float)(sc0 * c[1]), (float)(sc0 * c[0])),
+                           fmaf(-dm.x * f, (float)(mn0 * xp), acc0[v]));
+            acc1[v] = fmaf(d.y * f, fmaf(256.f, (float)(sc1 * c[3]), (float)(sc1 * c[2])),
+                           fmaf(-dm.y * f, (float)(mn1 * xp), acc1[v]));
+        }
+    }
+}
+
+template <int NX>
+struct UnitsN<NTX_Q4_K_T, NX> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, int XW,
+                                               const Lane& L, float (&acc0)[NX], float (&acc1)[NX])
+    {
+        units_k4<false, NX>(U, xs, fs, XW, L, acc0, acc1);
+    }
+};
+
+template <int NX>
+struct UnitsN<NTX_Q5_K_T, NX> {
+    static __device__ __forceinline__ void run(const uint8_t* U, const uint32_t* xs, const float* fs, int XW,
+                                               const Lane& L, float (&acc0)[NX], float (&acc1)[NX])
+    {
+        units_k4<true, NX>(U, xs, fs, XW, L, acc0, acc1);
+    }
+};
+
 // ------------------------------------------------------------------ epilogue
 
 // Output row `row` of vector v (t = row total, t_up the up-projection total for SwiGLU).
@@ -308,13 +471,15 @@ __device__ __forceinline__ void epilogue_v(const Params& P, const Vecs& V, int v
 
 // ------------------------------------------------------------------ kernel
 
-template <int QT, int EPI, int PRO, int NX>
+// CORE 1: dp4a on the CUDA cores (RowsN); CORE 0: the integer tensor cores (UnitsN).
+template <int QT, int EPI, int PRO, int NX, int CORE>
 __global__ void __launch_bounds__(kThreads, 1) qmma_multi_kernel(const Params P, const Vecs V)
 {
     using T = gemv::Tiled<QT>;
     constexpr int NM = EPI == gemv::EPI_SWIGLU ? 2 : 1;
     constexpr int SPU = T::UK / 32;
-    constexpr bool XSUMS = QT != NTX_Q8_0_T;   // the Q8_0 lane units read no limb sums
+    constexpr bool ROWS = CORE == 1 && QT != NTX_Q8_0_T;           // row-pair units
+    constexpr bool XSUMS = !(CORE == 1 && QT == NTX_Q8_0_T);       // the Q8_0 lane units read no limb sums
     constexpr bool RMS = PRO == gemv::PRO_RMSNORM;
     constexpr int RG = kWarps * NX * NM * 16;   // floats of one reduction buffer
 
@@ -474,8 +639,8 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_multi_kernel(const Params P,
             for (int k = 0; k < 4; ++k) {
                 const int u = (tid + (j0 + k) * kCons) >> 3;
                 if (u < n_steps) {
-                    x_store<QT == NTX_Q6_K_T, QT == NTX_Q8_0_T, XSUMS, false>(
-                        xv + 32 * u, wl, r[k], QT != NTX_Q8_0_T ? 8 * (u & 3) : 0, fk[k]);
+                    x_store<QT == NTX_Q6_K_T, CORE == 1 && QT == NTX_Q8_0_T, XSUMS, CORE == 0>(
+                        xv + 32 * u, wl, r[k], ROWS ? 8 * (u & 3) : 0, fk[k]);
                     if (wl == 0) xsf[u] = fk[k];
                 }
             }
@@ -507,7 +672,11 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_multi_kernel(const Params P,
                 const uint8_t* st = stages + (size_t)s * P.stage_bytes;
                 if (!dead) {
                     const int u0 = c * CE / 32;   // first step of the chunk
-                    if constexpr (QT == NTX_Q8_0_T) {
+                    if constexpr (CORE == 0) {
+                        for (int un = warp; un < n_units; un += kWarps)
+                            UnitsN<QT, NX>::run(st + (size_t)un * T::UB, xq + 32 * (u0 + SPU * un), fs0 + u0 + SPU * un,
+                                                XW, L, acc0, acc1);
+                    } else if constexpr (QT == NTX_Q8_0_T) {
                         for (int un = warp; un < n_units; un += kWarps)
                             RowsN<QT, NX>::run(st + (size_t)un * T::UB, xq + 32 * (u0 + un), XW, L, acc0, acc1);
                     } else if constexpr (QT == NTX_Q4_0_T) {
@@ -531,10 +700,12 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_multi_kernel(const Params P,
                     ph ^= 1u;
                 }
             }
+            // CORE 0: this lane's C columns hold limbs 0, 1 or limb 2
+            const float limb_w = (CORE == 0 && (L.tig & 1)) ? 65536.f : 1.f;
 #pragma unroll
             for (int v = 0; v < NX; ++v) {
                 float a0 = acc0[v], a1 = acc1[v];
-                if constexpr (QT != NTX_Q8_0_T) {
+                if constexpr (ROWS) {
                     // sum over the 4 threads of each gid: lane g < 8 ends with rows g, g + 8
                     a0 += __shfl_xor_sync(0xffffffffu, a0, 8);
                     a1 += __shfl_xor_sync(0xffffffffu, a1, 8);
@@ -545,7 +716,10 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_multi_kernel(const Params P,
                         rg[((warp * NX + v) * NM + mat) * 16 + lane + 8] = a1;
                     }
                 } else {
-                    // quad reduction: lane tig 0 ends with rows gid, gid + 8
+                    // quad reduction (with the limb weights of the MMA's C columns): lane tig 0
+                    // ends with rows gid, gid + 8
+                    a0 *= limb_w;
+                    a1 *= limb_w;
                     a0 += __shfl_xor_sync(0xffffffffu, a0, 1);
                     a1 += __shfl_xor_sync(0xffffffffu, a1, 1);
                     a0 += __shfl_xor_sync(0xffffffffu, a0, 2);

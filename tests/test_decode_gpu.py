@@ -345,19 +345,25 @@ def test_verify_tokens_against_oracle(ntx, syn, n_resident):
         assert elem_err(got[i], want[i]) <= TOL, i
 
 
-VERIFY_BATCH = [(0, 4), (1, 4), (2, 4), (3, 4), (4, 4), (0, 6), (3, 3), (0, 2)]
+VERIFY_BATCH = [(0, 4, "dp4a"), (1, 4, "dp4a"), (2, 4, "dp4a"), (3, 4, "dp4a"), (4, 4, "dp4a"), (0, 6, "dp4a"),
+                (3, 3, "dp4a"), (0, 2, "dp4a"), (0, 4, "tc"), (1, 4, "tc"), (2, 4, "tc"), (3, 4, "tc"), (4, 4, "tc"),
+                (3, 6, "tc")]
 
 
-@pytest.mark.parametrize("qtype,k", VERIFY_BATCH, ids=[f"{NAMES_T[q]}-{k}tokens" for q, k in VERIFY_BATCH])
-def test_verify_pass_batches_tokens(ntx, syn, monkeypatch, qtype, k):
+@pytest.mark.parametrize("qtype,k,core", VERIFY_BATCH,
+                         ids=[f"{NAMES_T[q]}-{k}tokens-{c}" for q, k, c in VERIFY_BATCH])
+def test_verify_pass_batches_tokens(ntx, syn, monkeypatch, qtype, k, core):
     """The verification pass runs each fused GEMV kind once for up to four tokens (every
     weight streamed once for all of them: 4 + 2 launches for six tokens; three for the
     14336-column down projection, whose four x vectors do not fit in shared memory, then
-    one).  Per vector the arithmetic is the one-token kernel's, so with whole rows per CTA
+    one), on the CUDA cores (dp4a) or the integer tensor cores (tc).  Per vector the
+    arithmetic is the one-token kernel's on the same cores, so with whole rows per CTA
     (every shape here is below 16384 columns) the logits equal those of one launch per
     token bit for bit, and they match the oracle."""
     from oracle import model as om
     from synth.device_model import DeviceModel
+    monkeypatch.setenv("NTX_VERIFY_CORE", core)
+    monkeypatch.setenv("NTX_GEMV_CORE", core)
     spec = small_spec(syn, qtype, n_layers=2, tiled=True, vocab=1008)
     tokens = [17, 5, 1007, 0, 333, 64][:k]
     pos0 = spec.n_prefill
