@@ -369,9 +369,12 @@ ntx_status ntx_model_set_layer_skip(ntx_model* model, const uint8_t* skip);
  * copied once per pass, and each fused GEMV of the layer (and the LM head) runs once for up
  * to 4 tokens, streaming its weights once for all of them (tiled formats whose x vectors
  * fit in shared memory; otherwise, and with NTX_VERIFY_PER_TOKEN=1 in the environment, one
- * launch per token).  Per token the arithmetic is that of a one-token step.  Queued on
- * `compute` (and `copy` for a partly resident model, which must differ); returns after
- * queueing.
+ * launch per token).  Per token the arithmetic is that of a one-token step.  On a fully
+ * resident model the pass is recorded as a CUDA graph on first use (per token count and
+ * logits buffer; recorded again after ntx_model_set_layer_skip) and replayed, reading the
+ * tokens and positions from device memory; so are the draft steps of
+ * ntx_speculative_step.  Queued on `compute` (and `copy` for a partly resident model, which
+ * must differ); returns after queueing.
  *
  * ntx_speculative_step: from `token` at `pos`, drafts k - 1 tokens (2 <= k <= 8) greedily
  * with the draft model (the resident layers, minus the layers draft_skip marks: host array

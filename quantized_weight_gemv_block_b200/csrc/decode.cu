@@ -66,6 +66,12 @@ struct ntx_model {
     // CUDA graph of the resident step
     cudaGraphExec_t graph = nullptr;
     float* graph_logits = nullptr;
+    // CUDA graphs of resident verification passes, by token count (1 .. 8), and their logits
+    cudaGraphExec_t vgraph[9] = {};
+    float* vgraph_logits[9] = {};
+    // CUDA graph of a draft step of self-speculative decoding, and the layers it leaves out
+    cudaGraphExec_t dgraph = nullptr;
+    std::vector<uint8_t> dgraph_also;
     // streaming ring
     uint8_t* ring = nullptr;
     size_t slot_bytes = 0;
@@ -545,6 +551,7 @@ size_t hbm_bytes_for(const ntx_model_desc* d, int n)
 }
 
 constexpr int kMaxLanes = 8;   // tokens of one verification pass
+static_assert(sizeof(ntx_model::vgraph) / sizeof(cudaGraphExec_t) == kMaxLanes + 1, "one graph per token count");
 
 void free_model(ntx_model* m)
 {
@@ -557,6 +564,9 @@ void free_model(ntx_model* m)
     cudaFree(m->spec_logits);
     for (void* p : m->registered) cudaHostUnregister(p);
     if (m->graph) cudaGraphExecDestroy(m->graph);
+    for (cudaGraphExec_t g : m->vgraph)
+        if (g) cudaGraphExecDestroy(g);
+    if (m->dgraph) cudaGraphExecDestroy(m->dgraph);
     for (int i = 0; i < 2; ++i) {
         if (m->copy_done[i]) cudaEventDestroy(m->copy_done[i]);
         if (m->slot_free[i]) cudaEventDestroy(m->slot_free[i]);
@@ -671,6 +681,42 @@ NTX_EXPORT ntx_status ntx_model_destroy(ntx_model* model)
     return NTX_OK;
 }
 
+namespace ntx {
+namespace {
+
+// Record what `enqueue` queues on a capture stream as an instantiated CUDA graph (*out).
+template <typename Enqueue>
+ntx_status record_graph(Enqueue enqueue, cudaGraphExec_t* out, const char* who)
+{
+    const std::string w(who);
+    cudaStream_t cap;
+    NTX_CUDA_TRY(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
+    cudaGraph_t g = nullptr;
+    cudaError_t e = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal);
+    if (e != cudaSuccess) {
+        cudaStreamDestroy(cap);
+        return fail(NTX_ECUDA, w + ": begin capture: " + cudaGetErrorString(e));
+    }
+    const ntx_status st = enqueue(cap);
+    e = cudaStreamEndCapture(cap, &g);
+    cudaStreamDestroy(cap);
+    if (st != NTX_OK) {
+        if (g) cudaGraphDestroy(g);
+        return st;
+    }
+    if (e != cudaSuccess) return fail(NTX_ECUDA, w + ": end capture: " + cudaGetErrorString(e));
+    e = cudaGraphInstantiate(out, g, 0);
+    cudaGraphDestroy(g);
+    if (e != cudaSuccess) {
+        *out = nullptr;
+        return fail(NTX_ECUDA, w + ": instantiate: " + cudaGetErrorString(e));
+    }
+    return NTX_OK;
+}
+
+}  // namespace
+}  // namespace ntx
+
 NTX_EXPORT ntx_status ntx_decode_step(ntx_model* m, int32_t token, int32_t pos, float* logits, void* stream)
 {
     if (!m || !logits) return fail(NTX_EINVAL, "ntx_decode_step: null pointer");
@@ -688,28 +734,9 @@ NTX_EXPORT ntx_status ntx_decode_step(ntx_model* m, int32_t token, int32_t pos, 
             cudaGraphExecDestroy(m->graph);
             m->graph = nullptr;
         }
-        cudaStream_t cap;
-        NTX_CUDA_TRY(cudaStreamCreateWithFlags(&cap, cudaStreamNonBlocking));
-        cudaGraph_t g = nullptr;
-        cudaError_t e = cudaStreamBeginCapture(cap, cudaStreamCaptureModeThreadLocal);
-        if (e != cudaSuccess) {
-            cudaStreamDestroy(cap);
-            return fail(NTX_ECUDA, std::string("ntx_decode_step: begin capture: ") + cudaGetErrorString(e));
-        }
-        st = enqueue_resident(m, m->d.n_layers, logits, cap, true);
-        e = cudaStreamEndCapture(cap, &g);
-        cudaStreamDestroy(cap);
-        if (st != NTX_OK) {
-            if (g) cudaGraphDestroy(g);
-            return st;
-        }
-        if (e != cudaSuccess) return fail(NTX_ECUDA, std::string("ntx_decode_step: end capture: ") + cudaGetErrorString(e));
-        e = cudaGraphInstantiate(&m->graph, g, 0);
-        cudaGraphDestroy(g);
-        if (e != cudaSuccess) {
-            m->graph = nullptr;
-            return fail(NTX_ECUDA, std::string("ntx_decode_step: instantiate: ") + cudaGetErrorString(e));
-        }
+        st = record_graph([&](cudaStream_t cap) { return enqueue_resident(m, m->d.n_layers, logits, cap, true); },
+                          &m->graph, "ntx_decode_step");
+        if (st != NTX_OK) return st;
         m->graph_logits = logits;
     }
     NTX_CUDA_TRY(cudaGraphLaunch(m->graph, s));
@@ -900,10 +927,18 @@ NTX_EXPORT ntx_status ntx_model_set_layer_skip(ntx_model* m, const uint8_t* skip
 {
     if (!m) return fail(NTX_EINVAL, "ntx_model_set_layer_skip: null model");
     for (int l = 0; l < m->d.n_layers; ++l) m->skip[l] = skip && skip[l] ? 1 : 0;
-    // the recorded step holds the old set of layers: record it again on the next call
+    // the recorded step and passes hold the old set of layers: record them again on the next call
     if (m->graph) {
         cudaGraphExecDestroy(m->graph);
         m->graph = nullptr;
+    }
+    for (cudaGraphExec_t& g : m->vgraph) {
+        if (g) cudaGraphExecDestroy(g);
+        g = nullptr;
+    }
+    if (m->dgraph) {
+        cudaGraphExecDestroy(m->dgraph);
+        m->dgraph = nullptr;
     }
     return NTX_OK;
 }
@@ -1030,8 +1065,25 @@ ntx_status enqueue_multi(ntx_model* m, const int32_t* tokens, const int32_t* tok
         if (st != NTX_OK) return st;
     }
     if (d.n_resident == d.n_layers) {
-        const ntx_status st = enqueue_resident(m, d.n_layers, logits, cs, lanes, n);
-        if (st != NTX_OK) return st;
+        // the pass body reads every token and position from the lanes' step words, so it is
+        // recorded once per token count (and logits buffer) and replayed
+        if (!m->use_graph) {
+            const ntx_status st = enqueue_resident(m, d.n_layers, logits, cs, lanes, n);
+            if (st != NTX_OK) return st;
+        } else {
+            if (!m->vgraph[n] || m->vgraph_logits[n] != logits) {
+                if (m->vgraph[n]) {
+                    cudaGraphExecDestroy(m->vgraph[n]);
+                    m->vgraph[n] = nullptr;
+                }
+                const ntx_status st = record_graph(
+                    [&](cudaStream_t cap) { return enqueue_resident(m, d.n_layers, logits, cap, lanes, n); },
+                    &m->vgraph[n], "verification pass");
+                if (st != NTX_OK) return st;
+                m->vgraph_logits[n] = logits;
+            }
+            NTX_CUDA_TRY(cudaGraphLaunch(m->vgraph[n], cs));
+        }
         NTX_CUDA_TRY(cudaEventRecord(m->ev_end, cs));
         return NTX_OK;
     }
@@ -1082,12 +1134,32 @@ NTX_EXPORT ntx_status ntx_speculative_step(ntx_model* m, int32_t token, int32_t 
     for (int l = 0; l < d.n_layers; ++l) also[l] = (l >= d.n_resident || (draft_skip && draft_skip[l])) ? 1 : 0;
     NTX_CUDA_TRY(cudaMemcpyAsync(drafted, &token, 4, cudaMemcpyHostToDevice, cs));
     const Lane ln = lane0(m);
+    // the draft step's body reads its token and position from the step word: recorded once
+    // per set of draft layers and replayed
+    if (m->use_graph && (!m->dgraph || m->dgraph_also != also)) {
+        if (m->dgraph) {
+            cudaGraphExecDestroy(m->dgraph);
+            m->dgraph = nullptr;
+        }
+        st = record_graph(
+            [&](cudaStream_t cap) { return enqueue_resident(m, d.n_layers, m->spec_logits, cap, &ln, 1, also.data()); },
+            &m->dgraph, "draft step");
+        if (st != NTX_OK) return st;
+        m->dgraph_also = also;
+    }
     for (int i = 0; i + 1 < k && st == NTX_OK; ++i) {
         // draft step i: the token drafted last, at pos + i; greedy pick of the next one (the
         // step word, written by a plain launch that reads the drafted token, precedes every
         // programmatic dependent of the step, as in ntx_decode_step)
         st = set_step_launch(ln.step, 0, pos + i, ln.rope, d.rope_theta, d.head_dim, cs, drafted + i);
-        if (st == NTX_OK) st = enqueue_resident(m, d.n_layers, m->spec_logits, cs, &ln, 1, also.data());
+        if (st == NTX_OK) {
+            if (m->use_graph) {
+                const cudaError_t e = cudaGraphLaunch(m->dgraph, cs);
+                if (e != cudaSuccess) st = fail(NTX_ECUDA, std::string("draft step: ") + cudaGetErrorString(e));
+            } else {
+                st = enqueue_resident(m, d.n_layers, m->spec_logits, cs, &ln, 1, also.data());
+            }
+        }
         if (st == NTX_OK) st = argmax_launch(m->spec_logits, d.vocab, drafted + i + 1, cs);
     }
     if (st != NTX_OK) return st;

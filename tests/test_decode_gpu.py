@@ -367,25 +367,59 @@ def test_verify_pass_batches_tokens(ntx, syn, monkeypatch, qtype, k, core):
     spec = small_spec(syn, qtype, n_layers=2, tiled=True, vocab=1008)
     tokens = [17, 5, 1007, 0, 333, 64][:k]
     pos0 = spec.n_prefill
-    m = DeviceModel(spec)
     cs, ks = torch.cuda.Stream(), torch.cuda.Stream()
 
     def verify():
+        # a model of its own: a resident pass is recorded as a CUDA graph on first use
+        m = DeviceModel(spec)
         out = torch.full((k, spec.vocab), float("nan"), dtype=torch.float32, device="cuda")
         ntx.ntx_verify_tokens(m.handle, tokens, pos0, out, cs.cuda_stream, ks.cuda_stream)
         torch.cuda.synchronize()
         assert ntx.ntx_device_error() == 0
+        again = torch.full_like(out, float("nan"))
+        ntx.ntx_verify_tokens(m.handle, tokens, pos0, again, cs.cuda_stream, ks.cuda_stream)   # replayed
+        torch.cuda.synchronize()
+        m.close()
+        assert torch.equal(out, again)
         return out.cpu().numpy()
 
     batched = verify()
     monkeypatch.setenv("NTX_VERIFY_PER_TOKEN", "1")
     per_token = verify()
-    m.close()
     assert np.array_equal(batched, per_token)
     want = om.decode_sequence(spec, tokens, pos0)
     for i in range(k):
         assert rel_err(batched[i], want[i]) <= TOL, i
         assert elem_err(batched[i], want[i]) <= TOL, i
+
+
+def test_verify_pass_graph_equals_direct_launches(ntx, syn, monkeypatch):
+    """A resident verification pass replayed from its CUDA graph (tokens and positions read
+    from the lanes' step words) gives the bits of the same pass launched directly, at a
+    second set of tokens and positions too (the graph recorded once is replayed)."""
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, 0, n_layers=2, tiled=True, vocab=1008)
+    cs, ks = torch.cuda.Stream(), torch.cuda.Stream()
+
+    def passes(m):
+        outs = []
+        for tokens, pos0 in (([17, 5, 1007], spec.n_prefill), ([2, 900, 44], spec.n_prefill - 20)):
+            out = torch.full((3, spec.vocab), float("nan"), dtype=torch.float32, device="cuda")
+            ntx.ntx_verify_tokens(m.handle, tokens, pos0, out, cs.cuda_stream, ks.cuda_stream)
+            torch.cuda.synchronize()
+            outs.append(out.cpu().numpy())
+        return outs
+
+    g = DeviceModel(spec)
+    graphed = passes(g)
+    g.close()
+    monkeypatch.setenv("NTX_NO_GRAPH", "1")
+    dm = DeviceModel(spec)
+    direct = passes(dm)
+    dm.close()
+    for a, b in zip(graphed, direct):
+        assert np.array_equal(a, b)
+    assert not np.array_equal(graphed[0], graphed[1])
 
 
 def greedy(ntx, m, token, pos, n, streamed):

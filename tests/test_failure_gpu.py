@@ -62,9 +62,11 @@ def test_batched_gemv_bounded_wait_runs_out_and_the_pass_recovers(ntx, syn, monk
     batched): with its producer stopped, the pass still completes and records the consumer
     wait bit; the next pass on the same context matches one launch per token bit for bit."""
     from synth.device_model import DeviceModel
-    # one layer: each of its four batched GEMVs and the head waits out its poll limit once
+    # one layer: each of its four batched GEMVs and the head waits out its poll limit once;
+    # direct launches (no recorded pass), so each pass reads the test switches anew
     spec = syn.ModelSpec(n_layers=1, hidden=1024, n_q_heads=16, n_kv_heads=4, head_dim=128, ffn=2816, vocab=512,
                          max_ctx=80, n_prefill=64, qtype=syn.Q8_0, seed=2, tiled=True)
+    monkeypatch.setenv("NTX_NO_GRAPH", "1")
     m = DeviceModel(spec)
     tokens = [3, 400]
     s = torch.cuda.current_stream().cuda_stream
