@@ -57,6 +57,7 @@ struct KArgs {
     int32_t n_ctx;
     const int32_t* pos_dev;
     int use_pdl;
+    KvPrefetch pf;              // the next layer's rows [0, pos), fetched into L2 (k null: none)
 };
 
 // Tensor-core helpers (mma.sync m16n8k16, fp16 in, fp32 accumulate).
@@ -115,6 +116,28 @@ __device__ __forceinline__ void tma_box(void* dst, const CUtensorMap* map, int x
         "[%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_addr(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(smem_addr(bar)), "l"(policy)
         : "memory");
+}
+
+// This CTA's share (b of G) of the rows of p (none when p.k is null): CTA b takes head
+// region r = b mod R (R = 2 n_kv: the K heads, then the V heads) and slice j = b / R of the
+// CTAs that share it.  32-bit index arithmetic only (a 64-bit division would raise the
+// register count of the whole kernel).
+__device__ __forceinline__ void kv_prefetch_share(const KvPrefetch& p, int b, int G, int pos)
+{
+    const int R = 2 * p.n_kv;
+    if (!p.k || pos <= 0 || R <= 0) return;
+    const int r = b % R, j = b / R, k = (G - r + R - 1) / R;
+    const int r0 = (int)((unsigned)pos * (unsigned)j / (unsigned)k);
+    const int r1 = (int)((unsigned)pos * (unsigned)(j + 1) / (unsigned)k);
+    const uint8_t* base = (r < p.n_kv ? p.k : p.v) + (int64_t)(r < p.n_kv ? r : r - p.n_kv) * p.head_stride;
+    const uint8_t* q = base + (int64_t)r0 * p.row_b;
+    int64_t n = (int64_t)(r1 - r0) * p.row_b;   // a multiple of 16: row_b is
+    while (n > 0) {
+        const uint32_t c = (uint32_t)(n < 65536 ? n : 65536);
+        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(q), "r"(c) : "memory");
+        q += c;
+        n -= c;
+    }
 }
 
 template <int G>
@@ -204,6 +227,10 @@ __global__ void __launch_bounds__(kThreads, 1) attn_kernel(const __grid_constant
                 ph ^= 1u;
             }
         }
+        // every copy of this CTA is under way: the rows the next layer's attention will read
+        // at this position come from HBM into L2 now, while the GEMVs in between stream
+        // their weights with the evict-first policy
+        if (lane == 0) kv_prefetch_share(a.pf, blockIdx.x, gridDim.x, n_ctx - 1);
     } else if (warp < kSWarps) {
         // ------------------------------------------- score and softmax warps
         // S^T[position][head] = K q^T for positions 16 warp .. +15 of each stage.  q^T is
@@ -575,6 +602,7 @@ ntx_status attn_launch(const AttnArgs& a, cudaStream_t s)
     k.n_ctx = a.n_ctx;
     k.pos_dev = a.pos_dev;
     k.use_pdl = a.pdl ? 1 : 0;
+    k.pf = a.pf;
     switch (G) {
     case 1: return launch_g<1>(k, a.n_q_heads, s, a.pdl);
     case 2: return launch_g<2>(k, a.n_q_heads, s, a.pdl);

@@ -31,6 +31,17 @@ ntx_status repack_launch(int qtype, const void* W, void* W_tiled, int64_t rows, 
 bool gemv_fast_path_ok(int qtype, const void* W, int64_t cols);
 
 // Split-KV decode attention (attn.cu).
+
+// An L2 prefetch of K / V rows that a later kernel will read (a hint: it changes no result):
+// rows [0, pos) of the n_kv heads of one layer's caches, K at k, V at v, head h at
+// h * head_stride bytes, row_b bytes per position.
+struct KvPrefetch {
+    const uint8_t* k;
+    const uint8_t* v;
+    int64_t head_stride;
+    int n_kv, row_b;
+};
+
 struct AttnArgs {
     const float* q;
     const __half* k_cache;
@@ -42,6 +53,8 @@ struct AttnArgs {
     void* workspace;            // split partials (no initialisation needed)
     int n_split;                // CTAs per kv head
     bool pdl;
+    KvPrefetch pf;              // rows of another layer to fetch into L2 once the copies are
+                                // under way (the step's next layer; k null: none)
 };
 ntx_status attn_check(const void* q, const void* k_cache, const void* v_cache, const void* out, int n_q_heads,
                       int n_kv_heads, int head_dim, int32_t n_ctx, int32_t max_ctx, const char* who);

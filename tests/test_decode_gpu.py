@@ -149,6 +149,26 @@ def test_graph_and_direct_launches_agree(ntx, syn, monkeypatch):
     assert np.array_equal(la, lb)
 
 
+def test_kv_prefetch_changes_nothing(ntx, syn, monkeypatch):
+    """The attention launch of each layer fetches the next layer's K / V rows into L2 (a
+    hint); with it turned off the step's logits are the same bits, and with it on they
+    match the oracle (tiled weights, 4 layers, so three layers prefetch for the next)."""
+    from oracle import model as om
+    from synth.device_model import DeviceModel
+    spec = small_spec(syn, 3, n_layers=4, tiled=True)
+    a = DeviceModel(spec)
+    la = run_decode(ntx, a, spec.token(), spec.n_prefill)
+    a.close()
+    monkeypatch.setenv("NTX_L2_PF", "0")
+    b = DeviceModel(spec)
+    lb = run_decode(ntx, b, spec.token(), spec.n_prefill)
+    b.close()
+    assert np.array_equal(la, lb)
+    want, _ = om.decode(spec)
+    assert rel_err(la, want) <= TOL
+    assert elem_err(la, want) <= TOL
+
+
 def test_streamed_equals_resident(ntx, syn):
     """Same kernels, same bytes: streaming layers through the HBM ring is bit-identical."""
     from synth.device_model import DeviceModel
