@@ -193,23 +193,23 @@ def gemv_kinds(spec):
 #       --clock-control none -k regex:qmma_kernel -c 40 --csv --log-file traffic.csv \
 #       python bench.py --workload <workload> --layers 2 --profile-step-gemv --warmup 3
 # (the last five launches: QKV, O, gate/up, down, LM head).
-GEMV_TRAFFIC_SRC_SHA = "c5f1243411b8b1b8"
+GEMV_TRAFFIC_SRC_SHA = "edad805671c881a8"
 GEMV_TRAFFIC = {
-    "q6_k_t:qkv:10240x8192": 68967424,
-    "q6_k_t:o:8192x8192": 55161600,
-    "q6_k_t:gate_up:28672x8192": 385580544,
-    "q6_k_t:down:8192x28672": 192949760,
-    "q6_k_t:lm_head:128256x8192": 862400512,
-    "q8_0_t:qkv:6144x4096": 26833664,
-    "q8_0_t:o:4096x4096": 17900288,
-    "q8_0_t:gate_up:14336x4096": 124925184,
-    "q8_0_t:down:4096x14336": 62507776,
-    "q8_0_t:lm_head:128256x4096": 558641408,
-    "q4_k_t:qkv:10240x8192": 47324160,
-    "q4_k_t:o:8192x8192": 37860608,
-    "q4_k_t:gate_up:28672x8192": 264496128,
-    "q4_k_t:down:8192x28672": 132431872,
-    "q4_k_t:lm_head:128256x8192": 591378688,
+    "q6_k_t:qkv:10240x8192": 68951296,
+    "q6_k_t:o:8192x8192": 55166464,
+    "q6_k_t:gate_up:28672x8192": 385856512,
+    "q6_k_t:down:8192x28672": 192995840,
+    "q6_k_t:lm_head:128256x8192": 862166272,
+    "q8_0_t:qkv:6144x4096": 26833920,
+    "q8_0_t:o:4096x4096": 17900032,
+    "q8_0_t:gate_up:14336x4096": 124950272,
+    "q8_0_t:down:4096x14336": 62517760,
+    "q8_0_t:lm_head:128256x4096": 558389248,
+    "q4_k_t:qkv:10240x8192": 47322624,
+    "q4_k_t:o:8192x8192": 37869568,
+    "q4_k_t:gate_up:28672x8192": 264761600,
+    "q4_k_t:down:8192x28672": 132520960,
+    "q4_k_t:lm_head:128256x8192": 591300352,
 }
 
 

@@ -199,8 +199,14 @@ bool shape(Params& P, int n_clusters, int csize, int n_mats)
     const int max_groups = (P.M / 16 + n_clusters - 1) / n_clusters;
     P.recv_bytes = max_groups * n_mats * 16 * 4;
     const int avail = kSmemLimit - kHeader - P.x_bytes - P.recv_bytes - 128;
-    // chunks of up to 2048 columns (whole units), shrunk until at least 3 stages fit
-    int ce = std::min(kh, 2048) / T::UK * T::UK;
+    // chunks of up to 4096 columns (whole units), shrunk until at least 3 stages fit: each
+    // consumer warp then takes two K-quant units (or 16 Q8_0 units) per stage, two
+    // independent dot chains to interleave, and crosses half as many stage barriers.
+    // Measured on B200 against 2048: Llama-70B Q6_K decode 80.6 -> 85.1 tok/s, Llama-8B
+    // Q8_0 493.4 -> 503.2.  NTX_GEMV_CE overrides the first choice (a tuning override).
+    const char* ce_env = std::getenv("NTX_GEMV_CE");
+    const int ce_max = (ce_env && ce_env[0]) ? std::max(T::UK, std::atoi(ce_env)) : 4096;
+    int ce = std::min(kh, ce_max) / T::UK * T::UK;
     while (ce > T::UK && avail / (ce / T::UK * T::UB) < 3) ce = std::max(T::UK, ce / 2 / T::UK * T::UK);
     if (ce < T::UK || avail <= 0) return false;
     P.chunk_elems = ce;

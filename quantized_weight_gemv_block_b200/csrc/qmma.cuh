@@ -1164,6 +1164,7 @@ __global__ void __launch_bounds__(kThreads, 1) qmma_kernel(const Params P)
                                     Row<QT>::run(st + (size_t)un * T::UB, xc + 32 * un, sx, fc[un], rgid, acc0, acc1);
                             }
                         } else {
+#pragma unroll 2
                             for (int un = warp; un < n_units; un += kWarps)
                                 Row<QT>::run(st + (size_t)un * T::UB, xc + 32 * SPU * un, fc + SPU * un, rgid, rj,
                                              acc0, acc1);

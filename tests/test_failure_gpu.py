@@ -33,11 +33,11 @@ def tiled_q8_0(ntx, syn, rows, cols, seed=3):
 @pytest.mark.parametrize("stage", [0, 1])
 def test_gemv_bounded_wait_runs_out_and_the_context_stays_usable(ntx, orc, syn, monkeypatch, stage):
     """With the producer stopped before stage `stage` (each CTA streams one 16-row group in
-    two 2048-column stages here, so stage 1 stops it half way), every consumer warp's wait
+    two 4096-column stages here, so stage 1 stops it half way), every consumer warp's wait
     for that stage gives up after its poll limit: the kernel still finishes, records the
     consumer wait bit for ntx_device_error(), and the next launch on the same context is
     correct."""
-    rows, cols = 32, 4096
+    rows, cols = 32, 8192
     host, W = tiled_q8_0(ntx, syn, rows, cols)
     x = torch.from_numpy(syn.normal_f32_host(3, 12, cols)).cuda()
     y = torch.empty(rows, dtype=torch.float32, device="cuda")

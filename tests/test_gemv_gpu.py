@@ -250,9 +250,10 @@ def make_tiled(ntx, syn, qtype, rows, cols, seed=1):
     return host, tiled
 
 
-# 16-row groups: one group, fewer groups than SMs, several per SM; several 2048-column
+# 16-row groups: one group, fewer groups than SMs, several per SM; several 4096-column
 # chunks and a partial one; a row shorter than one chunk
 TILED_FAST = [(Q8_0, 48, 4096 + 256), (Q4_0, 48, 4096 + 256), (Q4_K, 48, 8192 + 256), (Q6_K, 48, 8192 + 256),
+              (Q8_0, 48, 8192 + 1024 + 32), (Q4_0, 48, 8192 + 96),
               (Q8_0, 4096, 4096), (Q6_K, 16, 2048), (Q4_0, 304, 1024), (Q8_0, 16, 32), (Q4_K, 16, 256),
               (Q6_K, 4096, 1024 + 256), (Q4_0, 32, 96)]
 
