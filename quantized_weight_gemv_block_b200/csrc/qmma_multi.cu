@@ -26,8 +26,9 @@ bool shape_multi(Params& P, int nx, int n_ctas, int n_mats)
     const int avail = kSmemLimit - kMHeader - nx * P.x_bytes - P.recv_bytes - 128;
     if (avail <= 0) return false;
     // chunks of 2048 columns, shrunk for a third stage only while a chunk keeps at least 8
-    // units: every consumer warp then has a unit of each stage (and takes the same units
-    // as in the single-vector kernel, so each vector's sums are added in the same order)
+    // units: every consumer warp then has a unit of each stage and takes the same columns, in
+    // the same order, as in the single-vector kernel (whose 4096-column chunks hand each warp
+    // the units of two such chunks at once), so each vector's sums are added in the same order
     int ce = std::min(K, 2048) / T::UK * T::UK;
     while (ce / T::UK > 8 && avail / (ce / T::UK * T::UB) < 3) ce = std::max(8 * T::UK, ce / 2 / T::UK * T::UK);
     P.chunk_elems = ce;
